@@ -1,0 +1,231 @@
+"""Plain, slow fp64 CPU oracle for the Llama-3 decoder forward pass.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path may import, call or
+execute this module: only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline / reference legs of ``bench.py`` use it.  It shares no code, table
+or constant with the CUDA library; both sides only receive the same seeded
+inputs from ``llama_decoder_only_rmsnorm_b200.inputs``.
+
+Every quantity is evaluated in float64 with NumPy.  The inputs (bf16- or
+fp32-valued weights and activations) are upcast exactly, so a comparison with
+the GPU measures only the GPU's own rounding.
+
+Sources (the five web pages on the Llama-3 decoder; cited by title + section):
+  [S1] "从0开发大模型—译llama3-from-scratch" (sunaigc.com), sections 1-12.
+  [S2] "Build your own Llama 3 from scratch" (gitcode.csdn.net), sections
+       二 (input block), 三 3.1-3.6 (decoder block), 四 (output block), 六 (inference).
+  [S3] "llama3-from-scratch：输出层与预测" (agent.csdn.net), "预测流程的完整实现".
+  [S4] "Llama3 architecture" blog (joto.ai), GQA and RoPE paragraphs.
+
+Readings taken where the pages are silent or disagree (each also listed in
+the design doc):
+  * RoPE pairs adjacent elements (2i, 2i+1) as one complex number, real part
+    first ([S1] §6.6-6.9, [S2] §3.2); the exponent uses head_dim ([S2] §3.2,
+    frequencies built for dim=head_dim); angles are evaluated exactly in fp64.
+  * A query at position start_pos+t sees keys j <= start_pos+t (the training
+    mask of [S2] §3.4 / [S1] §7.1, shifted by the cache offset).
+  * Query head h reads KV head h // n_rep ([S2] §3.4 repeat_kv, [S1] §8 head//4).
+  * RMSNorm is not rounded between normalising and weighting.
+  * argmax breaks ties toward the lowest vocabulary index.
+
+Parity status: every function below is pinned by ``tests/test_oracle_pins.py``
+except ``forward_stack`` on real checkpoints (parity unpinned for real Meta
+weights: the checkpoint and tokenizer are not available, so the worked
+"42"/token-2983 example of [S1] §12 cannot be reproduced).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "rms_norm", "ffn_hidden_dim", "rope_inverse_frequencies", "rope_angles",
+    "apply_rope", "causal_mask", "gqa_attention", "silu", "swiglu_ffn",
+    "decoder_block", "lm_head", "embed", "forward_stack",
+]
+
+
+def _f64(a):
+    return np.asarray(a, dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------
+# RMSNorm  ([S1] §5 rms_norm; [S2] §3.1 RMSNorm)
+# ---------------------------------------------------------------------------
+def rms_norm(x, weight, eps):
+    """x / sqrt(mean(x^2 over the last axis) + eps) * weight, in fp64."""
+    x = _f64(x)
+    mean_sq = np.mean(x * x, axis=-1, keepdims=True)
+    return x / np.sqrt(mean_sq + eps) * _f64(weight)
+
+
+# ---------------------------------------------------------------------------
+# FFN hidden size rule  ([S2] §3.5 FeedForward.__init__, §3.6 4*dim input)
+# ---------------------------------------------------------------------------
+def ffn_hidden_dim(dim, multiple_of, ffn_dim_multiplier=None):
+    """The block is built with hidden = 4*dim; keep two thirds (truncated),
+    optionally scale by the multiplier (truncated), then round up to a
+    multiple of ``multiple_of``."""
+    hidden = int(2 * (4 * dim) / 3)
+    if ffn_dim_multiplier is not None:
+        hidden = int(ffn_dim_multiplier * hidden)
+    return multiple_of * ((hidden + multiple_of - 1) // multiple_of)
+
+
+# ---------------------------------------------------------------------------
+# RoPE  ([S1] §6.6-6.10; [S2] §3.2; [S4] RoPE paragraphs)
+# ---------------------------------------------------------------------------
+def rope_inverse_frequencies(head_dim, theta):
+    """theta_i = theta ** (-(2i)/head_dim) for pair i in [0, head_dim/2)."""
+    i = np.arange(head_dim // 2, dtype=np.float64)
+    return np.power(np.float64(theta), -(2.0 * i) / head_dim)
+
+
+def rope_angles(positions, head_dim, theta):
+    """Angle m * theta_i for every position m and pair i -> [len(pos), hd/2]."""
+    m = _f64(positions)
+    return np.outer(m, rope_inverse_frequencies(head_dim, theta))
+
+
+def apply_rope(x, positions, theta):
+    """Rotate pairs (x[2i], x[2i+1]) of the last axis by e^{i*m*theta_i}.
+
+    ``x`` has shape [..., S, n_heads, head_dim] and ``positions`` has length S
+    (the token axis is the third from last).  Each pair is read as the complex
+    number x[2i] + 1j*x[2i+1], multiplied by the unit phasor, and written back
+    with the real part first -- the view_as_complex reading of [S2] §3.2.
+    """
+    x = _f64(x)
+    hd = x.shape[-1]
+    ang = rope_angles(positions, hd, theta)                 # [S, hd/2]
+    phasor = np.exp(1j * ang)[:, None, :]                   # [S, 1, hd/2]
+    z = x[..., 0::2] + 1j * x[..., 1::2]                    # [..., S, H, hd/2]
+    zr = z * phasor
+    out = np.empty_like(x)
+    out[..., 0::2] = zr.real
+    out[..., 1::2] = zr.imag
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Causal grouped-query attention  ([S1] §6.11-8; [S2] §3.4; [S4] GQA)
+# ---------------------------------------------------------------------------
+def causal_mask(n_queries, n_keys, start_pos=0):
+    """Additive mask: 0 where key j <= start_pos + t, -inf above ([S1] §7.1)."""
+    t = np.arange(n_queries)[:, None] + start_pos
+    j = np.arange(n_keys)[None, :]
+    return np.where(j <= t, 0.0, -np.inf)
+
+
+def gqa_attention(q, k, v, start_pos=0, return_probs=False):
+    """softmax(q k^T / sqrt(hd) + mask) v for one sequence.
+
+    q: [S, H, hd] (rotated); k, v: [T, KV, hd] with T = start_pos + S.
+    Query head h reads KV head h // (H // KV).  Returns [S, H, hd]
+    (and the [H, S, T] probabilities when ``return_probs``).
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    S, H, hd = q.shape
+    T, KV, _ = k.shape
+    assert H % KV == 0 and T == start_pos + S
+    n_rep = H // KV
+    mask = causal_mask(S, T, start_pos)
+    out = np.empty((S, H, hd))
+    probs = np.empty((H, S, T)) if return_probs else None
+    for h in range(H):
+        g = h // n_rep
+        scores = q[:, h, :] @ k[:, g, :].T / np.sqrt(hd) + mask
+        scores = scores - scores.max(axis=1, keepdims=True)
+        p = np.exp(scores)
+        p = p / p.sum(axis=1, keepdims=True)
+        out[:, h, :] = p @ v[:, g, :]
+        if return_probs:
+            probs[h] = p
+    return (out, probs) if return_probs else out
+
+
+# ---------------------------------------------------------------------------
+# SwiGLU FFN  ([S1] §9.3; [S2] §3.5)
+# ---------------------------------------------------------------------------
+def silu(z):
+    z = _f64(z)
+    return z / (1.0 + np.exp(-z))
+
+
+def swiglu_ffn(x, w1, w2, w3):
+    """w2( silu(x w1^T) * (x w3^T) ) with Linear weights stored [out, in]."""
+    x = _f64(x)
+    return (silu(x @ _f64(w1).T) * (x @ _f64(w3).T)) @ _f64(w2).T
+
+
+# ---------------------------------------------------------------------------
+# One pre-norm decoder block  ([S2] §3.6 TransformerBlock; [S1] §6-10)
+# ---------------------------------------------------------------------------
+def decoder_block(x, layer, cfg, k_cache, v_cache, start_pos=0):
+    """h = x + Attn(RMSNorm(x)); out = h + FFN(RMSNorm(h)).
+
+    x: [B, S, D].  ``layer`` maps the page's weight names (attention_norm, wq,
+    wk, wv, wo, ffn_norm, w1, w2, w3) to arrays in [out, in] layout.
+    k_cache / v_cache: fp64 arrays [B, cap, KV, hd]; positions
+    [start_pos, start_pos+S) are overwritten with this call's rotated k and v
+    ([S2] §3.3 / §3.4 inference branch).  Returns out [B, S, D].
+    """
+    x = _f64(x)
+    B, S, D = x.shape
+    H, KV, hd = cfg["n_heads"], cfg["n_kv_heads"], cfg["head_dim"]
+    eps, theta = cfg["norm_eps"], cfg["rope_theta"]
+    pos = start_pos + np.arange(S)
+
+    xn = rms_norm(x, layer["attention_norm"], eps)
+    q = (xn @ _f64(layer["wq"]).T).reshape(B, S, H, hd)
+    k = (xn @ _f64(layer["wk"]).T).reshape(B, S, KV, hd)
+    v = (xn @ _f64(layer["wv"]).T).reshape(B, S, KV, hd)
+    q = apply_rope(q, pos, theta)
+    k = apply_rope(k, pos, theta)
+    k_cache[:B, start_pos:start_pos + S] = k
+    v_cache[:B, start_pos:start_pos + S] = v
+
+    o = np.empty((B, S, H, hd))
+    for b in range(B):
+        o[b] = gqa_attention(q[b], k_cache[b, :start_pos + S],
+                             v_cache[b, :start_pos + S], start_pos)
+    h = x + o.reshape(B, S, H * hd) @ _f64(layer["wo"]).T
+    hn = rms_norm(h, layer["ffn_norm"], eps)
+    return h + swiglu_ffn(hn, layer["w1"], layer["w2"], layer["w3"])
+
+
+# ---------------------------------------------------------------------------
+# Output block  ([S1] §11-12; [S2] 四; [S3] 预测流程)
+# ---------------------------------------------------------------------------
+def lm_head(h_rows, norm_weight, w_out, eps):
+    """RMSNorm the rows, project onto the vocabulary, take argmax.
+
+    h_rows: [R, D].  Returns (logits [R, V], ids [R]); ids pick the lowest
+    index among equal maxima.
+    """
+    hn = rms_norm(h_rows, norm_weight, eps)
+    logits = hn @ _f64(w_out).T
+    return logits, np.argmax(logits, axis=-1).astype(np.int64)
+
+
+def embed(ids, table):
+    """Row gather x[t] = E[id[t]]  ([S1] §4; [S2] 四 tok_embeddings)."""
+    return _f64(table)[np.asarray(ids)]
+
+
+def forward_stack(x, layers, cfg, k_caches=None, v_caches=None, start_pos=0,
+                  cache_len=None):
+    """Run x through every block in ``layers`` (the layer loop of [S2] 四).
+
+    Creates fp64 caches of length ``cache_len`` (default start_pos+S) when none
+    are given.  Returns (h, k_caches, v_caches).
+    """
+    x = _f64(x)
+    B, S, _ = x.shape
+    cap = cache_len or (start_pos + S)
+    KV, hd = cfg["n_kv_heads"], cfg["head_dim"]
+    if k_caches is None:
+        k_caches = [np.zeros((B, cap, KV, hd)) for _ in layers]
+        v_caches = [np.zeros((B, cap, KV, hd)) for _ in layers]
+    for layer, kc, vc in zip(layers, k_caches, v_caches):
+        x = decoder_block(x, layer, cfg, kc, vc, start_pos)
+    return x, k_caches, v_caches
