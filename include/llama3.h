@@ -1,0 +1,250 @@
+/*
+ * llama3.h -- C ABI of the B200 (sm_100a) Llama-3 decoder forward pass.
+ *
+ * The library computes the decoder described by the Llama-3 pages:
+ *   RMSNorm -> Wq/Wk/Wv -> RoPE (pairwise complex rotation, theta = rope_theta)
+ *   -> causal grouped-query attention -> wo + residual -> RMSNorm
+ *   -> SwiGLU FFN w2(silu(w1 x) * w3 x) + residual,
+ * and after the last block: final RMSNorm -> output projection -> argmax.
+ *
+ * Sources (cited by page title and section):
+ *   [S1] "从0开发大模型—译llama3-from-scratch" (sunaigc.com) §2-§12
+ *   [S2] "Build your own Llama 3 from scratch" (gitcode.csdn.net) §1.2 ModelArgs,
+ *        §3.1 RMSNorm, §3.2 RoPE, §3.3 KV Cache, §3.4 GQA, §3.5 FeedForward,
+ *        §3.6 TransformerBlock, 四 output block, 六 inference
+ *   [S3] "llama3-from-scratch：输出层与预测" (agent.csdn.net) "预测流程的完整实现",
+ *        "性能优化考虑"
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - All tensor arguments are DEVICE pointers into memory the caller allocated
+ *    and owns (weights, activations, caches, RoPE table, workspace).  The
+ *    library never allocates or frees device memory and keeps no pointer
+ *    after a call returns.
+ *  - Row-major, densely packed.  Linear weights are [out, in] and a Linear
+ *    computes y = x W^T ([S1] §6.5, [S2] §3.4 nn.Linear(bias=False)).
+ *  - Element type of activations, weights and caches is cfg->dtype:
+ *    LLAMA3_DTYPE_BF16 (bfloat16, the fast tcgen05 path) or LLAMA3_DTYPE_F32
+ *    (float, SIMT kernels, meant for small models).  Accumulation is fp32.
+ *  - Every device pointer must be 16-byte aligned (LLAMA3_ERR_ALIGN).
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream) and may be captured in a CUDA graph.
+ *  - Return value: LLAMA3_OK (0) or an LLAMA3_ERR_* code.  Invalid arguments
+ *    are rejected on the host before anything is launched.  A device-side
+ *    problem (token id out of range, a bounded wait that gave up) does not
+ *    trap: it is recorded in a per-device status word that
+ *    llama3_device_status() reads and clears.
+ */
+#ifndef LLAMA3_H
+#define LLAMA3_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* llama3_stream_t; /* identical to cudaStream_t */
+
+enum llama3_dtype { LLAMA3_DTYPE_BF16 = 0, LLAMA3_DTYPE_F32 = 1 };
+
+enum llama3_status {
+  LLAMA3_OK = 0,
+  LLAMA3_ERR_ARG = 1,         /* inconsistent config or size argument          */
+  LLAMA3_ERR_ALIGN = 2,       /* pointer not 16-byte aligned / bad stride      */
+  LLAMA3_ERR_WORKSPACE = 3,   /* workspace missing or smaller than required    */
+  LLAMA3_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed             */
+  LLAMA3_ERR_TIMEOUT = 5,     /* device: a bounded wait gave up                */
+  LLAMA3_ERR_TOKEN = 6,       /* device: token id outside [0, vocab)           */
+  LLAMA3_ERR_UNSUPPORTED = 7  /* valid model, but no kernel for this shape     */
+};
+
+/*
+ * Model hyper-parameters -- the ModelArgs / params.json fields of [S1] §2 and
+ * [S2] §1.2.  Constraints checked by every call:
+ *   dim == n_heads * head_dim; n_heads % n_kv_heads == 0; head_dim even and
+ *   in {16, 32, 64, 96, 128} (bf16 needs head_dim >= 64); ffn_hidden >= 1;
+ *   norm_eps > 0; rope_theta > 1; for bf16, dim and ffn_hidden multiples of 8.
+ * ffn_hidden is taken as given (the caller applies the hidden-size rule of
+ * [S2] §3.5 if it wants it).  vocab is only needed by the LM head / embedding.
+ */
+typedef struct llama3_config {
+  int dim;         /* model width D                                   */
+  int n_heads;     /* query heads H                                   */
+  int n_kv_heads;  /* key/value heads KV (query head h uses h/(H/KV)) */
+  int head_dim;    /* hd = D / H                                      */
+  int ffn_hidden;  /* F                                               */
+  int vocab;       /* V (0 if no embedding / LM head is used)         */
+  float norm_eps;  /* RMSNorm epsilon                                 */
+  double rope_theta;
+  int dtype;       /* enum llama3_dtype                               */
+} llama3_config;
+
+/*
+ * Weights of one decoder block, checkpoint names of [S1] §2.  All [out, in]:
+ *   attention_norm, ffn_norm : [D]
+ *   wqkv : [(H + 2*KV) * hd, D]  -- the rows of wq, wk, wv stacked in that
+ *          order (torch.cat((wq, wk, wv), 0)); head j of q is rows j*hd..
+ *   wo   : [D, H*hd]
+ *   w1, w3 : [F, D]    (gate and value paths of SwiGLU, [S2] §3.5)
+ *   w2   : [D, F]
+ */
+typedef struct llama3_layer_weights {
+  const void* attention_norm;
+  const void* wqkv;
+  const void* wo;
+  const void* ffn_norm;
+  const void* w1;
+  const void* w2;
+  const void* w3;
+} llama3_layer_weights;
+
+/*
+ * RoPE table ([S1] §6.7, [S2] §3.2 precompute_freqs_cis).
+ * Writes cos_sin[m][i][0] = cos(m * theta_i), cos_sin[m][i][1] = sin(m * theta_i)
+ * with theta_i = theta^(-2i/head_dim), i < head_dim/2, 0 <= m < max_pos.
+ * Angles are evaluated in double precision on the host and stored as float;
+ * the table (max_pos * head_dim * 4 bytes, device memory) is copied with one
+ * cudaMemcpyAsync on `stream`.  The pages build 2*max_seq_len positions.
+ * Errors: LLAMA3_ERR_ARG (head_dim odd or < 2, max_pos < 1, theta <= 1).
+ */
+int llama3_init_rope_table(float* cos_sin, int head_dim, int max_pos, double theta,
+                           llama3_stream_t stream);
+
+/*
+ * Bytes of workspace that llama3_layer_forward (seq tokens per sequence),
+ * llama3_layer_decode and llama3_lm_head_argmax (up to lm_rows rows) need
+ * for this config and batch.  One buffer of that size serves all three.
+ */
+int llama3_workspace_size(const llama3_config* cfg, int batch, int seq, int lm_rows,
+                          size_t* bytes);
+
+/*
+ * Token embedding gather x[t] = table[ids[t]] ([S1] §4, [S2] 四 tok_embeddings).
+ * ids: int32 [n_tokens]; table: [vocab, D]; x: [n_tokens, D].  An id outside
+ * [0, vocab) writes a zero row and records LLAMA3_ERR_TOKEN on the device.
+ */
+int llama3_embed(const llama3_config* cfg, const int32_t* ids, const void* table, void* x,
+                 int n_tokens, llama3_stream_t stream);
+
+/*
+ * Prefill / chunked prefill of one decoder block ([S2] §3.6 TransformerBlock,
+ * §3.4 Attention.forward with start_pos), in place:
+ *   x <- h + FFN(RMSNorm(h)),  h = x + Attn(RMSNorm(x))
+ * x: [batch, seq, D] (in/out).  k_cache, v_cache: [batch, cache_cap, KV, hd];
+ * this call writes the rotated keys and the values of positions
+ * [start_pos, start_pos + seq) and attends, for the token at position
+ * p = start_pos + t, to cached positions 0..p (causal, diagonal included).
+ * rope: table from llama3_init_rope_table with rope_len >= start_pos + seq.
+ * ws: workspace of at least llama3_workspace_size(cfg, batch, seq, .) bytes.
+ * Errors: LLAMA3_ERR_ARG (start_pos + seq > cache_cap, batch/seq < 1, ...),
+ * LLAMA3_ERR_ALIGN, LLAMA3_ERR_WORKSPACE, LLAMA3_ERR_CUDA.
+ */
+int llama3_layer_forward(const llama3_config* cfg, const llama3_layer_weights* w,
+                         const float* rope, int rope_len, void* x, void* k_cache,
+                         void* v_cache, int cache_cap, int batch, int seq, int start_pos,
+                         void* ws, size_t ws_bytes, llama3_stream_t stream);
+
+/*
+ * One decode step of one block ([S2] 六 generate: one new token per sequence
+ * against the KV cache, §3.3).  Same as llama3_layer_forward with seq = 1:
+ * x: [batch, 1, D]; the new token of every sequence sits at position
+ * start_pos, its k/v are written there, and it attends to positions
+ * 0..start_pos.  Uses split-KV attention and split-K weight streaming.
+ */
+int llama3_layer_decode(const llama3_config* cfg, const llama3_layer_weights* w,
+                        const float* rope, int rope_len, void* x, void* k_cache,
+                        void* v_cache, int cache_cap, int batch, int start_pos, void* ws,
+                        size_t ws_bytes, llama3_stream_t stream);
+
+/*
+ * Output block ([S1] §11-12, [S3] 预测流程): for each of `rows` hidden rows
+ * h[r] = h + r*row_stride (elements), compute logits = RMSNorm(h[r], norm_w)
+ * W_out^T over the vocabulary and ids_out[r] = argmax (lowest index on ties).
+ * w_out: [vocab, D].  logits_out: float [rows, vocab] or NULL (not written).
+ * row_stride lets a caller pick e.g. the last position of every sequence
+ * without a copy (row_stride = seq*D, h = x + (seq-1)*D).
+ * Errors: LLAMA3_ERR_ARG (rows < 1, vocab < 1, row_stride < D), ALIGN,
+ * WORKSPACE, CUDA.
+ */
+int llama3_lm_head_argmax(const llama3_config* cfg, const void* norm_w, const void* w_out,
+                          const void* h, int rows, long long row_stride, int32_t* ids_out,
+                          float* logits_out, void* ws, size_t ws_bytes,
+                          llama3_stream_t stream);
+
+/* ---- building blocks (the steps of the calls above, exposed for tests) ---- */
+
+/* y[r] = x[r] / sqrt(mean(x[r]^2) + eps) * w  ([S1] §5, [S2] §3.1); x rows at
+ * x + r*row_stride, y dense [rows, D]. */
+int llama3_rmsnorm(const llama3_config* cfg, const void* x, long long row_stride,
+                   const void* w, void* y, int rows, llama3_stream_t stream);
+
+/* y[m, n] = sum_k x[m, k] * w[n, k] (+ residual[m, n] when residual != NULL);
+ * x: [m, k], w: [n, k], y/residual: [m, n] (residual may equal y).  k and n
+ * multiples of 8 for bf16.  Uses the same GEMM kernels as the layer calls. */
+int llama3_linear(const llama3_config* cfg, const void* x, const void* w, const void* residual,
+                  void* y, int m, int n, int k, void* ws, size_t ws_bytes,
+                  llama3_stream_t stream);
+
+/* Causal GQA attention alone ([S2] §3.4): q: [batch, seq, H, hd] (already
+ * rotated), caches as in llama3_layer_forward (already holding positions
+ * 0..start_pos+seq-1), out: [batch, seq, H*hd].  seq == 1 uses the decode
+ * (split-KV) kernel. */
+int llama3_attention(const llama3_config* cfg, const void* q, const void* k_cache,
+                     const void* v_cache, int cache_cap, int batch, int seq, int start_pos,
+                     void* out, void* ws, size_t ws_bytes, llama3_stream_t stream);
+
+/* ---- measurement hooks (for benchmarks; no effect on results) ---- */
+
+/* Kernel families a launch timer can follow. */
+enum llama3_kernel_kind {
+  LLAMA3_KERNEL_GEMM_QKV = 1,          /* prefill Wqkv GEMM + RoPE + cache scatter */
+  LLAMA3_KERNEL_GEMM_WO = 2,           /* prefill wo GEMM + residual               */
+  LLAMA3_KERNEL_GEMM_W13 = 3,          /* prefill w1|w3 GEMM + SwiGLU              */
+  LLAMA3_KERNEL_GEMM_W2 = 4,           /* prefill w2 GEMM + residual               */
+  LLAMA3_KERNEL_ATTENTION = 5,         /* prefill causal GQA attention             */
+  LLAMA3_KERNEL_DECODE_GEMM = 6,       /* weight-streaming split-K GEMMs (decode)  */
+  LLAMA3_KERNEL_DECODE_ATTENTION = 7,  /* split-KV decode attention (main kernel)  */
+  LLAMA3_KERNEL_LM_HEAD = 8,           /* LM-head GEMM + argmax                    */
+  LLAMA3_KERNEL_NORM = 9,              /* RMSNorm                                  */
+  LLAMA3_KERNEL_ELEMENTWISE = 10       /* embedding, split-K reductions, misc.     */
+};
+
+/* Record start_events[i] / stop_events[i] (cudaEvent_t handles created by the
+ * caller) on the launching stream around each of the next n_pairs launches
+ * of kernel family `kind`; n_pairs = 0 switches the timer off.  Not
+ * thread-safe: meant for a single benchmarking thread. */
+int llama3_set_launch_timer(int kind, void* const* start_events, void* const* stop_events, int n_pairs);
+
+/* Number of event pairs recorded since the last llama3_set_launch_timer. */
+int llama3_launch_timer_used(void);
+
+/* Kernels launched by this library since it was loaded (all threads). */
+unsigned long long llama3_launch_count(void);
+
+/* ---- status ---- */
+
+/* Static text for a status code. */
+const char* llama3_status_string(int status);
+
+/* Reads and clears the current device's status word (synchronises the
+ * device).  *out receives LLAMA3_OK or the first device-side LLAMA3_ERR_*
+ * recorded since the last call.  Returns LLAMA3_ERR_CUDA if the read fails. */
+int llama3_device_status(int* out);
+
+/* cudaError_t of the last call that returned LLAMA3_ERR_CUDA (0 if none). */
+int llama3_last_cuda_error(void);
+
+/* Kernel selection for diagnosis: 0 (default) = tcgen05/TMA kernels for bf16,
+ * 1 = the plain SIMT kernels for every dtype.  Returns the previous value. */
+int llama3_set_kernel_path(int path);
+
+/* Limit, in milliseconds, of every bounded device-side wait (default 2000). */
+int llama3_set_wait_limit_ms(int ms);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LLAMA3_H */

@@ -1,0 +1,826 @@
+// llama3.cu -- host side of the C ABI declared in include/llama3.h.
+//
+// One translation unit: it includes every kernel header so that the device
+// status word and the kernels live in one module.  Entry points validate
+// every argument before launching anything, build TMA descriptors for the
+// tcgen05 kernels, carve the caller's workspace, and launch on the caller's
+// stream.  No device memory is allocated here.
+#include <math.h>
+#include <string.h>
+
+#include <algorithm>
+#include <atomic>
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+#include "decode_attention.cuh"
+#include "flash_attention.cuh"
+#include "simt.cuh"
+#include "tc_gemm.cuh"
+
+using namespace l3;
+
+namespace {
+
+thread_local int t_last_cuda = 0;
+int g_kernel_path = 0;       // 0 = tcgen05 for bf16, 1 = SIMT everywhere
+int g_wait_ms = 2000;        // bounded device waits
+constexpr int kMaxDevices = 64;
+int g_num_sms[kMaxDevices];
+
+int cuda_fail(cudaError_t e) {
+  t_last_cuda = (int)e;
+  return LLAMA3_ERR_CUDA;
+}
+#define L3_CUDA(call)                            \
+  do {                                           \
+    cudaError_t e_ = (call);                     \
+    if (e_ != cudaSuccess) return cuda_fail(e_); \
+  } while (0)
+#define L3_TRY(call)              \
+  do {                            \
+    int s_ = (call);              \
+    if (s_ != LLAMA3_OK) return s_; \
+  } while (0)
+
+int launch_check() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? LLAMA3_OK : cuda_fail(e);
+}
+
+// Launch accounting and the optional per-family event timer.
+std::atomic<unsigned long long> g_launches{0};
+struct LaunchTimer {
+  int kind = 0, n = 0, used = 0;
+  std::vector<cudaEvent_t> start, stop;
+} g_timer;
+
+void timer_begin(int kind, cudaStream_t st) {
+  if (g_timer.kind == kind && g_timer.used < g_timer.n) cudaEventRecord(g_timer.start[g_timer.used], st);
+}
+void timer_end(int kind, cudaStream_t st) {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (g_timer.kind == kind && g_timer.used < g_timer.n) cudaEventRecord(g_timer.stop[g_timer.used++], st);
+}
+// Launch `call` (a kernel<<<...>>>(...) expression) as family `kind` on `st`.
+#define L3_LAUNCH(kind, st, ...) \
+  do {                             \
+    timer_begin((kind), (st));     \
+    __VA_ARGS__;                   \
+    timer_end((kind), (st));       \
+  } while (0)
+
+int current_device(int* dev) {
+  cudaError_t e = cudaGetDevice(dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (*dev < 0 || *dev >= kMaxDevices) return LLAMA3_ERR_UNSUPPORTED;
+  return LLAMA3_OK;
+}
+
+int num_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  if (!g_num_sms[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    g_num_sms[dev] = n;
+  }
+  return g_num_sms[dev];
+}
+
+unsigned long long wait_ns() { return (unsigned long long)g_wait_ms * 1000000ull; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t esize(const llama3_config* c) { return c->dtype == LLAMA3_DTYPE_F32 ? 4 : 2; }
+
+bool use_tc(const llama3_config* c) { return c->dtype == LLAMA3_DTYPE_BF16 && g_kernel_path == 0; }
+
+int check_config(const llama3_config* c) {
+  if (!c) return LLAMA3_ERR_ARG;
+  if (c->dtype != LLAMA3_DTYPE_BF16 && c->dtype != LLAMA3_DTYPE_F32) return LLAMA3_ERR_ARG;
+  if (c->dim < 1 || c->n_heads < 1 || c->n_kv_heads < 1 || c->head_dim < 2) return LLAMA3_ERR_ARG;
+  if (c->n_heads % c->n_kv_heads) return LLAMA3_ERR_ARG;
+  if (c->dim != c->n_heads * c->head_dim) return LLAMA3_ERR_ARG;
+  const int hd = c->head_dim;
+  if (hd != 16 && hd != 32 && hd != 64 && hd != 96 && hd != 128) return LLAMA3_ERR_ARG;
+  if (c->ffn_hidden < 1 || c->vocab < 0) return LLAMA3_ERR_ARG;
+  if (!(c->norm_eps > 0.f) || !(c->rope_theta > 1.0)) return LLAMA3_ERR_ARG;
+  if (c->dtype == LLAMA3_DTYPE_BF16) {
+    if (hd < 64) return LLAMA3_ERR_ARG;
+    if (c->dim % 8 || c->ffn_hidden % 8) return LLAMA3_ERR_ARG;
+  }
+  return LLAMA3_OK;
+}
+
+// ---------------------------------------------------------------------------
+// TMA descriptors (driver entry point fetched through the runtime, so the
+// library does not link libcuda directly)
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+std::once_flag g_encode_once;
+
+int encode_fn(EncodeTiledFn* fn) {
+  std::call_once(g_encode_once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  *fn = g_encode;
+  return g_encode ? LLAMA3_OK : LLAMA3_ERR_CUDA;
+}
+
+// bf16 matrix [rows, cols] row-major, box of 64 columns x box_rows rows,
+// 128-byte swizzle; out-of-range elements read as zero.
+int make_map(CUtensorMap* m, const void* ptr, long long rows, long long cols, int box_rows) {
+  EncodeTiledFn enc;
+  L3_TRY(encode_fn(&enc));
+  if (!aligned16(ptr) || (cols * 2) % 16) return LLAMA3_ERR_ALIGN;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+  cuuint32_t es[2] = {1u, 1u};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    t_last_cuda = (int)r;
+    return LLAMA3_ERR_CUDA;
+  }
+  return LLAMA3_OK;
+}
+
+// bf16 4-D tensor {d0 (contiguous), d1, d2, d3} with byte strides for d1..d3,
+// box {64, 1, 128, 1}, 128-byte swizzle (one 128-row slab of 64 elements).
+int make_map_4d(CUtensorMap* m, const void* ptr, long long d0, long long d1, long long d2, long long d3,
+                long long s1_bytes, long long s2_bytes, long long s3_bytes) {
+  EncodeTiledFn enc;
+  L3_TRY(encode_fn(&enc));
+  if (!aligned16(ptr) || s1_bytes % 16 || s2_bytes % 16 || s3_bytes % 16) return LLAMA3_ERR_ALIGN;
+  cuuint64_t dims[4] = {(cuuint64_t)d0, (cuuint64_t)d1, (cuuint64_t)d2, (cuuint64_t)d3};
+  cuuint64_t strides[3] = {(cuuint64_t)s1_bytes, (cuuint64_t)s2_bytes, (cuuint64_t)s3_bytes};
+  cuuint32_t box[4] = {64u, 1u, 128u, 1u};
+  cuuint32_t es[4] = {1u, 1u, 1u, 1u};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    t_last_cuda = (int)r;
+    return LLAMA3_ERR_CUDA;
+  }
+  return LLAMA3_OK;
+}
+
+bool flash_attention_supported(int hd, int H, int KV) {
+  (void)H; (void)KV;
+  return hd == 64 || hd == 96 || hd == 128;
+}
+
+template <int HD>
+int run_flash_attention_t(int H, int KV, const void* q, const void* kc, const void* vc, int cap, int B, int S,
+                          int P, void* out, int sms, unsigned long long wns, cudaStream_t st) {
+  using Cfg = FlashCfg<HD>;
+  CUtensorMap mq, mk, mv;
+  const long long e = 2;
+  L3_TRY(make_map_4d(&mq, q, HD, H, S, B, HD * e, (long long)H * HD * e, (long long)S * H * HD * e));
+  L3_TRY(make_map_4d(&mk, kc, HD, KV, P + S, B, HD * e, (long long)KV * HD * e, (long long)cap * KV * HD * e));
+  L3_TRY(make_map_4d(&mv, vc, HD, KV, P + S, B, HD * e, (long long)KV * HD * e, (long long)cap * KV * HD * e));
+  FlashShape fs;
+  fs.B = B; fs.S = S; fs.P = P; fs.H = H; fs.KV = KV;
+  fs.n_rep = H / KV;
+  fs.pairs = (fs.n_rep + 1) / 2;
+  fs.qtiles = (S + 127) / 128;
+  fs.units = B * KV * fs.pairs * fs.qtiles;
+  fs.ldo = H * HD;
+  fs.scale_log2 = (float)(1.4426950408889634 / sqrt((double)HD));
+  auto kern = flash_attention_kernel<HD>;
+  int dev = 0;
+  L3_TRY(current_device(&dev));
+  static bool attr_done[kMaxDevices];
+  if (!attr_done[dev]) {
+    L3_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES));
+    attr_done[dev] = true;
+  }
+  const int grid = std::min(fs.units, sms);
+  L3_LAUNCH(LLAMA3_KERNEL_ATTENTION, st, kern<<<grid, 384, Cfg::SMEM_BYTES, st>>>(mq, mk, mv, (bf16*)out, fs, wns));
+  return launch_check();
+}
+
+int run_flash_attention(int hd, int H, int KV, const void* q, const void* kc, const void* vc, int cap, int B, int S,
+                        int P, void* out, int sms, unsigned long long wns, cudaStream_t st) {
+  switch (hd) {
+    case 64: return run_flash_attention_t<64>(H, KV, q, kc, vc, cap, B, S, P, out, sms, wns, st);
+    case 96: return run_flash_attention_t<96>(H, KV, q, kc, vc, cap, B, S, P, out, sms, wns, st);
+    case 128: return run_flash_attention_t<128>(H, KV, q, kc, vc, cap, B, S, P, out, sms, wns, st);
+    default: return LLAMA3_ERR_UNSUPPORTED;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Workspace layout
+// ---------------------------------------------------------------------------
+constexpr int kMaxSplitK = 16;
+constexpr int kMaxKvSplits = 128;
+
+struct Workspace {
+  size_t xn, q, o, g, part, attn_part, lm_rows, keys, total;
+};
+
+size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+
+Workspace layout(const llama3_config* c, int batch, int seq, int lm_rows) {
+  Workspace w;
+  const size_t es = esize(c);
+  const size_t M = (size_t)batch * seq;
+  const int H = c->n_heads, KV = c->n_kv_heads, hd = c->head_dim, D = c->dim, F = c->ffn_hidden;
+  const size_t nqkv = (size_t)(H + 2 * KV) * hd;
+  const size_t widest = std::max(nqkv, std::max((size_t)D, (size_t)2 * F));
+  size_t off = 0;
+  w.xn = off; off += up256(M * D * es);
+  w.q = off; off += up256(M * H * hd * es);
+  w.o = off; off += up256(M * H * hd * es);
+  w.g = off; off += up256(M * F * es);
+  // fp32 partial sums: whole [M, widest] for the SIMT path; kMaxSplitK slabs of
+  // [batch, widest] for the split-K decode GEMMs.
+  size_t part = kMaxSplitK * (size_t)batch * widest * 4;
+  if (!use_tc(c)) part = std::max(part, M * widest * 4);
+  w.part = off; off += up256(part);
+  w.attn_part = off; off += up256((size_t)batch * H * kMaxKvSplits * (hd + 2) * 4);
+  const size_t R = (size_t)std::max(lm_rows, 1);
+  w.lm_rows = off; off += up256(R * D * es);
+  w.keys = off; off += up256(R * 8);
+  w.total = off;
+  return w;
+}
+
+template <typename T>
+T* ws_at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+// ---------------------------------------------------------------------------
+// tcgen05 GEMM launch helpers
+// ---------------------------------------------------------------------------
+GemmShape make_shape(int rows_a, int rows_a2, int rows_b, int k, int bn, int splits) {
+  GemmShape s;
+  s.rows_a = rows_a;
+  s.rows_a2 = rows_a2;
+  s.rows_b = rows_b;
+  s.k = k;
+  s.tiles_m1 = (rows_a + 127) / 128;
+  s.tiles_m = s.tiles_m1 + (rows_a2 + 127) / 128;
+  s.tiles_n = (rows_b + bn - 1) / bn;
+  s.kblocks = (k + 63) / 64;
+  splits = std::max(1, std::min(splits, s.kblocks));
+  s.kb_per_split = (s.kblocks + splits - 1) / splits;
+  s.splits = (s.kblocks + s.kb_per_split - 1) / s.kb_per_split;
+  s.units = s.splits * s.tiles_m * s.tiles_n;
+  return s;
+}
+
+// Split count that minimises the longest per-CTA stream (persistent grid of
+// one CTA per SM): ceil(units / SMs) * k-blocks per split.
+int choose_splits(int tiles, int kblocks, int sms) {
+  int best = 1;
+  long long best_t = -1;
+  for (int s = 1; s <= std::min(kMaxSplitK, kblocks); ++s) {
+    const int per = (kblocks + s - 1) / s;
+    const int real = (kblocks + per - 1) / per;
+    const long long units = (long long)tiles * real;
+    const long long t = ((units + sms - 1) / sms) * per;
+    if (best_t < 0 || t < best_t) { best_t = t; best = real; }
+  }
+  return best;
+}
+
+template <int BN, int STAGES, int EPI, bool DUAL>
+int launch_gemm(int kind, const CUtensorMap& a, const CUtensorMap& a2, const CUtensorMap& b, const CUtensorMap& b2,
+                const GemmShape& sh, const EpiParams& ep, cudaStream_t st) {
+  using Cfg = TcGemmCfg<BN, STAGES, DUAL>;
+  auto kern = tc_gemm_kernel<BN, STAGES, EPI, DUAL>;
+  int dev = 0;
+  L3_TRY(current_device(&dev));
+  static bool attr_done[kMaxDevices];
+  if (!attr_done[dev]) {
+    L3_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES));
+    attr_done[dev] = true;
+  }
+  if (sh.units <= 0) return LLAMA3_OK;
+  const int grid = std::min(sh.units, num_sms());
+  L3_LAUNCH(kind, st, kern<<<grid, 192, Cfg::SMEM_BYTES, st>>>(a, a2, b, b2, sh, ep, wait_ns()));
+  return launch_check();
+}
+
+EpiParams empty_epi() {
+  EpiParams e;
+  memset(&e, 0, sizeof(e));
+  return e;
+}
+
+// Swapped (weight-streaming) GEMM for few token rows: P[split][t][n] =
+// sum_k W[n, k] X[t, k], with W1|W3 stacked through `w_second`.
+int swapped_partial_gemm(const void* w, int rows_w, const void* w_second, int rows_w2, int out_offset2,
+                         const void* x, int rows_x, int k, float* P, int ldo, int* splits_out,
+                         cudaStream_t st) {
+  CUtensorMap ma, ma2, mb;
+  const int bn = rows_x <= 16 ? 16 : rows_x <= 32 ? 32 : rows_x <= 64 ? 64 : rows_x <= 128 ? 128 : 256;
+  L3_TRY(make_map(&ma, w, rows_w, k, 128));
+  if (w_second) L3_TRY(make_map(&ma2, w_second, rows_w2, k, 128)); else ma2 = ma;
+  L3_TRY(make_map(&mb, x, rows_x, k, bn));
+  const int tiles = ((rows_w + 127) / 128 + (rows_w2 + 127) / 128) * ((rows_x + bn - 1) / bn);
+  const int splits = choose_splits(tiles, (k + 63) / 64, num_sms());
+  GemmShape sh = make_shape(rows_w, w_second ? rows_w2 : 0, rows_x, k, bn, splits);
+  EpiParams ep = empty_epi();
+  ep.out = P;
+  ep.ldo = ldo;
+  ep.split_stride = (long long)rows_x * ldo;
+  ep.out_row_offset2 = out_offset2;
+  *splits_out = sh.splits;
+  switch (bn) {
+    case 16: return launch_gemm<16, 8, EPI_PARTIAL, false>(LLAMA3_KERNEL_DECODE_GEMM, ma, ma2, mb, mb, sh, ep, st);
+    case 32: return launch_gemm<32, 8, EPI_PARTIAL, false>(LLAMA3_KERNEL_DECODE_GEMM, ma, ma2, mb, mb, sh, ep, st);
+    case 64: return launch_gemm<64, 6, EPI_PARTIAL, false>(LLAMA3_KERNEL_DECODE_GEMM, ma, ma2, mb, mb, sh, ep, st);
+    case 128: return launch_gemm<128, 5, EPI_PARTIAL, false>(LLAMA3_KERNEL_DECODE_GEMM, ma, ma2, mb, mb, sh, ep, st);
+    default: return launch_gemm<256, 4, EPI_PARTIAL, false>(LLAMA3_KERNEL_DECODE_GEMM, ma, ma2, mb, mb, sh, ep, st);
+  }
+}
+
+constexpr int kPrefillBN = 256;
+
+// ---------------------------------------------------------------------------
+// SIMT helpers (templated on element type)
+// ---------------------------------------------------------------------------
+template <typename T>
+int simt_gemm(int kind, const void* A, const void* B, float* C, int M, int N, int K, int ldc, cudaStream_t st) {
+  dim3 grid((N + 63) / 64, (M + 63) / 64);
+  L3_LAUNCH(kind, st, gemm_simt_kernel<T><<<grid, 256, 0, st>>>((const T*)A, (const T*)B, C, M, N, K, ldc));
+  return launch_check();
+}
+
+unsigned blocks_for(long long n, int threads) { return (unsigned)((n + threads - 1) / threads); }
+
+template <typename T>
+int run_rmsnorm(const llama3_config* c, const void* x, long long row_stride, const void* w, void* y, int rows,
+                cudaStream_t st) {
+  L3_LAUNCH(LLAMA3_KERNEL_NORM, st, rmsnorm_kernel<T><<<rows, 256, 0, st>>>((const T*)x, row_stride, (const T*)w, (T*)y, c->dim, c->norm_eps));
+  return launch_check();
+}
+int rmsnorm_any(const llama3_config* c, const void* x, long long row_stride, const void* w, void* y, int rows,
+                cudaStream_t st) {
+  return c->dtype == LLAMA3_DTYPE_F32 ? run_rmsnorm<float>(c, x, row_stride, w, y, rows, st)
+                                      : run_rmsnorm<bf16>(c, x, row_stride, w, y, rows, st);
+}
+
+template <typename T>
+int run_attention_simt(const llama3_config* c, const void* q, const void* kc, const void* vc, int cap, int B,
+                       int S, int P, void* out, cudaStream_t st) {
+  const long long warps = (long long)B * S * c->n_heads;
+  const float scale = (float)(1.0 / sqrt((double)c->head_dim));
+  L3_LAUNCH(LLAMA3_KERNEL_ATTENTION, st, attention_simt_kernel<T><<<blocks_for(warps * 32, 256), 256, 0, st>>>(
+      (const T*)q, (const T*)kc, (const T*)vc, (T*)out, B, S, P, c->n_heads, c->n_kv_heads, c->head_dim, cap,
+      scale));
+  return launch_check();
+}
+
+// Decode attention (one query per sequence), split over the key range.
+template <int HD, int NREP>
+int run_decode_attention_t(const llama3_config* c, const void* q, const void* kc, const void* vc, int cap,
+                           int B, int n_keys, void* out, float* part, cudaStream_t st) {
+  const int KV = c->n_kv_heads, H = c->n_heads;
+  const int sms = num_sms();
+  // Enough CTAs for ~4 per SM, each with at least 128 keys.
+  int splits = std::max(1, std::min(kMaxKvSplits, (4 * sms + B * KV - 1) / (B * KV)));
+  splits = std::min(splits, std::max(1, n_keys / 128));
+  int kps = (n_keys + splits - 1) / splits;
+  splits = (n_keys + kps - 1) / kps;
+  const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)HD));
+  dim3 grid(splits, KV, B);
+  L3_LAUNCH(LLAMA3_KERNEL_DECODE_ATTENTION, st, decode_attention_split_kernel<HD, NREP><<<grid, 128, 0, st>>>(
+      (const bf16*)q, (const bf16*)kc, (const bf16*)vc, part, H, KV, cap, n_keys, kps, splits, scale_log2));
+  L3_TRY(launch_check());
+  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, decode_attention_combine_kernel<HD><<<B * H, 128, 0, st>>>(part, (bf16*)out, splits));
+  return launch_check();
+}
+
+template <int HD>
+int run_decode_attention_hd(const llama3_config* c, const void* q, const void* kc, const void* vc, int cap,
+                            int B, int n_keys, void* out, float* part, cudaStream_t st) {
+  switch (c->n_heads / c->n_kv_heads) {
+    case 1: return run_decode_attention_t<HD, 1>(c, q, kc, vc, cap, B, n_keys, out, part, st);
+    case 2: return run_decode_attention_t<HD, 2>(c, q, kc, vc, cap, B, n_keys, out, part, st);
+    case 4: return run_decode_attention_t<HD, 4>(c, q, kc, vc, cap, B, n_keys, out, part, st);
+    case 8: return run_decode_attention_t<HD, 8>(c, q, kc, vc, cap, B, n_keys, out, part, st);
+    default: return LLAMA3_ERR_UNSUPPORTED;
+  }
+}
+
+bool decode_attention_supported(const llama3_config* c) {
+  const int r = c->n_heads / c->n_kv_heads;
+  return use_tc(c) && (c->head_dim == 64 || c->head_dim == 96 || c->head_dim == 128) &&
+         (r == 1 || r == 2 || r == 4 || r == 8);
+}
+
+int attention_dispatch(const llama3_config* c, const void* q, const void* kc, const void* vc, int cap, int B,
+                       int S, int P, void* out, float* part, cudaStream_t st) {
+  if (S == 1 && decode_attention_supported(c)) {
+    switch (c->head_dim) {
+      case 64: return run_decode_attention_hd<64>(c, q, kc, vc, cap, B, P + 1, out, part, st);
+      case 96: return run_decode_attention_hd<96>(c, q, kc, vc, cap, B, P + 1, out, part, st);
+      default: return run_decode_attention_hd<128>(c, q, kc, vc, cap, B, P + 1, out, part, st);
+    }
+  }
+  if (use_tc(c) && flash_attention_supported(c->head_dim, c->n_heads, c->n_kv_heads))
+    return run_flash_attention(c->head_dim, c->n_heads, c->n_kv_heads, q, kc, vc, cap, B, S, P, out, num_sms(),
+                               wait_ns(), st);
+  return c->dtype == LLAMA3_DTYPE_F32 ? run_attention_simt<float>(c, q, kc, vc, cap, B, S, P, out, st)
+                                      : run_attention_simt<bf16>(c, q, kc, vc, cap, B, S, P, out, st);
+}
+
+// ---------------------------------------------------------------------------
+// Layer: SIMT path (any dtype)
+// ---------------------------------------------------------------------------
+template <typename T>
+int layer_simt(const llama3_config* c, const llama3_layer_weights* w, const float* rope, void* x, void* kc,
+               void* vc, int cap, int B, int S, int P, const Workspace& L, void* ws, cudaStream_t st) {
+  const int M = B * S, D = c->dim, H = c->n_heads, KV = c->n_kv_heads, hd = c->head_dim, F = c->ffn_hidden;
+  const int nqkv = (H + 2 * KV) * hd;
+  T* xn = ws_at<T>(ws, L.xn);
+  T* q = ws_at<T>(ws, L.q);
+  T* o = ws_at<T>(ws, L.o);
+  T* g = ws_at<T>(ws, L.g);
+  float* Pp = ws_at<float>(ws, L.part);
+  float* Ap = ws_at<float>(ws, L.attn_part);
+  L3_TRY(run_rmsnorm<T>(c, x, D, w->attention_norm, xn, M, st));
+  L3_TRY(simt_gemm<T>(LLAMA3_KERNEL_GEMM_QKV, xn, w->wqkv, Pp, M, nqkv, D, nqkv, st));
+  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, epi_qkv_rope_kernel<T><<<blocks_for((long long)M * nqkv / 2, 256), 256, 0, st>>>(
+      Pp, 1, 0, M, S, P, H, KV, hd, rope, q, (T*)kc, (T*)vc, cap));
+  L3_TRY(launch_check());
+  L3_TRY(attention_dispatch(c, q, kc, vc, cap, B, S, P, o, Ap, st));
+  L3_TRY(simt_gemm<T>(LLAMA3_KERNEL_GEMM_WO, o, w->wo, Pp, M, D, H * hd, D, st));
+  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, epi_residual_kernel<T><<<blocks_for((long long)M * D, 256), 256, 0, st>>>(Pp, 1, 0, D, (const T*)x, (T*)x, M, D));
+  L3_TRY(launch_check());
+  L3_TRY(run_rmsnorm<T>(c, x, D, w->ffn_norm, xn, M, st));
+  L3_TRY(simt_gemm<T>(LLAMA3_KERNEL_GEMM_W13, xn, w->w1, Pp, M, F, D, 2 * F, st));
+  L3_TRY(simt_gemm<T>(LLAMA3_KERNEL_GEMM_W13, xn, w->w3, Pp + F, M, F, D, 2 * F, st));
+  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, epi_swiglu_kernel<T><<<blocks_for((long long)M * F, 256), 256, 0, st>>>(Pp, 1, 0, g, M, F));
+  L3_TRY(launch_check());
+  L3_TRY(simt_gemm<T>(LLAMA3_KERNEL_GEMM_W2, g, w->w2, Pp, M, D, F, D, st));
+  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, epi_residual_kernel<T><<<blocks_for((long long)M * D, 256), 256, 0, st>>>(Pp, 1, 0, D, (const T*)x, (T*)x, M, D));
+  return launch_check();
+}
+
+// ---------------------------------------------------------------------------
+// Layer: tcgen05 prefill path (bf16)
+// ---------------------------------------------------------------------------
+int layer_tc_prefill(const llama3_config* c, const llama3_layer_weights* w, const float* rope, void* x, void* kc,
+                     void* vc, int cap, int B, int S, int P, const Workspace& L, void* ws, cudaStream_t st) {
+  const int M = B * S, D = c->dim, H = c->n_heads, KV = c->n_kv_heads, hd = c->head_dim, F = c->ffn_hidden;
+  const int nqkv = (H + 2 * KV) * hd;
+  bf16* xn = ws_at<bf16>(ws, L.xn);
+  bf16* q = ws_at<bf16>(ws, L.q);
+  bf16* o = ws_at<bf16>(ws, L.o);
+  bf16* g = ws_at<bf16>(ws, L.g);
+  float* Ap = ws_at<float>(ws, L.attn_part);
+  CUtensorMap mxn, mo, mg, mwqkv, mwo, mw1, mw3, mw2;
+  L3_TRY(make_map(&mxn, xn, M, D, 128));
+  L3_TRY(make_map(&mo, o, M, H * hd, 128));
+  L3_TRY(make_map(&mg, g, M, F, 128));
+  L3_TRY(make_map(&mwqkv, w->wqkv, nqkv, D, kPrefillBN));
+  L3_TRY(make_map(&mwo, w->wo, D, H * hd, kPrefillBN));
+  L3_TRY(make_map(&mw1, w->w1, F, D, 128));
+  L3_TRY(make_map(&mw3, w->w3, F, D, 128));
+  L3_TRY(make_map(&mw2, w->w2, D, F, kPrefillBN));
+
+  // attention half
+  L3_TRY(run_rmsnorm<bf16>(c, x, D, w->attention_norm, xn, M, st));
+  {
+    EpiParams ep = empty_epi();
+    ep.seq = S; ep.start_pos = P; ep.n_heads = H; ep.n_kv = KV; ep.head_dim = hd; ep.cache_cap = cap;
+    ep.rope = rope; ep.q_out = q; ep.k_cache = kc; ep.v_cache = vc;
+    GemmShape sh = make_shape(M, 0, nqkv, D, kPrefillBN, 1);
+    L3_TRY((launch_gemm<kPrefillBN, 4, EPI_QKV_ROPE, false>(LLAMA3_KERNEL_GEMM_QKV, mxn, mxn, mwqkv, mwqkv, sh, ep, st)));
+  }
+  L3_TRY(attention_dispatch(c, q, kc, vc, cap, B, S, P, o, Ap, st));
+  {
+    EpiParams ep = empty_epi();
+    ep.out = x; ep.res = x; ep.ldo = D;
+    GemmShape sh = make_shape(M, 0, D, H * hd, kPrefillBN, 1);
+    L3_TRY((launch_gemm<kPrefillBN, 4, EPI_RESIDUAL, false>(LLAMA3_KERNEL_GEMM_WO, mo, mo, mwo, mwo, sh, ep, st)));
+  }
+  // FFN half
+  L3_TRY(run_rmsnorm<bf16>(c, x, D, w->ffn_norm, xn, M, st));
+  {
+    EpiParams ep = empty_epi();
+    ep.out = g; ep.ldo = F;
+    GemmShape sh = make_shape(M, 0, F, D, 128, 1);
+    L3_TRY((launch_gemm<128, 4, EPI_SWIGLU, true>(LLAMA3_KERNEL_GEMM_W13, mxn, mxn, mw1, mw3, sh, ep, st)));
+  }
+  {
+    EpiParams ep = empty_epi();
+    ep.out = x; ep.res = x; ep.ldo = D;
+    GemmShape sh = make_shape(M, 0, D, F, kPrefillBN, 1);
+    L3_TRY((launch_gemm<kPrefillBN, 4, EPI_RESIDUAL, false>(LLAMA3_KERNEL_GEMM_W2, mg, mg, mw2, mw2, sh, ep, st)));
+  }
+  return LLAMA3_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Layer: tcgen05 decode path (bf16, few tokens): weight-streaming split-K
+// GEMMs + SIMT epilogues over the fp32 partials.
+// ---------------------------------------------------------------------------
+int layer_tc_decode(const llama3_config* c, const llama3_layer_weights* w, const float* rope, void* x, void* kc,
+                    void* vc, int cap, int B, int P, const Workspace& L, void* ws, cudaStream_t st) {
+  const int M = B, D = c->dim, H = c->n_heads, KV = c->n_kv_heads, hd = c->head_dim, F = c->ffn_hidden;
+  const int nqkv = (H + 2 * KV) * hd;
+  bf16* xn = ws_at<bf16>(ws, L.xn);
+  bf16* q = ws_at<bf16>(ws, L.q);
+  bf16* o = ws_at<bf16>(ws, L.o);
+  bf16* g = ws_at<bf16>(ws, L.g);
+  float* Pp = ws_at<float>(ws, L.part);
+  float* Ap = ws_at<float>(ws, L.attn_part);
+  int splits = 1;
+
+  L3_TRY(run_rmsnorm<bf16>(c, x, D, w->attention_norm, xn, M, st));
+  L3_TRY(swapped_partial_gemm(w->wqkv, nqkv, nullptr, 0, 0, xn, M, D, Pp, nqkv, &splits, st));
+  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, epi_qkv_rope_kernel<bf16><<<blocks_for((long long)M * nqkv / 2, 256), 256, 0, st>>>(
+      Pp, splits, (long long)M * nqkv, M, 1, P, H, KV, hd, rope, q, (bf16*)kc, (bf16*)vc, cap));
+  L3_TRY(launch_check());
+  L3_TRY(attention_dispatch(c, q, kc, vc, cap, B, 1, P, o, Ap, st));
+  L3_TRY(swapped_partial_gemm(w->wo, D, nullptr, 0, 0, o, M, H * hd, Pp, D, &splits, st));
+  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, epi_residual_kernel<bf16><<<blocks_for((long long)M * D, 256), 256, 0, st>>>(
+      Pp, splits, (long long)M * D, D, (const bf16*)x, (bf16*)x, M, D));
+  L3_TRY(launch_check());
+  L3_TRY(run_rmsnorm<bf16>(c, x, D, w->ffn_norm, xn, M, st));
+  L3_TRY(swapped_partial_gemm(w->w1, F, w->w3, F, F, xn, M, D, Pp, 2 * F, &splits, st));
+  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, epi_swiglu_kernel<bf16><<<blocks_for((long long)M * F, 256), 256, 0, st>>>(Pp, splits, (long long)M * 2 * F, g,
+                                                                                M, F));
+  L3_TRY(launch_check());
+  L3_TRY(swapped_partial_gemm(w->w2, D, nullptr, 0, 0, g, M, F, Pp, D, &splits, st));
+  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, epi_residual_kernel<bf16><<<blocks_for((long long)M * D, 256), 256, 0, st>>>(
+      Pp, splits, (long long)M * D, D, (const bf16*)x, (bf16*)x, M, D));
+  return launch_check();
+}
+
+int check_layer_args(const llama3_config* c, const llama3_layer_weights* w, const float* rope, int rope_len,
+                     const void* x, const void* kc, const void* vc, int cap, int B, int S, int P, const void* ws,
+                     size_t ws_bytes, Workspace* L) {
+  L3_TRY(check_config(c));
+  if (!w || !rope || !x || !kc || !vc) return LLAMA3_ERR_ARG;
+  if (B < 1 || S < 1 || P < 0 || cap < 1) return LLAMA3_ERR_ARG;
+  if ((long long)P + S > cap) return LLAMA3_ERR_ARG;
+  if ((long long)P + S > rope_len) return LLAMA3_ERR_ARG;
+  const void* ptrs[] = {w->attention_norm, w->wqkv, w->wo, w->ffn_norm, w->w1, w->w2, w->w3, rope, x, kc, vc};
+  for (const void* p : ptrs) {
+    if (!p) return LLAMA3_ERR_ARG;
+    if (!aligned16(p)) return LLAMA3_ERR_ALIGN;
+  }
+  *L = layout(c, B, S, 1);
+  if (!ws || ws_bytes < L->total) return LLAMA3_ERR_WORKSPACE;
+  if (!aligned16(ws)) return LLAMA3_ERR_ALIGN;
+  return LLAMA3_OK;
+}
+
+}  // namespace
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+extern "C" {
+
+const char* llama3_status_string(int s) {
+  switch (s) {
+    case LLAMA3_OK: return "ok";
+    case LLAMA3_ERR_ARG: return "invalid argument";
+    case LLAMA3_ERR_ALIGN: return "pointer or stride not 16-byte aligned";
+    case LLAMA3_ERR_WORKSPACE: return "workspace missing or too small";
+    case LLAMA3_ERR_CUDA: return "CUDA call failed (see llama3_last_cuda_error)";
+    case LLAMA3_ERR_TIMEOUT: return "device-side wait timed out";
+    case LLAMA3_ERR_TOKEN: return "token id out of range";
+    case LLAMA3_ERR_UNSUPPORTED: return "shape not supported by the kernels";
+    default: return "unknown status";
+  }
+}
+
+int llama3_last_cuda_error(void) { return t_last_cuda; }
+
+int llama3_set_launch_timer(int kind, void* const* start_events, void* const* stop_events, int n_pairs) {
+  if (n_pairs < 0 || (n_pairs > 0 && (!start_events || !stop_events))) return LLAMA3_ERR_ARG;
+  g_timer.kind = n_pairs ? kind : 0;
+  g_timer.n = n_pairs;
+  g_timer.used = 0;
+  g_timer.start.assign(n_pairs, nullptr);
+  g_timer.stop.assign(n_pairs, nullptr);
+  for (int i = 0; i < n_pairs; ++i) {
+    g_timer.start[i] = (cudaEvent_t)start_events[i];
+    g_timer.stop[i] = (cudaEvent_t)stop_events[i];
+  }
+  return LLAMA3_OK;
+}
+
+int llama3_launch_timer_used(void) { return g_timer.used; }
+
+unsigned long long llama3_launch_count(void) { return g_launches.load(); }
+
+int llama3_set_kernel_path(int path) {
+  int old = g_kernel_path;
+  g_kernel_path = path ? 1 : 0;
+  return old;
+}
+
+int llama3_set_wait_limit_ms(int ms) {
+  int old = g_wait_ms;
+  if (ms > 0) g_wait_ms = ms;
+  return old;
+}
+
+int llama3_device_status(int* out) {
+  if (!out) return LLAMA3_ERR_ARG;
+  int v = 0, zero = 0;
+  L3_CUDA(cudaDeviceSynchronize());
+  L3_CUDA(cudaMemcpyFromSymbol(&v, g_status, sizeof(int)));
+  L3_CUDA(cudaMemcpyToSymbol(g_status, &zero, sizeof(int)));
+  *out = v;
+  return LLAMA3_OK;
+}
+
+int llama3_init_rope_table(float* cos_sin, int head_dim, int max_pos, double theta, llama3_stream_t stream) {
+  if (!cos_sin || head_dim < 2 || (head_dim & 1) || max_pos < 1 || !(theta > 1.0)) return LLAMA3_ERR_ARG;
+  if (!aligned16(cos_sin)) return LLAMA3_ERR_ALIGN;
+  const int half = head_dim / 2;
+  const size_t n = (size_t)max_pos * half * 2;
+  std::vector<float> host(n);
+  for (int m = 0; m < max_pos; ++m) {
+    for (int i = 0; i < half; ++i) {
+      const double inv = pow(theta, -(2.0 * i) / (double)head_dim);
+      const double ang = (double)m * inv;
+      host[((size_t)m * half + i) * 2] = (float)cos(ang);
+      host[((size_t)m * half + i) * 2 + 1] = (float)sin(ang);
+    }
+  }
+  L3_CUDA(cudaMemcpyAsync(cos_sin, host.data(), n * sizeof(float), cudaMemcpyHostToDevice, (cudaStream_t)stream));
+  L3_CUDA(cudaStreamSynchronize((cudaStream_t)stream));
+  return LLAMA3_OK;
+}
+
+int llama3_workspace_size(const llama3_config* cfg, int batch, int seq, int lm_rows, size_t* bytes) {
+  L3_TRY(check_config(cfg));
+  if (!bytes || batch < 1 || seq < 1 || lm_rows < 0) return LLAMA3_ERR_ARG;
+  *bytes = layout(cfg, batch, seq, lm_rows).total;
+  return LLAMA3_OK;
+}
+
+int llama3_embed(const llama3_config* cfg, const int32_t* ids, const void* table, void* x, int n_tokens,
+                 llama3_stream_t stream) {
+  L3_TRY(check_config(cfg));
+  if (!ids || !table || !x || n_tokens < 1 || cfg->vocab < 1) return LLAMA3_ERR_ARG;
+  if (!aligned16(ids) || !aligned16(table) || !aligned16(x)) return LLAMA3_ERR_ALIGN;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cfg->dtype == LLAMA3_DTYPE_F32)
+    L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, embed_kernel<float><<<n_tokens, 128, 0, st>>>(ids, (const float*)table, (float*)x, cfg->dim, cfg->vocab));
+  else
+    L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, embed_kernel<bf16><<<n_tokens, 128, 0, st>>>(ids, (const bf16*)table, (bf16*)x, cfg->dim, cfg->vocab));
+  return launch_check();
+}
+
+int llama3_rmsnorm(const llama3_config* cfg, const void* x, long long row_stride, const void* w, void* y, int rows,
+                   llama3_stream_t stream) {
+  L3_TRY(check_config(cfg));
+  if (!x || !w || !y || rows < 1 || row_stride < cfg->dim) return LLAMA3_ERR_ARG;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(y)) return LLAMA3_ERR_ALIGN;
+  return rmsnorm_any(cfg, x, row_stride, w, y, rows, (cudaStream_t)stream);
+}
+
+int llama3_linear(const llama3_config* cfg, const void* x, const void* w, const void* residual, void* y, int m,
+                  int n, int k, void* ws, size_t ws_bytes, llama3_stream_t stream) {
+  L3_TRY(check_config(cfg));
+  if (!x || !w || !y || m < 1 || n < 1 || k < 1) return LLAMA3_ERR_ARG;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(y) || (residual && !aligned16(residual)))
+    return LLAMA3_ERR_ALIGN;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (use_tc(cfg)) {
+    if (k % 8 || n % 8) return LLAMA3_ERR_ALIGN;
+    CUtensorMap ma, mb;
+    L3_TRY(make_map(&ma, x, m, k, 128));
+    L3_TRY(make_map(&mb, w, n, k, kPrefillBN));
+    EpiParams ep = empty_epi();
+    ep.out = y; ep.res = residual; ep.ldo = n;
+    GemmShape sh = make_shape(m, 0, n, k, kPrefillBN, 1);
+    if (residual) return launch_gemm<kPrefillBN, 4, EPI_RESIDUAL, false>(LLAMA3_KERNEL_GEMM_WO, ma, ma, mb, mb, sh, ep, st);
+    return launch_gemm<kPrefillBN, 4, EPI_STORE, false>(LLAMA3_KERNEL_GEMM_WO, ma, ma, mb, mb, sh, ep, st);
+  }
+  const size_t need = (size_t)m * n * 4;
+  if (!ws || ws_bytes < need) return LLAMA3_ERR_WORKSPACE;
+  float* C = (float*)ws;
+  if (cfg->dtype == LLAMA3_DTYPE_F32) {
+    L3_TRY(simt_gemm<float>(LLAMA3_KERNEL_GEMM_WO, x, w, C, m, n, k, n, st));
+    L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, epi_residual_kernel<float><<<blocks_for((long long)m * n, 256), 256, 0, st>>>(C, 1, 0, n, (const float*)residual,
+                                                                                  (float*)y, m, n));
+  } else {
+    L3_TRY(simt_gemm<bf16>(LLAMA3_KERNEL_GEMM_WO, x, w, C, m, n, k, n, st));
+    L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, epi_residual_kernel<bf16><<<blocks_for((long long)m * n, 256), 256, 0, st>>>(C, 1, 0, n, (const bf16*)residual,
+                                                                                 (bf16*)y, m, n));
+  }
+  return launch_check();
+}
+
+int llama3_attention(const llama3_config* cfg, const void* q, const void* k_cache, const void* v_cache,
+                     int cache_cap, int batch, int seq, int start_pos, void* out, void* ws, size_t ws_bytes,
+                     llama3_stream_t stream) {
+  L3_TRY(check_config(cfg));
+  if (!q || !k_cache || !v_cache || !out || batch < 1 || seq < 1 || start_pos < 0) return LLAMA3_ERR_ARG;
+  if ((long long)start_pos + seq > cache_cap) return LLAMA3_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out)) return LLAMA3_ERR_ALIGN;
+  Workspace L = layout(cfg, batch, seq, 1);
+  if (!ws || ws_bytes < L.total) return LLAMA3_ERR_WORKSPACE;
+  return attention_dispatch(cfg, q, k_cache, v_cache, cache_cap, batch, seq, start_pos, out,
+                            ws_at<float>(ws, L.attn_part), (cudaStream_t)stream);
+}
+
+int llama3_layer_forward(const llama3_config* cfg, const llama3_layer_weights* w, const float* rope, int rope_len,
+                         void* x, void* k_cache, void* v_cache, int cache_cap, int batch, int seq, int start_pos,
+                         void* ws, size_t ws_bytes, llama3_stream_t stream) {
+  Workspace L;
+  L3_TRY(check_layer_args(cfg, w, rope, rope_len, x, k_cache, v_cache, cache_cap, batch, seq, start_pos, ws,
+                          ws_bytes, &L));
+  cudaStream_t st = (cudaStream_t)stream;
+  if (use_tc(cfg))
+    return layer_tc_prefill(cfg, w, rope, x, k_cache, v_cache, cache_cap, batch, seq, start_pos, L, ws, st);
+  if (cfg->dtype == LLAMA3_DTYPE_F32)
+    return layer_simt<float>(cfg, w, rope, x, k_cache, v_cache, cache_cap, batch, seq, start_pos, L, ws, st);
+  return layer_simt<bf16>(cfg, w, rope, x, k_cache, v_cache, cache_cap, batch, seq, start_pos, L, ws, st);
+}
+
+int llama3_layer_decode(const llama3_config* cfg, const llama3_layer_weights* w, const float* rope, int rope_len,
+                        void* x, void* k_cache, void* v_cache, int cache_cap, int batch, int start_pos, void* ws,
+                        size_t ws_bytes, llama3_stream_t stream) {
+  Workspace L;
+  L3_TRY(check_layer_args(cfg, w, rope, rope_len, x, k_cache, v_cache, cache_cap, batch, 1, start_pos, ws,
+                          ws_bytes, &L));
+  cudaStream_t st = (cudaStream_t)stream;
+  if (use_tc(cfg)) {
+    if (batch <= 256)
+      return layer_tc_decode(cfg, w, rope, x, k_cache, v_cache, cache_cap, batch, start_pos, L, ws, st);
+    return layer_tc_prefill(cfg, w, rope, x, k_cache, v_cache, cache_cap, batch, 1, start_pos, L, ws, st);
+  }
+  if (cfg->dtype == LLAMA3_DTYPE_F32)
+    return layer_simt<float>(cfg, w, rope, x, k_cache, v_cache, cache_cap, batch, 1, start_pos, L, ws, st);
+  return layer_simt<bf16>(cfg, w, rope, x, k_cache, v_cache, cache_cap, batch, 1, start_pos, L, ws, st);
+}
+
+int llama3_lm_head_argmax(const llama3_config* cfg, const void* norm_w, const void* w_out, const void* h, int rows,
+                          long long row_stride, int32_t* ids_out, float* logits_out, void* ws, size_t ws_bytes,
+                          llama3_stream_t stream) {
+  L3_TRY(check_config(cfg));
+  if (!norm_w || !w_out || !h || !ids_out || rows < 1 || cfg->vocab < 1 || row_stride < cfg->dim)
+    return LLAMA3_ERR_ARG;
+  if (!aligned16(norm_w) || !aligned16(w_out) || !aligned16(h) || !aligned16(ids_out) ||
+      (logits_out && !aligned16(logits_out)))
+    return LLAMA3_ERR_ALIGN;
+  if ((row_stride * (long long)esize(cfg)) % 16) return LLAMA3_ERR_ALIGN;
+  Workspace L = layout(cfg, 1, 1, rows);
+  if (!ws || ws_bytes < L.total) return LLAMA3_ERR_WORKSPACE;
+  if (!aligned16(ws)) return LLAMA3_ERR_ALIGN;
+  cudaStream_t st = (cudaStream_t)stream;
+  void* hn = ws_at<void>(ws, L.lm_rows);
+  unsigned long long* keys = ws_at<unsigned long long>(ws, L.keys);
+  const int V = cfg->vocab, D = cfg->dim;
+  L3_TRY(rmsnorm_any(cfg, h, row_stride, norm_w, hn, rows, st));
+  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, argmax_init_kernel<<<blocks_for(rows, 256), 256, 0, st>>>(keys, rows));
+  L3_TRY(launch_check());
+  if (use_tc(cfg)) {
+    const int bn = rows <= 16 ? 16 : rows <= 32 ? 32 : rows <= 64 ? 64 : rows <= 128 ? 128 : 256;
+    CUtensorMap ma, mb;
+    L3_TRY(make_map(&ma, w_out, V, D, 128));
+    L3_TRY(make_map(&mb, hn, rows, D, bn));
+    GemmShape sh = make_shape(V, 0, rows, D, bn, 1);
+    EpiParams ep = empty_epi();
+    ep.logits = logits_out;
+    ep.keys = keys;
+    switch (bn) {
+      case 16: L3_TRY((launch_gemm<16, 8, EPI_ARGMAX, false>(LLAMA3_KERNEL_LM_HEAD, ma, ma, mb, mb, sh, ep, st))); break;
+      case 32: L3_TRY((launch_gemm<32, 8, EPI_ARGMAX, false>(LLAMA3_KERNEL_LM_HEAD, ma, ma, mb, mb, sh, ep, st))); break;
+      case 64: L3_TRY((launch_gemm<64, 6, EPI_ARGMAX, false>(LLAMA3_KERNEL_LM_HEAD, ma, ma, mb, mb, sh, ep, st))); break;
+      case 128: L3_TRY((launch_gemm<128, 5, EPI_ARGMAX, false>(LLAMA3_KERNEL_LM_HEAD, ma, ma, mb, mb, sh, ep, st))); break;
+      default: L3_TRY((launch_gemm<256, 4, EPI_ARGMAX, false>(LLAMA3_KERNEL_LM_HEAD, ma, ma, mb, mb, sh, ep, st))); break;
+    }
+  } else {
+    const long long warps = (long long)rows * ((V + 31) / 32);
+    if (cfg->dtype == LLAMA3_DTYPE_F32)
+      L3_LAUNCH(LLAMA3_KERNEL_LM_HEAD, st, lm_head_simt_kernel<float><<<blocks_for(warps * 32, 256), 256, 0, st>>>((const float*)hn, (const float*)w_out,
+                                                                               logits_out, keys, rows, V, D));
+    else
+      L3_LAUNCH(LLAMA3_KERNEL_LM_HEAD, st, lm_head_simt_kernel<bf16><<<blocks_for(warps * 32, 256), 256, 0, st>>>((const bf16*)hn, (const bf16*)w_out,
+                                                                              logits_out, keys, rows, V, D));
+    L3_TRY(launch_check());
+  }
+  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, argmax_finalize_kernel<<<blocks_for(rows, 256), 256, 0, st>>>(keys, ids_out, rows));
+  return launch_check();
+}
+
+}  // extern "C"

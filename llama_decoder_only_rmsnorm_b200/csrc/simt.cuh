@@ -1,0 +1,255 @@
+// simt.cuh -- plain CUDA-core kernels for every step of the decoder.
+//
+// They serve the fp32 models (tiny configs where tensor cores would not meet
+// a 1e-4 tolerance) and act as the independent GPU-side cross-check of the
+// tcgen05 kernels.  Templated on the element type T (float or bf16); all
+// arithmetic is fp32.  Nothing here is tuned.
+#pragma once
+#include "common.cuh"
+
+namespace l3 {
+
+// ---- embedding gather ("从0开发大模型—译llama3-from-scratch" §4) -------------
+template <typename T>
+__global__ void embed_kernel(const int32_t* __restrict__ ids, const T* __restrict__ table,
+                             T* __restrict__ x, int D, int vocab) {
+  int t = blockIdx.x;
+  int id = ids[t];
+  bool ok = id >= 0 && id < vocab;
+  if (!ok && threadIdx.x == 0) record_error(LLAMA3_ERR_TOKEN);
+  const T* src = table + (size_t)(ok ? id : 0) * D;
+  T* dst = x + (size_t)t * D;
+  for (int i = threadIdx.x; i < D; i += blockDim.x) dst[i] = ok ? src[i] : from_f<T>(0.f);
+}
+
+// ---- RMSNorm ("Build your own Llama 3 from scratch" §3.1) -------------------
+// One CTA per row; fp32 sum of squares, one rounding on output.
+template <typename T>
+__global__ void rmsnorm_kernel(const T* __restrict__ x, long long row_stride,
+                               const T* __restrict__ w, T* __restrict__ y, int D, float eps) {
+  const T* xr = x + (size_t)blockIdx.x * row_stride;
+  T* yr = y + (size_t)blockIdx.x * D;
+  float ss = 0.f;
+  for (int i = threadIdx.x; i < D; i += blockDim.x) {
+    float v = to_f(xr[i]);
+    ss = fmaf(v, v, ss);
+  }
+  __shared__ float red[32];
+  ss = warp_sum(ss);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+    v = warp_sum(v);
+    if (threadIdx.x == 0) red[0] = v;
+  }
+  __syncthreads();
+  float r = rsqrtf(red[0] / (float)D + eps);
+  for (int i = threadIdx.x; i < D; i += blockDim.x) yr[i] = from_f<T>(to_f(xr[i]) * r * to_f(w[i]));
+}
+
+// ---- GEMM C[m, n] = sum_k A[m, k] * B[n, k]   (fp32 result) -----------------
+// 64x64 tile, 256 threads, 4x4 outputs per thread, K staged 16 at a time.
+template <typename T>
+__global__ void __launch_bounds__(256) gemm_simt_kernel(const T* __restrict__ A, const T* __restrict__ B,
+                                                        float* __restrict__ C, int M, int N, int K,
+                                                        int ldc) {
+  __shared__ float As[16][64 + 1];
+  __shared__ float Bs[16][64 + 1];
+  int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < K; k0 += 16) {
+    for (int i = threadIdx.x; i < 64 * 16; i += 256) {
+      int r = i >> 4, c = i & 15;
+      int gm = m0 + r, gn = n0 + r, gk = k0 + c;
+      As[c][r] = (gm < M && gk < K) ? to_f(A[(size_t)gm * K + gk]) : 0.f;
+      Bs[c][r] = (gn < N && gk < K) ? to_f(B[(size_t)gn * K + gk]) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = As[kk][ty * 4 + i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) b[j] = Bs[kk][tx * 4 + j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    int gm = m0 + ty * 4 + i;
+    if (gm >= M) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      int gn = n0 + tx * 4 + j;
+      if (gn < N) C[(size_t)gm * ldc + gn] = acc[i][j];
+    }
+  }
+}
+
+// ---- epilogues over fp32 partial sums P[split][m][n] ------------------------
+// (used after the SIMT GEMM with splits = 1 and after split-K tensor-core GEMMs)
+__device__ __forceinline__ float sum_splits(const float* P, int splits, long long split_stride,
+                                            long long idx) {
+  float s = 0.f;
+  for (int i = 0; i < splits; ++i) s += P[(size_t)i * split_stride + idx];
+  return s;
+}
+
+// out[m, n] = (res ? res[m, n] : 0) + P[m, n]
+template <typename T>
+__global__ void epi_residual_kernel(const float* __restrict__ P, int splits, long long split_stride,
+                                    int ldp, const T* res, T* out, int M, int N) {
+  long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (long long)M * N) return;
+  int m = (int)(i / N), n = (int)(i % N);
+  float v = sum_splits(P, splits, split_stride, (long long)m * ldp + n);
+  if (res) v += to_f(res[i]);
+  out[i] = from_f<T>(v);
+}
+
+// g[m, f] = silu(P[m, f]) * P[m, F + f],  silu(z) = z / (1 + e^-z)
+// ("Build your own Llama 3 from scratch" §3.5)
+template <typename T>
+__global__ void epi_swiglu_kernel(const float* __restrict__ P, int splits, long long split_stride,
+                                  T* __restrict__ g, int M, int F) {
+  long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (long long)M * F) return;
+  int m = (int)(i / F), f = (int)(i % F);
+  float a = sum_splits(P, splits, split_stride, (long long)m * 2 * F + f);
+  float b = sum_splits(P, splits, split_stride, (long long)m * 2 * F + F + f);
+  g[i] = from_f<T>(a / (1.f + expf(-a)) * b);
+}
+
+// QKV epilogue: rotate q and k pairs (2i, 2i+1) by the table's (cos, sin) of
+// position start_pos + t ("Build your own Llama 3 from scratch" §3.2), write
+// q to q_out [M, H*hd] and k, v to the caches at [b, pos, kvh, :] (§3.3).
+// One thread per pair.
+template <typename T>
+__global__ void epi_qkv_rope_kernel(const float* __restrict__ P, int splits, long long split_stride,
+                                    int M, int seq, int start_pos, int H, int KV, int hd,
+                                    const float* __restrict__ rope, T* __restrict__ q_out,
+                                    T* __restrict__ k_cache, T* __restrict__ v_cache, int cap) {
+  int Ntot = (H + 2 * KV) * hd;
+  long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (long long)M * (Ntot / 2)) return;
+  int m = (int)(i / (Ntot / 2));
+  int n = (int)(i % (Ntot / 2)) * 2;
+  int b = m / seq, t = m % seq, pos = start_pos + t;
+  float a = sum_splits(P, splits, split_stride, (long long)m * Ntot + n);
+  float c = sum_splits(P, splits, split_stride, (long long)m * Ntot + n + 1);
+  int d = n % hd, head = n / hd;
+  if (head < H + KV) {
+    const float* cs = rope + ((size_t)pos * (hd / 2) + d / 2) * 2;
+    float co = cs[0], si = cs[1];
+    float ra = a * co - c * si, rc = a * si + c * co;
+    a = ra;
+    c = rc;
+  }
+  if (head < H) {
+    T* dst = q_out + (size_t)m * H * hd + n;
+    dst[0] = from_f<T>(a);
+    dst[1] = from_f<T>(c);
+  } else {
+    bool is_k = head < H + KV;
+    int kvh = head - (is_k ? H : H + KV);
+    T* dst = (is_k ? k_cache : v_cache) + (((size_t)b * cap + pos) * KV + kvh) * hd + d;
+    dst[0] = from_f<T>(a);
+    dst[1] = from_f<T>(c);
+  }
+}
+
+// ---- causal GQA attention, one warp per (b, t, h) ---------------------------
+// ("Build your own Llama 3 from scratch" §3.4; query head h reads KV head
+// h / (H/KV); key j is visible to position start_pos + t iff j <= start_pos + t)
+// Online softmax in fp32.  Lane l owns dims l, l+32, ... of the output.
+template <typename T>
+__global__ void attention_simt_kernel(const T* __restrict__ q, const T* __restrict__ k_cache,
+                                      const T* __restrict__ v_cache, T* __restrict__ out, int B,
+                                      int S, int start_pos, int H, int KV, int hd, int cap,
+                                      float scale) {
+  long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  int lane = threadIdx.x & 31;
+  if (w >= (long long)B * S * H) return;
+  int h = (int)(w % H);
+  int t = (int)((w / H) % S);
+  int b = (int)(w / ((long long)H * S));
+  int g = h / (H / KV);
+  const T* qr = q + (((size_t)b * S + t) * H + h) * hd;
+  float qv[4], acc[4];
+  for (int i = 0; i < 4; ++i) {
+    int d = lane + 32 * i;
+    qv[i] = d < hd ? to_f(qr[d]) : 0.f;
+    acc[i] = 0.f;
+  }
+  float m = -INFINITY, l = 0.f;
+  int last = start_pos + t;
+  for (int j = 0; j <= last; ++j) {
+    const T* kr = k_cache + (((size_t)b * cap + j) * KV + g) * hd;
+    const T* vr = v_cache + (((size_t)b * cap + j) * KV + g) * hd;
+    float s = 0.f;
+    for (int i = 0; i < 4; ++i) {
+      int d = lane + 32 * i;
+      if (d < hd) s = fmaf(qv[i], to_f(kr[d]), s);
+    }
+    s = warp_sum(s) * scale;
+    float mn = fmaxf(m, s);
+    float corr = expf(m - mn);  // exp(-inf) = 0 on the first key
+    float p = expf(s - mn);
+    l = l * corr + p;
+    for (int i = 0; i < 4; ++i) {
+      int d = lane + 32 * i;
+      acc[i] = acc[i] * corr + (d < hd ? p * to_f(vr[d]) : 0.f);
+    }
+    m = mn;
+  }
+  T* orow = out + (((size_t)b * S + t) * H + h) * hd;
+  float inv = 1.f / l;
+  for (int i = 0; i < 4; ++i) {
+    int d = lane + 32 * i;
+    if (d < hd) orow[d] = from_f<T>(acc[i] * inv);
+  }
+}
+
+// ---- LM head: logits and argmax ("llama3-from-scratch：输出层与预测") --------
+// One warp per (row r, block of 32 vocabulary rows); one atomicMax per warp.
+template <typename T>
+__global__ void lm_head_simt_kernel(const T* __restrict__ hn, const T* __restrict__ W,
+                                    float* __restrict__ logits, unsigned long long* __restrict__ keys,
+                                    int R, int V, int D) {
+  long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  int lane = threadIdx.x & 31;
+  int vblocks = (V + 31) / 32;
+  if (w >= (long long)R * vblocks) return;
+  int r = (int)(w / vblocks);
+  int v0 = (int)(w % vblocks) * 32;
+  const T* hr = hn + (size_t)r * D;
+  unsigned long long best = 0;
+  for (int v = v0; v < min(v0 + 32, V); ++v) {
+    const T* wr = W + (size_t)v * D;
+    float s = 0.f;
+    for (int i = lane; i < D; i += 32) s = fmaf(to_f(hr[i]), to_f(wr[i]), s);
+    s = warp_sum(s);
+    if (logits && lane == 0) logits[(size_t)r * V + v] = s;
+    unsigned long long k = argmax_pack(s, (uint32_t)v);
+    best = k > best ? k : best;
+  }
+  if (lane == 0) atomicMax(&keys[r], best);
+}
+
+__global__ void argmax_init_kernel(unsigned long long* keys, int R) {
+  int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < R) keys[i] = 0ull;
+}
+__global__ void argmax_finalize_kernel(const unsigned long long* keys, int32_t* ids, int R) {
+  int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < R) ids[i] = (int32_t)(0xffffffffu - (uint32_t)(keys[i] & 0xffffffffull));
+}
+
+}  // namespace l3

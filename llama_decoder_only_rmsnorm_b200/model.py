@@ -1,0 +1,61 @@
+"""Host-side driver of the C ABI for a whole decoder stack.
+
+Owns the device buffers (through torch: weights are given, the RoPE table,
+workspace, KV caches and id/logit outputs are allocated here) and issues one
+library call per step: embed -> layer_forward/layer_decode per block ->
+lm_head_argmax.  It does no arithmetic of its own.  The layer loop follows
+the stack of "Build your own Llama 3 from scratch" 四 (Transformer.forward).
+"""
+from __future__ import annotations
+
+import torch
+
+from . import binding as B
+
+
+class Llama3Stack:
+    def __init__(self, cfg: dict, layers, out_weights, batch: int, cache_cap: int, max_seq: int,
+                 lm_rows: int = 0, device="cuda", rope_len: int | None = None, caches=None):
+        self.cfg_dict = dict(cfg)
+        self.cfg = B.make_config(cfg["dim"], cfg["n_heads"], cfg["n_kv_heads"], cfg["ffn_hidden"],
+                                 cfg.get("vocab", 0), cfg["norm_eps"], cfg["rope_theta"], cfg["dtype"])
+        self.dtype = torch.float32 if cfg["dtype"] == "f32" else torch.bfloat16
+        self.layers = list(layers)
+        self.wstructs = [B.make_layer_weights(l) for l in self.layers]
+        self.out = out_weights
+        self.batch, self.cache_cap, self.max_seq = batch, cache_cap, max_seq
+        self.device = device
+        hd = cfg["dim"] // cfg["n_heads"]
+        self.rope_len = rope_len or max(cache_cap, 1)
+        self.rope = torch.empty((self.rope_len, hd // 2, 2), dtype=torch.float32, device=device)
+        B.llama3_init_rope_table(self.rope, hd, self.rope_len, cfg["rope_theta"])
+        self.lm_rows = max(lm_rows, 1)
+        self.ws_bytes = B.llama3_workspace_size(self.cfg, batch, max_seq, self.lm_rows)
+        self.ws = torch.empty((self.ws_bytes,), dtype=torch.uint8, device=device)
+        if caches is None:
+            shape = (batch, cache_cap, cfg["n_kv_heads"], hd)
+            caches = [(torch.zeros(shape, dtype=self.dtype, device=device),
+                       torch.zeros(shape, dtype=self.dtype, device=device)) for _ in self.layers]
+        self.caches = caches
+        self.ids_out = torch.zeros((self.lm_rows,), dtype=torch.int32, device=device)
+
+    # -- steps --------------------------------------------------------------
+    def embed(self, ids, x, stream=None):
+        B.llama3_embed(self.cfg, ids, self.out["tok_embeddings"], x, ids.numel(), stream)
+
+    def forward_layers(self, x, seq, start_pos=0, stream=None, layers=None):
+        for i in (range(len(self.layers)) if layers is None else layers):
+            kc, vc = self.caches[i]
+            B.llama3_layer_forward(self.cfg, self.wstructs[i], self.rope, self.rope_len, x, kc, vc,
+                                   self.cache_cap, self.batch, seq, start_pos, self.ws, self.ws_bytes, stream)
+
+    def decode_layers(self, x, start_pos, stream=None, layers=None):
+        for i in (range(len(self.layers)) if layers is None else layers):
+            kc, vc = self.caches[i]
+            B.llama3_layer_decode(self.cfg, self.wstructs[i], self.rope, self.rope_len, x, kc, vc,
+                                  self.cache_cap, self.batch, start_pos, self.ws, self.ws_bytes, stream)
+
+    def lm_head(self, h, rows, row_stride, logits=None, stream=None):
+        B.llama3_lm_head_argmax(self.cfg, self.out["norm"], self.out["output"], h, rows, row_stride,
+                                self.ids_out, logits, self.ws, self.ws_bytes, stream)
+        return self.ids_out[:rows]

@@ -1,0 +1,263 @@
+"""GPU parity: every step of the decoder, through the C ABI, against the fp64
+oracle on the same seeded inputs.  Tolerance |gpu - oracle| <= 2e-2 +
+2e-2*|oracle| per element for bf16 paths, 1e-4 + 1e-4*|oracle| for fp32;
+argmax ids must match wherever the oracle's top-2 logit gap exceeds 1e-2."""
+import numpy as np
+import pytest
+import torch
+
+from helpers import assert_argmax, assert_close, f64, oracle_cfg, oracle_layer
+from llama_decoder_only_rmsnorm_b200 import binding as B
+from llama_decoder_only_rmsnorm_b200 import inputs as I
+from llama_decoder_only_rmsnorm_b200.model import Llama3Stack
+from oracle import llama3_oracle as O
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(autouse=True)
+def _gpu_state():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    B.llama3_set_kernel_path(0)
+    yield
+    B.llama3_set_kernel_path(0)
+    torch.cuda.synchronize()
+    assert B.llama3_device_status() == 0, "device status word set"
+
+
+def wl(name, **kw):
+    return I.WORKLOADS[name].replace(**kw)
+
+
+def small_bf16(**kw):
+    d = dict(name="small", dim=512, n_layers=2, n_heads=8, n_kv_heads=2, ffn_hidden=1024, vocab=1000,
+             batch=3, seq=70, dtype="bf16", input_kind="activations", seed=77)
+    d.update(kw)
+    return I.Workload(**d)
+
+
+# ------------------------------------------------------------------ RMSNorm
+@pytest.mark.parametrize("dtype,D,H", [("bf16", 4096, 32), ("bf16", 576, 9), ("f32", 64, 4)])
+def test_rmsnorm(dtype, D, H):
+    tdt = torch.float32 if dtype == "f32" else torch.bfloat16
+    g = torch.Generator(device="cpu").manual_seed(5)
+    rows, stride = 37, D + 64
+    x = (torch.randn((rows, stride), generator=g) * 3).to(tdt).to(DEV)
+    nw = (1 + 0.1 * torch.randn((D,), generator=g)).to(tdt).to(DEV)
+    y = torch.empty((rows, D), dtype=tdt, device=DEV)
+    cfg = B.make_config(D, H, 1, 8 * D, dtype=dtype)
+    B.llama3_rmsnorm(cfg, x, stride, nw, y, rows)
+    want = O.rms_norm(f64(x)[:, :D], f64(nw), 1e-5)
+    assert_close(y, want, dtype, "rmsnorm")
+
+
+# ------------------------------------------------------------------ Linear
+@pytest.mark.parametrize("m,n,k", [(128, 256, 64), (300, 264, 200), (1000, 1536, 512), (77, 4096, 4096),
+                                   (2048, 6144, 4096)])
+@pytest.mark.parametrize("residual", [False, True])
+@pytest.mark.parametrize("path", [0, 1])
+def test_linear(m, n, k, residual, path):
+    if path == 1 and m * n > 2_000_000:
+        pytest.skip("SIMT cross-check only on the smaller shapes")
+    B.llama3_set_kernel_path(path)
+    g = torch.Generator(device="cpu").manual_seed(m * 7 + n + k)
+    x = torch.randn((m, k), generator=g).to(torch.bfloat16).to(DEV)
+    w = (torch.randn((n, k), generator=g) * 0.05).to(torch.bfloat16).to(DEV)
+    r = torch.randn((m, n), generator=g).to(torch.bfloat16).to(DEV) if residual else None
+    y = torch.empty((m, n), dtype=torch.bfloat16, device=DEV)
+    cfg = B.make_config(512, 8, 8, 1024)
+    ws = torch.empty((m * n * 4,), dtype=torch.uint8, device=DEV)
+    B.llama3_linear(cfg, x, w, r, y, m, n, k, ws, ws.numel())
+    want = f64(x) @ f64(w).T + (f64(r) if residual else 0.0)
+    assert_close(y, want, "bf16", f"linear {m}x{n}x{k}")
+
+
+def test_linear_in_place_residual():
+    m, n, k = 256, 512, 512
+    g = torch.Generator(device="cpu").manual_seed(3)
+    x = torch.randn((m, k), generator=g).to(torch.bfloat16).to(DEV)
+    w = (torch.randn((n, k), generator=g) * 0.05).to(torch.bfloat16).to(DEV)
+    y = torch.randn((m, n), generator=g).to(torch.bfloat16).to(DEV)
+    want = f64(x) @ f64(w).T + f64(y)
+    B.llama3_linear(B.make_config(512, 8, 8, 1024), x, w, y, y, m, n, k)
+    assert_close(y, want, "bf16", "in-place residual")
+
+
+# --------------------------------------------------------------- attention
+def _attn_case(Bn, S, P, H, KV, hd, seed):
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    cap = P + S + 5
+    q = torch.randn((Bn, S, H, hd), generator=g).to(torch.bfloat16)
+    kc = torch.randn((Bn, cap, KV, hd), generator=g).to(torch.bfloat16)
+    vc = torch.randn((Bn, cap, KV, hd), generator=g).to(torch.bfloat16)
+    return q, kc, vc, cap
+
+
+@pytest.mark.parametrize("Bn,S,P,H,KV,hd", [
+    (2, 200, 0, 8, 2, 64), (2, 129, 37, 8, 2, 96), (1, 300, 0, 32, 8, 128), (3, 64, 500, 4, 4, 128),
+    (1, 1, 0, 8, 2, 128), (4, 1, 1, 8, 1, 64), (3, 1, 1000, 32, 8, 128), (2, 1, 300, 8, 2, 96),
+    (2, 1, 777, 16, 16, 64)])
+def test_attention(Bn, S, P, H, KV, hd):
+    q, kc, vc, cap = _attn_case(Bn, S, P, H, KV, hd, Bn * 1000 + S + P + hd)
+    cfg = B.make_config(H * hd, H, KV, 1024)
+    ws_bytes = B.llama3_workspace_size(cfg, Bn, S, 1)
+    ws = torch.empty((ws_bytes,), dtype=torch.uint8, device=DEV)
+    out = torch.empty((Bn, S, H * hd), dtype=torch.bfloat16, device=DEV)
+    B.llama3_attention(cfg, q.to(DEV), kc.to(DEV), vc.to(DEV), cap, Bn, S, P, out, ws, ws_bytes)
+    for b in range(Bn):
+        want = O.gqa_attention(f64(q[b]), f64(kc[b, :P + S]), f64(vc[b, :P + S]), P)
+        assert_close(out[b], want.reshape(S, H * hd), "bf16", f"attention b={b}")
+
+
+# ------------------------------------------------------- whole workloads
+def _run_layers_vs_oracle(w, norm_weight="random", path=0):
+    B.llama3_set_kernel_path(path)
+    layers = [I.layer_weights(w, i, DEV, norm_weight) for i in range(w.n_layers)]
+    outw = I.output_weights(w, DEV, norm_weight)
+    cfg = w.cfg()
+    rows = w.batch * w.seq if w.lm_rows == "all" else w.batch
+    st = Llama3Stack(cfg, layers, outw, w.batch, w.seq, w.seq, lm_rows=rows if w.vocab else 0)
+    if w.input_kind == "ids":
+        ids = I.token_ids(w, DEV)
+        x = torch.empty((w.batch, w.seq, w.dim), dtype=w.torch_dtype, device=DEV)
+        st.embed(ids, x)
+        x0 = O.embed(ids.cpu().numpy(), f64(outw["tok_embeddings"]))
+    else:
+        x = I.activations(w, DEV)
+        x0 = f64(x)
+    st.forward_layers(x, w.seq)
+    torch.cuda.synchronize()
+    oc = oracle_cfg(w)
+    h, kcs, vcs = O.forward_stack(x0, [oracle_layer(l) for l in layers], oc)
+    assert_close(x, h, w.dtype, f"{w.name} hidden")
+    for i, (kc, vc) in enumerate(st.caches):
+        assert_close(kc, kcs[i], w.dtype, f"{w.name} k cache layer {i}")
+        assert_close(vc, vcs[i], w.dtype, f"{w.name} v cache layer {i}")
+    if w.vocab:
+        logits = torch.empty((rows, w.vocab), dtype=torch.float32, device=DEV)
+        ids_out = st.lm_head(x, rows, w.dim, logits)
+        want_logits, _ = O.lm_head(h.reshape(rows, w.dim), f64(outw["norm"]), f64(outw["output"]), w.norm_eps)
+        assert_close(logits, want_logits, w.dtype, f"{w.name} logits")
+        assert_argmax(ids_out, want_logits, f"{w.name} ids")
+
+
+def test_tiny_f32_block_and_lm_head():
+    _run_layers_vs_oracle(wl("tiny_f32"))
+
+
+def test_tiny_f32_pages_init():
+    _run_layers_vs_oracle(wl("tiny_f32"), norm_weight="ones")
+
+
+@pytest.mark.parametrize("path", [0, 1])
+def test_char_8l_stack_and_lm_head(path):
+    _run_layers_vs_oracle(wl("char_8l"), path=path)
+
+
+def test_gqa_768_layer():
+    _run_layers_vs_oracle(wl("gqa_768"))
+
+
+def test_chunked_prefill_then_decode_steps():
+    """Prefill 70 tokens, prefill a second chunk of 50 at start_pos 70, then
+    three one-token decode steps -- against the oracle's full causal pass."""
+    w = small_bf16()
+    layers = [I.layer_weights(w, i, DEV, "random") for i in range(w.n_layers)]
+    cap, total = 200, 70 + 50 + 3
+    st = Llama3Stack(w.cfg(), layers, I.output_weights(w, DEV), w.batch, cap, 70)
+    g = torch.Generator(device="cpu").manual_seed(9)
+    xs = torch.randn((w.batch, total, w.dim), generator=g).to(torch.bfloat16)
+    outs = []
+    a = xs[:, :70].contiguous().to(DEV); st.forward_layers(a, 70, 0); outs.append(a)
+    b = xs[:, 70:120].contiguous().to(DEV); st.forward_layers(b, 50, 70); outs.append(b)
+    for t in range(120, total):
+        d = xs[:, t:t + 1].contiguous().to(DEV)
+        st.decode_layers(d, t)
+        outs.append(d)
+    got = torch.cat([o.cpu() for o in outs], 1)
+    want, kcs, vcs = O.forward_stack(f64(xs), [oracle_layer(l) for l in layers], oracle_cfg(w))
+    assert_close(got, want, "bf16", "chunked + decode")
+    for i, (kc, vc) in enumerate(st.caches):
+        assert_close(kc[:, :total], kcs[i], "bf16", f"k cache {i}")
+        assert_close(vc[:, :total], vcs[i], "bf16", f"v cache {i}")
+
+
+def test_decode_step_matches_prefill_path_for_large_batch():
+    """batch > 256 decode routes to the prefill GEMMs; same answer as the oracle."""
+    w = small_bf16(batch=300, n_layers=1, dim=256, n_heads=4, n_kv_heads=2, ffn_hidden=512)
+    layers = [I.layer_weights(w, 0, DEV, "random")]
+    st = Llama3Stack(w.cfg(), layers, I.output_weights(w, DEV), w.batch, 8, 3)
+    g = torch.Generator(device="cpu").manual_seed(11)
+    xs = torch.randn((w.batch, 4, w.dim), generator=g).to(torch.bfloat16)
+    a = xs[:, :3].contiguous().to(DEV)
+    st.forward_layers(a, 3, 0)
+    d = xs[:, 3:4].contiguous().to(DEV)
+    st.decode_layers(d, 3)
+    want, _, _ = O.forward_stack(f64(xs), [oracle_layer(l) for l in layers], oracle_cfg(w))
+    assert_close(torch.cat([a.cpu(), d.cpu()], 1), want, "bf16", "batch-300 decode")
+
+
+# -------------------------------------------------------------- LM head
+@pytest.mark.parametrize("rows", [1, 5, 32, 300])
+def test_lm_head_8b_vocab(rows):
+    w = wl("llama3_8b_prefill")
+    outw = I.output_weights(w, DEV, "random")
+    h = I.hidden_rows(w, rows, DEV, std=2.0)
+    cfg = B.make_config(w.dim, w.n_heads, w.n_kv_heads, w.ffn_hidden, w.vocab)
+    ws_bytes = B.llama3_workspace_size(cfg, 1, 1, rows)
+    ws = torch.empty((ws_bytes,), dtype=torch.uint8, device=DEV)
+    ids = torch.empty((rows,), dtype=torch.int32, device=DEV)
+    logits = torch.empty((rows, w.vocab), dtype=torch.float32, device=DEV)
+    B.llama3_lm_head_argmax(cfg, outw["norm"], outw["output"], h, rows, w.dim, ids, logits, ws, ws_bytes)
+    ids2 = torch.empty_like(ids)
+    B.llama3_lm_head_argmax(cfg, outw["norm"], outw["output"], h, rows, w.dim, ids2, None, ws, ws_bytes)
+    want, _ = O.lm_head(f64(h), f64(outw["norm"]), f64(outw["output"]), w.norm_eps)
+    assert_close(logits, want, "bf16", "8b logits")
+    assert_argmax(ids, want, "8b ids")
+    assert torch.equal(ids, ids2)
+
+
+def test_lm_head_row_stride_selects_last_positions():
+    w = small_bf16()
+    outw = I.output_weights(w, DEV, "random")
+    x = I.activations(w, DEV)  # [3, 70, 512]
+    cfg = B.make_config(w.dim, w.n_heads, w.n_kv_heads, w.ffn_hidden, w.vocab)
+    ws_bytes = B.llama3_workspace_size(cfg, 1, 1, w.batch)
+    ws = torch.empty((ws_bytes,), dtype=torch.uint8, device=DEV)
+    ids = torch.empty((w.batch,), dtype=torch.int32, device=DEV)
+    logits = torch.empty((w.batch, w.vocab), dtype=torch.float32, device=DEV)
+    B.llama3_lm_head_argmax(cfg, outw["norm"], outw["output"], x[:, -1], w.batch, w.seq * w.dim, ids, logits,
+                            ws, ws_bytes)
+    want, _ = O.lm_head(f64(x)[:, -1], f64(outw["norm"]), f64(outw["output"]), w.norm_eps)
+    assert_close(logits, want, "bf16", "last-position logits")
+    assert_argmax(ids, want, "last-position ids")
+
+
+def test_lm_head_ties_pick_lowest_index():
+    V, D = 300, 512
+    cfg = B.make_config(D, 8, 2, 1024, V)
+    wout = torch.zeros((V, D), dtype=torch.bfloat16, device=DEV)
+    wout[[17, 40, 299]] = 1.0
+    h = torch.ones((2, D), dtype=torch.bfloat16, device=DEV)
+    nw = torch.ones((D,), dtype=torch.bfloat16, device=DEV)
+    ws_bytes = B.llama3_workspace_size(cfg, 1, 1, 2)
+    ws = torch.empty((ws_bytes,), dtype=torch.uint8, device=DEV)
+    ids = torch.empty((2,), dtype=torch.int32, device=DEV)
+    for path in (0, 1):
+        B.llama3_set_kernel_path(path)
+        B.llama3_lm_head_argmax(cfg, nw, wout, h, 2, D, ids, None, ws, ws_bytes)
+        assert ids.tolist() == [17, 17]
+
+
+def test_embed_out_of_range_id_is_reported():
+    w = small_bf16()
+    outw = I.output_weights(w, DEV)
+    cfg = B.make_config(w.dim, w.n_heads, w.n_kv_heads, w.ffn_hidden, w.vocab)
+    ids = torch.tensor([0, 5, w.vocab + 3], dtype=torch.int32, device=DEV)
+    x = torch.empty((3, w.dim), dtype=torch.bfloat16, device=DEV)
+    B.llama3_embed(cfg, ids, outw["tok_embeddings"], x, 3)
+    assert B.llama3_device_status() == 6
+    assert torch.equal(x[1], outw["tok_embeddings"][5])
+    assert torch.count_nonzero(x[2]) == 0

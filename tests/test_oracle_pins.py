@@ -300,6 +300,20 @@ def test_block_brute_force_with_cache_offset():
     np.testing.assert_allclose(vc[0].reshape(P + S, 8), np.array(vs), rtol=1e-12, atol=1e-13)
 
 
+def test_block_rows_matches_brute_force_block():
+    cfg = tiny_cfg()
+    layer = tiny_layer(cfg)
+    P, S = 2, 6
+    k_hist, v_hist = rand(P, 8), rand(P, 8)
+    x = rand(S, 16)
+    want, ks, vs = brute_force_block(x, layer, cfg, P, k_hist, v_hist)
+    rows = [0, 3, 5]
+    got, k, v = O.decoder_block_rows(x, layer, cfg, rows, k_hist.reshape(P, 2, 4), v_hist.reshape(P, 2, 4), P)
+    np.testing.assert_allclose(got, want[rows], rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(k.reshape(S, 8), np.array(ks[P:]), rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(v.reshape(S, 8), np.array(vs[P:]), rtol=1e-12, atol=1e-13)
+
+
 def test_prefill_equals_chunked_prefill_equals_token_by_token_decode():
     # The KV-cache argument of "Build your own Llama 3 from scratch" §3.3: the
     # cached path must give the same result as the full causal pass.
