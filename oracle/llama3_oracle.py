@@ -40,7 +40,7 @@ import numpy as np
 __all__ = [
     "rms_norm", "ffn_hidden_dim", "rope_inverse_frequencies", "rope_angles",
     "apply_rope", "causal_mask", "gqa_attention", "silu", "swiglu_ffn",
-    "decoder_block", "lm_head", "embed", "forward_stack",
+    "decoder_block", "decoder_block_rows", "lm_head", "embed", "forward_stack",
 ]
 
 
@@ -191,6 +191,42 @@ def decoder_block(x, layer, cfg, k_cache, v_cache, start_pos=0):
     h = x + o.reshape(B, S, H * hd) @ _f64(layer["wo"]).T
     hn = rms_norm(h, layer["ffn_norm"], eps)
     return h + swiglu_ffn(hn, layer["w1"], layer["w2"], layer["w3"])
+
+
+def decoder_block_rows(x, layer, cfg, rows, k_prefix=None, v_prefix=None, start_pos=0):
+    """Selected output rows of ``decoder_block`` for ONE sequence.
+
+    x: [S, D] (tokens at positions start_pos..start_pos+S-1); k_prefix /
+    v_prefix: [start_pos, KV, hd] cached entries before them (or None when
+    start_pos == 0).  Keys and values are projected for every token (each row
+    attends to all earlier ones); queries, attention, wo, the FFN and both
+    residuals only for the tokens in ``rows``.  Returns (out [len(rows), D],
+    k [S, KV, hd], v [S, KV, hd]) with k rotated, i.e. what the cache receives.
+    """
+    x = _f64(x)
+    S, D = x.shape
+    H, KV, hd = cfg["n_heads"], cfg["n_kv_heads"], cfg["head_dim"]
+    eps, theta = cfg["norm_eps"], cfg["rope_theta"]
+    rows = list(rows)
+    xn = rms_norm(x, layer["attention_norm"], eps)
+    pos = start_pos + np.arange(S)
+    k = apply_rope((xn @ _f64(layer["wk"]).T).reshape(S, KV, hd), pos, theta)
+    v = (xn @ _f64(layer["wv"]).T).reshape(S, KV, hd)
+    if start_pos:
+        k_all = np.concatenate([_f64(k_prefix), k], 0)
+        v_all = np.concatenate([_f64(v_prefix), v], 0)
+    else:
+        k_all, v_all = k, v
+    xr = x[rows]
+    q = apply_rope((xn[rows] @ _f64(layer["wq"]).T).reshape(len(rows), H, hd),
+                   start_pos + np.asarray(rows), theta)
+    o = np.empty((len(rows), H, hd))
+    for i, t in enumerate(rows):
+        n_keys = start_pos + t + 1
+        o[i] = gqa_attention(q[i:i + 1], k_all[:n_keys], v_all[:n_keys], n_keys - 1)[0]
+    h = xr + o.reshape(len(rows), H * hd) @ _f64(layer["wo"]).T
+    hn = rms_norm(h, layer["ffn_norm"], eps)
+    return h + swiglu_ffn(hn, layer["w1"], layer["w2"], layer["w3"]), k, v
 
 
 # ---------------------------------------------------------------------------
