@@ -1,0 +1,445 @@
+#!/usr/bin/env python
+"""Throughput of the Llama-3-8B-shaped decoder on B200 through the C ABI.
+
+One JSON line (rank 0).  `value` is prefill tokens/s for batch 1 x 8192 tokens
+through embedding, 32 decoder blocks, final norm and LM-head argmax on the
+last position; the `decode` object is the same for one decode step of 32
+sequences against 8192 cached positions each (new token at position 8192).
+Weights are seeded random-init N(0, 0.02) bf16 of the 8B architecture, token
+ids uniform; everything is resident in HBM before the timed region, and the
+16 GB of weights streamed per step are far larger than L2.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun (N > 1) every rank runs its own replica (no collective on the
+data path; `scaling: weak`); times are the max over ranks.
+"""
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from llama_decoder_only_rmsnorm_b200 import binding as B  # noqa: E402
+from llama_decoder_only_rmsnorm_b200 import inputs as I  # noqa: E402
+from llama_decoder_only_rmsnorm_b200.model import Llama3Stack  # noqa: E402
+
+METRIC = "prefill & decode tokens/s on 1 B200; % of bf16 tensor / HBM roofline"
+PREFILL, DECODE = I.WORKLOADS["llama3_8b_prefill"], I.WORKLOADS["llama3_8b_decode"]
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_PATH = os.path.join(ROOT, "profiles", "traffic.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-decode", action="store_true")
+    p.add_argument("--layers", type=int, default=None, help=argparse.SUPPRESS)  # profiling captures only
+    return p.parse_args()
+
+
+# --------------------------------------------------------------- plumbing ---
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(v, world):
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_PATH) as f:
+            return json.load(f), "measured"
+    except OSError:
+        return FALLBACK_PEAKS, "fallback"
+
+
+def source_hash(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kind, files):
+    """Per-launch DRAM bytes from a committed ncu capture, if the kernel's
+    sources are unchanged since it was taken; else None."""
+    try:
+        with open(TRAFFIC_PATH) as f:
+            rec = json.load(f).get(kind)
+    except (OSError, ValueError):
+        return None
+    if not rec or rec.get("source_sha") != source_hash(files):
+        return None
+    return rec.get("traffic_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples every 200 ms while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.gpu), "-lms", "200"], stdout=open(self.path, "w"),
+                                         stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            for line in open(self.path):
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        except OSError:
+            pass
+        finally:
+            if self.path and os.path.exists(self.path):
+                os.remove(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        power = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        loaded = [s for s, p in zip(sm, power) if p > 300.0] or sm
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for n, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+def event_pairs(n):
+    """n (start, stop) event pairs, each recorded once so that its CUDA event
+    exists before its handle goes to the library (torch creates them lazily)."""
+    pairs = ([torch.cuda.Event(enable_timing=True) for _ in range(n)],
+             [torch.cuda.Event(enable_timing=True) for _ in range(n)])
+    for e in pairs[0] + pairs[1]:
+        e.record()
+    return pairs
+
+
+# ------------------------------------------------------------------ model ---
+def build(dev):
+    w = PREFILL
+    layers = [I.layer_weights(w, i, dev) for i in range(w.n_layers)]
+    outw = I.output_weights(w, dev)
+    return layers, outw
+
+
+def decode_caches(dev, n_layers):
+    wd = DECODE
+    return [I.kv_cache(wd, i, wd.cache_len + 1, dev) for i in range(n_layers)]
+
+
+def time_steps(fn, steps, warmup, world, timer=None, name="timed"):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    if B.llama3_device_status() != 0:
+        raise RuntimeError("device status word set during warm-up")
+    barrier(world)
+    if timer:
+        kind, n = timer
+        starts, stops = event_pairs(n)
+        B.llama3_set_launch_timer(kind, starts, stops)
+    l0 = B.llama3_launch_count()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.nvtx.range_push(name)
+    t0.record()
+    for _ in range(steps):
+        fn()
+    t1.record()
+    torch.cuda.nvtx.range_pop()
+    torch.cuda.synchronize()
+    launches = B.llama3_launch_count() - l0
+    if B.llama3_device_status() != 0:
+        raise RuntimeError("device status word set during the timed region")
+    barrier(world)
+    ms = t0.elapsed_time(t1) / steps
+    kernel_ms = None
+    if timer:
+        used = B.llama3_launch_timer_used()
+        B.llama3_set_launch_timer(kind, [], [])
+        if used:
+            kernel_ms = sum(s.elapsed_time(e) for s, e in zip(starts[:used], stops[:used])) / used
+    return max_over_ranks(ms, world), kernel_ms, launches
+
+
+# ------------------------------------------------------- oracle baseline ---
+def oracle_sample(layers, outw, caches, prefix, decode_seq=True):
+    """Time the fp64 oracle (as it stands) on a bounded sample of both
+    workloads: the first `prefix` tokens of the prefill through all blocks +
+    final norm + LM head, and one sequence's decode step at position 8192.
+    Weight conversion to fp64 is outside the timed region."""
+    from oracle import llama3_oracle as O
+    import threadpoolctl
+    cfg = {k: v for k, v in PREFILL.cfg().items() if k not in ("vocab", "dtype")}
+    f64 = lambda t: t.detach().to(torch.float32).cpu().numpy().astype(np.float64)
+    ids = I.token_ids(PREFILL, "cuda")[:, :prefix].cpu().numpy()
+    dids = I.token_ids(DECODE, "cuda")[:1].cpu().numpy()
+    table = outw["tok_embeddings"]
+
+    def embed(id_arr):
+        # the oracle's gather over the rows this sample uses (a small table)
+        uniq, inv = np.unique(id_arr, return_inverse=True)
+        sub = f64(table[torch.as_tensor(uniq, device=table.device).long()])
+        return O.embed(inv.reshape(id_arr.shape), sub)
+
+    x = embed(ids)
+    xd = embed(dids)
+    t_pre = t_dec = 0.0
+    P = DECODE.cache_len
+    for i, layer in enumerate(layers):
+        ol = {k: f64(layer[k]) for k in ("attention_norm", "wq", "wk", "wv", "wo", "ffn_norm", "w1", "w2", "w3")}
+        kc = np.zeros((1, prefix, cfg["n_kv_heads"], cfg["head_dim"]))
+        vc = np.zeros_like(kc)
+        t = time.perf_counter()
+        x = O.decoder_block(x, ol, cfg, kc, vc, 0)
+        t_pre += time.perf_counter() - t
+        if decode_seq:
+            kd = np.zeros((1, P + 1, cfg["n_kv_heads"], cfg["head_dim"]))
+            vd = np.zeros_like(kd)
+            kd[0, :P] = f64(caches[i][0][0, :P])
+            vd[0, :P] = f64(caches[i][1][0, :P])
+            t = time.perf_counter()
+            xd = O.decoder_block(xd, ol, cfg, kd, vd, P)
+            t_dec += time.perf_counter() - t
+        del ol
+    nw, wout = f64(outw["norm"]), f64(outw["output"])
+    t = time.perf_counter()
+    O.lm_head(x[:, -1], nw, wout, PREFILL.norm_eps)
+    t_pre += time.perf_counter() - t
+    if decode_seq:
+        t = time.perf_counter()
+        O.lm_head(xd[:, -1], nw, wout, PREFILL.norm_eps)
+        t_dec += time.perf_counter() - t
+    info = threadpoolctl.threadpool_info()
+    cores = max([d.get("num_threads", 1) for d in info] or [os.cpu_count()])
+    return t_pre, t_dec, cores
+
+
+# ------------------------------------------------------------- our arm ---
+def run_ours(args):
+    world, rank, local = dist_setup()
+    dev = f"cuda:{local}"
+    peaks, peak_kind = load_peaks()
+    layers, outw = build(dev)
+    n_layers = args.layers or PREFILL.n_layers
+    layers = layers[:n_layers]
+    cfg = PREFILL.cfg()
+    S, D = PREFILL.seq, PREFILL.dim
+
+    # ---------------- prefill
+    pst = Llama3Stack(cfg, layers, outw, batch=1, cache_cap=S, max_seq=S, lm_rows=DECODE.batch, device=dev)
+    ids = I.token_ids(PREFILL, dev)
+    x = torch.empty((1, S, D), dtype=torch.bfloat16, device=dev)
+
+    def prefill_step():
+        pst.embed(ids, x)
+        pst.forward_layers(x, S, 0)
+        return pst.lm_head(x[:, -1], 1, S * D)
+
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        ms, k_ms, launches = time_steps(prefill_step, args.steps, args.warmup, world,
+                                        timer=("gemm_w13", args.steps * n_layers), name="prefill_timed")
+    clocks = clk.summary()
+    value = world * S / (ms / 1e3)
+    F = PREFILL.ffn_hidden
+    w13_flop = 2.0 * S * (2 * F) * D
+    achieved = w13_flop / (k_ms / 1e3) / 1e12 if k_ms else None
+    peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    roofline = {"bound": "tensor", "kernel": "tc_gemm w1|w3 + SwiGLU (M=8192, N=2x14336, K=4096)",
+                "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": (achieved / peak) if achieved else None,
+                "peak_source": f"{peak_kind} bf16_tflops_sustained",
+                "traffic": recorded_traffic("gemm_w13", ["llama_decoder_only_rmsnorm_b200/csrc/tc_gemm.cuh"]),
+                "kernel_ms": k_ms}
+    total_flop = n_layers * (2.0 * S * 6.979e9 / 32) + 2.0 * D * PREFILL.vocab  # linear layers + LM head row
+    attn_flop = n_layers * PREFILL.n_heads * 2.0 * S * (S + 1) * PREFILL.head_dim
+    whole = {"flop_per_step": total_flop + attn_flop,
+             "tflops": (total_flop + attn_flop) / (ms / 1e3) / 1e12}
+    whole["frac_of_peak"] = whole["tflops"] / peak
+
+    # e2e through the public API with host buffers
+    ids_h = ids.cpu().pin_memory()
+    out_h = torch.empty((1,), dtype=torch.int32).pin_memory()
+
+    def prefill_e2e():
+        ids.copy_(ids_h, non_blocking=True)
+        out_h.copy_(prefill_step(), non_blocking=True)
+
+    e2e_ms, _, _ = time_steps(prefill_e2e, args.steps, 1, world, name="prefill_e2e")
+    e2e = {"value": world * S / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": ids_h.numel() * 4,
+           "d2h_bytes_per_step": 4}
+    del pst, x
+    torch.cuda.empty_cache()
+
+    # ---------------- decode
+    decode = None
+    caches = None
+    if not args.no_decode:
+        caches = decode_caches(dev, n_layers)
+        Bd, P = DECODE.batch, DECODE.cache_len
+        dst = Llama3Stack(cfg, layers, outw, batch=Bd, cache_cap=P + 1, max_seq=1, lm_rows=Bd, device=dev,
+                          caches=caches)
+        dids = I.token_ids(DECODE, dev)
+        xd = torch.empty((Bd, 1, D), dtype=torch.bfloat16, device=dev)
+
+        def decode_step():
+            dst.embed(dids, xd)
+            dst.decode_layers(xd, P)
+            return dst.lm_head(xd, Bd, D)
+
+        with ClockSampler(torch.cuda.current_device()) as clk2:
+            dms, dk_ms, dlaunch = time_steps(decode_step, args.steps, args.warmup, world,
+                                             timer=("decode_attention", args.steps * n_layers), name="decode_timed")
+        kv_bytes = Bd * (P + 1) * DECODE.n_kv_heads * DECODE.head_dim * 2 * 2
+        dach = kv_bytes / (dk_ms / 1e3) / 1e9 if dk_ms else None
+        hbm = peaks.get("hbm_gbs")
+        step_bytes = n_layers * (kv_bytes + 2 * 6.979e9 / 32) + 2.0 * DECODE.vocab * D
+        dids_h = dids.cpu().pin_memory()
+        dout_h = torch.empty((Bd,), dtype=torch.int32).pin_memory()
+
+        def decode_e2e():
+            dids.copy_(dids_h, non_blocking=True)
+            dout_h.copy_(decode_step(), non_blocking=True)
+
+        de2e_ms, _, _ = time_steps(decode_e2e, args.steps, 1, world, name="decode_e2e")
+        decode = {"metric": "decode tokens/s", "value": world * Bd / (dms / 1e3), "unit": "tokens/s",
+                  "ms_per_step": dms, "steps": args.steps, "warmup": args.warmup,
+                  "config": {"workload": "llama3_8b_decode", "batch": Bd, "cached_positions": P,
+                             "new_token_position": P},
+                  "roofline": {"bound": "hbm", "kernel": "split-KV decode attention (1.07 GB K/V per launch)",
+                               "achieved": dach, "peak": hbm, "unit": "GB/s",
+                               "frac": (dach / hbm) if dach else None, "peak_source": f"{peak_kind} hbm_gbs",
+                               "traffic": recorded_traffic("decode_attention", [
+                                   "llama_decoder_only_rmsnorm_b200/csrc/decode_attention.cuh"]),
+                               "kernel_ms": dk_ms},
+                  "whole_step": {"bytes_per_step": step_bytes, "gbs": step_bytes / (dms / 1e3) / 1e9,
+                                 "frac_of_hbm": step_bytes / (dms / 1e3) / 1e9 / hbm},
+                  "e2e": {"value": world * Bd / (de2e_ms / 1e3), "unit": "tokens/s",
+                          "h2d_bytes_per_step": Bd * 4, "d2h_bytes_per_step": Bd * 4},
+                  "gpu_launches": dlaunch, "clocks": clk2.summary()}
+
+    # ---------------- oracle on the host cores
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        prefix = 64
+        t_pre, t_dec, cores = oracle_sample(layers, outw, caches, prefix, decode_seq=caches is not None)
+        cpu = {"value": prefix / t_pre, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"fp64 oracle, first {prefix} tokens of the prefill through all {n_layers} blocks + "
+                         "final norm + LM head on the last position (weight fp64 conversion not timed)"}
+        if decode is not None and t_dec > 0:
+            decode["cpu_baseline"] = {"value": 1.0 / t_dec, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                      "sample": "fp64 oracle, one sequence's decode step at position 8192 "
+                                                f"through all {n_layers} blocks + LM head"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic: seeded random-init N(0,0.02) weights of the Llama-3-8B shape, uniform token ids",
+                "config": {"workload": "llama3_8b_prefill", "batch": 1, "seq_len": S, "layers": n_layers,
+                           "lm_head_rows": "last position", "parallelism": f"replicas x{world}",
+                           "l2": "inputs larger than L2 (16 GB of weights streamed per step)"},
+                "roofline": roofline, "whole_step": whole, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": launches, "clocks": clocks, "decode": decode}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+# ------------------------------------------------------- reference arm ---
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    dev = f"cuda:{int(os.environ.get('LOCAL_RANK', '0'))}"
+    torch.cuda.set_device(dev)
+    layers, outw = build(dev)
+    prefix = 16
+    times = []
+    for _ in range(args.warmup + args.steps):
+        t_pre, _, cores = oracle_sample(layers, outw, None, prefix, decode_seq=False)
+        times.append(t_pre)
+    ts = times[args.warmup:]
+    ms = 1e3 * sum(ts) / len(ts)
+    v = prefix / (ms / 1e3)
+    sample = (f"fp64 oracle, first {prefix} tokens of the 8B-shaped prefill through all 32 blocks + final norm "
+              "+ LM head on the last position, per step (weight fp64 conversion not timed)")
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (same seeds as ours)",
+            "config": {"workload": "llama3_8b_prefill", "batch": 1, "seq_len": PREFILL.seq,
+                       "sampled_tokens": prefix},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    a = parse()
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_ours(a)
