@@ -173,6 +173,35 @@ int llama3_lm_head_argmax(const llama3_config* cfg, const void* norm_w, const vo
                           float* logits_out, void* ws, size_t ws_bytes,
                           llama3_stream_t stream);
 
+/*
+ * LM head + argmax without a caller-provided workspace.
+ *
+ * No counterpart on the pages: this is a convenience for hosts that cannot
+ * hand the library a workspace -- for example a C program embedded in a
+ * server whose device memory is already carved up by another allocator, or
+ * a caller that is not allowed to grow its device footprint after start-up.
+ * Everything else is as llama3_lm_head_argmax: same arguments (minus ws and
+ * ws_bytes), same kernels, same results.
+ *
+ * Scratch: the normalised rows and the per-row argmax keys live in one fixed
+ * array of LLAMA3_NOALLOC_SCRATCH_BYTES (4 MiB) that the library declares as a
+ * device global, so every GPU that loads the library holds those 4 MiB until
+ * the process exits.  The call needs  roundup(rows * 8, 256) +
+ * rows * dim * sizeof(element)  bytes of it and returns LLAMA3_ERR_WORKSPACE
+ * when that exceeds the array (for dim 4096 in bf16: at most 511 rows).
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  All calls share the one array and find the
+ * previous call's contents there (the argmax keys are re-initialised by each
+ * call): calls whose executions overlap on the GPU (other streams, other
+ * host threads) race on it and must be serialised by the caller.  The
+ * library allocates nothing for this call.
+ */
+#define LLAMA3_NOALLOC_SCRATCH_BYTES (4u << 20)
+int llama3_lm_head_argmax_noalloc(const llama3_config* cfg, const void* norm_w, const void* w_out,
+                                  const void* h, int rows, long long row_stride,
+                                  int32_t* ids_out, float* logits_out, llama3_stream_t stream);
+
 /* ---- building blocks (the steps of the calls above, exposed for tests) ---- */
 
 /* y[r] = x[r] / sqrt(mean(x[r]^2) + eps) * w  ([S1] §5, [S2] §3.1); x rows at

@@ -52,6 +52,7 @@ _SIGNATURES = {
     "llama3_layer_forward": [_cfgp, _wp, _p, _i, _p, _p, _p, _i, _i, _i, _i, _p, _sz, _p],
     "llama3_layer_decode": [_cfgp, _wp, _p, _i, _p, _p, _p, _i, _i, _i, _p, _sz, _p],
     "llama3_lm_head_argmax": [_cfgp, _p, _p, _p, _i, _ll, _p, _p, _p, _sz, _p],
+    "llama3_lm_head_argmax_noalloc": [_cfgp, _p, _p, _p, _i, _ll, _p, _p, _p],
     "llama3_rmsnorm": [_cfgp, _p, _ll, _p, _p, _i, _p],
     "llama3_linear": [_cfgp, _p, _p, _p, _p, _i, _i, _i, _p, _sz, _p],
     "llama3_attention": [_cfgp, _p, _p, _p, _i, _i, _i, _i, _p, _p, _sz, _p],
@@ -164,6 +165,17 @@ def llama3_lm_head_argmax(cfg, norm_w, w_out, h, rows, row_stride, ids_out, logi
     _check("llama3_lm_head_argmax", lib().llama3_lm_head_argmax(
         ctypes.byref(cfg), _ptr(norm_w), _ptr(w_out), _ptr(h), rows, row_stride, _ptr(ids_out),
         _ptr(logits_out), _ptr(ws), ws_bytes, _stream(stream)))
+
+
+NOALLOC_SCRATCH_BYTES = 4 << 20
+
+
+def llama3_lm_head_argmax_noalloc(cfg, norm_w, w_out, h, rows, row_stride, ids_out, logits_out, stream=None):
+    """LM head + argmax for callers that cannot pass a workspace: the library
+    uses its own fixed 4 MiB device scratch (shared by all calls)."""
+    _check("llama3_lm_head_argmax_noalloc", lib().llama3_lm_head_argmax_noalloc(
+        ctypes.byref(cfg), _ptr(norm_w), _ptr(w_out), _ptr(h), rows, row_stride, _ptr(ids_out),
+        _ptr(logits_out), _stream(stream)))
 
 
 def llama3_rmsnorm(cfg, x, row_stride, w, y, rows, stream=None):

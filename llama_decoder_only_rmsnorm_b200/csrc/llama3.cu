@@ -824,3 +824,85 @@ int llama3_lm_head_argmax(const llama3_config* cfg, const void* norm_w, const vo
 }
 
 }  // extern "C"
+
+// ===========================================================================
+// LM head without a caller workspace: scratch in a fixed device global.
+// ===========================================================================
+// Callers that cannot supply device memory use this 4 MiB array instead of a
+// workspace.  It exists on every device that loads the library.  Host code
+// must not use the symbol as a pointer: its device address is looked up once
+// per device with cudaGetSymbolAddress and cached in g_noalloc_addr.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[LLAMA3_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+void* g_noalloc_addr[kMaxDevices];
+std::mutex g_noalloc_mu;
+
+// Device address of g_noalloc_scratch on the current device (set-up on first use).
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  L3_TRY(current_device(&dev));
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e);
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return LLAMA3_OK;
+}
+}  // namespace
+
+extern "C" int llama3_lm_head_argmax_noalloc(const llama3_config* cfg, const void* norm_w, const void* w_out,
+                                             const void* h, int rows, long long row_stride, int32_t* ids_out,
+                                             float* logits_out, llama3_stream_t stream) {
+  L3_TRY(check_config(cfg));
+  if (!norm_w || !w_out || !h || !ids_out || rows < 1 || cfg->vocab < 1 || row_stride < cfg->dim)
+    return LLAMA3_ERR_ARG;
+  if (!aligned16(norm_w) || !aligned16(w_out) || !aligned16(h) || !aligned16(ids_out) ||
+      (logits_out && !aligned16(logits_out)))
+    return LLAMA3_ERR_ALIGN;
+  if ((row_stride * (long long)esize(cfg)) % 16) return LLAMA3_ERR_ALIGN;
+  const size_t keys_bytes = up256((size_t)rows * 8);
+  const size_t rows_bytes = (size_t)rows * cfg->dim * esize(cfg);
+  if (keys_bytes + rows_bytes > (size_t)LLAMA3_NOALLOC_SCRATCH_BYTES) return LLAMA3_ERR_WORKSPACE;
+  void* base = nullptr;
+  L3_TRY(noalloc_scratch(&base));
+  unsigned long long* keys = reinterpret_cast<unsigned long long*>(base);
+  void* hn = static_cast<char*>(base) + keys_bytes;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int V = cfg->vocab, D = cfg->dim;
+  L3_TRY(rmsnorm_any(cfg, h, row_stride, norm_w, hn, rows, st));
+  // the keys hold the previous call's maxima: start from zero every call
+  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, argmax_init_kernel<<<blocks_for(rows, 256), 256, 0, st>>>(keys, rows));
+  L3_TRY(launch_check());
+  if (use_tc(cfg)) {
+    const int bn = rows <= 16 ? 16 : rows <= 32 ? 32 : rows <= 64 ? 64 : rows <= 128 ? 128 : 256;
+    CUtensorMap ma, mb;
+    L3_TRY(make_map(&ma, w_out, V, D, 128));
+    L3_TRY(make_map(&mb, hn, rows, D, bn));
+    GemmShape sh = make_shape(V, 0, rows, D, bn, 1);
+    EpiParams ep = empty_epi();
+    ep.logits = logits_out;
+    ep.keys = keys;
+    switch (bn) {
+      case 16: L3_TRY((launch_gemm<16, 8, EPI_ARGMAX, false>(LLAMA3_KERNEL_LM_HEAD, ma, ma, mb, mb, sh, ep, st))); break;
+      case 32: L3_TRY((launch_gemm<32, 8, EPI_ARGMAX, false>(LLAMA3_KERNEL_LM_HEAD, ma, ma, mb, mb, sh, ep, st))); break;
+      case 64: L3_TRY((launch_gemm<64, 6, EPI_ARGMAX, false>(LLAMA3_KERNEL_LM_HEAD, ma, ma, mb, mb, sh, ep, st))); break;
+      case 128: L3_TRY((launch_gemm<128, 5, EPI_ARGMAX, false>(LLAMA3_KERNEL_LM_HEAD, ma, ma, mb, mb, sh, ep, st))); break;
+      default: L3_TRY((launch_gemm<256, 4, EPI_ARGMAX, false>(LLAMA3_KERNEL_LM_HEAD, ma, ma, mb, mb, sh, ep, st))); break;
+    }
+  } else {
+    const long long warps = (long long)rows * ((V + 31) / 32);
+    if (cfg->dtype == LLAMA3_DTYPE_F32)
+      L3_LAUNCH(LLAMA3_KERNEL_LM_HEAD, st, lm_head_simt_kernel<float><<<blocks_for(warps * 32, 256), 256, 0, st>>>(
+                                               (const float*)hn, (const float*)w_out, logits_out, keys, rows, V, D));
+    else
+      L3_LAUNCH(LLAMA3_KERNEL_LM_HEAD, st, lm_head_simt_kernel<bf16><<<blocks_for(warps * 32, 256), 256, 0, st>>>(
+                                               (const bf16*)hn, (const bf16*)w_out, logits_out, keys, rows, V, D));
+    L3_TRY(launch_check());
+  }
+  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, argmax_finalize_kernel<<<blocks_for(rows, 256), 256, 0, st>>>(keys, ids_out, rows));
+  return launch_check();
+}
