@@ -12,130 +12,9 @@
 
 namespace l3 {
 
-// Partial record per (b, h, split): m (running max of the scaled scores),
-// l (sum of exp(s - m)), acc[hd] (sum of exp(s - m) * v).  Stored as floats
-// [B][H][splits][hd + 2].
-template <int HD, int NREP>
-__global__ void __launch_bounds__(128)
-    decode_attention_split_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k_cache,
-                                  const bf16* __restrict__ v_cache, float* __restrict__ part,
-                                  int H, int KV, int cap, int n_keys, int keys_per_split,
-                                  int splits, float scale_log2) {
-  constexpr int DPL = HD / 32;  // output dims per lane
-  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int j0 = split * keys_per_split;
-  const int j1 = min(j0 + keys_per_split, n_keys);
-
-  __shared__ __align__(16) float qs[NREP][HD];
-  __shared__ float red_m[4][NREP], red_l[4][NREP];
-  __shared__ float red_acc[4][NREP][HD];
-
-  for (int i = threadIdx.x; i < NREP * HD; i += 128) {
-    const int h = i / HD, d = i % HD;
-    qs[h][d] = __bfloat162float(q[((size_t)b * H + g * NREP + h) * HD + d]) * scale_log2;
-  }
-  __syncthreads();
-
-  float m[NREP], l[NREP], acc[NREP][DPL];
-#pragma unroll
-  for (int h = 0; h < NREP; ++h) {
-    m[h] = -INFINITY;
-    l[h] = 0.f;
-#pragma unroll
-    for (int i = 0; i < DPL; ++i) acc[h][i] = 0.f;
-  }
-
-  const size_t row_stride = (size_t)KV * HD;  // elements between consecutive positions
-  const bf16* kbase = k_cache + ((size_t)b * cap * KV + g) * HD;
-  const bf16* vbase = v_cache + ((size_t)b * cap * KV + g) * HD;
-
-  for (int c0 = j0 + warp * 32; c0 < j1; c0 += 128) {
-    // scores of key c0 + lane for every head (log2 domain)
-    const int j = c0 + lane;
-    float s[NREP];
-#pragma unroll
-    for (int h = 0; h < NREP; ++h) s[h] = 0.f;
-    if (j < j1) {
-      const uint4* kr = reinterpret_cast<const uint4*>(kbase + (size_t)j * row_stride);
-#pragma unroll 4
-      for (int d8 = 0; d8 < HD / 8; ++d8) {
-        const uint4 kk = __ldg(kr + d8);
-        const float k0 = bf16lo(kk.x), k1 = bf16hi(kk.x), k2 = bf16lo(kk.y), k3 = bf16hi(kk.y);
-        const float k4 = bf16lo(kk.z), k5 = bf16hi(kk.z), k6 = bf16lo(kk.w), k7 = bf16hi(kk.w);
-#pragma unroll
-        for (int h = 0; h < NREP; ++h) {
-          const float4 qa = *reinterpret_cast<const float4*>(&qs[h][d8 * 8]);
-          const float4 qb = *reinterpret_cast<const float4*>(&qs[h][d8 * 8 + 4]);
-          s[h] = fmaf(qa.x, k0, fmaf(qa.y, k1, fmaf(qa.z, k2, fmaf(qa.w, k3, s[h]))));
-          s[h] = fmaf(qb.x, k4, fmaf(qb.y, k5, fmaf(qb.z, k6, fmaf(qb.w, k7, s[h]))));
-        }
-      }
-    }
-    const int nvalid = min(32, j1 - c0);
-    float p[NREP];
-#pragma unroll
-    for (int h = 0; h < NREP; ++h) {
-      const float sv = lane < nvalid ? s[h] : -INFINITY;
-      const float cmax = warp_max(sv);
-      const float mn = fmaxf(m[h], cmax);
-      const float corr = exp2f(m[h] - mn);
-      p[h] = lane < nvalid ? exp2f(sv - mn) : 0.f;
-      l[h] = l[h] * corr + warp_sum(p[h]);
-#pragma unroll
-      for (int i = 0; i < DPL; ++i) acc[h][i] *= corr;
-      m[h] = mn;
-    }
-    // P.V: lane owns dims lane*DPL .. lane*DPL+DPL-1
-    for (int jj = 0; jj < nvalid; ++jj) {
-      const bf16* vr = vbase + (size_t)(c0 + jj) * row_stride + lane * DPL;
-      float vv[DPL];
-      if constexpr (DPL == 4) {
-        const uint2 u = __ldg(reinterpret_cast<const uint2*>(vr));
-        vv[0] = bf16lo(u.x); vv[1] = bf16hi(u.x); vv[2] = bf16lo(u.y); vv[3] = bf16hi(u.y);
-      } else if constexpr (DPL == 2) {
-        const uint32_t u = __ldg(reinterpret_cast<const unsigned int*>(vr));
-        vv[0] = bf16lo(u); vv[1] = bf16hi(u);
-      } else {
-#pragma unroll
-        for (int i = 0; i < DPL; ++i) vv[i] = __bfloat162float(vr[i]);
-      }
-#pragma unroll
-      for (int h = 0; h < NREP; ++h) {
-        const float ph = __shfl_sync(0xffffffffu, p[h], jj);
-#pragma unroll
-        for (int i = 0; i < DPL; ++i) acc[h][i] = fmaf(ph, vv[i], acc[h][i]);
-      }
-    }
-  }
-
-  // merge the four warps
-#pragma unroll
-  for (int h = 0; h < NREP; ++h) {
-    if (lane == 0) { red_m[warp][h] = m[h]; red_l[warp][h] = l[h]; }
-#pragma unroll
-    for (int i = 0; i < DPL; ++i) red_acc[warp][h][lane * DPL + i] = acc[h][i];
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; i < NREP * (HD + 2); i += 128) {
-    const int h = i / (HD + 2), c = i % (HD + 2);
-    float mx = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) mx = fmaxf(mx, red_m[w][h]);
-    float val = 0.f;
-    if (c == 0) {
-      val = mx;
-    } else {
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const float f = red_m[w][h] == -INFINITY ? 0.f : exp2f(red_m[w][h] - mx);
-        val += f * (c == 1 ? red_l[w][h] : red_acc[w][h][c - 2]);
-      }
-    }
-    part[(((size_t)b * H + g * NREP + h) * splits + split) * (HD + 2) + c] = val;
-  }
-}
-
+// Partial record per (b, h, split): m (running max of the scores, log2
+// domain), l (sum of 2^(s - m)), acc[hd] (sum of 2^(s - m) * v).  Stored as
+// floats [B][H][splits][hd + 2] and merged by the combine kernel.
 // out[b, h, :] = sum_s e^(m_s - M) acc_s / sum_s e^(m_s - M) l_s
 template <int HD>
 __global__ void decode_attention_combine_kernel(const float* __restrict__ part, bf16* __restrict__ out,
@@ -153,6 +32,331 @@ __global__ void decode_attention_combine_kernel(const float* __restrict__ part, 
       num += f * p[s * (HD + 2) + 2 + d];
     }
     out[(size_t)bh * HD + d] = __float2bfloat16_rn(num / den);
+  }
+}
+
+// ===========================================================================
+// Tensor-core variant: the same partial records, produced by TMA streaming
+// of K/V tiles and two tcgen05 MMAs per 128-key tile:
+//   S^T[key, head] = K_tile[128 x hd] . Q^T          (M = 128 keys, N = 16)
+//   O^T[dim, head] += V_tile^T[hd x 128] . P^T       (M = 128 dims, N = 16)
+// Keys sit on the MMA's 128-row side, so the n_rep query heads of a group
+// (padded to 16 columns) share every K/V byte read.  K/V tiles arrive through
+// a 3-stage ring of 64 KB; the CUDA cores only do the per-head softmax.
+// ===========================================================================
+struct DecodeShape {
+  int B, H, KV, nrep, n_keys, tiles, splits, tiles_per_split, units;
+  float scale_log2;
+};
+
+template <int HD>
+struct DecodeTcCfg {
+  static constexpr int SLAB = 128 * 128;            // 128 rows x 64 bf16
+  static constexpr int CHUNKS_K = (HD + 63) / 64;   // slabs holding a K tile
+  static constexpr int K_BYTES = CHUNKS_K * SLAB;
+  static constexpr int V_BYTES = 2 * SLAB;          // always 128 dims (zero beyond hd)
+  static constexpr int STAGE_BYTES = K_BYTES + V_BYTES;
+  static constexpr int STAGES = 3;
+  static constexpr int Q_SLAB = 16 * 128;           // 16 rows x 64 bf16
+  static constexpr int Q_BYTES = CHUNKS_K * Q_SLAB;
+  static constexpr int P_BYTES = 2 * Q_SLAB;        // 16 heads x 128 keys
+  static constexpr int OFF_STAGE = 0;
+  static constexpr int OFF_Q = STAGES * STAGE_BYTES;
+  static constexpr int OFF_P = OFF_Q + 2 * Q_BYTES;
+  static constexpr int OFF_RED = OFF_P + 2 * P_BYTES;               // [2][4][16] floats
+  static constexpr int OFF_BAR = OFF_RED + 2 * 4 * 16 * 4;
+  static constexpr int N_BARS = 2 * STAGES + 4 /*q*/ + 2 /*s_full*/ + 2 /*p_full*/ + 1 /*o_done*/ +
+                                2 /*red*/;
+  static constexpr int SMEM_BYTES = 1024 + OFF_BAR + N_BARS * 8 + 16;
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
+};
+
+__device__ __forceinline__ void decode_unit(const DecodeShape& ds, int u, int& b, int& g, int& split, int& t0,
+                                            int& t1) {
+  split = u % ds.splits;
+  const int bg = u / ds.splits;
+  g = bg % ds.KV;
+  b = bg / ds.KV;
+  t0 = split * ds.tiles_per_split;
+  t1 = min(t0 + ds.tiles_per_split, ds.tiles);
+}
+
+template <int HD, int NREP>
+__global__ void __launch_bounds__(256, 1)
+    decode_attention_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
+                               const __grid_constant__ CUtensorMap mapV, float* __restrict__ part,
+                               const DecodeShape ds, const unsigned long long wait_ns) {
+  using C = DecodeTcCfg<HD>;
+  static_assert(NREP >= 1 && NREP <= 16, "query heads per KV head (upper bound)");
+  const int nrep = ds.nrep;   // <= NREP
+  constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 16, 0, 0);
+  constexpr uint32_t IDESC_O = idesc_bf16_f32(128, 16, 1, 0);   // V^T: dims contiguous (MN-major A)
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* kv_full = bars;
+  uint64_t* kv_empty = kv_full + C::STAGES;
+  uint64_t* q_full = kv_empty + C::STAGES;   // [2]
+  uint64_t* q_empty = q_full + 2;            // [2]
+  uint64_t* s_full = q_empty + 2;       // [2]
+  uint64_t* p_full = s_full + 2;        // [2]
+  uint64_t* o_done = p_full + 2;        // [1]
+  uint64_t* red_bar = o_done + 1;       // [2] cross-warp reductions of the softmax warps
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red_bar + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&q_full[s], 1); mbar_init(&q_empty[s], 1);
+      mbar_init(&s_full[s], 1); mbar_init(&p_full[s], 128);
+    }
+    mbar_init(o_done, 1);
+    mbar_init(&red_bar[0], 4); mbar_init(&red_bar[1], 4);
+    fence_mbar_init();
+  }
+  // P rows >= NREP stay zero for the whole kernel; dims >= hd of the V slabs
+  // that TMA never writes (head_dim 64) stay zero as well.
+  for (int i = threadIdx.x; i < 2 * C::P_BYTES / 16; i += blockDim.x)
+    reinterpret_cast<uint4*>(smem + C::OFF_P)[i] = make_uint4(0, 0, 0, 0);
+  if (HD <= 64) {
+    for (int s = 0; s < C::STAGES; ++s)
+      for (int i = threadIdx.x; i < C::SLAB / 16; i += blockDim.x)
+        reinterpret_cast<uint4*>(smem + C::OFF_STAGE + s * C::STAGE_BYTES + C::K_BYTES + C::SLAB)[i] =
+            make_uint4(0, 0, 0, 0);
+  }
+  fence_proxy_async_smem();
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&mapQ); prefetch_tensormap(&mapK); prefetch_tensormap(&mapV);
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, 64);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;   // S buffers: cols [0,16) and [16,32); O: [32,48)
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      int st = 0, kq = 0;
+      uint32_t ph = 0, qph[2] = {0, 0};
+      uint32_t iss = 0, par = 0, qiss = 0, qpar = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < ds.units && ok; u += gridDim.x, ++kq) {
+        int b, g, split, t0, t1;
+        decode_unit(ds, u, b, g, split, t0, t1);
+        const int qb = kq & 1;
+        if (!mbar_wait(&q_empty[qb], qph[qb] ^ 1u, wait_ns)) break;
+        mbar_arrive_expect_tx(&q_full[qb], C::Q_BYTES);
+        for (int c = 0; c < C::CHUNKS_K; ++c)
+          tma_load_2d(smem + C::OFF_Q + qb * C::Q_BYTES + c * C::Q_SLAB, &mapQ, &q_full[qb], c * 64,
+                      b * ds.H + g * nrep);
+        qiss |= 1u << qb; qpar = (qpar & ~(1u << qb)) | (qph[qb] << qb);
+        qph[qb] ^= 1u;
+        for (int t = t0; t < t1; ++t) {
+          if (!mbar_wait(&kv_empty[st], ph ^ 1u, wait_ns)) { ok = false; break; }
+          uint8_t* base = smem + C::OFF_STAGE + st * C::STAGE_BYTES;
+          mbar_arrive_expect_tx(&kv_full[st], C::K_BYTES + C::CHUNKS_K * C::SLAB);
+          for (int c = 0; c < C::CHUNKS_K; ++c) {
+            tma_load_4d(base + c * C::SLAB, &mapK, &kv_full[st], c * 64, g, t * 128, b);
+            tma_load_4d(base + C::K_BYTES + c * C::SLAB, &mapV, &kv_full[st], c * 64, g, t * 128, b);
+          }
+          iss |= 1u << st; par = (par & ~(1u << st)) | (ph << st);
+          if (++st == C::STAGES) { st = 0; ph ^= 1u; }
+        }
+      }
+      for (int s = 0; s < 2; ++s)
+        if (qiss & (1u << s)) mbar_wait(&q_full[s], (qpar >> s) & 1u, wait_ns);
+      for (int s = 0; s < C::STAGES; ++s)
+        if (iss & (1u << s)) mbar_wait(&kv_full[s], (par >> s) & 1u, wait_ns);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      int st = 0, kq = 0;
+      uint32_t ph = 0, qph[2] = {0, 0}, pph[2] = {0, 0};
+      bool ok = true;
+      const uint32_t p_addr = smem_u32(smem + C::OFF_P);
+      for (int u = blockIdx.x; u < ds.units && ok; u += gridDim.x, ++kq) {
+        int b, g, split, t0, t1;
+        decode_unit(ds, u, b, g, split, t0, t1);
+        const int qb = kq & 1;
+        const uint32_t q_addr = smem_u32(smem + C::OFF_Q + qb * C::Q_BYTES);
+        if (!mbar_wait(&q_full[qb], qph[qb], wait_ns)) break;
+        qph[qb] ^= 1u;
+        tc_fence_after();
+        const int n = t1 - t0;
+        // S for tile i goes to buffer (i & 1); P.V of tile i follows its softmax.
+        int st_s = st;
+        uint32_t ph_s = ph;
+        auto issue_s = [&](int i) {
+          const uint32_t ka = smem_u32(smem + C::OFF_STAGE + st_s * C::STAGE_BYTES);
+#pragma unroll
+          for (int k = 0; k < HD / 16; ++k) {
+            const uint64_t a = sw128_desc(ka + (k >> 2) * C::SLAB + (k & 3) * 32, 1024, 16);
+            const uint64_t bq = sw128_desc(q_addr + (k >> 2) * C::Q_SLAB + (k & 3) * 32, 1024, 16);
+            tc_mma_f16_ss(tmem_base + (i & 1) * 16, a, bq, IDESC_S, k > 0);
+          }
+          tc_commit(&s_full[i & 1]);
+        };
+        // S(0)
+        if (!mbar_wait(&kv_full[st_s], ph_s, wait_ns)) break;
+        tc_fence_after();
+        issue_s(0);
+        for (int i = 0; i < n && ok; ++i) {
+          // S(i+1) as soon as its tile has landed
+          if (i + 1 < n) {
+            if (++st_s == C::STAGES) { st_s = 0; ph_s ^= 1u; }
+            if (!mbar_wait(&kv_full[st_s], ph_s, wait_ns)) { ok = false; break; }
+            tc_fence_after();
+            issue_s(i + 1);
+          }
+          // O^T += V^T P^T for tile i once its P is in shared memory
+          if (!mbar_wait(&p_full[i & 1], pph[i & 1], wait_ns)) { ok = false; break; }
+          pph[i & 1] ^= 1u;
+          tc_fence_after();
+          const uint32_t va = smem_u32(smem + C::OFF_STAGE + st * C::STAGE_BYTES + C::K_BYTES);
+          const uint32_t pa = p_addr + (i & 1) * C::P_BYTES;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint64_t a = sw128_desc(va + k * 2048, 1024, C::SLAB);
+            const uint64_t bp = sw128_desc(pa + (k >> 2) * C::Q_SLAB + (k & 3) * 32, 1024, 16);
+            tc_mma_f16_ss(tmem_base + 32, a, bp, IDESC_O, (i > 0 || k > 0) ? 1u : 0u);
+          }
+          tc_commit(&kv_empty[st]);
+          tc_commit(o_done);
+          if (++st == C::STAGES) { st = 0; ph ^= 1u; }
+        }
+        tc_commit(&q_empty[qb]);
+      }
+    }
+  } else if (warp >= 4) {
+    // ---------------------------------------------------------------- softmax + epilogue
+    const int w4 = warp - 4;
+    const int row = w4 * 32 + lane;                  // TMEM lane: key of the tile / dim of O^T
+    const uint32_t lane_off = (uint32_t)(w4 * 32) << 16;
+    uint32_t sph[2] = {0, 0}, oph = 0, rph[2] = {0, 0};
+    int rpar = 0;
+    // all four softmax warps meet here (bounded: a warp that gave up makes the
+    // others give up too instead of hanging)
+    auto exchange = [&]() -> bool {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&red_bar[rpar]);
+      const bool done = mbar_wait(&red_bar[rpar], rph[rpar], wait_ns);
+      rph[rpar] ^= 1u;
+      return done;
+    };
+    for (int u = blockIdx.x; u < ds.units; u += gridDim.x) {
+      int b, g, split, t0, t1;
+      decode_unit(ds, u, b, g, split, t0, t1);
+      const int n = t1 - t0;
+      float m_ref[NREP], l_part[NREP];
+#pragma unroll
+      for (int h = 0; h < NREP; ++h) { m_ref[h] = -INFINITY; l_part[h] = 0.f; }
+      bool ok = true;
+      for (int i = 0; i < n; ++i) {
+        const int sb = i & 1;
+        if (!mbar_wait(&s_full[sb], sph[sb], wait_ns)) { ok = false; break; }
+        sph[sb] ^= 1u;
+        tc_fence_after();
+        uint32_t r[16];
+        tmem_ld16(tmem_base + lane_off + sb * 16, r);
+        tc_wait_ld();
+        const int key = (t0 + i) * 128 + row;
+        const bool valid = key < ds.n_keys;
+        float s[NREP];
+#pragma unroll
+        for (int h = 0; h < NREP; ++h)
+          s[h] = (valid && h < nrep) ? __uint_as_float(r[h]) * ds.scale_log2 : -INFINITY;
+        // tile maximum per head over the 128 keys
+        float* rb = red + rpar * 64;
+#pragma unroll
+        for (int h = 0; h < NREP; ++h) {
+          const float mx = warp_max(s[h]);
+          if (lane == 0) rb[w4 * 16 + h] = mx;
+        }
+        if (!exchange()) { ok = false; break; }
+        rpar ^= 1;
+        bool grow = false;
+        float alpha[NREP];
+#pragma unroll
+        for (int h = 0; h < NREP; ++h) {
+          const float tm = fmaxf(fmaxf(rb[h], rb[16 + h]), fmaxf(rb[32 + h], rb[48 + h]));
+          alpha[h] = 1.f;
+          if (tm > m_ref[h] + 8.0f) {
+            alpha[h] = exp2f(m_ref[h] - tm);
+            m_ref[h] = tm;
+            l_part[h] *= alpha[h];
+            grow = true;
+          }
+        }
+        // the previous tile's P.V must be done before P is rewritten or O rescaled
+        if (i > 0) {
+          if (!mbar_wait(o_done, oph, wait_ns)) { ok = false; break; }
+          oph ^= 1u;
+          tc_fence_after();
+          if (grow) {   // uniform across the CTA (all threads hold the same maxima)
+            uint32_t o[16];
+            tmem_ld16(tmem_base + lane_off + 32, o);
+            tc_wait_ld();
+#pragma unroll
+            for (int h = 0; h < NREP; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
+            tmem_st16(tmem_base + lane_off + 32, o);
+            tc_wait_st();
+          }
+        }
+        // P^T[head][key] in bf16, 128-byte-swizzled K-major rows of 128 keys
+        uint8_t* pbuf = smem + C::OFF_P + sb * C::P_BYTES + (row >> 6) * C::Q_SLAB;
+        const int kin = row & 63;
+#pragma unroll
+        for (int h = 0; h < NREP; ++h) {
+          if (h >= nrep) break;
+          const float p = exp2f(s[h] - m_ref[h]);
+          l_part[h] += p;
+          *reinterpret_cast<bf16*>(pbuf + h * 128 + ((((kin >> 3) ^ (h & 7))) << 4) + (kin & 7) * 2) =
+              __float2bfloat16_rn(p);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&p_full[sb]);
+      }
+      if (!ok) break;
+      // epilogue: last P.V, then (m, l, acc) of this split
+      if (!mbar_wait(o_done, oph, wait_ns)) break;
+      oph ^= 1u;
+      tc_fence_after();
+      uint32_t o[16];
+      tmem_ld16(tmem_base + lane_off + 32, o);
+      tc_wait_ld();
+      tc_fence_before();
+      float* rb = red + rpar * 64;
+#pragma unroll
+      for (int h = 0; h < NREP; ++h) {
+        const float sum = warp_sum(l_part[h]);
+        if (lane == 0) rb[w4 * 16 + h] = sum;
+      }
+      if (!exchange()) break;
+      rpar ^= 1;
+#pragma unroll
+      for (int h = 0; h < NREP; ++h) {
+        if (h >= nrep) break;
+        float* rec = part + (((size_t)b * ds.H + g * nrep + h) * ds.splits + split) * (HD + 2);
+        if (row < HD) rec[2 + row] = __uint_as_float(o[h]);
+        if (row == 0) {
+          rec[0] = m_ref[h];
+          rec[1] = rb[h] + rb[16 + h] + rb[32 + h] + rb[48 + h];
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 64);
   }
 }
 

@@ -45,7 +45,7 @@ struct FlashCfg {
   static constexpr int Q_BYTES = CHUNKS * TILE_BYTES;
   static constexpr int KV_BYTES = CHUNKS * TILE_BYTES;
   static constexpr int P_BYTES = 2 * TILE_BYTES;    // 128 rows x 128 keys
-  static constexpr int KST = 2, VST = 1;
+  static constexpr int KST = 1, VST = 2;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
   static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
@@ -255,21 +255,22 @@ __global__ void __launch_bounds__(384, 1)
         sph ^= 1u;
         tc_fence_after();
         const bool need_mask = j * 128 + 127 > fs.P + qt * 128;
-        // pass 1: row maximum of the scaled scores
+        // pass 1: row maximum of the raw scores
         float mx = -INFINITY;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t r[32];
           tmem_ld32(s_tmem + c * 32, r);
           tc_wait_ld();
+          if (need_mask) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int key = j * 128 + c * 32 + i;
-            const float v = (need_mask && key > qpos) ? -INFINITY : __uint_as_float(r[i]);
-            mx = fmaxf(mx, v);
+            for (int i = 0; i < 32; ++i)
+              if (j * 128 + c * 32 + i > qpos) r[i] = __float_as_uint(-INFINITY);
           }
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) mx = max3f(mx, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
         }
-        const float m_tile = mx * fs.scale_log2;
+        const float m_tile = mx * fs.scale_log2;   // scale_log2 > 0: max commutes with the scale
         // the O written by the previous tile's P.V must be complete before P
         // (single buffer) is overwritten or O is rescaled
         if (j > 0) {
@@ -299,21 +300,25 @@ __global__ void __launch_bounds__(384, 1)
           tc_wait_st();
         }
         // pass 2: p = 2^(s*scale - m_ref), row sum, bf16 P into shared memory
-        float sum = 0.f;
+        const float scl = fs.scale_log2, neg_m = -m_ref;
+        float sum_a = 0.f, sum_b = 0.f;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t r[32];
           tmem_ld32(s_tmem + c * 32, r);
           tc_wait_ld();
+          if (need_mask) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (j * 128 + c * 32 + i > qpos) r[i] = __float_as_uint(-INFINITY);
+          }
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const int key = j * 128 + c * 32 + 2 * i;
-            const float s0 = (need_mask && key > qpos) ? -INFINITY : __uint_as_float(r[2 * i]);
-            const float s1 = (need_mask && key + 1 > qpos) ? -INFINITY : __uint_as_float(r[2 * i + 1]);
-            const float p0 = exp2f(fmaf(s0, fs.scale_log2, -m_ref));
-            const float p1 = exp2f(fmaf(s1, fs.scale_log2, -m_ref));
-            sum += p0 + p1;
+            float x0, x1;
+            fma2(x0, x1, __uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), scl, scl, neg_m, neg_m);
+            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+            add2(sum_a, sum_b, p0, p1);
             pk[i] = pack_bf16x2(p0, p1);
           }
           // chunk c covers keys 32c..32c+31: slab c/2, 16-byte pieces (c%2)*4 .. +3
@@ -325,6 +330,7 @@ __global__ void __launch_bounds__(384, 1)
                 make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
           }
         }
+        const float sum = sum_a + sum_b;
         l += sum;
         fence_proxy_async_smem();
         tc_fence_before();

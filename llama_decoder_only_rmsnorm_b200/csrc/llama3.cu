@@ -56,12 +56,21 @@ struct LaunchTimer {
   std::vector<cudaEvent_t> start, stop;
 } g_timer;
 
+// Inside a stream capture the record must become an external event node so
+// that every replay of the graph timestamps the event.
+void timer_record(cudaEvent_t ev, cudaStream_t st) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+    cudaEventRecordWithFlags(ev, st, cudaEventRecordExternal);
+  else
+    cudaEventRecord(ev, st);
+}
 void timer_begin(int kind, cudaStream_t st) {
-  if (g_timer.kind == kind && g_timer.used < g_timer.n) cudaEventRecord(g_timer.start[g_timer.used], st);
+  if (g_timer.kind == kind && g_timer.used < g_timer.n) timer_record(g_timer.start[g_timer.used], st);
 }
 void timer_end(int kind, cudaStream_t st) {
   g_launches.fetch_add(1, std::memory_order_relaxed);
-  if (g_timer.kind == kind && g_timer.used < g_timer.n) cudaEventRecord(g_timer.stop[g_timer.used++], st);
+  if (g_timer.kind == kind && g_timer.used < g_timer.n) timer_record(g_timer.stop[g_timer.used++], st);
 }
 // Launch `call` (a kernel<<<...>>>(...) expression) as family `kind` on `st`.
 #define L3_LAUNCH(kind, st, ...) \
@@ -371,10 +380,29 @@ int run_rmsnorm(const llama3_config* c, const void* x, long long row_stride, con
   L3_LAUNCH(LLAMA3_KERNEL_NORM, st, rmsnorm_kernel<T><<<rows, 256, 0, st>>>((const T*)x, row_stride, (const T*)w, (T*)y, c->dim, c->norm_eps));
   return launch_check();
 }
+template <int CPL>
+int run_rmsnorm_warp(const llama3_config* c, const void* x, long long row_stride, const void* w, void* y, int rows,
+                     cudaStream_t st) {
+  L3_LAUNCH(LLAMA3_KERNEL_NORM, st,
+            rmsnorm_bf16_warp_kernel<CPL><<<(rows + 3) / 4, 128, 0, st>>>(
+                (const bf16*)x, row_stride, (const bf16*)w, (bf16*)y, rows, c->dim, c->norm_eps));
+  return launch_check();
+}
+
 int rmsnorm_any(const llama3_config* c, const void* x, long long row_stride, const void* w, void* y, int rows,
                 cudaStream_t st) {
-  return c->dtype == LLAMA3_DTYPE_F32 ? run_rmsnorm<float>(c, x, row_stride, w, y, rows, st)
-                                      : run_rmsnorm<bf16>(c, x, row_stride, w, y, rows, st);
+  if (c->dtype == LLAMA3_DTYPE_F32) return run_rmsnorm<float>(c, x, row_stride, w, y, rows, st);
+  // bf16: the warp-per-row kernel when rows are 16-byte aligned and fit its registers
+  const int chunks = c->dim / 8;
+  if (c->dim % 8 == 0 && (row_stride * 2) % 16 == 0 && g_kernel_path == 0) {
+    if (chunks <= 32) return run_rmsnorm_warp<1>(c, x, row_stride, w, y, rows, st);
+    if (chunks <= 64) return run_rmsnorm_warp<2>(c, x, row_stride, w, y, rows, st);
+    if (chunks <= 128) return run_rmsnorm_warp<4>(c, x, row_stride, w, y, rows, st);
+    if (chunks <= 256) return run_rmsnorm_warp<8>(c, x, row_stride, w, y, rows, st);
+    if (chunks <= 512) return run_rmsnorm_warp<16>(c, x, row_stride, w, y, rows, st);
+    if (chunks <= 1024) return run_rmsnorm_warp<32>(c, x, row_stride, w, y, rows, st);
+  }
+  return run_rmsnorm<bf16>(c, x, row_stride, w, y, rows, st);
 }
 
 template <typename T>
@@ -388,51 +416,76 @@ int run_attention_simt(const llama3_config* c, const void* q, const void* kc, co
   return launch_check();
 }
 
-// Decode attention (one query per sequence), split over the key range.
+// Tensor-core decode attention: TMA-streamed K/V tiles, two tcgen05 MMAs per tile.
 template <int HD, int NREP>
-int run_decode_attention_t(const llama3_config* c, const void* q, const void* kc, const void* vc, int cap,
-                           int B, int n_keys, void* out, float* part, cudaStream_t st) {
+int run_decode_attention_tc_t(const llama3_config* c, const void* q, const void* kc, const void* vc, int cap,
+                              int B, int n_keys, void* out, float* part, cudaStream_t st) {
+  using Cfg = DecodeTcCfg<HD>;
   const int KV = c->n_kv_heads, H = c->n_heads;
+  const long long e = 2;
+  CUtensorMap mq, mk, mv;
+  L3_TRY(make_map(&mq, q, (long long)B * H, HD, 16));
+  L3_TRY(make_map_4d(&mk, kc, HD, KV, n_keys, B, HD * e, (long long)KV * HD * e, (long long)cap * KV * HD * e));
+  L3_TRY(make_map_4d(&mv, vc, HD, KV, n_keys, B, HD * e, (long long)KV * HD * e, (long long)cap * KV * HD * e));
+  DecodeShape ds;
+  ds.B = B; ds.H = H; ds.KV = KV; ds.nrep = H / KV; ds.n_keys = n_keys;
+  ds.tiles = (n_keys + 127) / 128;
+  // split count minimising the longest per-CTA stream on a persistent grid
   const int sms = num_sms();
-  // Enough CTAs for ~4 per SM, each with at least 128 keys.
-  int splits = std::max(1, std::min(kMaxKvSplits, (4 * sms + B * KV - 1) / (B * KV)));
-  splits = std::min(splits, std::max(1, n_keys / 128));
-  int kps = (n_keys + splits - 1) / splits;
-  splits = (n_keys + kps - 1) / kps;
-  const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)HD));
-  dim3 grid(splits, KV, B);
-  L3_LAUNCH(LLAMA3_KERNEL_DECODE_ATTENTION, st, decode_attention_split_kernel<HD, NREP><<<grid, 128, 0, st>>>(
-      (const bf16*)q, (const bf16*)kc, (const bf16*)vc, part, H, KV, cap, n_keys, kps, splits, scale_log2));
+  int best = 1;
+  long long best_t = -1;
+  for (int sp = 1; sp <= std::min(ds.tiles, kMaxKvSplits); ++sp) {
+    const int per = (ds.tiles + sp - 1) / sp;
+    const int real = (ds.tiles + per - 1) / per;
+    const long long units = (long long)B * KV * real;
+    const long long t = ((units + sms - 1) / sms) * per;
+    if (best_t < 0 || t < best_t) { best_t = t; best = real; }
+  }
+  ds.tiles_per_split = (ds.tiles + best - 1) / best;
+  ds.splits = (ds.tiles + ds.tiles_per_split - 1) / ds.tiles_per_split;
+  ds.units = B * KV * ds.splits;
+  ds.scale_log2 = (float)(1.4426950408889634 / sqrt((double)HD));
+  auto kern = decode_attention_tc_kernel<HD, NREP>;
+  int dev = 0;
+  L3_TRY(current_device(&dev));
+  static bool attr_done[kMaxDevices];
+  if (!attr_done[dev]) {
+    L3_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES));
+    attr_done[dev] = true;
+  }
+  const int grid = std::min(ds.units, sms);
+  L3_LAUNCH(LLAMA3_KERNEL_DECODE_ATTENTION, st,
+            kern<<<grid, 256, Cfg::SMEM_BYTES, st>>>(mq, mk, mv, part, ds, wait_ns()));
   L3_TRY(launch_check());
-  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, decode_attention_combine_kernel<HD><<<B * H, 128, 0, st>>>(part, (bf16*)out, splits));
+  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st,
+            decode_attention_combine_kernel<HD><<<B * H, 128, 0, st>>>(part, (bf16*)out, ds.splits));
   return launch_check();
 }
 
 template <int HD>
-int run_decode_attention_hd(const llama3_config* c, const void* q, const void* kc, const void* vc, int cap,
-                            int B, int n_keys, void* out, float* part, cudaStream_t st) {
-  switch (c->n_heads / c->n_kv_heads) {
-    case 1: return run_decode_attention_t<HD, 1>(c, q, kc, vc, cap, B, n_keys, out, part, st);
-    case 2: return run_decode_attention_t<HD, 2>(c, q, kc, vc, cap, B, n_keys, out, part, st);
-    case 4: return run_decode_attention_t<HD, 4>(c, q, kc, vc, cap, B, n_keys, out, part, st);
-    case 8: return run_decode_attention_t<HD, 8>(c, q, kc, vc, cap, B, n_keys, out, part, st);
-    default: return LLAMA3_ERR_UNSUPPORTED;
-  }
+int run_decode_attention_tc_hd(const llama3_config* c, const void* q, const void* kc, const void* vc, int cap,
+                               int B, int n_keys, void* out, float* part, cudaStream_t st) {
+  const int r = c->n_heads / c->n_kv_heads;
+  if (r <= 1) return run_decode_attention_tc_t<HD, 1>(c, q, kc, vc, cap, B, n_keys, out, part, st);
+  if (r <= 2) return run_decode_attention_tc_t<HD, 2>(c, q, kc, vc, cap, B, n_keys, out, part, st);
+  if (r <= 4) return run_decode_attention_tc_t<HD, 4>(c, q, kc, vc, cap, B, n_keys, out, part, st);
+  if (r <= 8) return run_decode_attention_tc_t<HD, 8>(c, q, kc, vc, cap, B, n_keys, out, part, st);
+  if (r <= 16) return run_decode_attention_tc_t<HD, 16>(c, q, kc, vc, cap, B, n_keys, out, part, st);
+  return LLAMA3_ERR_UNSUPPORTED;
 }
 
-bool decode_attention_supported(const llama3_config* c) {
-  const int r = c->n_heads / c->n_kv_heads;
+bool decode_attention_tc_supported(const llama3_config* c) {
   return use_tc(c) && (c->head_dim == 64 || c->head_dim == 96 || c->head_dim == 128) &&
-         (r == 1 || r == 2 || r == 4 || r == 8);
+         c->n_heads / c->n_kv_heads <= 16;
 }
 
 int attention_dispatch(const llama3_config* c, const void* q, const void* kc, const void* vc, int cap, int B,
                        int S, int P, void* out, float* part, cudaStream_t st) {
-  if (S == 1 && decode_attention_supported(c)) {
+  if (S == 1 && decode_attention_tc_supported(c)) {
     switch (c->head_dim) {
-      case 64: return run_decode_attention_hd<64>(c, q, kc, vc, cap, B, P + 1, out, part, st);
-      case 96: return run_decode_attention_hd<96>(c, q, kc, vc, cap, B, P + 1, out, part, st);
-      default: return run_decode_attention_hd<128>(c, q, kc, vc, cap, B, P + 1, out, part, st);
+      case 64: return run_decode_attention_tc_hd<64>(c, q, kc, vc, cap, B, P + 1, out, part, st);
+      case 96: return run_decode_attention_tc_hd<96>(c, q, kc, vc, cap, B, P + 1, out, part, st);
+      default: return run_decode_attention_tc_hd<128>(c, q, kc, vc, cap, B, P + 1, out, part, st);
     }
   }
   if (use_tc(c) && flash_attention_supported(c->head_dim, c->n_heads, c->n_kv_heads))
@@ -498,7 +551,7 @@ int layer_tc_prefill(const llama3_config* c, const llama3_layer_weights* w, cons
   L3_TRY(make_map(&mw2, w->w2, D, F, kPrefillBN));
 
   // attention half
-  L3_TRY(run_rmsnorm<bf16>(c, x, D, w->attention_norm, xn, M, st));
+  L3_TRY(rmsnorm_any(c, x, D, w->attention_norm, xn, M, st));
   {
     EpiParams ep = empty_epi();
     ep.seq = S; ep.start_pos = P; ep.n_heads = H; ep.n_kv = KV; ep.head_dim = hd; ep.cache_cap = cap;
@@ -514,7 +567,7 @@ int layer_tc_prefill(const llama3_config* c, const llama3_layer_weights* w, cons
     L3_TRY((launch_gemm<kPrefillBN, 4, EPI_RESIDUAL, false>(LLAMA3_KERNEL_GEMM_WO, mo, mo, mwo, mwo, sh, ep, st)));
   }
   // FFN half
-  L3_TRY(run_rmsnorm<bf16>(c, x, D, w->ffn_norm, xn, M, st));
+  L3_TRY(rmsnorm_any(c, x, D, w->ffn_norm, xn, M, st));
   {
     EpiParams ep = empty_epi();
     ep.out = g; ep.ldo = F;
@@ -546,7 +599,7 @@ int layer_tc_decode(const llama3_config* c, const llama3_layer_weights* w, const
   float* Ap = ws_at<float>(ws, L.attn_part);
   int splits = 1;
 
-  L3_TRY(run_rmsnorm<bf16>(c, x, D, w->attention_norm, xn, M, st));
+  L3_TRY(rmsnorm_any(c, x, D, w->attention_norm, xn, M, st));
   L3_TRY(swapped_partial_gemm(w->wqkv, nqkv, nullptr, 0, 0, xn, M, D, Pp, nqkv, &splits, st));
   L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, epi_qkv_rope_kernel<bf16><<<blocks_for((long long)M * nqkv / 2, 256), 256, 0, st>>>(
       Pp, splits, (long long)M * nqkv, M, 1, P, H, KV, hd, rope, q, (bf16*)kc, (bf16*)vc, cap));
@@ -556,7 +609,7 @@ int layer_tc_decode(const llama3_config* c, const llama3_layer_weights* w, const
   L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, epi_residual_kernel<bf16><<<blocks_for((long long)M * D, 256), 256, 0, st>>>(
       Pp, splits, (long long)M * D, D, (const bf16*)x, (bf16*)x, M, D));
   L3_TRY(launch_check());
-  L3_TRY(run_rmsnorm<bf16>(c, x, D, w->ffn_norm, xn, M, st));
+  L3_TRY(rmsnorm_any(c, x, D, w->ffn_norm, xn, M, st));
   L3_TRY(swapped_partial_gemm(w->w1, F, w->w3, F, F, xn, M, D, Pp, 2 * F, &splits, st));
   L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, epi_swiglu_kernel<bf16><<<blocks_for((long long)M * F, 256), 256, 0, st>>>(Pp, splits, (long long)M * 2 * F, g,
                                                                                 M, F));

@@ -48,6 +48,51 @@ __global__ void rmsnorm_kernel(const T* __restrict__ x, long long row_stride,
   for (int i = threadIdx.x; i < D; i += blockDim.x) yr[i] = from_f<T>(to_f(xr[i]) * r * to_f(w[i]));
 }
 
+// bf16 rows with D % 8 == 0 and D <= 8 * 32 * CPL: one warp per row, the row
+// held in registers as 16-byte chunks (one read of x, one write of y).
+template <int CPL>
+__global__ void __launch_bounds__(128) rmsnorm_bf16_warp_kernel(const bf16* __restrict__ x, long long row_stride,
+                                                               const bf16* __restrict__ w, bf16* __restrict__ y,
+                                                               int rows, int D, float eps) {
+  const int row = blockIdx.x * 4 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)row * row_stride);
+  const uint4* wr = reinterpret_cast<const uint4*>(w);
+  uint4* yr = reinterpret_cast<uint4*>(y + (size_t)row * D);
+  const int nchunk = D >> 3;
+  uint4 v[CPL];
+  float ss = 0.f;
+#pragma unroll
+  for (int j = 0; j < CPL; ++j) {
+    const int c = lane + 32 * j;
+    if (c < nchunk) {
+      v[j] = xr[c];
+      const uint32_t u[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float a = bf16lo(u[q]), b = bf16hi(u[q]);
+        ss = fmaf(a, a, fmaf(b, b, ss));
+      }
+    }
+  }
+  ss = warp_sum(ss);
+  const float r = rsqrtf(ss / (float)D + eps);
+#pragma unroll
+  for (int j = 0; j < CPL; ++j) {
+    const int c = lane + 32 * j;
+    if (c < nchunk) {
+      const uint4 wv = __ldg(wr + c);
+      const uint32_t u[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+      const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+      uint32_t o[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        o[q] = pack_bf16x2(bf16lo(u[q]) * r * bf16lo(ww[q]), bf16hi(u[q]) * r * bf16hi(ww[q]));
+      yr[c] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+}
+
 // ---- GEMM C[m, n] = sum_k A[m, k] * B[n, k]   (fp32 result) -----------------
 // 64x64 tile, 256 threads, 4x4 outputs per thread, K staged 16 at a time.
 template <typename T>
