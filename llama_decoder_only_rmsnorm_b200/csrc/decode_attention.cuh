@@ -36,13 +36,15 @@ __global__ void decode_attention_combine_kernel(const float* __restrict__ part, 
 }
 
 // ===========================================================================
-// Tensor-core variant: the same partial records, produced by TMA streaming
-// of K/V tiles and two tcgen05 MMAs per 128-key tile:
+// Tensor-core kernel.  K/V tiles of 128 keys arrive by TMA (3-stage ring of
+// 64 KB for head_dim 128); per tile two tcgen05 MMAs:
 //   S^T[key, head] = K_tile[128 x hd] . Q^T          (M = 128 keys, N = 16)
 //   O^T[dim, head] += V_tile^T[hd x 128] . P^T       (M = 128 dims, N = 16)
 // Keys sit on the MMA's 128-row side, so the n_rep query heads of a group
-// (padded to 16 columns) share every K/V byte read.  K/V tiles arrive through
-// a 3-stage ring of 64 KB; the CUDA cores only do the per-head softmax.
+// (padded to 16 columns) share every K/V byte read.  Two softmax warpgroups
+// take alternate tiles, each with its own running (m, l, O^T), so one tile's
+// softmax overlaps the next one's; a work unit therefore yields two partial
+// records (slot 2*split + warpgroup) that the combine kernel merges.
 // ===========================================================================
 struct DecodeShape {
   int B, H, KV, nrep, n_keys, tiles, splits, tiles_per_split, units;
@@ -61,12 +63,12 @@ struct DecodeTcCfg {
   static constexpr int Q_BYTES = CHUNKS_K * Q_SLAB;
   static constexpr int P_BYTES = 2 * Q_SLAB;        // 16 heads x 128 keys
   static constexpr int OFF_STAGE = 0;
-  static constexpr int OFF_Q = STAGES * STAGE_BYTES;
-  static constexpr int OFF_P = OFF_Q + 2 * Q_BYTES;
-  static constexpr int OFF_RED = OFF_P + 2 * P_BYTES;               // [2][4][16] floats
-  static constexpr int OFF_BAR = OFF_RED + 2 * 4 * 16 * 4;
-  static constexpr int N_BARS = 2 * STAGES + 4 /*q*/ + 2 /*s_full*/ + 2 /*p_full*/ + 1 /*o_done*/ +
-                                2 /*red*/;
+  static constexpr int OFF_Q = STAGES * STAGE_BYTES;              // 2 buffers
+  static constexpr int OFF_P = OFF_Q + 2 * Q_BYTES;               // [warpgroup][2] buffers
+  static constexpr int OFF_RED = OFF_P + 4 * P_BYTES;             // [warpgroup][2][4][16] floats
+  static constexpr int OFF_BAR = OFF_RED + 2 * 2 * 4 * 16 * 4;
+  // kv full/empty, q full/empty [2], per warpgroup: s_full[2], p_full[2], o_done, red[2]
+  static constexpr int N_BARS = 2 * STAGES + 4 + 2 * 7;
   static constexpr int SMEM_BYTES = 1024 + OFF_BAR + N_BARS * 8 + 16;
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
@@ -82,7 +84,7 @@ __device__ __forceinline__ void decode_unit(const DecodeShape& ds, int u, int& b
 }
 
 template <int HD, int NREP>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(384, 1)
     decode_attention_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
                                const __grid_constant__ CUtensorMap mapV, float* __restrict__ part,
                                const DecodeShape ds, const unsigned long long wait_ns) {
@@ -94,32 +96,35 @@ __global__ void __launch_bounds__(256, 1)
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* kv_full = bars;
   uint64_t* kv_empty = kv_full + C::STAGES;
   uint64_t* q_full = kv_empty + C::STAGES;   // [2]
   uint64_t* q_empty = q_full + 2;            // [2]
-  uint64_t* s_full = q_empty + 2;       // [2]
-  uint64_t* p_full = s_full + 2;        // [2]
-  uint64_t* o_done = p_full + 2;        // [1]
-  uint64_t* red_bar = o_done + 1;       // [2] cross-warp reductions of the softmax warps
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red_bar + 2);
+  uint64_t* wg_bars = q_empty + 2;           // [warpgroup][7]: s_full[2], p_full[2], o_done, red[2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(wg_bars + 14);
+  auto s_full = [&](int wg, int i) { return &wg_bars[wg * 7 + i]; };
+  auto p_full = [&](int wg, int i) { return &wg_bars[wg * 7 + 2 + i]; };
+  auto o_done = [&](int wg) { return &wg_bars[wg * 7 + 4]; };
+  auto red_bar = [&](int wg, int i) { return &wg_bars[wg * 7 + 5 + i]; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&q_full[s], 1); mbar_init(&q_empty[s], 1);
-      mbar_init(&s_full[s], 1); mbar_init(&p_full[s], 128);
+    for (int s = 0; s < 2; ++s) { mbar_init(&q_full[s], 1); mbar_init(&q_empty[s], 1); }
+    for (int wg = 0; wg < 2; ++wg) {
+      for (int s = 0; s < 2; ++s) {
+        mbar_init(s_full(wg, s), 1);
+        mbar_init(p_full(wg, s), 128);
+        mbar_init(red_bar(wg, s), 4);
+      }
+      mbar_init(o_done(wg), 1);
     }
-    mbar_init(o_done, 1);
-    mbar_init(&red_bar[0], 4); mbar_init(&red_bar[1], 4);
     fence_mbar_init();
   }
-  // P rows >= NREP stay zero for the whole kernel; dims >= hd of the V slabs
+  // P rows >= n_rep stay zero for the whole kernel; dims >= hd of the V slabs
   // that TMA never writes (head_dim 64) stay zero as well.
-  for (int i = threadIdx.x; i < 2 * C::P_BYTES / 16; i += blockDim.x)
+  for (int i = threadIdx.x; i < 4 * C::P_BYTES / 16; i += blockDim.x)
     reinterpret_cast<uint4*>(smem + C::OFF_P)[i] = make_uint4(0, 0, 0, 0);
   if (HD <= 64) {
     for (int s = 0; s < C::STAGES; ++s)
@@ -131,11 +136,12 @@ __global__ void __launch_bounds__(256, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&mapQ); prefetch_tensormap(&mapK); prefetch_tensormap(&mapV);
   }
-  if (warp == 1) tmem_alloc(tmem_slot, 64);
+  if (warp == 1) tmem_alloc(tmem_slot, 128);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;   // S buffers: cols [0,16) and [16,32); O: [32,48)
+  // TMEM columns: warpgroup w owns S buffers [64w, 64w+16), [64w+16, 64w+32) and O^T [64w+32, 64w+48)
+  const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
@@ -176,9 +182,9 @@ __global__ void __launch_bounds__(256, 1)
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       int st = 0, kq = 0;
-      uint32_t ph = 0, qph[2] = {0, 0}, pph[2] = {0, 0};
+      uint32_t ph = 0, qph[2] = {0, 0};
+      uint32_t pph[2][2] = {{0, 0}, {0, 0}};
       bool ok = true;
-      const uint32_t p_addr = smem_u32(smem + C::OFF_P);
       for (int u = blockIdx.x; u < ds.units && ok; u += gridDim.x, ++kq) {
         int b, g, split, t0, t1;
         decode_unit(ds, u, b, g, split, t0, t1);
@@ -188,63 +194,65 @@ __global__ void __launch_bounds__(256, 1)
         qph[qb] ^= 1u;
         tc_fence_after();
         const int n = t1 - t0;
-        // S for tile i goes to buffer (i & 1); P.V of tile i follows its softmax.
+        // tile i: warpgroup wg = i & 1, its (i >> 1)-th tile, S buffer (i >> 1) & 1
         int st_s = st;
         uint32_t ph_s = ph;
-        auto issue_s = [&](int i) {
+        auto issue_s = [&](int i) -> bool {
+          if (!mbar_wait(&kv_full[st_s], ph_s, wait_ns)) return false;
+          tc_fence_after();
           const uint32_t ka = smem_u32(smem + C::OFF_STAGE + st_s * C::STAGE_BYTES);
+          const int wg = i & 1, sb = (i >> 1) & 1;
 #pragma unroll
           for (int k = 0; k < HD / 16; ++k) {
             const uint64_t a = sw128_desc(ka + (k >> 2) * C::SLAB + (k & 3) * 32, 1024, 16);
             const uint64_t bq = sw128_desc(q_addr + (k >> 2) * C::Q_SLAB + (k & 3) * 32, 1024, 16);
-            tc_mma_f16_ss(tmem_base + (i & 1) * 16, a, bq, IDESC_S, k > 0);
+            tc_mma_f16_ss(tmem_base + wg * 64 + sb * 16, a, bq, IDESC_S, k > 0);
           }
-          tc_commit(&s_full[i & 1]);
+          tc_commit(s_full(wg, sb));
+          if (++st_s == C::STAGES) { st_s = 0; ph_s ^= 1u; }
+          return true;
         };
-        // S(0)
-        if (!mbar_wait(&kv_full[st_s], ph_s, wait_ns)) break;
-        tc_fence_after();
-        issue_s(0);
+        if (n > 0 && !issue_s(0)) break;
+        if (n > 1 && !issue_s(1)) break;
         for (int i = 0; i < n && ok; ++i) {
-          // S(i+1) as soon as its tile has landed
-          if (i + 1 < n) {
-            if (++st_s == C::STAGES) { st_s = 0; ph_s ^= 1u; }
-            if (!mbar_wait(&kv_full[st_s], ph_s, wait_ns)) { ok = false; break; }
-            tc_fence_after();
-            issue_s(i + 1);
-          }
-          // O^T += V^T P^T for tile i once its P is in shared memory
-          if (!mbar_wait(&p_full[i & 1], pph[i & 1], wait_ns)) { ok = false; break; }
-          pph[i & 1] ^= 1u;
+          const int wg = i & 1, sb = (i >> 1) & 1;
+          // O^T += V^T P^T for tile i once its warpgroup has written P
+          if (!mbar_wait(p_full(wg, sb), pph[wg][sb], wait_ns)) { ok = false; break; }
+          pph[wg][sb] ^= 1u;
           tc_fence_after();
           const uint32_t va = smem_u32(smem + C::OFF_STAGE + st * C::STAGE_BYTES + C::K_BYTES);
-          const uint32_t pa = p_addr + (i & 1) * C::P_BYTES;
+          const uint32_t pa = smem_u32(smem + C::OFF_P + (wg * 2 + sb) * C::P_BYTES);
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
             const uint64_t a = sw128_desc(va + k * 2048, 1024, C::SLAB);
             const uint64_t bp = sw128_desc(pa + (k >> 2) * C::Q_SLAB + (k & 3) * 32, 1024, 16);
-            tc_mma_f16_ss(tmem_base + 32, a, bp, IDESC_O, (i > 0 || k > 0) ? 1u : 0u);
+            tc_mma_f16_ss(tmem_base + wg * 64 + 32, a, bp, IDESC_O, (i > 1 || k > 0) ? 1u : 0u);
           }
           tc_commit(&kv_empty[st]);
-          tc_commit(o_done);
+          tc_commit(o_done(wg));
           if (++st == C::STAGES) { st = 0; ph ^= 1u; }
+          // S for tile i + 2 (same warpgroup, its other S buffer)
+          if (i + 2 < n && !issue_s(i + 2)) { ok = false; break; }
         }
         tc_commit(&q_empty[qb]);
       }
     }
   } else if (warp >= 4) {
     // ---------------------------------------------------------------- softmax + epilogue
-    const int w4 = warp - 4;
-    const int row = w4 * 32 + lane;                  // TMEM lane: key of the tile / dim of O^T
+    const int wg = (warp - 4) >> 2;                 // 0 or 1: takes tiles i with i % 2 == wg
+    const int w4 = warp & 3;                        // quarter of the TMEM lanes
+    const int row = w4 * 32 + lane;                 // TMEM lane: key of the tile / dim of O^T
     const uint32_t lane_off = (uint32_t)(w4 * 32) << 16;
+    const uint32_t wg_tmem = tmem_base + lane_off + wg * 64;
+    float* red = reinterpret_cast<float*>(smem + C::OFF_RED) + wg * 128;
     uint32_t sph[2] = {0, 0}, oph = 0, rph[2] = {0, 0};
     int rpar = 0;
-    // all four softmax warps meet here (bounded: a warp that gave up makes the
-    // others give up too instead of hanging)
+    // the four warps of this warpgroup meet here (bounded: a warp that gave up
+    // makes the others give up too instead of hanging)
     auto exchange = [&]() -> bool {
       __syncwarp();
-      if (lane == 0) mbar_arrive(&red_bar[rpar]);
-      const bool done = mbar_wait(&red_bar[rpar], rph[rpar], wait_ns);
+      if (lane == 0) mbar_arrive(red_bar(wg, rpar));
+      const bool done = mbar_wait(red_bar(wg, rpar), rph[rpar], wait_ns);
       rph[rpar] ^= 1u;
       return done;
     };
@@ -252,17 +260,18 @@ __global__ void __launch_bounds__(256, 1)
       int b, g, split, t0, t1;
       decode_unit(ds, u, b, g, split, t0, t1);
       const int n = t1 - t0;
+      const int mine = n > wg ? (n - wg + 1) / 2 : 0;   // tiles wg, wg+2, ...
       float m_ref[NREP], l_part[NREP];
 #pragma unroll
       for (int h = 0; h < NREP; ++h) { m_ref[h] = -INFINITY; l_part[h] = 0.f; }
       bool ok = true;
-      for (int i = 0; i < n; ++i) {
-        const int sb = i & 1;
-        if (!mbar_wait(&s_full[sb], sph[sb], wait_ns)) { ok = false; break; }
+      for (int k = 0; k < mine; ++k) {
+        const int i = wg + 2 * k, sb = k & 1;
+        if (!mbar_wait(s_full(wg, sb), sph[sb], wait_ns)) { ok = false; break; }
         sph[sb] ^= 1u;
         tc_fence_after();
         uint32_t r[16];
-        tmem_ld16(tmem_base + lane_off + sb * 16, r);
+        tmem_ld16(wg_tmem + sb * 16, r);
         tc_wait_ld();
         const int key = (t0 + i) * 128 + row;
         const bool valid = key < ds.n_keys;
@@ -292,45 +301,55 @@ __global__ void __launch_bounds__(256, 1)
             grow = true;
           }
         }
-        // the previous tile's P.V must be done before P is rewritten or O rescaled
-        if (i > 0) {
-          if (!mbar_wait(o_done, oph, wait_ns)) { ok = false; break; }
+        // this warpgroup's previous P.V must be done before P is rewritten or O rescaled
+        if (k > 0) {
+          if (!mbar_wait(o_done(wg), oph, wait_ns)) { ok = false; break; }
           oph ^= 1u;
           tc_fence_after();
-          if (grow) {   // uniform across the CTA (all threads hold the same maxima)
+          if (grow) {   // uniform across the warpgroup (all threads hold the same maxima)
             uint32_t o[16];
-            tmem_ld16(tmem_base + lane_off + 32, o);
+            tmem_ld16(wg_tmem + 32, o);
             tc_wait_ld();
 #pragma unroll
             for (int h = 0; h < NREP; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
-            tmem_st16(tmem_base + lane_off + 32, o);
+            tmem_st16(wg_tmem + 32, o);
             tc_wait_st();
           }
         }
-        // P^T[head][key] in bf16, 128-byte-swizzled K-major rows of 128 keys
-        uint8_t* pbuf = smem + C::OFF_P + sb * C::P_BYTES + (row >> 6) * C::Q_SLAB;
+        // P^T[head][key] in bf16, 128-byte-swizzled K-major rows of 128 keys;
+        // even lanes store the (key, key+1) pair as one 32-bit word
+        uint8_t* pbuf = smem + C::OFF_P + (wg * 2 + sb) * C::P_BYTES + (row >> 6) * C::Q_SLAB;
         const int kin = row & 63;
 #pragma unroll
         for (int h = 0; h < NREP; ++h) {
-          if (h >= nrep) break;
-          const float p = exp2f(s[h] - m_ref[h]);
+          const float p = (h < nrep) ? exp2f(s[h] - m_ref[h]) : 0.f;
           l_part[h] += p;
-          *reinterpret_cast<bf16*>(pbuf + h * 128 + ((((kin >> 3) ^ (h & 7))) << 4) + (kin & 7) * 2) =
-              __float2bfloat16_rn(p);
+          const float p_next = __shfl_down_sync(0xffffffffu, p, 1);
+          if ((lane & 1) == 0 && h < nrep)
+            *reinterpret_cast<uint32_t*>(pbuf + h * 128 + ((((kin >> 3) ^ (h & 7))) << 4) + (kin & 7) * 2) =
+                pack_bf16x2(p, p_next);
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(&p_full[sb]);
+        mbar_arrive(p_full(wg, sb));
       }
       if (!ok) break;
-      // epilogue: last P.V, then (m, l, acc) of this split
-      if (!mbar_wait(o_done, oph, wait_ns)) break;
-      oph ^= 1u;
-      tc_fence_after();
-      uint32_t o[16];
-      tmem_ld16(tmem_base + lane_off + 32, o);
-      tc_wait_ld();
-      tc_fence_before();
+      // epilogue: last P.V of this warpgroup, then its (m, l, acc) record
+      float o_val[NREP];
+      if (mine > 0) {
+        if (!mbar_wait(o_done(wg), oph, wait_ns)) break;
+        oph ^= 1u;
+        tc_fence_after();
+        uint32_t o[16];
+        tmem_ld16(wg_tmem + 32, o);
+        tc_wait_ld();
+        tc_fence_before();
+#pragma unroll
+        for (int h = 0; h < NREP; ++h) o_val[h] = __uint_as_float(o[h]);
+      } else {
+#pragma unroll
+        for (int h = 0; h < NREP; ++h) o_val[h] = 0.f;
+      }
       float* rb = red + rpar * 64;
 #pragma unroll
       for (int h = 0; h < NREP; ++h) {
@@ -339,11 +358,12 @@ __global__ void __launch_bounds__(256, 1)
       }
       if (!exchange()) break;
       rpar ^= 1;
+      const int slot = 2 * split + wg;
 #pragma unroll
       for (int h = 0; h < NREP; ++h) {
         if (h >= nrep) break;
-        float* rec = part + (((size_t)b * ds.H + g * nrep + h) * ds.splits + split) * (HD + 2);
-        if (row < HD) rec[2 + row] = __uint_as_float(o[h]);
+        float* rec = part + (((size_t)b * ds.H + g * nrep + h) * (2 * ds.splits) + slot) * (HD + 2);
+        if (row < HD) rec[2 + row] = o_val[h];
         if (row == 0) {
           rec[0] = m_ref[h];
           rec[1] = rb[h] + rb[16 + h] + rb[32 + h] + rb[48 + h];
@@ -356,7 +376,7 @@ __global__ void __launch_bounds__(256, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, 64);
+    tmem_dealloc(tmem_base, 128);
   }
 }
 

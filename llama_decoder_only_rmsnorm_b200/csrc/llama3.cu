@@ -290,6 +290,10 @@ GemmShape make_shape(int rows_a, int rows_a2, int rows_b, int k, int bn, int spl
   s.kb_per_split = (s.kblocks + splits - 1) / splits;
   s.splits = (s.kblocks + s.kb_per_split - 1) / s.kb_per_split;
   s.units = s.splits * s.tiles_m * s.tiles_n;
+  // Groups of 16 m-tiles: with a 148-CTA persistent grid the tiles in flight
+  // span 16 A row-blocks x ~9 B column-blocks.  The swapped (weight-streaming)
+  // launches have one n-tile, where grouping changes nothing.
+  s.group_m = std::max(1, std::min(16, s.tiles_m));
   return s;
 }
 
@@ -434,7 +438,7 @@ int run_decode_attention_tc_t(const llama3_config* c, const void* q, const void*
   const int sms = num_sms();
   int best = 1;
   long long best_t = -1;
-  for (int sp = 1; sp <= std::min(ds.tiles, kMaxKvSplits); ++sp) {
+  for (int sp = 1; sp <= std::min(ds.tiles, kMaxKvSplits / 2); ++sp) {
     const int per = (ds.tiles + sp - 1) / sp;
     const int real = (ds.tiles + per - 1) / per;
     const long long units = (long long)B * KV * real;
@@ -455,10 +459,10 @@ int run_decode_attention_tc_t(const llama3_config* c, const void* q, const void*
   }
   const int grid = std::min(ds.units, sms);
   L3_LAUNCH(LLAMA3_KERNEL_DECODE_ATTENTION, st,
-            kern<<<grid, 256, Cfg::SMEM_BYTES, st>>>(mq, mk, mv, part, ds, wait_ns()));
+            kern<<<grid, 384, Cfg::SMEM_BYTES, st>>>(mq, mk, mv, part, ds, wait_ns()));
   L3_TRY(launch_check());
   L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st,
-            decode_attention_combine_kernel<HD><<<B * H, 128, 0, st>>>(part, (bf16*)out, ds.splits));
+            decode_attention_combine_kernel<HD><<<B * H, 128, 0, st>>>(part, (bf16*)out, 2 * ds.splits));
   return launch_check();
 }
 

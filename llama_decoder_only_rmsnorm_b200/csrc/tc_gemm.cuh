@@ -14,8 +14,8 @@
 // The accumulator is double-buffered in TMEM so the epilogue of one tile
 // overlaps the main loop of the next.
 //
-// Work unit = (split, m-tile, n-tile); m varies fastest so CTAs running at the
-// same time share the same B tile (the weights in the prefill layout).
+// Work unit = (split, m-tile, n-tile), visited in groups of m-tiles (see
+// gemm_unit) so that the tiles in flight share their operands through L2.
 //
 // "A" may consist of two tensors stacked along rows (tiles of the second one
 // come after those of the first; their output rows are offset by
@@ -48,7 +48,25 @@ struct GemmShape {
   int kb_per_split;
   int splits;
   int units;           // splits * tiles_m * tiles_n
+  int group_m;         // raster: m-tiles per group (tiles of a group share A rows and B columns)
 };
+
+// Work unit -> (split, m-tile, n-tile).  Within a split, tiles are visited in
+// groups of `group_m` m-tiles: n varies across the group, m fastest inside it,
+// so the CTAs running at the same time touch group_m A row-blocks and a few B
+// column-blocks, which stay in L2.
+__device__ __forceinline__ void gemm_unit(const GemmShape& sh, int u, int& split, int& mt, int& nt) {
+  const int per_split = sh.tiles_m * sh.tiles_n;
+  split = u / per_split;
+  const int r = u % per_split;
+  const int per_group = sh.group_m * sh.tiles_n;
+  const int group = r / per_group;
+  const int first_m = group * sh.group_m;
+  const int gm = min(sh.group_m, sh.tiles_m - first_m);
+  const int q = r % per_group;
+  mt = first_m + q % gm;
+  nt = q / gm;
+}
 
 struct EpiParams {
   void* out;           // STORE/RESIDUAL/SWIGLU: bf16 [rows_a, ldo]; PARTIAL: float
@@ -262,8 +280,6 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int per_split = sh.tiles_m * sh.tiles_n;
-
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -272,8 +288,8 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t issued_mask = 0, issued_parity = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < sh.units && ok; u += gridDim.x) {
-        const int split = u / per_split, rem = u % per_split;
-        const int mt = rem % sh.tiles_m, nt = rem / sh.tiles_m;
+        int split, mt, nt;
+        gemm_unit(sh, u, split, mt, nt);
         const bool second = mt >= sh.tiles_m1;
         const CUtensorMap* ma = second ? &mapA2 : &mapA;
         const int arow = (second ? mt - sh.tiles_m1 : mt) * C::BM;
@@ -304,7 +320,8 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t last_parity = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < sh.units && ok; u += gridDim.x) {
-        const int split = u / per_split;
+        int split, mt_unused, nt_unused;
+        gemm_unit(sh, u, split, mt_unused, nt_unused);
         const int kb0 = split * sh.kb_per_split;
         const int kb1 = min(kb0 + sh.kb_per_split, sh.kblocks);
         if (!mbar_wait(&acc_empty[abuf], aphase ^ 1u, wait_ns)) break;
@@ -345,8 +362,8 @@ __global__ void __launch_bounds__(192, 1)
     int abuf = 0;
     uint32_t aphase = 0;
     for (int u = blockIdx.x; u < sh.units; u += gridDim.x) {
-      const int split = u / per_split, rem = u % per_split;
-      const int mt = rem % sh.tiles_m, nt = rem / sh.tiles_m;
+      int split, mt, nt;
+      gemm_unit(sh, u, split, mt, nt);
       const bool second = mt >= sh.tiles_m1;
       const int local_row = (second ? mt - sh.tiles_m1 : mt) * C::BM + row_in_tile;
       const bool arow_ok = local_row < (second ? sh.rows_a2 : sh.rows_a);
