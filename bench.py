@@ -51,6 +51,8 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--layers", type=int, default=None, help=argparse.SUPPRESS)  # profiling captures only
+    p.add_argument("--no-pdl", action="store_true", help=argparse.SUPPRESS)   # A/B of programmatic launch
+    p.add_argument("--kernel-path", type=int, default=0, help=argparse.SUPPRESS)  # A/B of GEMM variants
     return p.parse_args()
 
 
@@ -282,6 +284,9 @@ def oracle_sample(layers, outw, caches, prefix, decode_seq=True):
 def run_ours(args):
     world, rank, local = dist_setup()
     dev = f"cuda:{local}"
+    if args.no_pdl:
+        B.llama3_set_programmatic_launch(False)
+    B.llama3_set_kernel_path(args.kernel_path)
     peaks, peak_kind = load_peaks()
     layers, outw = build(dev)
     n_layers = args.layers or PREFILL.n_layers

@@ -65,7 +65,8 @@ enum llama3_status {
  * [S2] §1.2.  Constraints checked by every call:
  *   dim == n_heads * head_dim; n_heads % n_kv_heads == 0; head_dim even and
  *   in {16, 32, 64, 96, 128} (bf16 needs head_dim >= 64); ffn_hidden >= 1;
- *   norm_eps > 0; rope_theta > 1; for bf16, dim and ffn_hidden multiples of 8.
+ *   norm_eps > 0; rope_theta > 1; dim and ffn_hidden multiples of 8 for bf16,
+ *   of 4 for fp32.
  * ffn_hidden is taken as given (the caller applies the hidden-size rule of
  * [S2] §3.5 if it wants it).  vocab is only needed by the LM head / embedding.
  */
@@ -211,7 +212,8 @@ int llama3_rmsnorm(const llama3_config* cfg, const void* x, long long row_stride
 
 /* y[m, n] = sum_k x[m, k] * w[n, k] (+ residual[m, n] when residual != NULL);
  * x: [m, k], w: [n, k], y/residual: [m, n] (residual may equal y).  k and n
- * multiples of 8 for bf16.  Uses the same GEMM kernels as the layer calls. */
+ * multiples of 8 for bf16, n a multiple of 4 for fp32.  Uses the same GEMM
+ * kernels as the layer calls. */
 int llama3_linear(const llama3_config* cfg, const void* x, const void* w, const void* residual,
                   void* y, int m, int n, int k, void* ws, size_t ws_bytes,
                   llama3_stream_t stream);
@@ -265,12 +267,20 @@ int llama3_device_status(int* out);
 /* cudaError_t of the last call that returned LLAMA3_ERR_CUDA (0 if none). */
 int llama3_last_cuda_error(void);
 
-/* Kernel selection for diagnosis: 0 (default) = tcgen05/TMA kernels for bf16,
- * 1 = the plain SIMT kernels for every dtype.  Returns the previous value. */
+/* Kernel selection: 0 (default) = tcgen05/TMA kernels for bf16, 1 = the plain
+ * SIMT kernels for every dtype, 2 = as 0 but the prefill GEMMs (m >= 256) run
+ * on CTA pairs (tcgen05 cta_group::2, 256-row tiles).  Returns the previous
+ * value. */
 int llama3_set_kernel_path(int path);
 
 /* Limit, in milliseconds, of every bounded device-side wait (default 2000). */
 int llama3_set_wait_limit_ms(int ms);
+
+/* 1 (default): kernels are launched with programmatic stream serialization,
+ * so a kernel's launch and set-up overlap the end of the previous kernel in
+ * the stream (each kernel waits for its predecessor before touching memory);
+ * 0: ordinary launches.  Returns the previous value. */
+int llama3_set_programmatic_launch(int on);
 
 #ifdef __cplusplus
 }

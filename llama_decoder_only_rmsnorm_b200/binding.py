@@ -61,6 +61,7 @@ _SIGNATURES = {
     "llama3_last_cuda_error": [],
     "llama3_set_kernel_path": [_i],
     "llama3_set_wait_limit_ms": [_i],
+    "llama3_set_programmatic_launch": [_i],
     "llama3_set_launch_timer": [_i, _p, _p, _i],
     "llama3_launch_timer_used": [],
     "llama3_launch_count": [],
@@ -214,6 +215,10 @@ def llama3_set_kernel_path(path):
 
 def llama3_set_wait_limit_ms(ms):
     return lib().llama3_set_wait_limit_ms(ms)
+
+
+def llama3_set_programmatic_launch(on):
+    return lib().llama3_set_programmatic_launch(1 if on else 0)
 
 
 KERNEL_KINDS = {"gemm_qkv": 1, "gemm_wo": 2, "gemm_w13": 3, "gemm_w2": 4, "attention": 5, "decode_gemm": 6,

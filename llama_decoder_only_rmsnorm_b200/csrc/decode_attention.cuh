@@ -19,6 +19,7 @@ namespace l3 {
 template <int HD>
 __global__ void decode_attention_combine_kernel(const float* __restrict__ part, bf16* __restrict__ out,
                                                 int splits) {
+  griddep_wait_and_release();
   const int bh = blockIdx.x;  // b * H + h
   const float* p = part + (size_t)bh * splits * (HD + 2);
   float mx = -INFINITY;
@@ -142,6 +143,7 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_after();
   // TMEM columns: warpgroup w owns S buffers [64w, 64w+16), [64w+16, 64w+32) and O^T [64w+32, 64w+48)
   const uint32_t tmem_base = *tmem_slot;
+  griddep_wait_and_release();
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer

@@ -113,6 +113,7 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  griddep_wait_and_release();
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
@@ -313,13 +314,29 @@ __global__ void __launch_bounds__(384, 1)
               if (j * 128 + c * 32 + i > qpos) r[i] = __float_as_uint(-INFINITY);
           }
           uint32_t pk[16];
+          if (need_mask) {   // masked keys must give exactly 0: MUFU path only
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float x0, x1;
-            fma2(x0, x1, __uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), scl, scl, neg_m, neg_m);
-            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-            add2(sum_a, sum_b, p0, p1);
-            pk[i] = pack_bf16x2(p0, p1);
+            for (int i = 0; i < 16; ++i) {
+              float x0, x1;
+              fma2(x0, x1, __uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), scl, scl, neg_m, neg_m);
+              const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+              add2(sum_a, sum_b, p0, p1);
+              pk[i] = pack_bf16x2(p0, p1);
+            }
+          } else {           // 6 of every 16 pairs on the FMA pipe, the rest on MUFU
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              float x0, x1, p0, p1;
+              fma2(x0, x1, __uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), scl, scl, neg_m, neg_m);
+              if ((i & 7) < 3) {
+                exp2_poly2(x0, x1, p0, p1);
+              } else {
+                p0 = ex2_approx(x0);
+                p1 = ex2_approx(x1);
+              }
+              add2(sum_a, sum_b, p0, p1);
+              pk[i] = pack_bf16x2(p0, p1);
+            }
           }
           // chunk c covers keys 32c..32c+31: slab c/2, 16-byte pieces (c%2)*4 .. +3
           uint8_t* slab = p_smem + (c >> 1) * C::TILE_BYTES + row * 128;

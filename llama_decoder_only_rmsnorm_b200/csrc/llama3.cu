@@ -18,13 +18,15 @@
 #include "flash_attention.cuh"
 #include "simt.cuh"
 #include "tc_gemm.cuh"
+#include "tc_gemm_pair.cuh"
 
 using namespace l3;
 
 namespace {
 
 thread_local int t_last_cuda = 0;
-int g_kernel_path = 0;       // 0 = tcgen05 for bf16, 1 = SIMT everywhere
+int g_kernel_path = 0;       // 0 = tcgen05 for bf16, 1 = SIMT everywhere,
+                             // 2 = tcgen05 with CTA-pair prefill GEMMs
 int g_wait_ms = 2000;        // bounded device waits
 constexpr int kMaxDevices = 64;
 int g_num_sms[kMaxDevices];
@@ -72,13 +74,36 @@ void timer_end(int kind, cudaStream_t st) {
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (g_timer.kind == kind && g_timer.used < g_timer.n) timer_record(g_timer.stop[g_timer.used++], st);
 }
-// Launch `call` (a kernel<<<...>>>(...) expression) as family `kind` on `st`.
-#define L3_LAUNCH(kind, st, ...) \
-  do {                             \
-    timer_begin((kind), (st));     \
-    __VA_ARGS__;                   \
-    timer_end((kind), (st));       \
+// Launch `call` (a launch_k(...) expression) as family `kind` on `st`.
+#define L3_LAUNCH(kind, st, ...)                        \
+  do {                                                  \
+    timer_begin((kind), (st));                          \
+    const cudaError_t le_ = (__VA_ARGS__);              \
+    timer_end((kind), (st));                            \
+    if (le_ != cudaSuccess) return cuda_fail(le_);      \
   } while (0)
+
+// Every kernel is launched with programmatic stream serialization: it may be
+// scheduled while its predecessor in the stream finishes, and it waits for
+// that predecessor (griddepcontrol.wait) after its own set-up and before it
+// touches memory.  g_pdl = false launches them the ordinary way.
+bool g_pdl = true;
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                     Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = g_pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
 
 int current_device(int* dev) {
   cudaError_t e = cudaGetDevice(dev);
@@ -104,7 +129,8 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 size_t esize(const llama3_config* c) { return c->dtype == LLAMA3_DTYPE_F32 ? 4 : 2; }
 
-bool use_tc(const llama3_config* c) { return c->dtype == LLAMA3_DTYPE_BF16 && g_kernel_path == 0; }
+bool use_tc(const llama3_config* c) { return c->dtype == LLAMA3_DTYPE_BF16 && g_kernel_path != 1; }
+bool use_pair_gemm(int m) { return g_kernel_path == 2 && m >= 256; }
 
 int check_config(const llama3_config* c) {
   if (!c) return LLAMA3_ERR_ARG;
@@ -119,6 +145,8 @@ int check_config(const llama3_config* c) {
   if (c->dtype == LLAMA3_DTYPE_BF16) {
     if (hd < 64) return LLAMA3_ERR_ARG;
     if (c->dim % 8 || c->ffn_hidden % 8) return LLAMA3_ERR_ARG;
+  } else if (c->dim % 4 || c->ffn_hidden % 4) {
+    return LLAMA3_ERR_ARG;
   }
   return LLAMA3_OK;
 }
@@ -217,7 +245,7 @@ int run_flash_attention_t(int H, int KV, const void* q, const void* kc, const vo
     attr_done[dev] = true;
   }
   const int grid = std::min(fs.units, sms);
-  L3_LAUNCH(LLAMA3_KERNEL_ATTENTION, st, kern<<<grid, 384, Cfg::SMEM_BYTES, st>>>(mq, mk, mv, (bf16*)out, fs, wns));
+  L3_LAUNCH(LLAMA3_KERNEL_ATTENTION, st, launch_k(kern, grid, 384, Cfg::SMEM_BYTES, st, mq, mk, mv, (bf16*)out, fs, wns));
   return launch_check();
 }
 
@@ -326,7 +354,49 @@ int launch_gemm(int kind, const CUtensorMap& a, const CUtensorMap& a2, const CUt
   }
   if (sh.units <= 0) return LLAMA3_OK;
   const int grid = std::min(sh.units, num_sms());
-  L3_LAUNCH(kind, st, kern<<<grid, 192, Cfg::SMEM_BYTES, st>>>(a, a2, b, b2, sh, ep, wait_ns()));
+  L3_LAUNCH(kind, st, launch_k(kern, grid, 192, Cfg::SMEM_BYTES, st, a, a2, b, b2, sh, ep, wait_ns()));
+  return launch_check();
+}
+
+// Prefill GEMM tile shape for CTA pairs: 256-row tiles of A.
+GemmShape make_shape_pair(int rows_a, int rows_b, int k, int bn) {
+  GemmShape s = make_shape(rows_a, 0, rows_b, k, bn, 1);
+  s.tiles_m1 = s.tiles_m = (rows_a + 255) / 256;
+  s.units = s.tiles_m * s.tiles_n;
+  s.group_m = std::max(1, std::min(8, s.tiles_m));
+  return s;
+}
+
+template <int BN, int STAGES, int EPI, bool DUAL>
+int launch_gemm_pair(int kind, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2,
+                     const GemmShape& sh, const EpiParams& ep, cudaStream_t st) {
+  using Cfg = TcGemmPairCfg<BN, STAGES, DUAL>;
+  auto kern = tc_gemm_pair_kernel<BN, STAGES, EPI, DUAL>;
+  int dev = 0;
+  L3_TRY(current_device(&dev));
+  static bool attr_done[kMaxDevices];
+  if (!attr_done[dev]) {
+    L3_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES));
+    attr_done[dev] = true;
+  }
+  if (sh.units <= 0) return LLAMA3_OK;
+  const int pairs = std::min(sh.units, std::max(1, num_sms() / 2));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs);
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = g_pdl ? 2 : 1;
+  const unsigned long long wns = wait_ns();
+  L3_LAUNCH(kind, st, cudaLaunchKernelEx(&cfg, kern, a, b, b2, sh, ep, wns));
   return launch_check();
 }
 
@@ -372,7 +442,7 @@ constexpr int kPrefillBN = 256;
 template <typename T>
 int simt_gemm(int kind, const void* A, const void* B, float* C, int M, int N, int K, int ldc, cudaStream_t st) {
   dim3 grid((N + 63) / 64, (M + 63) / 64);
-  L3_LAUNCH(kind, st, gemm_simt_kernel<T><<<grid, 256, 0, st>>>((const T*)A, (const T*)B, C, M, N, K, ldc));
+  L3_LAUNCH(kind, st, launch_k((gemm_simt_kernel<T>), grid, 256, 0, st, (const T*)A, (const T*)B, C, M, N, K, ldc));
   return launch_check();
 }
 
@@ -381,15 +451,15 @@ unsigned blocks_for(long long n, int threads) { return (unsigned)((n + threads -
 template <typename T>
 int run_rmsnorm(const llama3_config* c, const void* x, long long row_stride, const void* w, void* y, int rows,
                 cudaStream_t st) {
-  L3_LAUNCH(LLAMA3_KERNEL_NORM, st, rmsnorm_kernel<T><<<rows, 256, 0, st>>>((const T*)x, row_stride, (const T*)w, (T*)y, c->dim, c->norm_eps));
+  L3_LAUNCH(LLAMA3_KERNEL_NORM, st, launch_k((rmsnorm_kernel<T>), rows, 256, 0, st, (const T*)x, row_stride, (const T*)w, (T*)y, c->dim, c->norm_eps));
   return launch_check();
 }
 template <int CPL>
 int run_rmsnorm_warp(const llama3_config* c, const void* x, long long row_stride, const void* w, void* y, int rows,
                      cudaStream_t st) {
   L3_LAUNCH(LLAMA3_KERNEL_NORM, st,
-            rmsnorm_bf16_warp_kernel<CPL><<<(rows + 3) / 4, 128, 0, st>>>(
-                (const bf16*)x, row_stride, (const bf16*)w, (bf16*)y, rows, c->dim, c->norm_eps));
+            launch_k((rmsnorm_bf16_warp_kernel<CPL>), (rows + 3) / 4, 128, 0, st, (const bf16*)x, row_stride,
+                     (const bf16*)w, (bf16*)y, rows, c->dim, c->norm_eps));
   return launch_check();
 }
 
@@ -414,7 +484,7 @@ int run_attention_simt(const llama3_config* c, const void* q, const void* kc, co
                        int S, int P, void* out, cudaStream_t st) {
   const long long warps = (long long)B * S * c->n_heads;
   const float scale = (float)(1.0 / sqrt((double)c->head_dim));
-  L3_LAUNCH(LLAMA3_KERNEL_ATTENTION, st, attention_simt_kernel<T><<<blocks_for(warps * 32, 256), 256, 0, st>>>(
+  L3_LAUNCH(LLAMA3_KERNEL_ATTENTION, st, launch_k((attention_simt_kernel<T>), blocks_for(warps * 32, 256), 256, 0, st, 
       (const T*)q, (const T*)kc, (const T*)vc, (T*)out, B, S, P, c->n_heads, c->n_kv_heads, c->head_dim, cap,
       scale));
   return launch_check();
@@ -459,10 +529,10 @@ int run_decode_attention_tc_t(const llama3_config* c, const void* q, const void*
   }
   const int grid = std::min(ds.units, sms);
   L3_LAUNCH(LLAMA3_KERNEL_DECODE_ATTENTION, st,
-            kern<<<grid, 384, Cfg::SMEM_BYTES, st>>>(mq, mk, mv, part, ds, wait_ns()));
+            launch_k(kern, grid, 384, Cfg::SMEM_BYTES, st, mq, mk, mv, part, ds, wait_ns()));
   L3_TRY(launch_check());
   L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st,
-            decode_attention_combine_kernel<HD><<<B * H, 128, 0, st>>>(part, (bf16*)out, 2 * ds.splits));
+            launch_k((decode_attention_combine_kernel<HD>), B * H, 128, 0, st, part, (bf16*)out, 2 * ds.splits));
   return launch_check();
 }
 
@@ -515,20 +585,20 @@ int layer_simt(const llama3_config* c, const llama3_layer_weights* w, const floa
   float* Ap = ws_at<float>(ws, L.attn_part);
   L3_TRY(run_rmsnorm<T>(c, x, D, w->attention_norm, xn, M, st));
   L3_TRY(simt_gemm<T>(LLAMA3_KERNEL_GEMM_QKV, xn, w->wqkv, Pp, M, nqkv, D, nqkv, st));
-  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, epi_qkv_rope_kernel<T><<<blocks_for((long long)M * nqkv / 2, 256), 256, 0, st>>>(
+  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_qkv_rope_kernel<T>), blocks_for((long long)M * nqkv / 4, 256), 256, 0, st, 
       Pp, 1, 0, M, S, P, H, KV, hd, rope, q, (T*)kc, (T*)vc, cap));
   L3_TRY(launch_check());
   L3_TRY(attention_dispatch(c, q, kc, vc, cap, B, S, P, o, Ap, st));
   L3_TRY(simt_gemm<T>(LLAMA3_KERNEL_GEMM_WO, o, w->wo, Pp, M, D, H * hd, D, st));
-  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, epi_residual_kernel<T><<<blocks_for((long long)M * D, 256), 256, 0, st>>>(Pp, 1, 0, D, (const T*)x, (T*)x, M, D));
+  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_residual_kernel<T>), blocks_for((long long)M * D / 4, 256), 256, 0, st, Pp, 1, 0, D, (const T*)x, (T*)x, M, D));
   L3_TRY(launch_check());
   L3_TRY(run_rmsnorm<T>(c, x, D, w->ffn_norm, xn, M, st));
   L3_TRY(simt_gemm<T>(LLAMA3_KERNEL_GEMM_W13, xn, w->w1, Pp, M, F, D, 2 * F, st));
   L3_TRY(simt_gemm<T>(LLAMA3_KERNEL_GEMM_W13, xn, w->w3, Pp + F, M, F, D, 2 * F, st));
-  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, epi_swiglu_kernel<T><<<blocks_for((long long)M * F, 256), 256, 0, st>>>(Pp, 1, 0, g, M, F));
+  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_swiglu_kernel<T>), blocks_for((long long)M * F / 4, 256), 256, 0, st, Pp, 1, 0, g, M, F));
   L3_TRY(launch_check());
   L3_TRY(simt_gemm<T>(LLAMA3_KERNEL_GEMM_W2, g, w->w2, Pp, M, D, F, D, st));
-  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, epi_residual_kernel<T><<<blocks_for((long long)M * D, 256), 256, 0, st>>>(Pp, 1, 0, D, (const T*)x, (T*)x, M, D));
+  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_residual_kernel<T>), blocks_for((long long)M * D / 4, 256), 256, 0, st, Pp, 1, 0, D, (const T*)x, (T*)x, M, D));
   return launch_check();
 }
 
@@ -544,15 +614,19 @@ int layer_tc_prefill(const llama3_config* c, const llama3_layer_weights* w, cons
   bf16* o = ws_at<bf16>(ws, L.o);
   bf16* g = ws_at<bf16>(ws, L.g);
   float* Ap = ws_at<float>(ws, L.attn_part);
+  // CTA-pair GEMMs take B in halves per CTA (box rows BN/2); single-CTA ones whole.
+  const bool pair = use_pair_gemm(M);
+  const int bb = pair ? kPrefillBN / 2 : kPrefillBN;
+  const int bd = pair ? 64 : 128;
   CUtensorMap mxn, mo, mg, mwqkv, mwo, mw1, mw3, mw2;
   L3_TRY(make_map(&mxn, xn, M, D, 128));
   L3_TRY(make_map(&mo, o, M, H * hd, 128));
   L3_TRY(make_map(&mg, g, M, F, 128));
-  L3_TRY(make_map(&mwqkv, w->wqkv, nqkv, D, kPrefillBN));
-  L3_TRY(make_map(&mwo, w->wo, D, H * hd, kPrefillBN));
-  L3_TRY(make_map(&mw1, w->w1, F, D, 128));
-  L3_TRY(make_map(&mw3, w->w3, F, D, 128));
-  L3_TRY(make_map(&mw2, w->w2, D, F, kPrefillBN));
+  L3_TRY(make_map(&mwqkv, w->wqkv, nqkv, D, bb));
+  L3_TRY(make_map(&mwo, w->wo, D, H * hd, bb));
+  L3_TRY(make_map(&mw1, w->w1, F, D, bd));
+  L3_TRY(make_map(&mw3, w->w3, F, D, bd));
+  L3_TRY(make_map(&mw2, w->w2, D, F, bb));
 
   // attention half
   L3_TRY(rmsnorm_any(c, x, D, w->attention_norm, xn, M, st));
@@ -560,29 +634,45 @@ int layer_tc_prefill(const llama3_config* c, const llama3_layer_weights* w, cons
     EpiParams ep = empty_epi();
     ep.seq = S; ep.start_pos = P; ep.n_heads = H; ep.n_kv = KV; ep.head_dim = hd; ep.cache_cap = cap;
     ep.rope = rope; ep.q_out = q; ep.k_cache = kc; ep.v_cache = vc;
-    GemmShape sh = make_shape(M, 0, nqkv, D, kPrefillBN, 1);
-    L3_TRY((launch_gemm<kPrefillBN, 4, EPI_QKV_ROPE, false>(LLAMA3_KERNEL_GEMM_QKV, mxn, mxn, mwqkv, mwqkv, sh, ep, st)));
+    if (pair)
+      L3_TRY((launch_gemm_pair<kPrefillBN, 6, EPI_QKV_ROPE, false>(
+          LLAMA3_KERNEL_GEMM_QKV, mxn, mwqkv, mwqkv, make_shape_pair(M, nqkv, D, kPrefillBN), ep, st)));
+    else
+      L3_TRY((launch_gemm<kPrefillBN, 4, EPI_QKV_ROPE, false>(LLAMA3_KERNEL_GEMM_QKV, mxn, mxn, mwqkv, mwqkv,
+                                                               make_shape(M, 0, nqkv, D, kPrefillBN, 1), ep, st)));
   }
   L3_TRY(attention_dispatch(c, q, kc, vc, cap, B, S, P, o, Ap, st));
   {
     EpiParams ep = empty_epi();
     ep.out = x; ep.res = x; ep.ldo = D;
-    GemmShape sh = make_shape(M, 0, D, H * hd, kPrefillBN, 1);
-    L3_TRY((launch_gemm<kPrefillBN, 4, EPI_RESIDUAL, false>(LLAMA3_KERNEL_GEMM_WO, mo, mo, mwo, mwo, sh, ep, st)));
+    if (pair)
+      L3_TRY((launch_gemm_pair<kPrefillBN, 6, EPI_RESIDUAL, false>(
+          LLAMA3_KERNEL_GEMM_WO, mo, mwo, mwo, make_shape_pair(M, D, H * hd, kPrefillBN), ep, st)));
+    else
+      L3_TRY((launch_gemm<kPrefillBN, 4, EPI_RESIDUAL, false>(LLAMA3_KERNEL_GEMM_WO, mo, mo, mwo, mwo,
+                                                               make_shape(M, 0, D, H * hd, kPrefillBN, 1), ep, st)));
   }
   // FFN half
   L3_TRY(rmsnorm_any(c, x, D, w->ffn_norm, xn, M, st));
   {
     EpiParams ep = empty_epi();
     ep.out = g; ep.ldo = F;
-    GemmShape sh = make_shape(M, 0, F, D, 128, 1);
-    L3_TRY((launch_gemm<128, 4, EPI_SWIGLU, true>(LLAMA3_KERNEL_GEMM_W13, mxn, mxn, mw1, mw3, sh, ep, st)));
+    if (pair)
+      L3_TRY((launch_gemm_pair<128, 6, EPI_SWIGLU, true>(LLAMA3_KERNEL_GEMM_W13, mxn, mw1, mw3,
+                                                          make_shape_pair(M, F, D, 128), ep, st)));
+    else
+      L3_TRY((launch_gemm<128, 4, EPI_SWIGLU, true>(LLAMA3_KERNEL_GEMM_W13, mxn, mxn, mw1, mw3,
+                                                     make_shape(M, 0, F, D, 128, 1), ep, st)));
   }
   {
     EpiParams ep = empty_epi();
     ep.out = x; ep.res = x; ep.ldo = D;
-    GemmShape sh = make_shape(M, 0, D, F, kPrefillBN, 1);
-    L3_TRY((launch_gemm<kPrefillBN, 4, EPI_RESIDUAL, false>(LLAMA3_KERNEL_GEMM_W2, mg, mg, mw2, mw2, sh, ep, st)));
+    if (pair)
+      L3_TRY((launch_gemm_pair<kPrefillBN, 6, EPI_RESIDUAL, false>(
+          LLAMA3_KERNEL_GEMM_W2, mg, mw2, mw2, make_shape_pair(M, D, F, kPrefillBN), ep, st)));
+    else
+      L3_TRY((launch_gemm<kPrefillBN, 4, EPI_RESIDUAL, false>(LLAMA3_KERNEL_GEMM_W2, mg, mg, mw2, mw2,
+                                                               make_shape(M, 0, D, F, kPrefillBN, 1), ep, st)));
   }
   return LLAMA3_OK;
 }
@@ -605,21 +695,21 @@ int layer_tc_decode(const llama3_config* c, const llama3_layer_weights* w, const
 
   L3_TRY(rmsnorm_any(c, x, D, w->attention_norm, xn, M, st));
   L3_TRY(swapped_partial_gemm(w->wqkv, nqkv, nullptr, 0, 0, xn, M, D, Pp, nqkv, &splits, st));
-  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, epi_qkv_rope_kernel<bf16><<<blocks_for((long long)M * nqkv / 2, 256), 256, 0, st>>>(
+  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_qkv_rope_kernel<bf16>), blocks_for((long long)M * nqkv / 4, 256), 256, 0, st, 
       Pp, splits, (long long)M * nqkv, M, 1, P, H, KV, hd, rope, q, (bf16*)kc, (bf16*)vc, cap));
   L3_TRY(launch_check());
   L3_TRY(attention_dispatch(c, q, kc, vc, cap, B, 1, P, o, Ap, st));
   L3_TRY(swapped_partial_gemm(w->wo, D, nullptr, 0, 0, o, M, H * hd, Pp, D, &splits, st));
-  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, epi_residual_kernel<bf16><<<blocks_for((long long)M * D, 256), 256, 0, st>>>(
+  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_residual_kernel<bf16>), blocks_for((long long)M * D / 4, 256), 256, 0, st, 
       Pp, splits, (long long)M * D, D, (const bf16*)x, (bf16*)x, M, D));
   L3_TRY(launch_check());
   L3_TRY(rmsnorm_any(c, x, D, w->ffn_norm, xn, M, st));
   L3_TRY(swapped_partial_gemm(w->w1, F, w->w3, F, F, xn, M, D, Pp, 2 * F, &splits, st));
-  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, epi_swiglu_kernel<bf16><<<blocks_for((long long)M * F, 256), 256, 0, st>>>(Pp, splits, (long long)M * 2 * F, g,
+  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_swiglu_kernel<bf16>), blocks_for((long long)M * F / 4, 256), 256, 0, st, Pp, splits, (long long)M * 2 * F, g,
                                                                                 M, F));
   L3_TRY(launch_check());
   L3_TRY(swapped_partial_gemm(w->w2, D, nullptr, 0, 0, g, M, F, Pp, D, &splits, st));
-  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, epi_residual_kernel<bf16><<<blocks_for((long long)M * D, 256), 256, 0, st>>>(
+  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_residual_kernel<bf16>), blocks_for((long long)M * D / 4, 256), 256, 0, st, 
       Pp, splits, (long long)M * D, D, (const bf16*)x, (bf16*)x, M, D));
   return launch_check();
 }
@@ -686,7 +776,13 @@ unsigned long long llama3_launch_count(void) { return g_launches.load(); }
 
 int llama3_set_kernel_path(int path) {
   int old = g_kernel_path;
-  g_kernel_path = path ? 1 : 0;
+  g_kernel_path = (path >= 0 && path <= 2) ? path : 0;
+  return old;
+}
+
+int llama3_set_programmatic_launch(int on) {
+  const int old = g_pdl ? 1 : 0;
+  g_pdl = on != 0;
   return old;
 }
 
@@ -739,9 +835,9 @@ int llama3_embed(const llama3_config* cfg, const int32_t* ids, const void* table
   if (!aligned16(ids) || !aligned16(table) || !aligned16(x)) return LLAMA3_ERR_ALIGN;
   cudaStream_t st = (cudaStream_t)stream;
   if (cfg->dtype == LLAMA3_DTYPE_F32)
-    L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, embed_kernel<float><<<n_tokens, 128, 0, st>>>(ids, (const float*)table, (float*)x, cfg->dim, cfg->vocab));
+    L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((embed_kernel<float>), n_tokens, 128, 0, st, ids, (const float*)table, (float*)x, cfg->dim, cfg->vocab));
   else
-    L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, embed_kernel<bf16><<<n_tokens, 128, 0, st>>>(ids, (const bf16*)table, (bf16*)x, cfg->dim, cfg->vocab));
+    L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((embed_kernel<bf16>), n_tokens, 128, 0, st, ids, (const bf16*)table, (bf16*)x, cfg->dim, cfg->vocab));
   return launch_check();
 }
 
@@ -763,24 +859,33 @@ int llama3_linear(const llama3_config* cfg, const void* x, const void* w, const 
   if (use_tc(cfg)) {
     if (k % 8 || n % 8) return LLAMA3_ERR_ALIGN;
     CUtensorMap ma, mb;
-    L3_TRY(make_map(&ma, x, m, k, 128));
-    L3_TRY(make_map(&mb, w, n, k, kPrefillBN));
     EpiParams ep = empty_epi();
     ep.out = y; ep.res = residual; ep.ldo = n;
+    if (use_pair_gemm(m)) {
+      L3_TRY(make_map(&ma, x, m, k, 128));
+      L3_TRY(make_map(&mb, w, n, k, kPrefillBN / 2));
+      const GemmShape sp = make_shape_pair(m, n, k, kPrefillBN);
+      if (residual)
+        return launch_gemm_pair<kPrefillBN, 6, EPI_RESIDUAL, false>(LLAMA3_KERNEL_GEMM_WO, ma, mb, mb, sp, ep, st);
+      return launch_gemm_pair<kPrefillBN, 6, EPI_STORE, false>(LLAMA3_KERNEL_GEMM_WO, ma, mb, mb, sp, ep, st);
+    }
+    L3_TRY(make_map(&ma, x, m, k, 128));
+    L3_TRY(make_map(&mb, w, n, k, kPrefillBN));
     GemmShape sh = make_shape(m, 0, n, k, kPrefillBN, 1);
     if (residual) return launch_gemm<kPrefillBN, 4, EPI_RESIDUAL, false>(LLAMA3_KERNEL_GEMM_WO, ma, ma, mb, mb, sh, ep, st);
     return launch_gemm<kPrefillBN, 4, EPI_STORE, false>(LLAMA3_KERNEL_GEMM_WO, ma, ma, mb, mb, sh, ep, st);
   }
+  if (n % 4) return LLAMA3_ERR_ALIGN;
   const size_t need = (size_t)m * n * 4;
   if (!ws || ws_bytes < need) return LLAMA3_ERR_WORKSPACE;
   float* C = (float*)ws;
   if (cfg->dtype == LLAMA3_DTYPE_F32) {
     L3_TRY(simt_gemm<float>(LLAMA3_KERNEL_GEMM_WO, x, w, C, m, n, k, n, st));
-    L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, epi_residual_kernel<float><<<blocks_for((long long)m * n, 256), 256, 0, st>>>(C, 1, 0, n, (const float*)residual,
+    L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_residual_kernel<float>), blocks_for(((long long)m * n + 3) / 4, 256), 256, 0, st, C, 1, 0, n, (const float*)residual,
                                                                                   (float*)y, m, n));
   } else {
     L3_TRY(simt_gemm<bf16>(LLAMA3_KERNEL_GEMM_WO, x, w, C, m, n, k, n, st));
-    L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, epi_residual_kernel<bf16><<<blocks_for((long long)m * n, 256), 256, 0, st>>>(C, 1, 0, n, (const bf16*)residual,
+    L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_residual_kernel<bf16>), blocks_for(((long long)m * n + 3) / 4, 256), 256, 0, st, C, 1, 0, n, (const bf16*)residual,
                                                                                  (bf16*)y, m, n));
   }
   return launch_check();
@@ -848,7 +953,7 @@ int llama3_lm_head_argmax(const llama3_config* cfg, const void* norm_w, const vo
   unsigned long long* keys = ws_at<unsigned long long>(ws, L.keys);
   const int V = cfg->vocab, D = cfg->dim;
   L3_TRY(rmsnorm_any(cfg, h, row_stride, norm_w, hn, rows, st));
-  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, argmax_init_kernel<<<blocks_for(rows, 256), 256, 0, st>>>(keys, rows));
+  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((argmax_init_kernel), blocks_for(rows, 256), 256, 0, st, keys, rows));
   L3_TRY(launch_check());
   if (use_tc(cfg)) {
     const int bn = rows <= 16 ? 16 : rows <= 32 ? 32 : rows <= 64 ? 64 : rows <= 128 ? 128 : 256;
@@ -869,14 +974,14 @@ int llama3_lm_head_argmax(const llama3_config* cfg, const void* norm_w, const vo
   } else {
     const long long warps = (long long)rows * ((V + 31) / 32);
     if (cfg->dtype == LLAMA3_DTYPE_F32)
-      L3_LAUNCH(LLAMA3_KERNEL_LM_HEAD, st, lm_head_simt_kernel<float><<<blocks_for(warps * 32, 256), 256, 0, st>>>((const float*)hn, (const float*)w_out,
+      L3_LAUNCH(LLAMA3_KERNEL_LM_HEAD, st, launch_k((lm_head_simt_kernel<float>), blocks_for(warps * 32, 256), 256, 0, st, (const float*)hn, (const float*)w_out,
                                                                                logits_out, keys, rows, V, D));
     else
-      L3_LAUNCH(LLAMA3_KERNEL_LM_HEAD, st, lm_head_simt_kernel<bf16><<<blocks_for(warps * 32, 256), 256, 0, st>>>((const bf16*)hn, (const bf16*)w_out,
+      L3_LAUNCH(LLAMA3_KERNEL_LM_HEAD, st, launch_k((lm_head_simt_kernel<bf16>), blocks_for(warps * 32, 256), 256, 0, st, (const bf16*)hn, (const bf16*)w_out,
                                                                               logits_out, keys, rows, V, D));
     L3_TRY(launch_check());
   }
-  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, argmax_finalize_kernel<<<blocks_for(rows, 256), 256, 0, st>>>(keys, ids_out, rows));
+  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((argmax_finalize_kernel), blocks_for(rows, 256), 256, 0, st, keys, ids_out, rows));
   return launch_check();
 }
 
@@ -932,7 +1037,7 @@ extern "C" int llama3_lm_head_argmax_noalloc(const llama3_config* cfg, const voi
   const int V = cfg->vocab, D = cfg->dim;
   L3_TRY(rmsnorm_any(cfg, h, row_stride, norm_w, hn, rows, st));
   // the keys hold the previous call's maxima: start from zero every call
-  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, argmax_init_kernel<<<blocks_for(rows, 256), 256, 0, st>>>(keys, rows));
+  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((argmax_init_kernel), blocks_for(rows, 256), 256, 0, st, keys, rows));
   L3_TRY(launch_check());
   if (use_tc(cfg)) {
     const int bn = rows <= 16 ? 16 : rows <= 32 ? 32 : rows <= 64 ? 64 : rows <= 128 ? 128 : 256;
@@ -953,13 +1058,13 @@ extern "C" int llama3_lm_head_argmax_noalloc(const llama3_config* cfg, const voi
   } else {
     const long long warps = (long long)rows * ((V + 31) / 32);
     if (cfg->dtype == LLAMA3_DTYPE_F32)
-      L3_LAUNCH(LLAMA3_KERNEL_LM_HEAD, st, lm_head_simt_kernel<float><<<blocks_for(warps * 32, 256), 256, 0, st>>>(
+      L3_LAUNCH(LLAMA3_KERNEL_LM_HEAD, st, launch_k((lm_head_simt_kernel<float>), blocks_for(warps * 32, 256), 256, 0, st, 
                                                (const float*)hn, (const float*)w_out, logits_out, keys, rows, V, D));
     else
-      L3_LAUNCH(LLAMA3_KERNEL_LM_HEAD, st, lm_head_simt_kernel<bf16><<<blocks_for(warps * 32, 256), 256, 0, st>>>(
+      L3_LAUNCH(LLAMA3_KERNEL_LM_HEAD, st, launch_k((lm_head_simt_kernel<bf16>), blocks_for(warps * 32, 256), 256, 0, st, 
                                                (const bf16*)hn, (const bf16*)w_out, logits_out, keys, rows, V, D));
     L3_TRY(launch_check());
   }
-  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, argmax_finalize_kernel<<<blocks_for(rows, 256), 256, 0, st>>>(keys, ids_out, rows));
+  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((argmax_finalize_kernel), blocks_for(rows, 256), 256, 0, st, keys, ids_out, rows));
   return launch_check();
 }

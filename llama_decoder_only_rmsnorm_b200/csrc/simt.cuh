@@ -13,13 +13,21 @@ namespace l3 {
 template <typename T>
 __global__ void embed_kernel(const int32_t* __restrict__ ids, const T* __restrict__ table,
                              T* __restrict__ x, int D, int vocab) {
-  int t = blockIdx.x;
-  int id = ids[t];
-  bool ok = id >= 0 && id < vocab;
+  griddep_wait_and_release();
+  const int t = blockIdx.x;
+  const int id = ids[t];
+  const bool ok = id >= 0 && id < vocab;
   if (!ok && threadIdx.x == 0) record_error(LLAMA3_ERR_TOKEN);
   const T* src = table + (size_t)(ok ? id : 0) * D;
   T* dst = x + (size_t)t * D;
-  for (int i = threadIdx.x; i < D; i += blockDim.x) dst[i] = ok ? src[i] : from_f<T>(0.f);
+  if ((D * sizeof(T)) % 16 == 0) {   // rows are 16-byte aligned: copy 16 bytes per thread
+    const int n16 = D * (int)sizeof(T) / 16;
+    const uint4* s4 = reinterpret_cast<const uint4*>(src);
+    uint4* d4 = reinterpret_cast<uint4*>(dst);
+    for (int i = threadIdx.x; i < n16; i += blockDim.x) d4[i] = ok ? s4[i] : make_uint4(0, 0, 0, 0);
+  } else {
+    for (int i = threadIdx.x; i < D; i += blockDim.x) dst[i] = ok ? src[i] : from_f<T>(0.f);
+  }
 }
 
 // ---- RMSNorm ("Build your own Llama 3 from scratch" §3.1) -------------------
@@ -27,6 +35,7 @@ __global__ void embed_kernel(const int32_t* __restrict__ ids, const T* __restric
 template <typename T>
 __global__ void rmsnorm_kernel(const T* __restrict__ x, long long row_stride,
                                const T* __restrict__ w, T* __restrict__ y, int D, float eps) {
+  griddep_wait_and_release();
   const T* xr = x + (size_t)blockIdx.x * row_stride;
   T* yr = y + (size_t)blockIdx.x * D;
   float ss = 0.f;
@@ -54,6 +63,7 @@ template <int CPL>
 __global__ void __launch_bounds__(128) rmsnorm_bf16_warp_kernel(const bf16* __restrict__ x, long long row_stride,
                                                                const bf16* __restrict__ w, bf16* __restrict__ y,
                                                                int rows, int D, float eps) {
+  griddep_wait_and_release();
   const int row = blockIdx.x * 4 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (row >= rows) return;
   const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)row * row_stride);
@@ -99,6 +109,7 @@ template <typename T>
 __global__ void __launch_bounds__(256) gemm_simt_kernel(const T* __restrict__ A, const T* __restrict__ B,
                                                         float* __restrict__ C, int M, int N, int K,
                                                         int ldc) {
+  griddep_wait_and_release();
   __shared__ float As[16][64 + 1];
   __shared__ float Bs[16][64 + 1];
   int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
@@ -140,23 +151,49 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(const T* __restrict__ A,
 
 // ---- epilogues over fp32 partial sums P[split][m][n] ------------------------
 // (used after the SIMT GEMM with splits = 1 and after split-K tensor-core GEMMs)
-__device__ __forceinline__ float sum_splits(const float* P, int splits, long long split_stride,
-                                            long long idx) {
-  float s = 0.f;
-  for (int i = 0; i < splits; ++i) s += P[(size_t)i * split_stride + idx];
-  return s;
+// Four consecutive elements per thread: every row length here is a multiple of 4.
+__device__ __forceinline__ void load4(const float* p, float (&v)[4]) {
+  const float4 x = *reinterpret_cast<const float4*>(p);
+  v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+}
+__device__ __forceinline__ void load4(const bf16* p, float (&v)[4]) {
+  const uint2 x = *reinterpret_cast<const uint2*>(p);
+  v[0] = bf16lo(x.x); v[1] = bf16hi(x.x); v[2] = bf16lo(x.y); v[3] = bf16hi(x.y);
+}
+__device__ __forceinline__ void store4(float* p, const float (&v)[4]) {
+  *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+}
+__device__ __forceinline__ void store4(bf16* p, const float (&v)[4]) {
+  *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
+}
+__device__ __forceinline__ void sum4_splits(const float* P, int splits, long long split_stride, long long idx,
+                                            float (&v)[4]) {
+  load4(P + idx, v);
+  for (int i = 1; i < splits; ++i) {
+    float w[4];
+    load4(P + (size_t)i * split_stride + idx, w);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) v[q] += w[q];
+  }
 }
 
 // out[m, n] = (res ? res[m, n] : 0) + P[m, n]
 template <typename T>
 __global__ void epi_residual_kernel(const float* __restrict__ P, int splits, long long split_stride,
                                     int ldp, const T* res, T* out, int M, int N) {
-  long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  griddep_wait_and_release();
+  const long long i = ((long long)blockIdx.x * blockDim.x + threadIdx.x) * 4;
   if (i >= (long long)M * N) return;
-  int m = (int)(i / N), n = (int)(i % N);
-  float v = sum_splits(P, splits, split_stride, (long long)m * ldp + n);
-  if (res) v += to_f(res[i]);
-  out[i] = from_f<T>(v);
+  const int m = (int)(i / N), n = (int)(i % N);
+  float v[4];
+  sum4_splits(P, splits, split_stride, (long long)m * ldp + n, v);
+  if (res) {
+    float r[4];
+    load4(res + i, r);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) v[q] += r[q];
+  }
+  store4(out + i, v);
 }
 
 // g[m, f] = silu(P[m, f]) * P[m, F + f],  silu(z) = z / (1 + e^-z)
@@ -164,49 +201,51 @@ __global__ void epi_residual_kernel(const float* __restrict__ P, int splits, lon
 template <typename T>
 __global__ void epi_swiglu_kernel(const float* __restrict__ P, int splits, long long split_stride,
                                   T* __restrict__ g, int M, int F) {
-  long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  griddep_wait_and_release();
+  const long long i = ((long long)blockIdx.x * blockDim.x + threadIdx.x) * 4;
   if (i >= (long long)M * F) return;
-  int m = (int)(i / F), f = (int)(i % F);
-  float a = sum_splits(P, splits, split_stride, (long long)m * 2 * F + f);
-  float b = sum_splits(P, splits, split_stride, (long long)m * 2 * F + F + f);
-  g[i] = from_f<T>(a / (1.f + expf(-a)) * b);
+  const int m = (int)(i / F), f = (int)(i % F);
+  float a[4], b[4], o[4];
+  sum4_splits(P, splits, split_stride, (long long)m * 2 * F + f, a);
+  sum4_splits(P, splits, split_stride, (long long)m * 2 * F + F + f, b);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) o[q] = a[q] / (1.f + expf(-a[q])) * b[q];
+  store4(g + i, o);
 }
 
 // QKV epilogue: rotate q and k pairs (2i, 2i+1) by the table's (cos, sin) of
 // position start_pos + t ("Build your own Llama 3 from scratch" §3.2), write
 // q to q_out [M, H*hd] and k, v to the caches at [b, pos, kvh, :] (§3.3).
-// One thread per pair.
+// Two pairs (four elements, inside one head) per thread.
 template <typename T>
 __global__ void epi_qkv_rope_kernel(const float* __restrict__ P, int splits, long long split_stride,
                                     int M, int seq, int start_pos, int H, int KV, int hd,
                                     const float* __restrict__ rope, T* __restrict__ q_out,
                                     T* __restrict__ k_cache, T* __restrict__ v_cache, int cap) {
-  int Ntot = (H + 2 * KV) * hd;
-  long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= (long long)M * (Ntot / 2)) return;
-  int m = (int)(i / (Ntot / 2));
-  int n = (int)(i % (Ntot / 2)) * 2;
-  int b = m / seq, t = m % seq, pos = start_pos + t;
-  float a = sum_splits(P, splits, split_stride, (long long)m * Ntot + n);
-  float c = sum_splits(P, splits, split_stride, (long long)m * Ntot + n + 1);
-  int d = n % hd, head = n / hd;
+  griddep_wait_and_release();
+  const int Ntot = (H + 2 * KV) * hd;
+  const long long i = ((long long)blockIdx.x * blockDim.x + threadIdx.x) * 4;
+  if (i >= (long long)M * Ntot) return;
+  const int m = (int)(i / Ntot);
+  const int n = (int)(i % Ntot);
+  const int b = m / seq, t = m % seq, pos = start_pos + t;
+  float v[4];
+  sum4_splits(P, splits, split_stride, (long long)m * Ntot + n, v);
+  const int d = n % hd, head = n / hd;
   if (head < H + KV) {
-    const float* cs = rope + ((size_t)pos * (hd / 2) + d / 2) * 2;
-    float co = cs[0], si = cs[1];
-    float ra = a * co - c * si, rc = a * si + c * co;
-    a = ra;
-    c = rc;
+    const float4 cs = *reinterpret_cast<const float4*>(rope + ((size_t)pos * (hd / 2) + d / 2) * 2);
+    const float a0 = v[0], b0 = v[1], a1 = v[2], b1 = v[3];
+    v[0] = a0 * cs.x - b0 * cs.y;
+    v[1] = a0 * cs.y + b0 * cs.x;
+    v[2] = a1 * cs.z - b1 * cs.w;
+    v[3] = a1 * cs.w + b1 * cs.z;
   }
   if (head < H) {
-    T* dst = q_out + (size_t)m * H * hd + n;
-    dst[0] = from_f<T>(a);
-    dst[1] = from_f<T>(c);
+    store4(q_out + (size_t)m * H * hd + n, v);
   } else {
-    bool is_k = head < H + KV;
-    int kvh = head - (is_k ? H : H + KV);
-    T* dst = (is_k ? k_cache : v_cache) + (((size_t)b * cap + pos) * KV + kvh) * hd + d;
-    dst[0] = from_f<T>(a);
-    dst[1] = from_f<T>(c);
+    const bool is_k = head < H + KV;
+    const int kvh = head - (is_k ? H : H + KV);
+    store4((is_k ? k_cache : v_cache) + (((size_t)b * cap + pos) * KV + kvh) * hd + d, v);
   }
 }
 
@@ -219,6 +258,7 @@ __global__ void attention_simt_kernel(const T* __restrict__ q, const T* __restri
                                       const T* __restrict__ v_cache, T* __restrict__ out, int B,
                                       int S, int start_pos, int H, int KV, int hd, int cap,
                                       float scale) {
+  griddep_wait_and_release();
   long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   int lane = threadIdx.x & 31;
   if (w >= (long long)B * S * H) return;
@@ -268,6 +308,7 @@ template <typename T>
 __global__ void lm_head_simt_kernel(const T* __restrict__ hn, const T* __restrict__ W,
                                     float* __restrict__ logits, unsigned long long* __restrict__ keys,
                                     int R, int V, int D) {
+  griddep_wait_and_release();
   long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   int lane = threadIdx.x & 31;
   int vblocks = (V + 31) / 32;
@@ -289,10 +330,12 @@ __global__ void lm_head_simt_kernel(const T* __restrict__ hn, const T* __restric
 }
 
 __global__ void argmax_init_kernel(unsigned long long* keys, int R) {
+  griddep_wait_and_release();
   int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < R) keys[i] = 0ull;
 }
 __global__ void argmax_finalize_kernel(const unsigned long long* keys, int32_t* ids, int R) {
+  griddep_wait_and_release();
   int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < R) ids[i] = (int32_t)(0xffffffffu - (uint32_t)(keys[i] & 0xffffffffull));
 }

@@ -279,6 +279,7 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  griddep_wait_and_release();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer

@@ -57,7 +57,7 @@ def test_rmsnorm(dtype, D, H):
 @pytest.mark.parametrize("m,n,k", [(128, 256, 64), (300, 264, 200), (1000, 1536, 512), (77, 4096, 4096),
                                    (2048, 6144, 4096)])
 @pytest.mark.parametrize("residual", [False, True])
-@pytest.mark.parametrize("path", [0, 1])
+@pytest.mark.parametrize("path", [0, 1, 2])
 def test_linear(m, n, k, residual, path):
     if path == 1 and m * n > 2_000_000:
         pytest.skip("SIMT cross-check only on the smaller shapes")
@@ -157,8 +157,9 @@ def test_char_8l_stack_and_lm_head(path):
     _run_layers_vs_oracle(wl("char_8l"), path=path)
 
 
-def test_gqa_768_layer():
-    _run_layers_vs_oracle(wl("gqa_768"))
+@pytest.mark.parametrize("path", [0, 2])
+def test_gqa_768_layer(path):
+    _run_layers_vs_oracle(wl("gqa_768"), path=path)
 
 
 def test_chunked_prefill_then_decode_steps():
