@@ -53,6 +53,7 @@ def parse():
     p.add_argument("--layers", type=int, default=None, help=argparse.SUPPRESS)  # profiling captures only
     p.add_argument("--no-pdl", action="store_true", help=argparse.SUPPRESS)   # A/B of programmatic launch
     p.add_argument("--kernel-path", type=int, default=0, help=argparse.SUPPRESS)  # A/B of GEMM variants
+    p.add_argument("--flash-variant", type=int, default=None, help=argparse.SUPPRESS)  # A/B of attention designs
     return p.parse_args()
 
 
@@ -287,6 +288,8 @@ def run_ours(args):
     if args.no_pdl:
         B.llama3_set_programmatic_launch(False)
     B.llama3_set_kernel_path(args.kernel_path)
+    if args.flash_variant is not None:
+        B.llama3_set_flash_variant(args.flash_variant)
     peaks, peak_kind = load_peaks()
     layers, outw = build(dev)
     n_layers = args.layers or PREFILL.n_layers
@@ -324,6 +327,18 @@ def run_ours(args):
     whole = {"flop_per_step": total_flop + attn_flop,
              "tflops": (total_flop + attn_flop) / (ms / 1e3) / 1e12}
     whole["frac_of_peak"] = whole["tflops"] / peak
+    # the causal attention kernel, timed in a second, shorter pass (its own
+    # events; one timer family at a time).  Algorithmic flops: QK^T and PV over
+    # the visible (causal) keys only.
+    a_steps = max(1, min(3, args.steps))
+    _, a_ms, _ = time_steps(prefill_step, a_steps, 1, world, timer=("attention", a_steps * n_layers),
+                            name="prefill_attention")
+    a_flop = PREFILL.n_heads * 2.0 * 2.0 * (S * (S + 1) / 2) * PREFILL.head_dim
+    attention = {"kernel": "causal GQA flash attention (S=8192, 32 q heads, 8 kv heads, hd 128)",
+                 "kernel_ms": a_ms, "flop_per_launch": a_flop,
+                 "tflops": a_flop / (a_ms / 1e3) / 1e12 if a_ms else None}
+    if attention["tflops"]:
+        attention["frac_of_peak"] = attention["tflops"] / peak
 
     # e2e through the public API with host buffers
     ids_h = ids.cpu().pin_memory()
@@ -424,7 +439,7 @@ def run_ours(args):
                 "config": {"workload": "llama3_8b_prefill", "batch": 1, "seq_len": S, "layers": n_layers,
                            "lm_head_rows": "last position", "parallelism": f"replicas x{world}",
                            "l2": "inputs larger than L2 (16 GB of weights streamed per step)"},
-                "roofline": roofline, "whole_step": whole, "cpu_baseline": cpu, "e2e": e2e,
+                "roofline": roofline, "whole_step": whole, "attention": attention, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": launches, "clocks": clocks, "decode": decode}
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -148,6 +148,22 @@ int llama3_layer_forward(const llama3_config* cfg, const llama3_layer_weights* w
                          void* ws, size_t ws_bytes, llama3_stream_t stream);
 
 /*
+ * llama3_layer_forward with the document-level attention mask of
+ * "Build your own Llama 3 from scratch" 附 1: several documents packed into one
+ * sequence must not attend to each other.  doc_start: device int32
+ * [batch, seq]; doc_start[b][t] is the position where the document of token t
+ * (position start_pos + t) begins.  The token then attends to positions
+ * doc_start[b][t] .. start_pos + t.  Values must be non-decreasing in t and
+ * lie in [0, start_pos + t] (larger values are clamped to start_pos + t).
+ * Errors as llama3_layer_forward, plus LLAMA3_ERR_ARG for a NULL doc_start.
+ */
+int llama3_layer_forward_docs(const llama3_config* cfg, const llama3_layer_weights* w,
+                              const float* rope, int rope_len, void* x, void* k_cache,
+                              void* v_cache, int cache_cap, int batch, int seq, int start_pos,
+                              const int32_t* doc_start, void* ws, size_t ws_bytes,
+                              llama3_stream_t stream);
+
+/*
  * One decode step of one block ([S2] 六 generate: one new token per sequence
  * against the KV cache, §3.3).  Same as llama3_layer_forward with seq = 1:
  * x: [batch, 1, D]; the new token of every sequence sits at position
@@ -254,6 +270,13 @@ int llama3_launch_timer_used(void);
 /* Kernels launched by this library since it was loaded (all threads). */
 unsigned long long llama3_launch_count(void);
 
+/* llama3_attention with the document mask (doc_start as in
+ * llama3_layer_forward_docs); always uses the prefill kernels. */
+int llama3_attention_docs(const llama3_config* cfg, const void* q, const void* k_cache,
+                          const void* v_cache, int cache_cap, int batch, int seq, int start_pos,
+                          const int32_t* doc_start, void* out, void* ws, size_t ws_bytes,
+                          llama3_stream_t stream);
+
 /* ---- status ---- */
 
 /* Static text for a status code. */
@@ -281,6 +304,13 @@ int llama3_set_wait_limit_ms(int ms);
  * the stream (each kernel waits for its predecessor before touching memory);
  * 0: ordinary launches.  Returns the previous value. */
 int llama3_set_programmatic_launch(int on);
+
+/* Prefill attention kernel design (bf16, tcgen05 path): 1 (default) = one
+ * softmax thread per query row with P staged in shared memory; 2 = two
+ * softmax threads per row (each over half the keys of a tile) with P written
+ * back into tensor memory.  Both compute the same attention.  Any other value
+ * selects 1.  Returns the previous value. */
+int llama3_set_flash_variant(int variant);
 
 #ifdef __cplusplus
 }

@@ -51,6 +51,8 @@ _SIGNATURES = {
     "llama3_embed": [_cfgp, _p, _p, _p, _i, _p],
     "llama3_layer_forward": [_cfgp, _wp, _p, _i, _p, _p, _p, _i, _i, _i, _i, _p, _sz, _p],
     "llama3_layer_decode": [_cfgp, _wp, _p, _i, _p, _p, _p, _i, _i, _i, _p, _sz, _p],
+    "llama3_layer_forward_docs": [_cfgp, _wp, _p, _i, _p, _p, _p, _i, _i, _i, _i, _p, _p, _sz, _p],
+    "llama3_attention_docs": [_cfgp, _p, _p, _p, _i, _i, _i, _i, _p, _p, _p, _sz, _p],
     "llama3_lm_head_argmax": [_cfgp, _p, _p, _p, _i, _ll, _p, _p, _p, _sz, _p],
     "llama3_lm_head_argmax_noalloc": [_cfgp, _p, _p, _p, _i, _ll, _p, _p, _p],
     "llama3_rmsnorm": [_cfgp, _p, _ll, _p, _p, _i, _p],
@@ -62,6 +64,7 @@ _SIGNATURES = {
     "llama3_set_kernel_path": [_i],
     "llama3_set_wait_limit_ms": [_i],
     "llama3_set_programmatic_launch": [_i],
+    "llama3_set_flash_variant": [_i],
     "llama3_set_launch_timer": [_i, _p, _p, _i],
     "llama3_launch_timer_used": [],
     "llama3_launch_count": [],
@@ -154,6 +157,20 @@ def llama3_layer_forward(cfg, w, rope, rope_len, x, k_cache, v_cache, cache_cap,
         cache_cap, batch, seq, start_pos, _ptr(ws), ws_bytes, _stream(stream)))
 
 
+def llama3_layer_forward_docs(cfg, w, rope, rope_len, x, k_cache, v_cache, cache_cap, batch, seq, start_pos,
+                              doc_start, ws, ws_bytes, stream=None):
+    _check("llama3_layer_forward_docs", lib().llama3_layer_forward_docs(
+        ctypes.byref(cfg), ctypes.byref(w), _ptr(rope), rope_len, _ptr(x), _ptr(k_cache), _ptr(v_cache),
+        cache_cap, batch, seq, start_pos, _ptr(doc_start), _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def llama3_attention_docs(cfg, q, k_cache, v_cache, cache_cap, batch, seq, start_pos, doc_start, out, ws,
+                          ws_bytes, stream=None):
+    _check("llama3_attention_docs", lib().llama3_attention_docs(
+        ctypes.byref(cfg), _ptr(q), _ptr(k_cache), _ptr(v_cache), cache_cap, batch, seq, start_pos,
+        _ptr(doc_start), _ptr(out), _ptr(ws), ws_bytes, _stream(stream)))
+
+
 def llama3_layer_decode(cfg, w, rope, rope_len, x, k_cache, v_cache, cache_cap, batch, start_pos, ws, ws_bytes,
                         stream=None):
     _check("llama3_layer_decode", lib().llama3_layer_decode(
@@ -219,6 +236,10 @@ def llama3_set_wait_limit_ms(ms):
 
 def llama3_set_programmatic_launch(on):
     return lib().llama3_set_programmatic_launch(1 if on else 0)
+
+
+def llama3_set_flash_variant(variant):
+    return lib().llama3_set_flash_variant(int(variant))
 
 
 KERNEL_KINDS = {"gemm_qkv": 1, "gemm_wo": 2, "gemm_w13": 3, "gemm_w2": 4, "attention": 5, "decode_gemm": 6,

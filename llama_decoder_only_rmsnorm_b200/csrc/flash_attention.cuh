@@ -36,6 +36,10 @@ struct FlashShape {
   int B, S, P, H, KV, n_rep, pairs, qtiles, units;
   int ldo;            // H * hd (output row length)
   float scale_log2;   // log2(e) / sqrt(hd)
+  // Optional document mask: doc_start[b * S + t] is the position where the
+  // document of token t begins (non-decreasing in t, <= start_pos + t); keys
+  // before it are invisible ("Build your own Llama 3 from scratch" 附 1).
+  const int32_t* doc_start;
 };
 
 template <int HD>
@@ -70,6 +74,17 @@ __device__ __forceinline__ void flash_unit(const FlashShape& fs, int u, int& b, 
 __device__ __forceinline__ int flash_ntiles(const FlashShape& fs, int qt) {
   const int last_key = min(fs.P + qt * 128 + 127, fs.P + fs.S - 1);
   return last_key / 128 + 1;
+}
+// Lowest visible key of query row t (document mask), clamped so that a row
+// always keeps its own key.
+__device__ __forceinline__ int flash_row_lo(const FlashShape& fs, int b, int t) {
+  if (!fs.doc_start) return 0;
+  const int tt = min(t, fs.S - 1);
+  return max(0, min(fs.doc_start[(size_t)b * fs.S + tt], fs.P + tt));
+}
+// First key tile a query tile needs: the tile of its first row's document start.
+__device__ __forceinline__ int flash_first_tile(const FlashShape& fs, int b, int qt) {
+  return flash_row_lo(fs, b, qt * 128) / 128;
 }
 
 template <int HD>
@@ -138,7 +153,8 @@ __global__ void __launch_bounds__(384, 1)
           qiss |= 1u << s; qpar = (qpar & ~(1u << s)) | (qph[s] << s);
           qph[s] ^= 1u;
         }
-        for (int j = 0; j < nt && ok; ++j) {
+        const int jt0 = flash_first_tile(fs, b, qt);
+        for (int j = jt0; j < nt && ok; ++j) {
           if (!mbar_wait(&k_empty[ks], kph ^ 1u, wait_ns)) { ok = false; break; }
           mbar_arrive_expect_tx(&k_full[ks], C::KV_BYTES);
           for (int c = 0; c < C::CHUNKS; ++c)
@@ -205,22 +221,29 @@ __global__ void __launch_bounds__(384, 1)
         }
         if (!ok) break;
         tc_fence_after();
-        // S(0) for every slot
+        const int jt0 = flash_first_tile(fs, b, qt);
+        // S of the first key tile for every slot
         if (!mbar_wait(&k_full[ks], kph, wait_ns)) break;
         tc_fence_after();
         for (int s = 0; s < nslots; ++s) issue_s(s, ks);
         tc_commit(&k_empty[ks]);
         if (++ks == C::KST) { ks = 0; kph ^= 1u; }
-        for (int j = 0; j < nt && ok; ++j) {
+        for (int j = jt0; j < nt && ok; ++j) {
           if (!mbar_wait(&v_full[vs], vph, wait_ns)) { ok = false; break; }
           const bool more = j + 1 < nt;
-          if (more && !mbar_wait(&k_full[ks], kph, wait_ns)) { ok = false; break; }
+          bool k_ready = false;
           for (int s = 0; s < nslots; ++s) {
             if (!mbar_wait(&p_full[s], pph[s], wait_ns)) { ok = false; break; }
             pph[s] ^= 1u;
             tc_fence_after();
-            issue_pv(s, vs, j > 0);
-            if (more) issue_s(s, ks);
+            issue_pv(s, vs, j > jt0);
+            if (more) {
+              // K of the next tile is only needed from here on: P.V above does not wait for it
+              if (!k_ready && !mbar_wait(&k_full[ks], kph, wait_ns)) { ok = false; break; }
+              k_ready = true;
+              tc_fence_after();
+              issue_s(s, ks);
+            }
           }
           if (!ok) break;
           tc_commit(&v_empty[vs]);
@@ -248,33 +271,43 @@ __global__ void __launch_bounds__(384, 1)
       flash_unit(fs, u, b, g, pair, qt);
       if (slot == 1 && !(pair * 2 + 1 < fs.n_rep)) continue;
       const int nt = flash_ntiles(fs, qt);
+      const int jt0 = flash_first_tile(fs, b, qt);
       const int qpos = fs.P + qt * 128 + row;
+      const int lo = flash_row_lo(fs, b, qt * 128 + row);
+      const int lo_last = flash_row_lo(fs, b, qt * 128 + 127);   // largest lower bound in the tile
       float m_ref = -INFINITY, l = 0.f;
       bool ok = true;
-      for (int j = 0; j < nt; ++j) {
+      for (int j = jt0; j < nt; ++j) {
         if (!mbar_wait(&s_full[slot], sph, wait_ns)) { ok = false; break; }
         sph ^= 1u;
         tc_fence_after();
-        const bool need_mask = j * 128 + 127 > fs.P + qt * 128;
-        // pass 1: row maximum of the raw scores
+        const bool need_mask = j * 128 + 127 > fs.P + qt * 128 || j * 128 < lo_last;
+        // pass 1: row maximum of the raw scores (the next chunk's TMEM load is
+        // in flight while the current one is reduced)
         float mx = -INFINITY;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tmem_ld32(s_tmem + c * 32, r);
+        {
+          uint32_t ra[32], rb[32];
+          tmem_ld32(s_tmem, ra);
           tc_wait_ld();
-          if (need_mask) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (j * 128 + c * 32 + i > qpos) r[i] = __float_as_uint(-INFINITY);
+          for (int c = 0; c < 4; ++c) {
+            uint32_t(&cur)[32] = (c & 1) ? rb : ra;
+            uint32_t(&nxt)[32] = (c & 1) ? ra : rb;
+            if (c + 1 < 4) tmem_ld32(s_tmem + (c + 1) * 32, nxt);
+            if (need_mask) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (j * 128 + c * 32 + i > qpos || j * 128 + c * 32 + i < lo) cur[i] = __float_as_uint(-INFINITY);
+            }
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) mx = max3f(mx, __uint_as_float(cur[i]), __uint_as_float(cur[i + 1]));
+            if (c + 1 < 4) tc_wait_ld();
           }
-#pragma unroll
-          for (int i = 0; i < 32; i += 2) mx = max3f(mx, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
         }
         const float m_tile = mx * fs.scale_log2;   // scale_log2 > 0: max commutes with the scale
         // the O written by the previous tile's P.V must be complete before P
         // (single buffer) is overwritten or O is rescaled
-        if (j > 0) {
+        if (j > jt0) {
           if (!mbar_wait(&o_done[slot], oph, wait_ns)) { ok = false; break; }
           oph ^= 1u;
           tc_fence_after();
@@ -288,7 +321,7 @@ __global__ void __launch_bounds__(384, 1)
         }
         // rescale this warp's rows of O in TMEM when any of them grew (the
         // TMEM accesses are warp-collective; rows that did not grow use 1)
-        if (j > 0 && __any_sync(0xffffffffu, grow)) {
+        if (j > jt0 && __any_sync(0xffffffffu, grow)) {
 #pragma unroll 1
           for (int c = 0; c < HD / 16; ++c) {
             uint32_t r[16];
@@ -301,50 +334,58 @@ __global__ void __launch_bounds__(384, 1)
           tc_wait_st();
         }
         // pass 2: p = 2^(s*scale - m_ref), row sum, bf16 P into shared memory
-        const float scl = fs.scale_log2, neg_m = -m_ref;
+        // (again with the next chunk's TMEM load overlapping this chunk's math)
+        const float scl = fs.scale_log2;
+        const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;   // a row with no visible key yet: p = 0
         float sum_a = 0.f, sum_b = 0.f;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tmem_ld32(s_tmem + c * 32, r);
+        {
+          uint32_t ra[32], rb[32];
+          tmem_ld32(s_tmem, ra);
           tc_wait_ld();
-          if (need_mask) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (j * 128 + c * 32 + i > qpos) r[i] = __float_as_uint(-INFINITY);
-          }
-          uint32_t pk[16];
-          if (need_mask) {   // masked keys must give exactly 0: MUFU path only
+          for (int c = 0; c < 4; ++c) {
+            uint32_t(&r)[32] = (c & 1) ? rb : ra;
+            uint32_t(&nxt)[32] = (c & 1) ? ra : rb;
+            if (c + 1 < 4) tmem_ld32(s_tmem + (c + 1) * 32, nxt);
+            if (need_mask) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              float x0, x1;
-              fma2(x0, x1, __uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), scl, scl, neg_m, neg_m);
-              const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-              add2(sum_a, sum_b, p0, p1);
-              pk[i] = pack_bf16x2(p0, p1);
+              for (int i = 0; i < 32; ++i)
+                if (j * 128 + c * 32 + i > qpos || j * 128 + c * 32 + i < lo) r[i] = __float_as_uint(-INFINITY);
             }
-          } else {           // 6 of every 16 pairs on the FMA pipe, the rest on MUFU
+            uint32_t pk[16];
+            if (need_mask) {   // masked keys must give exactly 0: MUFU path only
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              float x0, x1, p0, p1;
-              fma2(x0, x1, __uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), scl, scl, neg_m, neg_m);
-              if ((i & 7) < 3) {
-                exp2_poly2(x0, x1, p0, p1);
-              } else {
-                p0 = ex2_approx(x0);
-                p1 = ex2_approx(x1);
+              for (int i = 0; i < 16; ++i) {
+                float x0, x1;
+                fma2(x0, x1, __uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), scl, scl, neg_m, neg_m);
+                const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                add2(sum_a, sum_b, p0, p1);
+                pk[i] = pack_bf16x2(p0, p1);
               }
-              add2(sum_a, sum_b, p0, p1);
-              pk[i] = pack_bf16x2(p0, p1);
-            }
-          }
-          // chunk c covers keys 32c..32c+31: slab c/2, 16-byte pieces (c%2)*4 .. +3
-          uint8_t* slab = p_smem + (c >> 1) * C::TILE_BYTES + row * 128;
+            } else {           // 6 of every 16 pairs on the FMA pipe, the rest on MUFU
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int piece = (c & 1) * 4 + q;
-            *reinterpret_cast<uint4*>(slab + ((piece ^ (row & 7)) << 4)) =
-                make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+              for (int i = 0; i < 16; ++i) {
+                float x0, x1, p0, p1;
+                fma2(x0, x1, __uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), scl, scl, neg_m, neg_m);
+                if ((i & 7) < 3) {
+                  exp2_poly2(x0, x1, p0, p1);
+                } else {
+                  p0 = ex2_approx(x0);
+                  p1 = ex2_approx(x1);
+                }
+                add2(sum_a, sum_b, p0, p1);
+                pk[i] = pack_bf16x2(p0, p1);
+              }
+            }
+            // chunk c covers keys 32c..32c+31: slab c/2, 16-byte pieces (c%2)*4 .. +3
+            uint8_t* slab = p_smem + (c >> 1) * C::TILE_BYTES + row * 128;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int piece = (c & 1) * 4 + q;
+              *reinterpret_cast<uint4*>(slab + ((piece ^ (row & 7)) << 4)) =
+                  make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+            }
+            if (c + 1 < 4) tc_wait_ld();
           }
         }
         const float sum = sum_a + sum_b;

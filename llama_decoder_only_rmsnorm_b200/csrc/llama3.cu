@@ -16,6 +16,7 @@
 #include "common.cuh"
 #include "decode_attention.cuh"
 #include "flash_attention.cuh"
+#include "flash_attention2.cuh"
 #include "simt.cuh"
 #include "tc_gemm.cuh"
 #include "tc_gemm_pair.cuh"
@@ -88,6 +89,10 @@ void timer_end(int kind, cudaStream_t st) {
 // that predecessor (griddepcontrol.wait) after its own set-up and before it
 // touches memory.  g_pdl = false launches them the ordinary way.
 bool g_pdl = true;
+
+// Prefill attention kernel design: 1 = one softmax thread per query row, P
+// through shared memory; 2 = two softmax threads per row, P kept in TMEM.
+int g_flash_variant = 1;
 
 template <typename... KArgs, typename... Args>
 cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
@@ -219,10 +224,10 @@ bool flash_attention_supported(int hd, int H, int KV) {
   return hd == 64 || hd == 96 || hd == 128;
 }
 
-template <int HD>
+template <int HD, int VARIANT>
 int run_flash_attention_t(int H, int KV, const void* q, const void* kc, const void* vc, int cap, int B, int S,
-                          int P, void* out, int sms, unsigned long long wns, cudaStream_t st) {
-  using Cfg = FlashCfg<HD>;
+                          int P, void* out, const int32_t* doc_start, int sms, unsigned long long wns,
+                          cudaStream_t st) {
   CUtensorMap mq, mk, mv;
   const long long e = 2;
   L3_TRY(make_map_4d(&mq, q, HD, H, S, B, HD * e, (long long)H * HD * e, (long long)S * H * HD * e));
@@ -236,25 +241,38 @@ int run_flash_attention_t(int H, int KV, const void* q, const void* kc, const vo
   fs.units = B * KV * fs.pairs * fs.qtiles;
   fs.ldo = H * HD;
   fs.scale_log2 = (float)(1.4426950408889634 / sqrt((double)HD));
-  auto kern = flash_attention_kernel<HD>;
+  fs.doc_start = doc_start;
+  constexpr int smem = VARIANT == 2 ? Flash2Cfg<HD>::SMEM_BYTES : FlashCfg<HD>::SMEM_BYTES;
+  constexpr int threads = VARIANT == 2 ? 640 : 384;
+  auto kern = VARIANT == 2 ? flash_attention2_kernel<HD> : flash_attention_kernel<HD>;
   int dev = 0;
   L3_TRY(current_device(&dev));
   static bool attr_done[kMaxDevices];
   if (!attr_done[dev]) {
-    L3_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES));
+    L3_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
     attr_done[dev] = true;
   }
   const int grid = std::min(fs.units, sms);
-  L3_LAUNCH(LLAMA3_KERNEL_ATTENTION, st, launch_k(kern, grid, 384, Cfg::SMEM_BYTES, st, mq, mk, mv, (bf16*)out, fs, wns));
+  L3_LAUNCH(LLAMA3_KERNEL_ATTENTION, st, launch_k(kern, grid, threads, smem, st, mq, mk, mv, (bf16*)out, fs, wns));
   return launch_check();
 }
 
+template <int HD>
+int run_flash_attention_v(int H, int KV, const void* q, const void* kc, const void* vc, int cap, int B, int S,
+                          int P, void* out, const int32_t* doc_start, int sms, unsigned long long wns,
+                          cudaStream_t st) {
+  if (g_flash_variant == 2)
+    return run_flash_attention_t<HD, 2>(H, KV, q, kc, vc, cap, B, S, P, out, doc_start, sms, wns, st);
+  return run_flash_attention_t<HD, 1>(H, KV, q, kc, vc, cap, B, S, P, out, doc_start, sms, wns, st);
+}
+
 int run_flash_attention(int hd, int H, int KV, const void* q, const void* kc, const void* vc, int cap, int B, int S,
-                        int P, void* out, int sms, unsigned long long wns, cudaStream_t st) {
+                        int P, void* out, const int32_t* doc_start, int sms, unsigned long long wns,
+                        cudaStream_t st) {
   switch (hd) {
-    case 64: return run_flash_attention_t<64>(H, KV, q, kc, vc, cap, B, S, P, out, sms, wns, st);
-    case 96: return run_flash_attention_t<96>(H, KV, q, kc, vc, cap, B, S, P, out, sms, wns, st);
-    case 128: return run_flash_attention_t<128>(H, KV, q, kc, vc, cap, B, S, P, out, sms, wns, st);
+    case 64: return run_flash_attention_v<64>(H, KV, q, kc, vc, cap, B, S, P, out, doc_start, sms, wns, st);
+    case 96: return run_flash_attention_v<96>(H, KV, q, kc, vc, cap, B, S, P, out, doc_start, sms, wns, st);
+    case 128: return run_flash_attention_v<128>(H, KV, q, kc, vc, cap, B, S, P, out, doc_start, sms, wns, st);
     default: return LLAMA3_ERR_UNSUPPORTED;
   }
 }
@@ -481,12 +499,12 @@ int rmsnorm_any(const llama3_config* c, const void* x, long long row_stride, con
 
 template <typename T>
 int run_attention_simt(const llama3_config* c, const void* q, const void* kc, const void* vc, int cap, int B,
-                       int S, int P, void* out, cudaStream_t st) {
+                       int S, int P, void* out, const int32_t* doc_start, cudaStream_t st) {
   const long long warps = (long long)B * S * c->n_heads;
   const float scale = (float)(1.0 / sqrt((double)c->head_dim));
   L3_LAUNCH(LLAMA3_KERNEL_ATTENTION, st, launch_k((attention_simt_kernel<T>), blocks_for(warps * 32, 256), 256, 0, st, 
       (const T*)q, (const T*)kc, (const T*)vc, (T*)out, B, S, P, c->n_heads, c->n_kv_heads, c->head_dim, cap,
-      scale));
+      scale, doc_start));
   return launch_check();
 }
 
@@ -504,7 +522,9 @@ int run_decode_attention_tc_t(const llama3_config* c, const void* q, const void*
   DecodeShape ds;
   ds.B = B; ds.H = H; ds.KV = KV; ds.nrep = H / KV; ds.n_keys = n_keys;
   ds.tiles = (n_keys + 127) / 128;
-  // split count minimising the longest per-CTA stream on a persistent grid
+  // Split count minimising the longest per-CTA stream on a persistent grid,
+  // counting one tile of fixed cost per work unit (Q load, per-warpgroup
+  // epilogue, partial records for the combine kernel); ties go to fewer splits.
   const int sms = num_sms();
   int best = 1;
   long long best_t = -1;
@@ -512,7 +532,7 @@ int run_decode_attention_tc_t(const llama3_config* c, const void* q, const void*
     const int per = (ds.tiles + sp - 1) / sp;
     const int real = (ds.tiles + per - 1) / per;
     const long long units = (long long)B * KV * real;
-    const long long t = ((units + sms - 1) / sms) * per;
+    const long long t = ((units + sms - 1) / sms) * (per + 1);
     if (best_t < 0 || t < best_t) { best_t = t; best = real; }
   }
   ds.tiles_per_split = (ds.tiles + best - 1) / best;
@@ -554,8 +574,8 @@ bool decode_attention_tc_supported(const llama3_config* c) {
 }
 
 int attention_dispatch(const llama3_config* c, const void* q, const void* kc, const void* vc, int cap, int B,
-                       int S, int P, void* out, float* part, cudaStream_t st) {
-  if (S == 1 && decode_attention_tc_supported(c)) {
+                       int S, int P, void* out, float* part, cudaStream_t st, const int32_t* doc_start = nullptr) {
+  if (S == 1 && !doc_start && decode_attention_tc_supported(c)) {
     switch (c->head_dim) {
       case 64: return run_decode_attention_tc_hd<64>(c, q, kc, vc, cap, B, P + 1, out, part, st);
       case 96: return run_decode_attention_tc_hd<96>(c, q, kc, vc, cap, B, P + 1, out, part, st);
@@ -563,10 +583,10 @@ int attention_dispatch(const llama3_config* c, const void* q, const void* kc, co
     }
   }
   if (use_tc(c) && flash_attention_supported(c->head_dim, c->n_heads, c->n_kv_heads))
-    return run_flash_attention(c->head_dim, c->n_heads, c->n_kv_heads, q, kc, vc, cap, B, S, P, out, num_sms(),
-                               wait_ns(), st);
-  return c->dtype == LLAMA3_DTYPE_F32 ? run_attention_simt<float>(c, q, kc, vc, cap, B, S, P, out, st)
-                                      : run_attention_simt<bf16>(c, q, kc, vc, cap, B, S, P, out, st);
+    return run_flash_attention(c->head_dim, c->n_heads, c->n_kv_heads, q, kc, vc, cap, B, S, P, out, doc_start,
+                               num_sms(), wait_ns(), st);
+  return c->dtype == LLAMA3_DTYPE_F32 ? run_attention_simt<float>(c, q, kc, vc, cap, B, S, P, out, doc_start, st)
+                                      : run_attention_simt<bf16>(c, q, kc, vc, cap, B, S, P, out, doc_start, st);
 }
 
 // ---------------------------------------------------------------------------
@@ -574,7 +594,8 @@ int attention_dispatch(const llama3_config* c, const void* q, const void* kc, co
 // ---------------------------------------------------------------------------
 template <typename T>
 int layer_simt(const llama3_config* c, const llama3_layer_weights* w, const float* rope, void* x, void* kc,
-               void* vc, int cap, int B, int S, int P, const Workspace& L, void* ws, cudaStream_t st) {
+               void* vc, int cap, int B, int S, int P, const Workspace& L, void* ws, cudaStream_t st,
+               const int32_t* doc_start = nullptr) {
   const int M = B * S, D = c->dim, H = c->n_heads, KV = c->n_kv_heads, hd = c->head_dim, F = c->ffn_hidden;
   const int nqkv = (H + 2 * KV) * hd;
   T* xn = ws_at<T>(ws, L.xn);
@@ -588,7 +609,7 @@ int layer_simt(const llama3_config* c, const llama3_layer_weights* w, const floa
   L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_qkv_rope_kernel<T>), blocks_for((long long)M * nqkv / 4, 256), 256, 0, st, 
       Pp, 1, 0, M, S, P, H, KV, hd, rope, q, (T*)kc, (T*)vc, cap));
   L3_TRY(launch_check());
-  L3_TRY(attention_dispatch(c, q, kc, vc, cap, B, S, P, o, Ap, st));
+  L3_TRY(attention_dispatch(c, q, kc, vc, cap, B, S, P, o, Ap, st, doc_start));
   L3_TRY(simt_gemm<T>(LLAMA3_KERNEL_GEMM_WO, o, w->wo, Pp, M, D, H * hd, D, st));
   L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_residual_kernel<T>), blocks_for((long long)M * D / 4, 256), 256, 0, st, Pp, 1, 0, D, (const T*)x, (T*)x, M, D));
   L3_TRY(launch_check());
@@ -606,7 +627,8 @@ int layer_simt(const llama3_config* c, const llama3_layer_weights* w, const floa
 // Layer: tcgen05 prefill path (bf16)
 // ---------------------------------------------------------------------------
 int layer_tc_prefill(const llama3_config* c, const llama3_layer_weights* w, const float* rope, void* x, void* kc,
-                     void* vc, int cap, int B, int S, int P, const Workspace& L, void* ws, cudaStream_t st) {
+                     void* vc, int cap, int B, int S, int P, const Workspace& L, void* ws, cudaStream_t st,
+                     const int32_t* doc_start = nullptr) {
   const int M = B * S, D = c->dim, H = c->n_heads, KV = c->n_kv_heads, hd = c->head_dim, F = c->ffn_hidden;
   const int nqkv = (H + 2 * KV) * hd;
   bf16* xn = ws_at<bf16>(ws, L.xn);
@@ -641,7 +663,7 @@ int layer_tc_prefill(const llama3_config* c, const llama3_layer_weights* w, cons
       L3_TRY((launch_gemm<kPrefillBN, 4, EPI_QKV_ROPE, false>(LLAMA3_KERNEL_GEMM_QKV, mxn, mxn, mwqkv, mwqkv,
                                                                make_shape(M, 0, nqkv, D, kPrefillBN, 1), ep, st)));
   }
-  L3_TRY(attention_dispatch(c, q, kc, vc, cap, B, S, P, o, Ap, st));
+  L3_TRY(attention_dispatch(c, q, kc, vc, cap, B, S, P, o, Ap, st, doc_start));
   {
     EpiParams ep = empty_epi();
     ep.out = x; ep.res = x; ep.ldo = D;
@@ -700,10 +722,30 @@ int layer_tc_decode(const llama3_config* c, const llama3_layer_weights* w, const
   L3_TRY(launch_check());
   L3_TRY(attention_dispatch(c, q, kc, vc, cap, B, 1, P, o, Ap, st));
   L3_TRY(swapped_partial_gemm(w->wo, D, nullptr, 0, 0, o, M, H * hd, Pp, D, &splits, st));
-  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_residual_kernel<bf16>), blocks_for((long long)M * D / 4, 256), 256, 0, st, 
-      Pp, splits, (long long)M * D, D, (const bf16*)x, (bf16*)x, M, D));
-  L3_TRY(launch_check());
-  L3_TRY(rmsnorm_any(c, x, D, w->ffn_norm, xn, M, st));
+  // h = x + o Wo^T and hn = RMSNorm(h) in one pass over each row
+  if (D <= 8 * 4 * 256) {
+    const int G = (D + 1023) / 1024;
+    const long long sstride = (long long)M * D;
+    if (G <= 1)
+      L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_residual_rmsnorm_kernel<1>), M, 256, 0, st, Pp, splits,
+                                                        sstride, (bf16*)x, (const bf16*)w->ffn_norm, xn, D, c->norm_eps));
+    else if (G <= 2)
+      L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_residual_rmsnorm_kernel<2>), M, 256, 0, st, Pp, splits,
+                                                        sstride, (bf16*)x, (const bf16*)w->ffn_norm, xn, D, c->norm_eps));
+    else if (G <= 4)
+      L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_residual_rmsnorm_kernel<4>), M, 256, 0, st, Pp, splits,
+                                                        sstride, (bf16*)x, (const bf16*)w->ffn_norm, xn, D, c->norm_eps));
+    else
+      L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_residual_rmsnorm_kernel<8>), M, 256, 0, st, Pp, splits,
+                                                        sstride, (bf16*)x, (const bf16*)w->ffn_norm, xn, D, c->norm_eps));
+    L3_TRY(launch_check());
+  } else {
+    L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_residual_kernel<bf16>), blocks_for((long long)M * D / 4, 256),
+                                                      256, 0, st, Pp, splits, (long long)M * D, D, (const bf16*)x,
+                                                      (bf16*)x, M, D));
+    L3_TRY(launch_check());
+    L3_TRY(rmsnorm_any(c, x, D, w->ffn_norm, xn, M, st));
+  }
   L3_TRY(swapped_partial_gemm(w->w1, F, w->w3, F, F, xn, M, D, Pp, 2 * F, &splits, st));
   L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_swiglu_kernel<bf16>), blocks_for((long long)M * F / 4, 256), 256, 0, st, Pp, splits, (long long)M * 2 * F, g,
                                                                                 M, F));
@@ -777,6 +819,12 @@ unsigned long long llama3_launch_count(void) { return g_launches.load(); }
 int llama3_set_kernel_path(int path) {
   int old = g_kernel_path;
   g_kernel_path = (path >= 0 && path <= 2) ? path : 0;
+  return old;
+}
+
+int llama3_set_flash_variant(int variant) {
+  const int old = g_flash_variant;
+  g_flash_variant = (variant == 2) ? 2 : 1;
   return old;
 }
 
@@ -933,6 +981,41 @@ int llama3_layer_decode(const llama3_config* cfg, const llama3_layer_weights* w,
   if (cfg->dtype == LLAMA3_DTYPE_F32)
     return layer_simt<float>(cfg, w, rope, x, k_cache, v_cache, cache_cap, batch, 1, start_pos, L, ws, st);
   return layer_simt<bf16>(cfg, w, rope, x, k_cache, v_cache, cache_cap, batch, 1, start_pos, L, ws, st);
+}
+
+int llama3_layer_forward_docs(const llama3_config* cfg, const llama3_layer_weights* w, const float* rope,
+                              int rope_len, void* x, void* k_cache, void* v_cache, int cache_cap, int batch, int seq,
+                              int start_pos, const int32_t* doc_start, void* ws, size_t ws_bytes,
+                              llama3_stream_t stream) {
+  Workspace L;
+  L3_TRY(check_layer_args(cfg, w, rope, rope_len, x, k_cache, v_cache, cache_cap, batch, seq, start_pos, ws,
+                          ws_bytes, &L));
+  if (!doc_start) return LLAMA3_ERR_ARG;
+  if (!aligned16(doc_start)) return LLAMA3_ERR_ALIGN;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (use_tc(cfg))
+    return layer_tc_prefill(cfg, w, rope, x, k_cache, v_cache, cache_cap, batch, seq, start_pos, L, ws, st,
+                            doc_start);
+  if (cfg->dtype == LLAMA3_DTYPE_F32)
+    return layer_simt<float>(cfg, w, rope, x, k_cache, v_cache, cache_cap, batch, seq, start_pos, L, ws, st,
+                             doc_start);
+  return layer_simt<bf16>(cfg, w, rope, x, k_cache, v_cache, cache_cap, batch, seq, start_pos, L, ws, st,
+                          doc_start);
+}
+
+int llama3_attention_docs(const llama3_config* cfg, const void* q, const void* k_cache, const void* v_cache,
+                          int cache_cap, int batch, int seq, int start_pos, const int32_t* doc_start, void* out,
+                          void* ws, size_t ws_bytes, llama3_stream_t stream) {
+  L3_TRY(check_config(cfg));
+  if (!q || !k_cache || !v_cache || !out || !doc_start || batch < 1 || seq < 1 || start_pos < 0)
+    return LLAMA3_ERR_ARG;
+  if ((long long)start_pos + seq > cache_cap) return LLAMA3_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) || !aligned16(doc_start))
+    return LLAMA3_ERR_ALIGN;
+  Workspace L = layout(cfg, batch, seq, 1);
+  if (!ws || ws_bytes < L.total) return LLAMA3_ERR_WORKSPACE;
+  return attention_dispatch(cfg, q, k_cache, v_cache, cache_cap, batch, seq, start_pos, out,
+                            ws_at<float>(ws, L.attn_part), (cudaStream_t)stream, doc_start);
 }
 
 int llama3_lm_head_argmax(const llama3_config* cfg, const void* norm_w, const void* w_out, const void* h, int rows,

@@ -196,6 +196,57 @@ __global__ void epi_residual_kernel(const float* __restrict__ P, int splits, lon
   store4(out + i, v);
 }
 
+// Residual add fused with the RMSNorm that follows it (decode, few rows):
+//   x[m] <- round(x[m] + sum_s P[s][m]);  xn[m] = round(x[m] * r * w),
+//   r = 1 / sqrt(mean(x[m]^2) + eps) over the rounded x ("Build your own
+// Llama 3 from scratch" §3.6 residual, §3.1 RMSNorm).  One CTA of 256 threads
+// per row, 4*G consecutive-by-4 elements per thread held in registers.
+template <int G>
+__global__ void __launch_bounds__(256) epi_residual_rmsnorm_kernel(const float* __restrict__ P, int splits,
+                                                                  long long split_stride, bf16* __restrict__ x,
+                                                                  const bf16* __restrict__ w,
+                                                                  bf16* __restrict__ xn, int D, float eps) {
+  griddep_wait_and_release();
+  const int m = blockIdx.x;
+  float v[G][4];
+  float ss = 0.f;
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const int n = 4 * (threadIdx.x + 256 * g);
+    if (n < D) {
+      float r[4];
+      sum4_splits(P, splits, split_stride, (long long)m * D + n, v[g]);
+      load4(x + (size_t)m * D + n, r);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        // round to bf16 exactly as the stored residual stream, then square that
+        v[g][q] = __bfloat162float(__float2bfloat16_rn(v[g][q] + r[q]));
+        ss = fmaf(v[g][q], v[g][q], ss);
+      }
+      store4(x + (size_t)m * D + n, v[g]);
+    }
+  }
+  __shared__ float red[8];
+  ss = warp_sum(ss);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  float tot = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) tot += red[i];
+  const float rs = rsqrtf(tot / (float)D + eps);
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const int n = 4 * (threadIdx.x + 256 * g);
+    if (n < D) {
+      float wv[4], o[4];
+      load4(w + n, wv);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) o[q] = v[g][q] * rs * wv[q];
+      store4(xn + (size_t)m * D + n, o);
+    }
+  }
+}
+
 // g[m, f] = silu(P[m, f]) * P[m, F + f],  silu(z) = z / (1 + e^-z)
 // ("Build your own Llama 3 from scratch" §3.5)
 template <typename T>
@@ -257,7 +308,7 @@ template <typename T>
 __global__ void attention_simt_kernel(const T* __restrict__ q, const T* __restrict__ k_cache,
                                       const T* __restrict__ v_cache, T* __restrict__ out, int B,
                                       int S, int start_pos, int H, int KV, int hd, int cap,
-                                      float scale) {
+                                      float scale, const int32_t* __restrict__ doc_start) {
   griddep_wait_and_release();
   long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   int lane = threadIdx.x & 31;
@@ -274,8 +325,10 @@ __global__ void attention_simt_kernel(const T* __restrict__ q, const T* __restri
     acc[i] = 0.f;
   }
   float m = -INFINITY, l = 0.f;
-  int last = start_pos + t;
-  for (int j = 0; j <= last; ++j) {
+  const int last = start_pos + t;
+  // document mask: keys before the start of this token's document are invisible
+  const int first = doc_start ? max(0, min(doc_start[(size_t)b * S + t], last)) : 0;
+  for (int j = first; j <= last; ++j) {
     const T* kr = k_cache + (((size_t)b * cap + j) * KV + g) * hd;
     const T* vr = v_cache + (((size_t)b * cap + j) * KV + g) * hd;
     float s = 0.f;

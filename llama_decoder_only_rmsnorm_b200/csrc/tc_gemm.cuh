@@ -279,7 +279,12 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  griddep_wait_and_release();
+  // In the swapped launches A is a weight matrix, which no earlier kernel
+  // writes: the producer starts streaming it before waiting for the previous
+  // kernel (programmatic launch) and waits only before loading B.  Every other
+  // thread waits here, before its first global access.
+  constexpr bool kEarlyA = (EPI == EPI_PARTIAL || EPI == EPI_ARGMAX);
+  if (!(kEarlyA && warp == 0)) griddep_wait_and_release();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -288,14 +293,40 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t phase = 0;
       uint32_t issued_mask = 0, issued_parity = 0;
       bool ok = true;
+      int pre = 0;   // k-blocks of the first unit whose A tile went out before the dependency wait
+      if constexpr (kEarlyA) {
+        if ((int)blockIdx.x < sh.units) {
+          int split, mt, nt;
+          gemm_unit(sh, blockIdx.x, split, mt, nt);
+          const bool second = mt >= sh.tiles_m1;
+          const int arow = (second ? mt - sh.tiles_m1 : mt) * C::BM;
+          const int kb0 = split * sh.kb_per_split;
+          pre = min(STAGES, min(kb0 + sh.kb_per_split, sh.kblocks) - kb0);
+          for (int i = 0; i < pre; ++i) {   // fresh ring: these stages are free
+            mbar_arrive_expect_tx(&full[i], C::STAGE_BYTES);
+            tma_load_2d(sA + i * C::A_BYTES, second ? &mapA2 : &mapA, &full[i], (kb0 + i) * C::BK, arow);
+          }
+          griddep_wait_and_release();
+          for (int i = 0; i < pre; ++i) {
+            tma_load_2d(sB + (i * C::NB) * C::B_BYTES, &mapB, &full[i], (kb0 + i) * C::BK, nt * BN);
+            if constexpr (DUAL)
+              tma_load_2d(sB + (i * C::NB + 1) * C::B_BYTES, &mapB2, &full[i], (kb0 + i) * C::BK, nt * BN);
+            issued_mask |= 1u << i;
+          }
+          stage = pre % STAGES;
+          phase = pre == STAGES ? 1u : 0u;
+        } else {
+          griddep_wait_and_release();
+        }
+      }
       for (int u = blockIdx.x; u < sh.units && ok; u += gridDim.x) {
         int split, mt, nt;
         gemm_unit(sh, u, split, mt, nt);
         const bool second = mt >= sh.tiles_m1;
         const CUtensorMap* ma = second ? &mapA2 : &mapA;
         const int arow = (second ? mt - sh.tiles_m1 : mt) * C::BM;
-        const int kb0 = split * sh.kb_per_split;
-        const int kb1 = min(kb0 + sh.kb_per_split, sh.kblocks);
+        const int kb0 = split * sh.kb_per_split + (u == (int)blockIdx.x ? pre : 0);
+        const int kb1 = min(split * sh.kb_per_split + sh.kb_per_split, sh.kblocks);
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, wait_ns)) { ok = false; break; }
           mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);

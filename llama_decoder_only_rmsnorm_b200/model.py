@@ -59,3 +59,37 @@ class Llama3Stack:
         B.llama3_lm_head_argmax(self.cfg, self.out["norm"], self.out["output"], h, rows, row_stride,
                                 self.ids_out, logits, self.ws, self.ws_bytes, stream)
         return self.ids_out[:rows]
+
+    # -- greedy generation ("Build your own Llama 3 from scratch" 六, temperature 0)
+    def generate(self, prompt_ids, n_new, eos_id=None, stream=None):
+        """Prefill the prompts (int32 [batch, S] on the device), then decode
+        n_new tokens greedily.  Each step's LM head writes its argmax straight
+        into row `step` of a [n_new, batch] device buffer, which the next
+        step's embedding reads, so no token leaves the device in the loop.
+        Returns the [batch, n_new] tokens as a host array; after a sequence's
+        first eos_id the rest of its row is eos_id (the pages stop the loop
+        there)."""
+        import torch
+        Bn, S = prompt_ids.shape
+        assert Bn == self.batch and S + n_new - 1 <= self.cache_cap
+        D = self.cfg_dict["dim"]
+        x = torch.empty((Bn, S, D), dtype=self.dtype, device=self.device)
+        self.embed(prompt_ids, x, stream)
+        self.forward_layers(x, S, 0, stream)
+        row = (Bn + 3) // 4 * 4            # keeps every step's ids 16-byte aligned
+        out = torch.empty((n_new, row), dtype=torch.int32, device=self.device)
+        B.llama3_lm_head_argmax(self.cfg, self.out["norm"], self.out["output"], x[:, -1], Bn, S * D, out[0], None,
+                                self.ws, self.ws_bytes, stream)
+        xd = torch.empty((Bn, 1, D), dtype=self.dtype, device=self.device)
+        for step in range(1, n_new):
+            B.llama3_embed(self.cfg, out[step - 1], self.out["tok_embeddings"], xd, Bn, stream)
+            self.decode_layers(xd, S + step - 1, stream)
+            B.llama3_lm_head_argmax(self.cfg, self.out["norm"], self.out["output"], xd, Bn, D, out[step], None,
+                                    self.ws, self.ws_bytes, stream)
+        toks = out[:, :Bn].t().cpu().numpy()
+        if eos_id is not None:   # host-side: hold the end token once emitted
+            for b in range(Bn):
+                hits = (toks[b] == eos_id).nonzero()[0]
+                if hits.size:
+                    toks[b, hits[0]:] = eos_id
+        return toks

@@ -41,6 +41,7 @@ __all__ = [
     "rms_norm", "ffn_hidden_dim", "rope_inverse_frequencies", "rope_angles",
     "apply_rope", "causal_mask", "gqa_attention", "silu", "swiglu_ffn",
     "decoder_block", "decoder_block_rows", "lm_head", "embed", "forward_stack",
+    "generate_greedy",
 ]
 
 
@@ -109,14 +110,22 @@ def apply_rope(x, positions, theta):
 # ---------------------------------------------------------------------------
 # Causal grouped-query attention  ([S1] §6.11-8; [S2] §3.4; [S4] GQA)
 # ---------------------------------------------------------------------------
-def causal_mask(n_queries, n_keys, start_pos=0):
-    """Additive mask: 0 where key j <= start_pos + t, -inf above ([S1] §7.1)."""
+def causal_mask(n_queries, n_keys, start_pos=0, doc_start=None):
+    """Additive mask: 0 where key j <= start_pos + t, -inf above ([S1] §7.1).
+
+    With ``doc_start`` (one position per query: where that query's document
+    begins) keys before it are masked too -- the document-level mask that
+    keeps packed documents from attending to each other ([S2] 附 1).
+    """
     t = np.arange(n_queries)[:, None] + start_pos
     j = np.arange(n_keys)[None, :]
-    return np.where(j <= t, 0.0, -np.inf)
+    ok = j <= t
+    if doc_start is not None:
+        ok &= j >= np.asarray(doc_start)[:, None]
+    return np.where(ok, 0.0, -np.inf)
 
 
-def gqa_attention(q, k, v, start_pos=0, return_probs=False):
+def gqa_attention(q, k, v, start_pos=0, return_probs=False, doc_start=None):
     """softmax(q k^T / sqrt(hd) + mask) v for one sequence.
 
     q: [S, H, hd] (rotated); k, v: [T, KV, hd] with T = start_pos + S.
@@ -128,7 +137,7 @@ def gqa_attention(q, k, v, start_pos=0, return_probs=False):
     T, KV, _ = k.shape
     assert H % KV == 0 and T == start_pos + S
     n_rep = H // KV
-    mask = causal_mask(S, T, start_pos)
+    mask = causal_mask(S, T, start_pos, doc_start)
     out = np.empty((S, H, hd))
     probs = np.empty((H, S, T)) if return_probs else None
     for h in range(H):
@@ -160,14 +169,16 @@ def swiglu_ffn(x, w1, w2, w3):
 # ---------------------------------------------------------------------------
 # One pre-norm decoder block  ([S2] §3.6 TransformerBlock; [S1] §6-10)
 # ---------------------------------------------------------------------------
-def decoder_block(x, layer, cfg, k_cache, v_cache, start_pos=0):
+def decoder_block(x, layer, cfg, k_cache, v_cache, start_pos=0, doc_start=None):
     """h = x + Attn(RMSNorm(x)); out = h + FFN(RMSNorm(h)).
 
     x: [B, S, D].  ``layer`` maps the page's weight names (attention_norm, wq,
     wk, wv, wo, ffn_norm, w1, w2, w3) to arrays in [out, in] layout.
     k_cache / v_cache: fp64 arrays [B, cap, KV, hd]; positions
     [start_pos, start_pos+S) are overwritten with this call's rotated k and v
-    ([S2] §3.3 / §3.4 inference branch).  Returns out [B, S, D].
+    ([S2] §3.3 / §3.4 inference branch).  ``doc_start`` [B, S] (optional):
+    the position where each token's document begins (document mask).
+    Returns out [B, S, D].
     """
     x = _f64(x)
     B, S, D = x.shape
@@ -186,8 +197,8 @@ def decoder_block(x, layer, cfg, k_cache, v_cache, start_pos=0):
 
     o = np.empty((B, S, H, hd))
     for b in range(B):
-        o[b] = gqa_attention(q[b], k_cache[b, :start_pos + S],
-                             v_cache[b, :start_pos + S], start_pos)
+        o[b] = gqa_attention(q[b], k_cache[b, :start_pos + S], v_cache[b, :start_pos + S], start_pos,
+                             doc_start=None if doc_start is None else np.asarray(doc_start)[b])
     h = x + o.reshape(B, S, H * hd) @ _f64(layer["wo"]).T
     hn = rms_norm(h, layer["ffn_norm"], eps)
     return h + swiglu_ffn(hn, layer["w1"], layer["w2"], layer["w3"])
@@ -249,7 +260,7 @@ def embed(ids, table):
 
 
 def forward_stack(x, layers, cfg, k_caches=None, v_caches=None, start_pos=0,
-                  cache_len=None):
+                  cache_len=None, doc_start=None):
     """Run x through every block in ``layers`` (the layer loop of [S2] 四).
 
     Creates fp64 caches of length ``cache_len`` (default start_pos+S) when none
@@ -263,5 +274,40 @@ def forward_stack(x, layers, cfg, k_caches=None, v_caches=None, start_pos=0,
         k_caches = [np.zeros((B, cap, KV, hd)) for _ in layers]
         v_caches = [np.zeros((B, cap, KV, hd)) for _ in layers]
     for layer, kc, vc in zip(layers, k_caches, v_caches):
-        x = decoder_block(x, layer, cfg, kc, vc, start_pos)
+        x = decoder_block(x, layer, cfg, kc, vc, start_pos, doc_start)
     return x, k_caches, v_caches
+
+
+# ---------------------------------------------------------------------------
+# Greedy generation  ([S2] 六 generate with temperature 0: argmax of the last
+# position's logits, fed back one token per step through the KV cache)
+# ---------------------------------------------------------------------------
+def generate_greedy(prompt_ids, table, layers, norm_weight, w_out, cfg, n_new, eos_id=None):
+    """Greedy continuation of every prompt (all the same length).
+
+    Prefills the prompts, then for each new token: embed it, run one cached
+    decode step at the next position, take the argmax of the final-norm LM
+    head.  Returns (tokens [B, n_new], gaps [B, n_new]) where gaps are the
+    top-2 logit differences of each decision.  After a sequence emits eos_id
+    its later tokens are eos_id as well (the page stops the loop there).
+    """
+    ids = np.asarray(prompt_ids)
+    B, S = ids.shape
+    cap = S + n_new
+    h, kc, vc = forward_stack(embed(ids, table), layers, cfg, cache_len=cap)
+    logits, nxt = lm_head(h[:, -1], norm_weight, w_out, cfg["norm_eps"])
+    toks = np.zeros((B, n_new), dtype=np.int64)
+    gaps = np.zeros((B, n_new))
+    done = np.zeros(B, dtype=bool)
+    for step in range(n_new):
+        top2 = np.sort(logits, axis=1)[:, -2:]
+        gaps[:, step] = top2[:, 1] - top2[:, 0]
+        nxt = np.where(done, eos_id if eos_id is not None else nxt, nxt)
+        toks[:, step] = nxt
+        if eos_id is not None:
+            done |= nxt == eos_id
+        if step + 1 == n_new:
+            break
+        h, kc, vc = forward_stack(embed(nxt[:, None], table), layers, cfg, kc, vc, start_pos=S + step)
+        logits, nxt = lm_head(h[:, -1], norm_weight, w_out, cfg["norm_eps"])
+    return toks, gaps

@@ -19,7 +19,7 @@ def assert_close(gpu, oracle, dtype, what=""):
     atol, rtol = TOL[dtype]
     err = np.abs(g - o)
     bound = atol + rtol * np.abs(o)
-    bad = err > bound
+    bad = ~(err <= bound)   # a NaN on either side counts as out of tolerance
     if bad.any():
         i = np.unravel_index(np.argmax(err - bound), err.shape)
         raise AssertionError(f"{what}: {bad.sum()} of {bad.size} elements out of tolerance; worst at {i}: "

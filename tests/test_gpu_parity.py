@@ -21,8 +21,11 @@ def _gpu_state():
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
     B.llama3_set_kernel_path(0)
+    flash = B.llama3_set_flash_variant(1)
+    B.llama3_set_flash_variant(flash)
     yield
     B.llama3_set_kernel_path(0)
+    B.llama3_set_flash_variant(flash)
     torch.cuda.synchronize()
     assert B.llama3_device_status() == 0, "device status word set"
 
@@ -100,7 +103,11 @@ def _attn_case(Bn, S, P, H, KV, hd, seed):
     (1, 1, 0, 8, 2, 128), (4, 1, 1, 8, 1, 64), (3, 1, 1000, 32, 8, 128), (2, 1, 300, 8, 2, 96),
     (2, 1, 777, 16, 16, 64), (2, 1, 500, 12, 4, 64), (1, 150, 20, 12, 4, 64), (2, 1, 130, 16, 1, 128),
     (1, 1, 8192, 32, 8, 128), (2, 300, 0, 6, 2, 96)])
-def test_attention(Bn, S, P, H, KV, hd):
+@pytest.mark.parametrize("variant", [1, 2])
+def test_attention(Bn, S, P, H, KV, hd, variant):
+    if variant == 2 and S == 1:
+        pytest.skip("single-token steps take the decode kernel")
+    B.llama3_set_flash_variant(variant)
     q, kc, vc, cap = _attn_case(Bn, S, P, H, KV, hd, Bn * 1000 + S + P + hd)
     cfg = B.make_config(H * hd, H, KV, 1024)
     ws_bytes = B.llama3_workspace_size(cfg, Bn, S, 1)
@@ -263,3 +270,81 @@ def test_embed_out_of_range_id_is_reported():
     assert B.llama3_device_status() == 6
     assert torch.equal(x[1], outw["tok_embeddings"][5])
     assert torch.count_nonzero(x[2]) == 0
+
+
+def test_greedy_generation_matches_oracle():
+    """Prefill + greedy decode loop on the device vs the oracle's greedy
+    generation; tokens must agree at every step whose oracle top-2 gap exceeds
+    1e-2 (after an undecided step a sequence may legitimately diverge)."""
+    w = small_bf16(batch=3, seq=20, vocab=1000)
+    layers = [I.layer_weights(w, i, DEV, "random") for i in range(w.n_layers)]
+    outw = I.output_weights(w, DEV, "random")
+    n_new = 12
+    st = Llama3Stack(w.cfg(), layers, outw, w.batch, w.seq + n_new, w.seq, lm_rows=w.batch)
+    prompt = I.token_ids(w, DEV)
+    got = st.generate(prompt, n_new)
+    toks, gaps = O.generate_greedy(prompt.cpu().numpy(), f64(outw["tok_embeddings"]),
+                                   [oracle_layer(l) for l in layers], f64(outw["norm"]), f64(outw["output"]),
+                                   oracle_cfg(w), n_new)
+    compared = 0
+    for b in range(w.batch):
+        for t in range(n_new):
+            if gaps[b, t] <= 1e-2:
+                break
+            assert got[b, t] == toks[b, t], (b, t, got[b], toks[b])
+            compared += 1
+    assert compared >= n_new  # the check covered a real stretch of tokens
+
+
+# ------------------------------------------------------------ document mask
+def _doc_starts(Bn, S, P, seed):
+    """Per-token document start positions: random document lengths packed
+    after `P` already-cached positions of one document starting at 0."""
+    rng = np.random.default_rng(seed)
+    ds = np.zeros((Bn, S), dtype=np.int32)
+    for b in range(Bn):
+        start, t = 0, 0
+        while t < S:
+            n = int(rng.integers(1, max(2, S // 2)))
+            if t > 0 or P == 0:
+                start = P + t if t > 0 else 0
+            ds[b, t:t + n] = start
+            t += n
+    return ds
+
+
+@pytest.mark.parametrize("Bn,S,P,H,KV,hd,path", [
+    (2, 300, 0, 8, 2, 128, 0), (2, 200, 37, 8, 2, 64, 0), (1, 257, 0, 12, 4, 96, 0), (2, 130, 5, 8, 2, 64, 1)])
+@pytest.mark.parametrize("variant", [1, 2])
+def test_attention_document_mask(Bn, S, P, H, KV, hd, path, variant):
+    if variant == 2 and path != 0:
+        pytest.skip("the SIMT path has one attention kernel")
+    B.llama3_set_kernel_path(path)
+    B.llama3_set_flash_variant(variant)
+    q, kc, vc, cap = _attn_case(Bn, S, P, H, KV, hd, 77 + S + P)
+    ds = _doc_starts(Bn, S, P, S + hd)
+    cfg = B.make_config(H * hd, H, KV, 1024)
+    ws_bytes = B.llama3_workspace_size(cfg, Bn, S, 1)
+    ws = torch.empty((ws_bytes,), dtype=torch.uint8, device=DEV)
+    out = torch.empty((Bn, S, H * hd), dtype=torch.bfloat16, device=DEV)
+    B.llama3_attention_docs(cfg, q.to(DEV), kc.to(DEV), vc.to(DEV), cap, Bn, S, P, torch.from_numpy(ds).to(DEV), out,
+                            ws, ws_bytes)
+    for b in range(Bn):
+        want = O.gqa_attention(f64(q[b]), f64(kc[b, :P + S]), f64(vc[b, :P + S]), P, doc_start=ds[b])
+        assert_close(out[b], want.reshape(S, H * hd), "bf16", f"doc attention b={b}")
+
+
+def test_layer_forward_packed_documents():
+    w = small_bf16(n_layers=2, seq=150)
+    layers = [I.layer_weights(w, i, DEV, "random") for i in range(w.n_layers)]
+    st = Llama3Stack(w.cfg(), layers, I.output_weights(w, DEV), w.batch, w.seq, w.seq)
+    ds = _doc_starts(w.batch, w.seq, 0, 11)
+    dsd = torch.from_numpy(ds).to(DEV)
+    x = I.activations(w, DEV)
+    x0 = f64(x)
+    for i in range(w.n_layers):
+        kc, vc = st.caches[i]
+        B.llama3_layer_forward_docs(st.cfg, st.wstructs[i], st.rope, st.rope_len, x, kc, vc, st.cache_cap,
+                                    w.batch, w.seq, 0, dsd, st.ws, st.ws_bytes)
+    want, _, _ = O.forward_stack(x0, [oracle_layer(l) for l in layers], oracle_cfg(w), doc_start=ds)
+    assert_close(x, want, "bf16", "packed documents")

@@ -403,3 +403,70 @@ def test_pins_catch_planted_mistakes():
     for pin, override in cases:
         with pytest.raises(AssertionError):
             pin(mutated(**override))
+
+
+def test_greedy_generation_with_cache_equals_recomputing_the_whole_sequence():
+    # The KV-cache path of the inference section must pick the same tokens as
+    # re-running the full causal model on the growing sequence every step.
+    cfg = tiny_cfg()
+    layers = [tiny_layer(cfg, scale=0.4) for _ in range(2)]
+    V, D = 23, 16
+    table, w_out, nw = rand(V, D), rand(V, D), 1 + 0.1 * rand(D)
+    prompt = RNG.integers(0, V, (2, 5))
+    toks, gaps = O.generate_greedy(prompt, table, layers, nw, w_out, cfg, 6)
+    seq = prompt.copy()
+    for step in range(6):
+        h, _, _ = O.forward_stack(O.embed(seq, table), layers, cfg)
+        logits, nxt = O.lm_head(h[:, -1], nw, w_out, cfg["norm_eps"])
+        np.testing.assert_array_equal(toks[:, step], nxt)
+        seq = np.concatenate([seq, nxt[:, None]], 1)
+    assert np.all(gaps >= 0)
+
+
+def test_greedy_generation_holds_eos():
+    cfg = tiny_cfg()
+    layers = [tiny_layer(cfg)]
+    V, D = 7, 16
+    table, w_out = rand(V, D), np.zeros((V, D))
+    # all logits tie at 0, so the lowest index (0) wins every step; with 0 as
+    # the end token every sequence ends at once and stays ended
+    toks, _ = O.generate_greedy(RNG.integers(0, V, (2, 3)), table, layers, np.ones(D), w_out, cfg, 4, eos_id=0)
+    assert np.all(toks == 0)
+
+
+# ----------------------------------------------------------- document mask ---
+def test_document_mask_single_document_is_plain_causal():
+    q, k, v = rand(9, 4, 8), rand(9, 2, 8), rand(9, 2, 8)
+    np.testing.assert_array_equal(O.gqa_attention(q, k, v, doc_start=np.zeros(9, int)), O.gqa_attention(q, k, v))
+
+
+def test_document_mask_brute_force():
+    S, H, KV, hd = 8, 4, 2, 4
+    q, k, v = rand(S, H, hd), rand(S, KV, hd), rand(S, KV, hd)
+    ds = np.array([0, 0, 0, 3, 3, 5, 5, 5])
+    got = O.gqa_attention(q, k, v, doc_start=ds)
+    for t in range(S):
+        for h in range(H):
+            g = h // (H // KV)
+            keys = range(ds[t], t + 1)
+            sc = [sum(q[t, h, d] * k[j, g, d] for d in range(hd)) / math.sqrt(hd) for j in keys]
+            mx = max(sc); e = [math.exp(x - mx) for x in sc]; z = sum(e)
+            want = [sum(e[i] * v[j, g, d] for i, j in enumerate(keys)) / z for d in range(hd)]
+            np.testing.assert_allclose(got[t, h], want, rtol=1e-11, atol=1e-12)
+
+
+def test_packed_documents_equal_separate_documents():
+    # Two documents packed into one sequence, positions running on: each
+    # document's block outputs equal running it alone from position 0 (the
+    # attention sees only its own document, and RoPE scores depend only on
+    # relative positions).
+    cfg = tiny_cfg()
+    layers = [tiny_layer(cfg) for _ in range(2)]
+    a, b = rand(1, 5, 16), rand(1, 7, 16)
+    packed = np.concatenate([a, b], 1)
+    ds = np.array([[0] * 5 + [5] * 7])
+    out, _, _ = O.forward_stack(packed, layers, cfg, doc_start=ds)
+    alone_a, _, _ = O.forward_stack(a, layers, cfg)
+    alone_b, _, _ = O.forward_stack(b, layers, cfg)
+    np.testing.assert_allclose(out[:, :5], alone_a, rtol=1e-10, atol=1e-11)
+    np.testing.assert_allclose(out[:, 5:], alone_b, rtol=1e-10, atol=1e-11)
