@@ -41,7 +41,7 @@ __all__ = [
     "rms_norm", "ffn_hidden_dim", "rope_inverse_frequencies", "rope_angles",
     "apply_rope", "causal_mask", "gqa_attention", "silu", "swiglu_ffn",
     "decoder_block", "decoder_block_rows", "lm_head", "embed", "forward_stack",
-    "generate_greedy",
+    "generate_greedy", "philox4x64", "sampling_word", "top_p_sample",
 ]
 
 
@@ -311,3 +311,80 @@ def generate_greedy(prompt_ids, table, layers, norm_weight, w_out, cfg, n_new, e
         h, kc, vc = forward_stack(embed(nxt[:, None], table), layers, cfg, kc, vc, start_pos=S + step)
         logits, nxt = lm_head(h[:, -1], norm_weight, w_out, cfg["norm_eps"])
     return toks, gaps
+
+
+# ---------------------------------------------------------------------------
+# Temperature / top-p sampling  ([S2] 六 generate and sample_top_p; [S3]
+# 预测流程 on temperature)
+# ---------------------------------------------------------------------------
+# The random numbers come from Philox-4x64-10, the counter-based generator of
+# Salmon, Moraes, Dror and Shaw, "Parallel random numbers: as easy as 1, 2, 3"
+# (SC 2011): ten rounds of two 64x64->128 multiplies with the constants below,
+# the key bumped by two Weyl increments between rounds.
+_MASK64 = (1 << 64) - 1
+_PHILOX_MUL = (0xD2E7470EE14C6C93, 0xCA5A826395121157)
+_PHILOX_WEYL = (0x9E3779B97F4A7C15, 0xBB67AE8584CAA73B)
+
+
+def philox4x64(counter, key, rounds=10):
+    """One Philox-4x64 block: 4 counter words and 2 key words -> 4 words."""
+    c = [int(w) & _MASK64 for w in counter]
+    k = [int(w) & _MASK64 for w in key]
+    for _ in range(rounds):
+        p0 = _PHILOX_MUL[0] * c[0]
+        p1 = _PHILOX_MUL[1] * c[2]
+        c = [(p1 >> 64) ^ c[1] ^ k[0], p1 & _MASK64, (p0 >> 64) ^ c[3] ^ k[1], p0 & _MASK64]
+        k = [(k[0] + _PHILOX_WEYL[0]) & _MASK64, (k[1] + _PHILOX_WEYL[1]) & _MASK64]
+    return c
+
+
+def sampling_word(seed, offset, row):
+    """The 64-bit random word of one draw: first output word of
+    Philox-4x64-10 with key (seed, 0) and counter (offset, row, 0, 0)."""
+    return philox4x64((offset, row, 0, 0), (seed, 0))[0]
+
+
+def top_p_sample(logits, temperature, top_p, word):
+    """Next token of one row as [S2] 六 generate draws it.
+
+    temperature <= 0: argmax (lowest index on ties).  Otherwise
+    p = softmax(logits / temperature); tokens are ranked by descending p
+    (ties by ascending index, a stable sort); a token is kept iff the mass
+    ranked before it is <= top_p (the page zeroes those whose cumulative sum
+    minus their own probability exceeds top_p); the kept probabilities are
+    renormalised and one token is drawn.  The draw maps u = word / 2^64 by the
+    inverse CDF over the kept tokens in ascending index order: the first kept
+    token whose running kept mass exceeds u * (kept mass).  (The page hands the
+    draw to a multinomial routine; any fixed order gives the same law, and this
+    one needs no sort.)
+
+    Returns (token, margins) where margins = (cut, draw): the distance of
+    top_p from the nearest kept/dropped decision, and of the draw target from
+    the nearest boundary of the running kept mass, both as fractions of the
+    row's total probability.
+    """
+    z = _f64(logits)
+    if temperature <= 0:
+        return int(np.argmax(z)), (np.inf, np.inf)
+    z = z / float(temperature)
+    e = np.exp(z - z.max())
+    p = e / e.sum()
+    order = np.argsort(-p, kind="stable")
+    ranked = p[order]
+    before = np.cumsum(ranked) - ranked
+    keep_ranked = before <= top_p
+    kept = np.zeros(p.shape, dtype=bool)
+    kept[order[keep_ranked]] = True
+    n_keep = int(keep_ranked.sum())
+    cut = top_p - before[n_keep - 1]
+    if n_keep < len(ranked):
+        cut = min(cut, before[n_keep] - top_p)
+    idx = np.nonzero(kept)[0]
+    run = np.cumsum(p[idx])
+    target = (int(word) / 2.0 ** 64) * run[-1]
+    i = int(np.searchsorted(run, target, side="right"))
+    i = min(i, len(idx) - 1)
+    draw = run[i] - target
+    if i > 0:
+        draw = min(draw, target - run[i - 1])
+    return int(idx[i]), (float(cut), float(draw))

@@ -470,3 +470,140 @@ def test_packed_documents_equal_separate_documents():
     alone_b, _, _ = O.forward_stack(b, layers, cfg)
     np.testing.assert_allclose(out[:, :5], alone_a, rtol=1e-10, atol=1e-11)
     np.testing.assert_allclose(out[:, 5:], alone_b, rtol=1e-10, atol=1e-11)
+
+
+# ------------------------------------------------------ top-p sampling ---
+def _word(u):
+    """The 64-bit word whose draw fraction is u (0 <= u < 1)."""
+    return int(u * 2.0 ** 64)
+
+
+def pin_philox(o):
+    # Philox-4x64-10 is also numpy's Philox bit generator, which advances its
+    # counter before each block: block for counter c = random_raw after
+    # starting from c - 1.
+    for key, ctr in [((0, 0), (1, 0, 0, 0)), ((7, 0), (5, 3, 0, 0)),
+                     ((0x0123456789ABCDEF, 0xFEDCBA9876543210), (2 ** 63 + 11, 17, 2 ** 40, 9))]:
+        k = key[0] | (key[1] << 64)
+        start = ((ctr[0] - 1) | (ctr[1] << 64) | (ctr[2] << 128) | (ctr[3] << 192))
+        bg = np.random.Philox(key=k, counter=start)
+        want = [int(w) for w in bg.random_raw(4)]
+        assert o.philox4x64(ctr, key) == want
+    # the published known-answer vector for zero counter and key
+    assert o.philox4x64((0, 0, 0, 0), (0, 0)) == [0x16554D9ECA36314C, 0xDB20FE9D672D0FDC,
+                                                  0xD7E772CEE186176B, 0x7E68B68AEC7BA23B]
+
+
+def pin_top_p_hand_example(o):
+    # p = (0.05, 0.5, 0.15, 0.3): ranked 1, 3, 2, 0 with mass before 0, .5, .8, .95.
+    # top_p = 0.6 keeps tokens 1 and 3 (kept mass 0.8, running 0.5, 0.8 by index).
+    lg = np.log([0.05, 0.5, 0.15, 0.3])
+    for u, want in [(0.0, 1), (0.3, 1), (0.62, 1), (0.63, 3), (0.9, 3), (0.999, 3)]:
+        assert o.top_p_sample(lg, 1.0, 0.6, _word(u))[0] == want, u
+    # p = (.25, .5, .25), top_p = 0.5: token 0 is kept (the mass ranked before
+    # it is exactly 0.5), its tie token 2 is ranked after it and dropped
+    tie = np.log([0.25, 0.5, 0.25])
+    assert o.top_p_sample(tie, 1.0, 0.5, _word(0.2))[0] == 0
+    assert o.top_p_sample(tie, 1.0, 0.5, _word(0.9))[0] == 1
+    # top_p = 0.49 keeps only the top token
+    assert o.top_p_sample(lg, 1.0, 0.49, _word(0.999))[0] == 1
+
+
+def pin_top_p_ties(o):
+    # eight equal logits: ranked by index, the mass before token k is k/8
+    # (exact in binary), so top_p = 0.5 keeps tokens 0..4 (draw floor(5u))
+    # and top_p = 0.45 keeps 0..3
+    lg = np.zeros(8)
+    for k in range(5):
+        assert o.top_p_sample(lg, 0.7, 0.5, _word((k + 0.5) / 5))[0] == k
+    for k in range(4):
+        assert o.top_p_sample(lg, 1.3, 0.45, _word((k + 0.5) / 4))[0] == k
+
+
+def pin_top_p_limits(o):
+    rng = np.random.default_rng(4)
+    for _ in range(20):
+        lg = rng.standard_normal(50) * 3
+        w = int(rng.integers(0, 2 ** 63)) * 2 + 1
+        # a vanishing top_p keeps only the most probable token; temperature 0 is argmax
+        assert o.top_p_sample(lg, 0.8, 1e-12, w)[0] == int(np.argmax(lg))
+        assert o.top_p_sample(lg, 0.0, 0.9, w)[0] == int(np.argmax(lg))
+        # dividing by T is the same as scaling the logits by 1/T (exact for T = 2)
+        assert o.top_p_sample(lg * 2, 2.0, 0.9, w)[0] == o.top_p_sample(lg, 1.0, 0.9, w)[0]
+
+
+def pin_top_p_frequencies(o):
+    # The law of the draw: frequencies over many independent words equal the
+    # renormalised kept probabilities (here p = (.4, .25, .2, .1, .05), top_p
+    # 0.7 keeps the three largest: .4/.85, .25/.85, .2/.85).
+    p = np.array([0.1, 0.4, 0.05, 0.25, 0.2])
+    lg = np.log(p)
+    n = 20000
+    counts = np.zeros(5)
+    for i in range(n):
+        counts[o.top_p_sample(lg, 1.0, 0.7, o.sampling_word(99, i, 3))[0]] += 1
+    want = np.array([0, 0.4, 0, 0.25, 0.2]) / 0.85
+    sigma = np.sqrt(want * (1 - want) / n) + 1e-12
+    assert np.all(np.abs(counts / n - want) <= 5 * sigma + 1e-12), counts / n
+
+
+def test_philox_matches_numpy_and_known_answer():
+    pin_philox(O)
+
+
+def test_top_p_hand_example():
+    pin_top_p_hand_example(O)
+
+
+def test_top_p_ties_follow_index_order():
+    pin_top_p_ties(O)
+
+
+def test_top_p_limits_and_temperature():
+    pin_top_p_limits(O)
+
+
+def test_top_p_draw_frequencies():
+    pin_top_p_frequencies(O)
+
+
+def test_sampling_pins_catch_planted_mistakes():
+    def philox_swapped_constants(counter, key, rounds=10):
+        return O.philox4x64(counter, (key[1], key[0]), rounds)
+
+    def keep_by_inclusive_sum(logits, temperature, top_p, word):
+        # drops a token once the mass up to and INCLUDING it exceeds top_p
+        z = np.asarray(logits, float) / temperature
+        p = np.exp(z - z.max()); p /= p.sum()
+        order = np.argsort(-p, kind="stable")
+        keep = np.zeros(p.shape, bool)
+        keep[order[np.cumsum(p[order]) <= top_p]] = True
+        keep[order[0]] = True
+        idx = np.nonzero(keep)[0]
+        run = np.cumsum(p[idx])
+        return int(idx[min(np.searchsorted(run, word / 2.0 ** 64 * run[-1], "right"), len(idx) - 1)]), (0, 0)
+
+    def no_renormalisation(logits, temperature, top_p, word):
+        # draws u against the full mass instead of the kept mass
+        tok, m = O.top_p_sample(logits, temperature, top_p, word)
+        z = np.asarray(logits, float) / temperature
+        p = np.exp(z - z.max()); p /= p.sum()
+        u = word / 2.0 ** 64
+        order = np.argsort(-p, kind="stable")
+        before = np.cumsum(p[order]) - p[order]
+        idx = np.sort(order[before <= top_p])
+        run = np.cumsum(p[idx])
+        return int(idx[min(np.searchsorted(run, u, "right"), len(idx) - 1)]), m
+
+    def temperature_multiplies(logits, temperature, top_p, word):
+        return O.top_p_sample(np.asarray(logits, float) * temperature * temperature, temperature, top_p, word)
+
+    cases = [
+        (pin_philox, dict(philox4x64=philox_swapped_constants)),
+        (pin_top_p_hand_example, dict(top_p_sample=keep_by_inclusive_sum)),
+        (pin_top_p_frequencies, dict(top_p_sample=no_renormalisation)),
+        (pin_top_p_limits, dict(top_p_sample=temperature_multiplies)),
+    ]
+    for pin, override in cases:
+        with pytest.raises(AssertionError):
+            pin(mutated(**override))
