@@ -176,6 +176,25 @@ int llama3_layer_decode(const llama3_config* cfg, const llama3_layer_weights* w,
                         size_t ws_bytes, llama3_stream_t stream);
 
 /*
+ * One decode step of one block for a ragged batch ([S2] 六 generate with
+ * sequences of different lengths; the cache of §3.3): as llama3_layer_decode,
+ * but sequence b's new token sits at its own position positions[b] (device
+ * memory, int32 [batch]): its k/v are written there and it attends to
+ * positions 0..positions[b] of its own cache.  max_position is an upper bound
+ * of every positions[b], known to the caller without reading the device
+ * array (it sizes the launches; max_position + 1 <= cache_cap and <=
+ * rope_len).  A position outside [0, max_position] is clamped and reported as
+ * LLAMA3_ERR_ARG through llama3_device_status.  Errors as
+ * llama3_layer_decode, plus LLAMA3_ERR_ARG for positions == NULL and
+ * LLAMA3_ERR_ALIGN if it is not 4-byte aligned.
+ */
+int llama3_layer_decode_ragged(const llama3_config* cfg, const llama3_layer_weights* w,
+                               const float* rope, int rope_len, void* x, void* k_cache,
+                               void* v_cache, int cache_cap, int batch, const int32_t* positions,
+                               int max_position, void* ws, size_t ws_bytes,
+                               llama3_stream_t stream);
+
+/*
  * Output block ([S1] §11-12, [S3] 预测流程): for each of `rows` hidden rows
  * h[r] = h + r*row_stride (elements), compute logits = RMSNorm(h[r], norm_w)
  * W_out^T over the vocabulary and ids_out[r] = argmax (lowest index on ties).
@@ -219,6 +238,29 @@ int llama3_lm_head_argmax_noalloc(const llama3_config* cfg, const void* norm_w, 
                                   const void* h, int rows, long long row_stride,
                                   int32_t* ids_out, float* logits_out, llama3_stream_t stream);
 
+/*
+ * Temperature / top-p draw of the next token ([S2] 六 generate and
+ * sample_top_p).  For each row r of fp32 logits (row r at logits + r*ld,
+ * `vocab` entries) writes ids_out[r]:
+ *   temperature <= 0: the argmax (lowest index on ties), the page's T = 0 case;
+ *   otherwise p = softmax(logits / temperature); tokens ranked by descending p
+ *   (ties: lower index first) are kept while the probability ranked before
+ *   them is <= top_p (top_p >= 1 keeps all, top_p = 0 keeps the top token);
+ *   one kept token is drawn with probability proportional to p.
+ * The draw is deterministic in (seed, offset, row): the first 64-bit word of
+ * Philox-4x64-10 (Salmon et al., SC 2011) with key (seed, 0) and counter
+ * (offset, r, 0, 0) selects the token by the inverse CDF of the kept law
+ * taken in index order.  Probabilities are evaluated in fp32 and summed
+ * exactly as integers in units of 2^-40 of the largest one.  Pass the
+ * decoding step as `offset` to get a fresh draw per step.
+ * Errors: LLAMA3_ERR_ARG (null pointers, rows < 1, vocab < 1, ld < vocab,
+ * top_p < 0 or NaN, temperature NaN), LLAMA3_ERR_ALIGN (pointers not 4-byte
+ * aligned), LLAMA3_ERR_CUDA.  Allocates nothing; asynchronous on `stream`.
+ */
+int llama3_sample_top_p(const float* logits, int rows, long long ld, int vocab, float temperature,
+                        float top_p, unsigned long long seed, unsigned long long offset,
+                        int32_t* ids_out, llama3_stream_t stream);
+
 /* ---- building blocks (the steps of the calls above, exposed for tests) ---- */
 
 /* y[r] = x[r] / sqrt(mean(x[r]^2) + eps) * w  ([S1] §5, [S2] §3.1); x rows at
@@ -255,7 +297,8 @@ enum llama3_kernel_kind {
   LLAMA3_KERNEL_DECODE_ATTENTION = 7,  /* split-KV decode attention (main kernel)  */
   LLAMA3_KERNEL_LM_HEAD = 8,           /* LM-head GEMM + argmax                    */
   LLAMA3_KERNEL_NORM = 9,              /* RMSNorm                                  */
-  LLAMA3_KERNEL_ELEMENTWISE = 10       /* embedding, split-K reductions, misc.     */
+  LLAMA3_KERNEL_ELEMENTWISE = 10,      /* embedding, split-K reductions, misc.     */
+  LLAMA3_KERNEL_SAMPLE = 11            /* temperature / top-p draw                 */
 };
 
 /* Record start_events[i] / stop_events[i] (cudaEvent_t handles created by the
@@ -305,11 +348,14 @@ int llama3_set_wait_limit_ms(int ms);
  * 0: ordinary launches.  Returns the previous value. */
 int llama3_set_programmatic_launch(int on);
 
-/* Prefill attention kernel design (bf16, tcgen05 path): 1 (default) = one
- * softmax thread per query row with P staged in shared memory; 2 = two
- * softmax threads per row (each over half the keys of a tile) with P written
- * back into tensor memory.  Both compute the same attention.  Any other value
- * selects 1.  Returns the previous value. */
+/* Prefill attention kernel design (bf16, tcgen05 path): 2 (default) = two
+ * softmax threads per query row (each over half the keys of a tile) with P
+ * written back into tensor memory; 1 = one softmax thread per row with P
+ * staged in shared memory; 3 = one softmax thread per row holding the whole
+ * row of a tile in registers (warpgroup register reallocation) with P in
+ * tensor memory.  All compute the same attention.  Values other than 1 and 3
+ * select 2.  Variant 3 returns LLAMA3_ERR_UNSUPPORTED if the compiled kernel's
+ * register count cannot fund its register split.  Returns the previous value. */
 int llama3_set_flash_variant(int variant);
 
 #ifdef __cplusplus

@@ -51,6 +51,7 @@ _SIGNATURES = {
     "llama3_embed": [_cfgp, _p, _p, _p, _i, _p],
     "llama3_layer_forward": [_cfgp, _wp, _p, _i, _p, _p, _p, _i, _i, _i, _i, _p, _sz, _p],
     "llama3_layer_decode": [_cfgp, _wp, _p, _i, _p, _p, _p, _i, _i, _i, _p, _sz, _p],
+    "llama3_layer_decode_ragged": [_cfgp, _wp, _p, _i, _p, _p, _p, _i, _i, _p, _i, _p, _sz, _p],
     "llama3_layer_forward_docs": [_cfgp, _wp, _p, _i, _p, _p, _p, _i, _i, _i, _i, _p, _p, _sz, _p],
     "llama3_attention_docs": [_cfgp, _p, _p, _p, _i, _i, _i, _i, _p, _p, _p, _sz, _p],
     "llama3_lm_head_argmax": [_cfgp, _p, _p, _p, _i, _ll, _p, _p, _p, _sz, _p],
@@ -65,6 +66,7 @@ _SIGNATURES = {
     "llama3_set_wait_limit_ms": [_i],
     "llama3_set_programmatic_launch": [_i],
     "llama3_set_flash_variant": [_i],
+    "llama3_sample_top_p": [_p, _i, _ll, _i, ctypes.c_float, ctypes.c_float, ctypes.c_ulonglong, ctypes.c_ulonglong, _p, _p],
     "llama3_set_launch_timer": [_i, _p, _p, _i],
     "llama3_launch_timer_used": [],
     "llama3_launch_count": [],
@@ -178,11 +180,26 @@ def llama3_layer_decode(cfg, w, rope, rope_len, x, k_cache, v_cache, cache_cap, 
         cache_cap, batch, start_pos, _ptr(ws), ws_bytes, _stream(stream)))
 
 
+def llama3_layer_decode_ragged(cfg, w, rope, rope_len, x, k_cache, v_cache, cache_cap, batch, positions,
+                               max_position, ws, ws_bytes, stream=None):
+    """One decode step with every sequence at its own position (int32 device tensor [batch])."""
+    _check("llama3_layer_decode_ragged", lib().llama3_layer_decode_ragged(
+        ctypes.byref(cfg), ctypes.byref(w), _ptr(rope), rope_len, _ptr(x), _ptr(k_cache), _ptr(v_cache),
+        cache_cap, batch, _ptr(positions), max_position, _ptr(ws), ws_bytes, _stream(stream)))
+
+
 def llama3_lm_head_argmax(cfg, norm_w, w_out, h, rows, row_stride, ids_out, logits_out, ws, ws_bytes,
                           stream=None):
     _check("llama3_lm_head_argmax", lib().llama3_lm_head_argmax(
         ctypes.byref(cfg), _ptr(norm_w), _ptr(w_out), _ptr(h), rows, row_stride, _ptr(ids_out),
         _ptr(logits_out), _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def llama3_sample_top_p(logits, rows, ld, vocab, temperature, top_p, seed, offset, ids_out, stream=None):
+    """Temperature / top-p draw of one token per row of fp32 logits."""
+    _check("llama3_sample_top_p", lib().llama3_sample_top_p(
+        _ptr(logits), rows, ld, vocab, float(temperature), float(top_p), int(seed) & (2 ** 64 - 1),
+        int(offset) & (2 ** 64 - 1), _ptr(ids_out), _stream(stream)))
 
 
 NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -243,7 +260,7 @@ def llama3_set_flash_variant(variant):
 
 
 KERNEL_KINDS = {"gemm_qkv": 1, "gemm_wo": 2, "gemm_w13": 3, "gemm_w2": 4, "attention": 5, "decode_gemm": 6,
-                "decode_attention": 7, "lm_head": 8, "norm": 9, "elementwise": 10}
+                "decode_attention": 7, "lm_head": 8, "norm": 9, "elementwise": 10, "sample": 11}
 
 
 def llama3_set_launch_timer(kind, start_events, stop_events):

@@ -50,6 +50,9 @@ __global__ void decode_attention_combine_kernel(const float* __restrict__ part, 
 struct DecodeShape {
   int B, H, KV, nrep, n_keys, tiles, splits, tiles_per_split, units;
   float scale_log2;
+  // Optional per-sequence positions (device, [B]): sequence b's token sits at
+  // positions[b] and sees keys 0..positions[b] (at most n_keys of them).
+  const int32_t* positions;
 };
 
 template <int HD>
@@ -74,14 +77,18 @@ struct DecodeTcCfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
+// Unit u -> sequence b, KV head g, key tiles [t0, t1) and the number of keys
+// sequence b sees (n_keys, or positions[b] + 1 clamped to [1, n_keys]); a
+// unit past a short sequence's last tile is empty (t1 == t0).
 __device__ __forceinline__ void decode_unit(const DecodeShape& ds, int u, int& b, int& g, int& split, int& t0,
-                                            int& t1) {
+                                            int& t1, int& nk) {
   split = u % ds.splits;
   const int bg = u / ds.splits;
   g = bg % ds.KV;
   b = bg / ds.KV;
+  nk = ds.positions ? max(1, min(ds.positions[b] + 1, ds.n_keys)) : ds.n_keys;
   t0 = split * ds.tiles_per_split;
-  t1 = min(t0 + ds.tiles_per_split, ds.tiles);
+  t1 = max(t0, min(t0 + ds.tiles_per_split, (nk + 127) / 128));
 }
 
 template <int HD, int NREP>
@@ -153,8 +160,8 @@ __global__ void __launch_bounds__(384, 1)
       uint32_t iss = 0, par = 0, qiss = 0, qpar = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < ds.units && ok; u += gridDim.x, ++kq) {
-        int b, g, split, t0, t1;
-        decode_unit(ds, u, b, g, split, t0, t1);
+        int b, g, split, t0, t1, nk;
+        decode_unit(ds, u, b, g, split, t0, t1, nk);
         const int qb = kq & 1;
         if (!mbar_wait(&q_empty[qb], qph[qb] ^ 1u, wait_ns)) break;
         mbar_arrive_expect_tx(&q_full[qb], C::Q_BYTES);
@@ -188,8 +195,8 @@ __global__ void __launch_bounds__(384, 1)
       uint32_t pph[2][2] = {{0, 0}, {0, 0}};
       bool ok = true;
       for (int u = blockIdx.x; u < ds.units && ok; u += gridDim.x, ++kq) {
-        int b, g, split, t0, t1;
-        decode_unit(ds, u, b, g, split, t0, t1);
+        int b, g, split, t0, t1, nk;
+        decode_unit(ds, u, b, g, split, t0, t1, nk);
         const int qb = kq & 1;
         const uint32_t q_addr = smem_u32(smem + C::OFF_Q + qb * C::Q_BYTES);
         if (!mbar_wait(&q_full[qb], qph[qb], wait_ns)) break;
@@ -259,8 +266,8 @@ __global__ void __launch_bounds__(384, 1)
       return done;
     };
     for (int u = blockIdx.x; u < ds.units; u += gridDim.x) {
-      int b, g, split, t0, t1;
-      decode_unit(ds, u, b, g, split, t0, t1);
+      int b, g, split, t0, t1, nk;
+      decode_unit(ds, u, b, g, split, t0, t1, nk);
       const int n = t1 - t0;
       const int mine = n > wg ? (n - wg + 1) / 2 : 0;   // tiles wg, wg+2, ...
       float m_ref[NREP], l_part[NREP];
@@ -276,7 +283,7 @@ __global__ void __launch_bounds__(384, 1)
         tmem_ld16(wg_tmem + sb * 16, r);
         tc_wait_ld();
         const int key = (t0 + i) * 128 + row;
-        const bool valid = key < ds.n_keys;
+        const bool valid = key < nk;
         float s[NREP];
 #pragma unroll
         for (int h = 0; h < NREP; ++h)

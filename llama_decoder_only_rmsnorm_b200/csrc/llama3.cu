@@ -17,6 +17,8 @@
 #include "decode_attention.cuh"
 #include "flash_attention.cuh"
 #include "flash_attention2.cuh"
+#include "flash_attention3.cuh"
+#include "sampling.cuh"
 #include "simt.cuh"
 #include "tc_gemm.cuh"
 #include "tc_gemm_pair.cuh"
@@ -92,7 +94,7 @@ bool g_pdl = true;
 
 // Prefill attention kernel design: 1 = one softmax thread per query row, P
 // through shared memory; 2 = two softmax threads per row, P kept in TMEM.
-int g_flash_variant = 1;
+int g_flash_variant = 2;
 
 template <typename... KArgs, typename... Args>
 cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
@@ -242,16 +244,27 @@ int run_flash_attention_t(int H, int KV, const void* q, const void* kc, const vo
   fs.ldo = H * HD;
   fs.scale_log2 = (float)(1.4426950408889634 / sqrt((double)HD));
   fs.doc_start = doc_start;
-  constexpr int smem = VARIANT == 2 ? Flash2Cfg<HD>::SMEM_BYTES : FlashCfg<HD>::SMEM_BYTES;
-  constexpr int threads = VARIANT == 2 ? 640 : 384;
-  auto kern = VARIANT == 2 ? flash_attention2_kernel<HD> : flash_attention_kernel<HD>;
+  constexpr int smem = VARIANT == 3 ? Flash3Cfg<HD>::SMEM_BYTES
+                     : VARIANT == 2 ? Flash2Cfg<HD>::SMEM_BYTES : FlashCfg<HD>::SMEM_BYTES;
+  constexpr int threads = VARIANT == 3 ? kFlash3Threads : VARIANT == 2 ? 640 : 384;
+  auto kern = VARIANT == 3 ? flash_attention3_kernel<HD>
+            : VARIANT == 2 ? flash_attention2_kernel<HD> : flash_attention_kernel<HD>;
   int dev = 0;
   L3_TRY(current_device(&dev));
   static bool attr_done[kMaxDevices];
+  static bool regs_ok[kMaxDevices];
   if (!attr_done[dev]) {
     L3_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    if (VARIANT == 3) {
+      // The warpgroups' setmaxnreg shares must fit the registers the block is
+      // launched with, or the raising warpgroups would wait for ever.
+      cudaFuncAttributes fa;
+      L3_CUDA(cudaFuncGetAttributes(&fa, kern));
+      regs_ok[dev] = (long long)fa.numRegs * kFlash3Threads >= 128LL * kFlash3LowRegs + 256LL * kFlash3HighRegs;
+    }
     attr_done[dev] = true;
   }
+  if (VARIANT == 3 && !regs_ok[dev]) return LLAMA3_ERR_UNSUPPORTED;
   const int grid = std::min(fs.units, sms);
   L3_LAUNCH(LLAMA3_KERNEL_ATTENTION, st, launch_k(kern, grid, threads, smem, st, mq, mk, mv, (bf16*)out, fs, wns));
   return launch_check();
@@ -261,6 +274,8 @@ template <int HD>
 int run_flash_attention_v(int H, int KV, const void* q, const void* kc, const void* vc, int cap, int B, int S,
                           int P, void* out, const int32_t* doc_start, int sms, unsigned long long wns,
                           cudaStream_t st) {
+  if (g_flash_variant == 3)
+    return run_flash_attention_t<HD, 3>(H, KV, q, kc, vc, cap, B, S, P, out, doc_start, sms, wns, st);
   if (g_flash_variant == 2)
     return run_flash_attention_t<HD, 2>(H, KV, q, kc, vc, cap, B, S, P, out, doc_start, sms, wns, st);
   return run_flash_attention_t<HD, 1>(H, KV, q, kc, vc, cap, B, S, P, out, doc_start, sms, wns, st);
@@ -345,6 +360,12 @@ GemmShape make_shape(int rows_a, int rows_a2, int rows_b, int k, int bn, int spl
 
 // Split count that minimises the longest per-CTA stream (persistent grid of
 // one CTA per SM): ceil(units / SMs) * k-blocks per split.
+// Split-K count for a skinny GEMM: minimise the busiest CTA's load, counted
+// in k-blocks, where every work unit also costs L3_SPLIT_UNIT_COST k-blocks
+// for writing its fp32 partial tile and reading it back in the reduction.
+#ifndef L3_SPLIT_UNIT_COST
+#define L3_SPLIT_UNIT_COST 2
+#endif
 int choose_splits(int tiles, int kblocks, int sms) {
   int best = 1;
   long long best_t = -1;
@@ -352,7 +373,7 @@ int choose_splits(int tiles, int kblocks, int sms) {
     const int per = (kblocks + s - 1) / s;
     const int real = (kblocks + per - 1) / per;
     const long long units = (long long)tiles * real;
-    const long long t = ((units + sms - 1) / sms) * per;
+    const long long t = ((units + sms - 1) / sms) * (per + L3_SPLIT_UNIT_COST);
     if (best_t < 0 || t < best_t) { best_t = t; best = real; }
   }
   return best;
@@ -426,6 +447,8 @@ EpiParams empty_epi() {
 
 // Swapped (weight-streaming) GEMM for few token rows: P[split][t][n] =
 // sum_k W[n, k] X[t, k], with W1|W3 stacked through `w_second`.
+// Skinny GEMM with the weights as the MMA's M side and split-K: fp32 partials
+// P[split][token][feature], reduced by a separate kernel.
 int swapped_partial_gemm(const void* w, int rows_w, const void* w_second, int rows_w2, int out_offset2,
                          const void* x, int rows_x, int k, float* P, int ldo, int* splits_out,
                          cudaStream_t st) {
@@ -451,6 +474,7 @@ int swapped_partial_gemm(const void* w, int rows_w, const void* w_second, int ro
     default: return launch_gemm<256, 4, EPI_PARTIAL, false>(LLAMA3_KERNEL_DECODE_GEMM, ma, ma2, mb, mb, sh, ep, st);
   }
 }
+
 
 constexpr int kPrefillBN = 256;
 
@@ -481,8 +505,21 @@ int run_rmsnorm_warp(const llama3_config* c, const void* x, long long row_stride
   return launch_check();
 }
 
+bool rmsnorm_rows_kernel_ok(const llama3_config* c, long long row_stride, int rows) {
+  return c->dtype == LLAMA3_DTYPE_BF16 && c->dim % 8 == 0 && (row_stride * 2) % 16 == 0 && g_kernel_path == 0 &&
+         rows <= 512 && c->dim / 8 <= 1024;
+}
+
 int rmsnorm_any(const llama3_config* c, const void* x, long long row_stride, const void* w, void* y, int rows,
                 cudaStream_t st) {
+  if (rmsnorm_rows_kernel_ok(c, row_stride, rows)) {
+    // few rows (decode, LM head): one CTA per row spreads them over the SMs
+    const int threads = (c->dim / 8 + 31) / 32 * 32;
+    L3_LAUNCH(LLAMA3_KERNEL_NORM, st,
+              launch_k(rmsnorm_bf16_row_kernel, rows, threads, 0, st, (const bf16*)x, row_stride, (const bf16*)w,
+                       (bf16*)y, c->dim, c->norm_eps));
+    return launch_check();
+  }
   if (c->dtype == LLAMA3_DTYPE_F32) return run_rmsnorm<float>(c, x, row_stride, w, y, rows, st);
   // bf16: the warp-per-row kernel when rows are 16-byte aligned and fit its registers
   const int chunks = c->dim / 8;
@@ -499,19 +536,21 @@ int rmsnorm_any(const llama3_config* c, const void* x, long long row_stride, con
 
 template <typename T>
 int run_attention_simt(const llama3_config* c, const void* q, const void* kc, const void* vc, int cap, int B,
-                       int S, int P, void* out, const int32_t* doc_start, cudaStream_t st) {
+                       int S, int P, void* out, const int32_t* doc_start, cudaStream_t st,
+                       const int32_t* positions = nullptr) {
   const long long warps = (long long)B * S * c->n_heads;
   const float scale = (float)(1.0 / sqrt((double)c->head_dim));
   L3_LAUNCH(LLAMA3_KERNEL_ATTENTION, st, launch_k((attention_simt_kernel<T>), blocks_for(warps * 32, 256), 256, 0, st, 
       (const T*)q, (const T*)kc, (const T*)vc, (T*)out, B, S, P, c->n_heads, c->n_kv_heads, c->head_dim, cap,
-      scale, doc_start));
+      scale, doc_start, positions, P));
   return launch_check();
 }
 
 // Tensor-core decode attention: TMA-streamed K/V tiles, two tcgen05 MMAs per tile.
 template <int HD, int NREP>
 int run_decode_attention_tc_t(const llama3_config* c, const void* q, const void* kc, const void* vc, int cap,
-                              int B, int n_keys, void* out, float* part, cudaStream_t st) {
+                              int B, int n_keys, void* out, float* part, cudaStream_t st,
+                              const int32_t* positions) {
   using Cfg = DecodeTcCfg<HD>;
   const int KV = c->n_kv_heads, H = c->n_heads;
   const long long e = 2;
@@ -539,6 +578,7 @@ int run_decode_attention_tc_t(const llama3_config* c, const void* q, const void*
   ds.splits = (ds.tiles + ds.tiles_per_split - 1) / ds.tiles_per_split;
   ds.units = B * KV * ds.splits;
   ds.scale_log2 = (float)(1.4426950408889634 / sqrt((double)HD));
+  ds.positions = positions;
   auto kern = decode_attention_tc_kernel<HD, NREP>;
   int dev = 0;
   L3_TRY(current_device(&dev));
@@ -558,13 +598,14 @@ int run_decode_attention_tc_t(const llama3_config* c, const void* q, const void*
 
 template <int HD>
 int run_decode_attention_tc_hd(const llama3_config* c, const void* q, const void* kc, const void* vc, int cap,
-                               int B, int n_keys, void* out, float* part, cudaStream_t st) {
+                               int B, int n_keys, void* out, float* part, cudaStream_t st,
+                               const int32_t* positions) {
   const int r = c->n_heads / c->n_kv_heads;
-  if (r <= 1) return run_decode_attention_tc_t<HD, 1>(c, q, kc, vc, cap, B, n_keys, out, part, st);
-  if (r <= 2) return run_decode_attention_tc_t<HD, 2>(c, q, kc, vc, cap, B, n_keys, out, part, st);
-  if (r <= 4) return run_decode_attention_tc_t<HD, 4>(c, q, kc, vc, cap, B, n_keys, out, part, st);
-  if (r <= 8) return run_decode_attention_tc_t<HD, 8>(c, q, kc, vc, cap, B, n_keys, out, part, st);
-  if (r <= 16) return run_decode_attention_tc_t<HD, 16>(c, q, kc, vc, cap, B, n_keys, out, part, st);
+  if (r <= 1) return run_decode_attention_tc_t<HD, 1>(c, q, kc, vc, cap, B, n_keys, out, part, st, positions);
+  if (r <= 2) return run_decode_attention_tc_t<HD, 2>(c, q, kc, vc, cap, B, n_keys, out, part, st, positions);
+  if (r <= 4) return run_decode_attention_tc_t<HD, 4>(c, q, kc, vc, cap, B, n_keys, out, part, st, positions);
+  if (r <= 8) return run_decode_attention_tc_t<HD, 8>(c, q, kc, vc, cap, B, n_keys, out, part, st, positions);
+  if (r <= 16) return run_decode_attention_tc_t<HD, 16>(c, q, kc, vc, cap, B, n_keys, out, part, st, positions);
   return LLAMA3_ERR_UNSUPPORTED;
 }
 
@@ -573,13 +614,23 @@ bool decode_attention_tc_supported(const llama3_config* c) {
          c->n_heads / c->n_kv_heads <= 16;
 }
 
+// positions (device [B], with S == 1 and P = their upper bound): every
+// sequence's token at its own position (ragged decode).
 int attention_dispatch(const llama3_config* c, const void* q, const void* kc, const void* vc, int cap, int B,
-                       int S, int P, void* out, float* part, cudaStream_t st, const int32_t* doc_start = nullptr) {
+                       int S, int P, void* out, float* part, cudaStream_t st, const int32_t* doc_start = nullptr,
+                       const int32_t* positions = nullptr) {
+  if (positions) {
+    if (S != 1 || doc_start) return LLAMA3_ERR_ARG;
+    if (!decode_attention_tc_supported(c))
+      return c->dtype == LLAMA3_DTYPE_F32
+                 ? run_attention_simt<float>(c, q, kc, vc, cap, B, 1, P, out, nullptr, st, positions)
+                 : run_attention_simt<bf16>(c, q, kc, vc, cap, B, 1, P, out, nullptr, st, positions);
+  }
   if (S == 1 && !doc_start && decode_attention_tc_supported(c)) {
     switch (c->head_dim) {
-      case 64: return run_decode_attention_tc_hd<64>(c, q, kc, vc, cap, B, P + 1, out, part, st);
-      case 96: return run_decode_attention_tc_hd<96>(c, q, kc, vc, cap, B, P + 1, out, part, st);
-      default: return run_decode_attention_tc_hd<128>(c, q, kc, vc, cap, B, P + 1, out, part, st);
+      case 64: return run_decode_attention_tc_hd<64>(c, q, kc, vc, cap, B, P + 1, out, part, st, positions);
+      case 96: return run_decode_attention_tc_hd<96>(c, q, kc, vc, cap, B, P + 1, out, part, st, positions);
+      default: return run_decode_attention_tc_hd<128>(c, q, kc, vc, cap, B, P + 1, out, part, st, positions);
     }
   }
   if (use_tc(c) && flash_attention_supported(c->head_dim, c->n_heads, c->n_kv_heads))
@@ -595,7 +646,7 @@ int attention_dispatch(const llama3_config* c, const void* q, const void* kc, co
 template <typename T>
 int layer_simt(const llama3_config* c, const llama3_layer_weights* w, const float* rope, void* x, void* kc,
                void* vc, int cap, int B, int S, int P, const Workspace& L, void* ws, cudaStream_t st,
-               const int32_t* doc_start = nullptr) {
+               const int32_t* doc_start = nullptr, const int32_t* positions = nullptr) {
   const int M = B * S, D = c->dim, H = c->n_heads, KV = c->n_kv_heads, hd = c->head_dim, F = c->ffn_hidden;
   const int nqkv = (H + 2 * KV) * hd;
   T* xn = ws_at<T>(ws, L.xn);
@@ -607,9 +658,9 @@ int layer_simt(const llama3_config* c, const llama3_layer_weights* w, const floa
   L3_TRY(run_rmsnorm<T>(c, x, D, w->attention_norm, xn, M, st));
   L3_TRY(simt_gemm<T>(LLAMA3_KERNEL_GEMM_QKV, xn, w->wqkv, Pp, M, nqkv, D, nqkv, st));
   L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_qkv_rope_kernel<T>), blocks_for((long long)M * nqkv / 4, 256), 256, 0, st, 
-      Pp, 1, 0, M, S, P, H, KV, hd, rope, q, (T*)kc, (T*)vc, cap));
+      Pp, 1, 0, M, S, P, H, KV, hd, rope, q, (T*)kc, (T*)vc, cap, positions, P));
   L3_TRY(launch_check());
-  L3_TRY(attention_dispatch(c, q, kc, vc, cap, B, S, P, o, Ap, st, doc_start));
+  L3_TRY(attention_dispatch(c, q, kc, vc, cap, B, S, P, o, Ap, st, doc_start, positions));
   L3_TRY(simt_gemm<T>(LLAMA3_KERNEL_GEMM_WO, o, w->wo, Pp, M, D, H * hd, D, st));
   L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_residual_kernel<T>), blocks_for((long long)M * D / 4, 256), 256, 0, st, Pp, 1, 0, D, (const T*)x, (T*)x, M, D));
   L3_TRY(launch_check());
@@ -704,7 +755,8 @@ int layer_tc_prefill(const llama3_config* c, const llama3_layer_weights* w, cons
 // GEMMs + SIMT epilogues over the fp32 partials.
 // ---------------------------------------------------------------------------
 int layer_tc_decode(const llama3_config* c, const llama3_layer_weights* w, const float* rope, void* x, void* kc,
-                    void* vc, int cap, int B, int P, const Workspace& L, void* ws, cudaStream_t st) {
+                    void* vc, int cap, int B, int P, const Workspace& L, void* ws, cudaStream_t st,
+                    const int32_t* positions = nullptr) {
   const int M = B, D = c->dim, H = c->n_heads, KV = c->n_kv_heads, hd = c->head_dim, F = c->ffn_hidden;
   const int nqkv = (H + 2 * KV) * hd;
   bf16* xn = ws_at<bf16>(ws, L.xn);
@@ -714,29 +766,25 @@ int layer_tc_decode(const llama3_config* c, const llama3_layer_weights* w, const
   float* Pp = ws_at<float>(ws, L.part);
   float* Ap = ws_at<float>(ws, L.attn_part);
   int splits = 1;
-
   L3_TRY(rmsnorm_any(c, x, D, w->attention_norm, xn, M, st));
   L3_TRY(swapped_partial_gemm(w->wqkv, nqkv, nullptr, 0, 0, xn, M, D, Pp, nqkv, &splits, st));
-  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_qkv_rope_kernel<bf16>), blocks_for((long long)M * nqkv / 4, 256), 256, 0, st, 
-      Pp, splits, (long long)M * nqkv, M, 1, P, H, KV, hd, rope, q, (bf16*)kc, (bf16*)vc, cap));
+  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_qkv_rope_kernel<bf16>), blocks_for((long long)M * nqkv / 4, 256), 256, 0, st,
+      Pp, splits, (long long)M * nqkv, M, 1, P, H, KV, hd, rope, q, (bf16*)kc, (bf16*)vc, cap, positions, P));
   L3_TRY(launch_check());
-  L3_TRY(attention_dispatch(c, q, kc, vc, cap, B, 1, P, o, Ap, st));
+  L3_TRY(attention_dispatch(c, q, kc, vc, cap, B, 1, P, o, Ap, st, nullptr, positions));
   L3_TRY(swapped_partial_gemm(w->wo, D, nullptr, 0, 0, o, M, H * hd, Pp, D, &splits, st));
   // h = x + o Wo^T and hn = RMSNorm(h) in one pass over each row
-  if (D <= 8 * 4 * 256) {
-    const int G = (D + 1023) / 1024;
+  if (D <= 4 * 4 * 1024) {
+    const int G = (D + 4095) / 4096;
     const long long sstride = (long long)M * D;
     if (G <= 1)
-      L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_residual_rmsnorm_kernel<1>), M, 256, 0, st, Pp, splits,
+      L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_residual_rmsnorm_kernel<1>), M, 1024, 0, st, Pp, splits,
                                                         sstride, (bf16*)x, (const bf16*)w->ffn_norm, xn, D, c->norm_eps));
     else if (G <= 2)
-      L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_residual_rmsnorm_kernel<2>), M, 256, 0, st, Pp, splits,
-                                                        sstride, (bf16*)x, (const bf16*)w->ffn_norm, xn, D, c->norm_eps));
-    else if (G <= 4)
-      L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_residual_rmsnorm_kernel<4>), M, 256, 0, st, Pp, splits,
+      L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_residual_rmsnorm_kernel<2>), M, 1024, 0, st, Pp, splits,
                                                         sstride, (bf16*)x, (const bf16*)w->ffn_norm, xn, D, c->norm_eps));
     else
-      L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_residual_rmsnorm_kernel<8>), M, 256, 0, st, Pp, splits,
+      L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_residual_rmsnorm_kernel<4>), M, 1024, 0, st, Pp, splits,
                                                         sstride, (bf16*)x, (const bf16*)w->ffn_norm, xn, D, c->norm_eps));
     L3_TRY(launch_check());
   } else {
@@ -751,7 +799,7 @@ int layer_tc_decode(const llama3_config* c, const llama3_layer_weights* w, const
                                                                                 M, F));
   L3_TRY(launch_check());
   L3_TRY(swapped_partial_gemm(w->w2, D, nullptr, 0, 0, g, M, F, Pp, D, &splits, st));
-  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_residual_kernel<bf16>), blocks_for((long long)M * D / 4, 256), 256, 0, st, 
+  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_residual_kernel<bf16>), blocks_for((long long)M * D / 4, 256), 256, 0, st,
       Pp, splits, (long long)M * D, D, (const bf16*)x, (bf16*)x, M, D));
   return launch_check();
 }
@@ -822,9 +870,37 @@ int llama3_set_kernel_path(int path) {
   return old;
 }
 
+int llama3_sample_top_p(const float* logits, int rows, long long ld, int vocab, float temperature, float top_p,
+                        unsigned long long seed, unsigned long long offset, int32_t* ids_out,
+                        llama3_stream_t stream) {
+  if (!logits || !ids_out || rows < 1 || vocab < 1 || ld < vocab) return LLAMA3_ERR_ARG;
+  if (std::isnan(temperature) || std::isnan(top_p) || top_p < 0.f) return LLAMA3_ERR_ARG;
+  if ((reinterpret_cast<uintptr_t>(logits) & 3) || (reinterpret_cast<uintptr_t>(ids_out) & 3))
+    return LLAMA3_ERR_ALIGN;
+  cudaStream_t st = (cudaStream_t)stream;
+  int dev = 0;
+  L3_TRY(current_device(&dev));
+  static bool attr_done[kMaxDevices];
+  if (!attr_done[dev]) {
+    L3_CUDA(cudaFuncSetAttribute(sample_top_p_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSampleSmem));
+    attr_done[dev] = true;
+  }
+  SampleParams sp;
+  sp.logits = logits;
+  sp.ld = ld;
+  sp.V = vocab;
+  sp.temperature = temperature;
+  sp.top_p = top_p;
+  sp.seed = seed;
+  sp.offset = offset;
+  sp.ids = ids_out;
+  L3_LAUNCH(LLAMA3_KERNEL_SAMPLE, st, launch_k(sample_top_p_kernel, rows, kSampleThreads, kSampleSmem, st, sp));
+  return launch_check();
+}
+
 int llama3_set_flash_variant(int variant) {
   const int old = g_flash_variant;
-  g_flash_variant = (variant == 2) ? 2 : 1;
+  g_flash_variant = (variant == 1 || variant == 3) ? variant : 2;
   return old;
 }
 
@@ -981,6 +1057,25 @@ int llama3_layer_decode(const llama3_config* cfg, const llama3_layer_weights* w,
   if (cfg->dtype == LLAMA3_DTYPE_F32)
     return layer_simt<float>(cfg, w, rope, x, k_cache, v_cache, cache_cap, batch, 1, start_pos, L, ws, st);
   return layer_simt<bf16>(cfg, w, rope, x, k_cache, v_cache, cache_cap, batch, 1, start_pos, L, ws, st);
+}
+
+int llama3_layer_decode_ragged(const llama3_config* cfg, const llama3_layer_weights* w, const float* rope,
+                               int rope_len, void* x, void* k_cache, void* v_cache, int cache_cap, int batch,
+                               const int32_t* positions, int max_position, void* ws, size_t ws_bytes,
+                               llama3_stream_t stream) {
+  if (!positions) return LLAMA3_ERR_ARG;
+  if (reinterpret_cast<uintptr_t>(positions) & 3) return LLAMA3_ERR_ALIGN;
+  Workspace L;
+  L3_TRY(check_layer_args(cfg, w, rope, rope_len, x, k_cache, v_cache, cache_cap, batch, 1, max_position, ws,
+                          ws_bytes, &L));
+  cudaStream_t st = (cudaStream_t)stream;
+  if (use_tc(cfg))
+    return layer_tc_decode(cfg, w, rope, x, k_cache, v_cache, cache_cap, batch, max_position, L, ws, st, positions);
+  if (cfg->dtype == LLAMA3_DTYPE_F32)
+    return layer_simt<float>(cfg, w, rope, x, k_cache, v_cache, cache_cap, batch, 1, max_position, L, ws, st,
+                             nullptr, positions);
+  return layer_simt<bf16>(cfg, w, rope, x, k_cache, v_cache, cache_cap, batch, 1, max_position, L, ws, st,
+                          nullptr, positions);
 }
 
 int llama3_layer_forward_docs(const llama3_config* cfg, const llama3_layer_weights* w, const float* rope,

@@ -103,6 +103,45 @@ __global__ void __launch_bounds__(128) rmsnorm_bf16_warp_kernel(const bf16* __re
   }
 }
 
+// bf16 rows, few of them (decode): one CTA per row, one 16-byte chunk per
+// thread (D % 8 == 0, D <= 8192), the weight chunk fetched before the
+// reduction so both loads are in flight together.
+__global__ void __launch_bounds__(1024) rmsnorm_bf16_row_kernel(const bf16* __restrict__ x, long long row_stride,
+                                                               const bf16* __restrict__ w, bf16* __restrict__ y,
+                                                               int D, float eps) {
+  griddep_wait_and_release();
+  const int row = blockIdx.x, c = threadIdx.x, lane = c & 31;
+  const int nchunk = D >> 3;
+  uint4 v = make_uint4(0, 0, 0, 0), wv = make_uint4(0, 0, 0, 0);
+  if (c < nchunk) {
+    v = reinterpret_cast<const uint4*>(x + (size_t)row * row_stride)[c];
+    wv = __ldg(reinterpret_cast<const uint4*>(w) + c);
+  }
+  const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+  float ss = 0.f;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float a = bf16lo(u[q]), b = bf16hi(u[q]);
+    ss = fmaf(a, a, fmaf(b, b, ss));
+  }
+  __shared__ float red[32];
+  ss = warp_sum(ss);
+  if (lane == 0) red[c >> 5] = ss;
+  __syncthreads();
+  float tot = 0.f;
+  const int nw = (blockDim.x + 31) >> 5;
+  for (int i = 0; i < nw; ++i) tot += red[i];
+  const float r = rsqrtf(tot / (float)D + eps);
+  if (c < nchunk) {
+    const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      o[q] = pack_bf16x2(bf16lo(u[q]) * r * bf16lo(ww[q]), bf16hi(u[q]) * r * bf16hi(ww[q]));
+    reinterpret_cast<uint4*>(y + (size_t)row * D)[c] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
 // ---- GEMM C[m, n] = sum_k A[m, k] * B[n, k]   (fp32 result) -----------------
 // 64x64 tile, 256 threads, 4x4 outputs per thread, K staged 16 at a time.
 template <typename T>
@@ -166,10 +205,22 @@ __device__ __forceinline__ void store4(float* p, const float (&v)[4]) {
 __device__ __forceinline__ void store4(bf16* p, const float (&v)[4]) {
   *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
 }
+// v = sum over s of P[s * split_stride + idx .. +3], added in split order;
+// loads are issued four splits at a time so their latencies overlap.
 __device__ __forceinline__ void sum4_splits(const float* P, int splits, long long split_stride, long long idx,
                                             float (&v)[4]) {
   load4(P + idx, v);
-  for (int i = 1; i < splits; ++i) {
+  int i = 1;
+  for (; i + 4 <= splits; i += 4) {
+    float w[4][4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) load4(P + (size_t)(i + u) * split_stride + idx, w[u]);
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) v[q] += w[u][q];
+  }
+  for (; i < splits; ++i) {
     float w[4];
     load4(P + (size_t)i * split_stride + idx, w);
 #pragma unroll
@@ -199,44 +250,50 @@ __global__ void epi_residual_kernel(const float* __restrict__ P, int splits, lon
 // Residual add fused with the RMSNorm that follows it (decode, few rows):
 //   x[m] <- round(x[m] + sum_s P[s][m]);  xn[m] = round(x[m] * r * w),
 //   r = 1 / sqrt(mean(x[m]^2) + eps) over the rounded x ("Build your own
-// Llama 3 from scratch" §3.6 residual, §3.1 RMSNorm).  One CTA of 256 threads
-// per row, 4*G consecutive-by-4 elements per thread held in registers.
+// Llama 3 from scratch" §3.6 residual, §3.1 RMSNorm).  One CTA of 1024 threads
+// per row, 4*G consecutive-by-4 elements per thread held in registers; all
+// of a thread's loads are issued before any of its stores.
 template <int G>
-__global__ void __launch_bounds__(256) epi_residual_rmsnorm_kernel(const float* __restrict__ P, int splits,
-                                                                  long long split_stride, bf16* __restrict__ x,
-                                                                  const bf16* __restrict__ w,
-                                                                  bf16* __restrict__ xn, int D, float eps) {
+__global__ void __launch_bounds__(1024) epi_residual_rmsnorm_kernel(const float* __restrict__ P, int splits,
+                                                                   long long split_stride, bf16* __restrict__ x,
+                                                                   const bf16* __restrict__ w,
+                                                                   bf16* __restrict__ xn, int D, float eps) {
   griddep_wait_and_release();
   const int m = blockIdx.x;
-  float v[G][4];
+  float v[G][4], r[G][4];
   float ss = 0.f;
 #pragma unroll
   for (int g = 0; g < G; ++g) {
-    const int n = 4 * (threadIdx.x + 256 * g);
+    const int n = 4 * (threadIdx.x + 1024 * g);
     if (n < D) {
-      float r[4];
       sum4_splits(P, splits, split_stride, (long long)m * D + n, v[g]);
-      load4(x + (size_t)m * D + n, r);
+      load4(x + (size_t)m * D + n, r[g]);
+    }
+  }
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const int n = 4 * (threadIdx.x + 1024 * g);
+    if (n < D) {
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         // round to bf16 exactly as the stored residual stream, then square that
-        v[g][q] = __bfloat162float(__float2bfloat16_rn(v[g][q] + r[q]));
+        v[g][q] = __bfloat162float(__float2bfloat16_rn(v[g][q] + r[g][q]));
         ss = fmaf(v[g][q], v[g][q], ss);
       }
       store4(x + (size_t)m * D + n, v[g]);
     }
   }
-  __shared__ float red[8];
+  __shared__ float red[32];
   ss = warp_sum(ss);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
   __syncthreads();
   float tot = 0.f;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) tot += red[i];
+  for (int i = 0; i < 32; ++i) tot += red[i];
   const float rs = rsqrtf(tot / (float)D + eps);
 #pragma unroll
   for (int g = 0; g < G; ++g) {
-    const int n = 4 * (threadIdx.x + 256 * g);
+    const int n = 4 * (threadIdx.x + 1024 * g);
     if (n < D) {
       float wv[4], o[4];
       load4(w + n, wv);
@@ -272,14 +329,23 @@ template <typename T>
 __global__ void epi_qkv_rope_kernel(const float* __restrict__ P, int splits, long long split_stride,
                                     int M, int seq, int start_pos, int H, int KV, int hd,
                                     const float* __restrict__ rope, T* __restrict__ q_out,
-                                    T* __restrict__ k_cache, T* __restrict__ v_cache, int cap) {
+                                    T* __restrict__ k_cache, T* __restrict__ v_cache, int cap,
+                                    const int32_t* __restrict__ positions, int max_pos) {
   griddep_wait_and_release();
   const int Ntot = (H + 2 * KV) * hd;
   const long long i = ((long long)blockIdx.x * blockDim.x + threadIdx.x) * 4;
   if (i >= (long long)M * Ntot) return;
   const int m = (int)(i / Ntot);
   const int n = (int)(i % Ntot);
-  const int b = m / seq, t = m % seq, pos = start_pos + t;
+  const int b = m / seq, t = m % seq;
+  int pos = start_pos + t;
+  if (positions) {   // one token per sequence at its own position (out of range: flagged, clamped)
+    pos = positions[b];
+    if (pos < 0 || pos > max_pos) {
+      if (n == 0) record_error(LLAMA3_ERR_ARG);
+      pos = max(0, min(pos, max_pos));
+    }
+  }
   float v[4];
   sum4_splits(P, splits, split_stride, (long long)m * Ntot + n, v);
   const int d = n % hd, head = n / hd;
@@ -308,7 +374,8 @@ template <typename T>
 __global__ void attention_simt_kernel(const T* __restrict__ q, const T* __restrict__ k_cache,
                                       const T* __restrict__ v_cache, T* __restrict__ out, int B,
                                       int S, int start_pos, int H, int KV, int hd, int cap,
-                                      float scale, const int32_t* __restrict__ doc_start) {
+                                      float scale, const int32_t* __restrict__ doc_start,
+                                      const int32_t* __restrict__ positions, int max_pos) {
   griddep_wait_and_release();
   long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   int lane = threadIdx.x & 31;
@@ -325,7 +392,8 @@ __global__ void attention_simt_kernel(const T* __restrict__ q, const T* __restri
     acc[i] = 0.f;
   }
   float m = -INFINITY, l = 0.f;
-  const int last = start_pos + t;
+  // per-sequence positions (one token per sequence): clamped into range
+  const int last = positions ? max(0, min(positions[b], max_pos)) : start_pos + t;
   // document mask: keys before the start of this token's document are invisible
   const int first = doc_start ? max(0, min(doc_start[(size_t)b * S + t], last)) : 0;
   for (int j = first; j <= last; ++j) {

@@ -55,41 +55,67 @@ class Llama3Stack:
             B.llama3_layer_decode(self.cfg, self.wstructs[i], self.rope, self.rope_len, x, kc, vc,
                                   self.cache_cap, self.batch, start_pos, self.ws, self.ws_bytes, stream)
 
+    def decode_layers_ragged(self, x, positions, max_position, stream=None, layers=None):
+        """One decode step where sequence b's token sits at positions[b]
+        (int32 device tensor); max_position bounds them all."""
+        for i in (range(len(self.layers)) if layers is None else layers):
+            kc, vc = self.caches[i]
+            B.llama3_layer_decode_ragged(self.cfg, self.wstructs[i], self.rope, self.rope_len, x, kc, vc,
+                                         self.cache_cap, self.batch, positions, max_position, self.ws,
+                                         self.ws_bytes, stream)
+
     def lm_head(self, h, rows, row_stride, logits=None, stream=None):
         B.llama3_lm_head_argmax(self.cfg, self.out["norm"], self.out["output"], h, rows, row_stride,
                                 self.ids_out, logits, self.ws, self.ws_bytes, stream)
         return self.ids_out[:rows]
 
-    # -- greedy generation ("Build your own Llama 3 from scratch" 六, temperature 0)
-    def generate(self, prompt_ids, n_new, eos_id=None, stream=None):
+    # -- generation ("Build your own Llama 3 from scratch" 六 generate)
+    def generate(self, prompt_ids, n_new, eos_id=None, stream=None, temperature=0.0, top_p=0.9, seed=0,
+                 return_logits=False):
         """Prefill the prompts (int32 [batch, S] on the device), then decode
-        n_new tokens greedily.  Each step's LM head writes its argmax straight
-        into row `step` of a [n_new, batch] device buffer, which the next
-        step's embedding reads, so no token leaves the device in the loop.
-        Returns the [batch, n_new] tokens as a host array; after a sequence's
-        first eos_id the rest of its row is eos_id (the pages stop the loop
-        there)."""
+        n_new tokens.  temperature <= 0 is greedy (the LM head's argmax);
+        otherwise each step's fp32 logits go through llama3_sample_top_p with
+        the step number as the draw's counter offset.  Each step writes its
+        tokens straight into row `step` of a [n_new, batch] device buffer,
+        which the next step's embedding reads, so no token leaves the device
+        in the loop.  Returns the [batch, n_new] tokens as a host array (and,
+        with return_logits, the [n_new, batch, vocab] fp32 logits); after a
+        sequence's first eos_id the rest of its row is eos_id (the page stops
+        the loop there)."""
         import torch
         Bn, S = prompt_ids.shape
         assert Bn == self.batch and S + n_new - 1 <= self.cache_cap
-        D = self.cfg_dict["dim"]
+        D, V = self.cfg_dict["dim"], self.cfg_dict["vocab"]
+        sampling = temperature > 0
         x = torch.empty((Bn, S, D), dtype=self.dtype, device=self.device)
         self.embed(prompt_ids, x, stream)
         self.forward_layers(x, S, 0, stream)
         row = (Bn + 3) // 4 * 4            # keeps every step's ids 16-byte aligned
         out = torch.empty((n_new, row), dtype=torch.int32, device=self.device)
-        B.llama3_lm_head_argmax(self.cfg, self.out["norm"], self.out["output"], x[:, -1], Bn, S * D, out[0], None,
-                                self.ws, self.ws_bytes, stream)
+        keep = return_logits or sampling
+        logits = torch.empty((n_new if return_logits else 1, Bn, V), dtype=torch.float32,
+                             device=self.device) if keep else None
+        pick = torch.empty((row,), dtype=torch.int32, device=self.device) if sampling else None
+
+        def head(h, stride, step):
+            lg = logits[step if return_logits else 0] if keep else None
+            B.llama3_lm_head_argmax(self.cfg, self.out["norm"], self.out["output"], h, Bn, stride,
+                                    pick if sampling else out[step], lg, self.ws, self.ws_bytes, stream)
+            if sampling:
+                B.llama3_sample_top_p(lg, Bn, V, V, temperature, top_p, seed, step, out[step], stream)
+
+        head(x[:, -1], S * D, 0)
         xd = torch.empty((Bn, 1, D), dtype=self.dtype, device=self.device)
         for step in range(1, n_new):
             B.llama3_embed(self.cfg, out[step - 1], self.out["tok_embeddings"], xd, Bn, stream)
             self.decode_layers(xd, S + step - 1, stream)
-            B.llama3_lm_head_argmax(self.cfg, self.out["norm"], self.out["output"], xd, Bn, D, out[step], None,
-                                    self.ws, self.ws_bytes, stream)
+            head(xd, D, step)
         toks = out[:, :Bn].t().cpu().numpy()
         if eos_id is not None:   # host-side: hold the end token once emitted
             for b in range(Bn):
                 hits = (toks[b] == eos_id).nonzero()[0]
                 if hits.size:
                     toks[b, hits[0]:] = eos_id
+        if return_logits:
+            return toks, logits.cpu().numpy()
         return toks

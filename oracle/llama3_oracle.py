@@ -376,9 +376,15 @@ def top_p_sample(logits, temperature, top_p, word):
     kept = np.zeros(p.shape, dtype=bool)
     kept[order[keep_ranked]] = True
     n_keep = int(keep_ranked.sum())
-    cut = top_p - before[n_keep - 1]
-    if n_keep < len(ranked):
-        cut = min(cut, before[n_keep] - top_p)
+    # Decisions that rounding cannot flip are no boundary: the top token (mass
+    # before it exactly 0) and, for top_p >= 1, every token (the mass before
+    # any token is below 1).
+    cut = np.inf
+    if top_p < 1:
+        if n_keep > 1:
+            cut = top_p - before[n_keep - 1]
+        if n_keep < len(ranked):
+            cut = min(cut, before[n_keep] - top_p)
     idx = np.nonzero(kept)[0]
     run = np.cumsum(p[idx])
     target = (int(word) / 2.0 ** 64) * run[-1]

@@ -42,11 +42,12 @@ def small_bf16(**kw):
 
 
 # ------------------------------------------------------------------ RMSNorm
-@pytest.mark.parametrize("dtype,D,H", [("bf16", 4096, 32), ("bf16", 576, 9), ("f32", 64, 4)])
-def test_rmsnorm(dtype, D, H):
+@pytest.mark.parametrize("dtype,D,H,rows", [("bf16", 4096, 32, 37), ("bf16", 576, 9, 37), ("f32", 64, 4, 37),
+                                            ("bf16", 4096, 32, 600), ("bf16", 8192, 64, 3), ("bf16", 960, 10, 513), ("bf16", 960, 10, 5)])
+def test_rmsnorm(dtype, D, H, rows):
     tdt = torch.float32 if dtype == "f32" else torch.bfloat16
     g = torch.Generator(device="cpu").manual_seed(5)
-    rows, stride = 37, D + 64
+    stride = D + 64
     x = (torch.randn((rows, stride), generator=g) * 3).to(tdt).to(DEV)
     nw = (1 + 0.1 * torch.randn((D,), generator=g)).to(tdt).to(DEV)
     y = torch.empty((rows, D), dtype=tdt, device=DEV)
@@ -103,9 +104,9 @@ def _attn_case(Bn, S, P, H, KV, hd, seed):
     (1, 1, 0, 8, 2, 128), (4, 1, 1, 8, 1, 64), (3, 1, 1000, 32, 8, 128), (2, 1, 300, 8, 2, 96),
     (2, 1, 777, 16, 16, 64), (2, 1, 500, 12, 4, 64), (1, 150, 20, 12, 4, 64), (2, 1, 130, 16, 1, 128),
     (1, 1, 8192, 32, 8, 128), (2, 300, 0, 6, 2, 96)])
-@pytest.mark.parametrize("variant", [1, 2])
+@pytest.mark.parametrize("variant", [1, 2, 3])
 def test_attention(Bn, S, P, H, KV, hd, variant):
-    if variant == 2 and S == 1:
+    if variant != 2 and S == 1:
         pytest.skip("single-token steps take the decode kernel")
     B.llama3_set_flash_variant(variant)
     q, kc, vc, cap = _attn_case(Bn, S, P, H, KV, hd, Bn * 1000 + S + P + hd)
@@ -167,6 +168,12 @@ def test_char_8l_stack_and_lm_head(path):
 @pytest.mark.parametrize("path", [0, 2])
 def test_gqa_768_layer(path):
     _run_layers_vs_oracle(wl("gqa_768"), path=path)
+
+
+@pytest.mark.parametrize("variant", [1, 3])
+def test_gqa_768_layer_other_attention_designs(variant):
+    B.llama3_set_flash_variant(variant)
+    _run_layers_vs_oracle(wl("gqa_768"))
 
 
 def test_chunked_prefill_then_decode_steps():
@@ -315,9 +322,9 @@ def _doc_starts(Bn, S, P, seed):
 
 @pytest.mark.parametrize("Bn,S,P,H,KV,hd,path", [
     (2, 300, 0, 8, 2, 128, 0), (2, 200, 37, 8, 2, 64, 0), (1, 257, 0, 12, 4, 96, 0), (2, 130, 5, 8, 2, 64, 1)])
-@pytest.mark.parametrize("variant", [1, 2])
+@pytest.mark.parametrize("variant", [1, 2, 3])
 def test_attention_document_mask(Bn, S, P, H, KV, hd, path, variant):
-    if variant == 2 and path != 0:
+    if variant != 2 and path != 0:
         pytest.skip("the SIMT path has one attention kernel")
     B.llama3_set_kernel_path(path)
     B.llama3_set_flash_variant(variant)
@@ -348,3 +355,39 @@ def test_layer_forward_packed_documents():
                                     w.batch, w.seq, 0, dsd, st.ws, st.ws_bytes)
     want, _, _ = O.forward_stack(x0, [oracle_layer(l) for l in layers], oracle_cfg(w), doc_start=ds)
     assert_close(x, want, "bf16", "packed documents")
+
+
+# ------------------------------------------------------------ ragged decode
+@pytest.mark.parametrize("dtype,path", [("bf16", 0), ("bf16", 1), ("f32", 0)])
+def test_ragged_decode_step_matches_per_sequence_oracle(dtype, path):
+    """One decode step where every sequence's token sits at its own position
+    (empty prefix, tile boundaries, the maximum): each sequence equals the
+    oracle's block run alone at that position; new K/V land at their rows."""
+    B.llama3_set_kernel_path(path)
+    if dtype == "f32":
+        w = I.Workload(name="tiny", dim=64, n_layers=1, n_heads=4, n_kv_heads=2, ffn_hidden=192, vocab=100,
+                       batch=5, seq=1, dtype="f32", input_kind="activations", seed=13)
+    else:
+        w = small_bf16(batch=5, n_layers=1)
+    layer = I.layer_weights(w, 0, DEV, "random")
+    cap = 200
+    positions = np.array([0, 37, 128, 129, 150], dtype=np.int32)
+    st = Llama3Stack(w.cfg(), [layer], I.output_weights(w, DEV), w.batch, cap, 1)
+    kc, vc = st.caches[0]
+    g = torch.Generator(device="cpu").manual_seed(21)
+    k0 = torch.randn(kc.shape, generator=g).to(kc.dtype)
+    v0 = torch.randn(vc.shape, generator=g).to(vc.dtype)
+    kc.copy_(k0.to(DEV)); vc.copy_(v0.to(DEV))
+    x = torch.randn((w.batch, 1, w.dim), generator=g).to(kc.dtype)
+    xd = x.to(DEV)
+    st.decode_layers_ragged(xd, torch.from_numpy(positions).to(DEV), int(positions.max()))
+    torch.cuda.synchronize()
+    lo, oc = oracle_layer(layer), oracle_cfg(w)
+    for b, p in enumerate(positions):
+        kb, vb = f64(k0[b:b + 1]), f64(v0[b:b + 1])
+        want = O.decoder_block(f64(x[b:b + 1]), lo, oc, kb, vb, start_pos=int(p))
+        assert_close(xd[b:b + 1], want, dtype, f"ragged decode b={b} pos={p}")
+        assert_close(kc[b, p], kb[0, p], dtype, f"k row b={b}")
+        assert_close(vc[b, p], vb[0, p], dtype, f"v row b={b}")
+        # the rest of the cache is untouched
+        np.testing.assert_array_equal(f64(kc[b, :p]), f64(k0[b, :p]))

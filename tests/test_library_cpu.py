@@ -105,3 +105,26 @@ def test_kernel_path_and_wait_limit_switches():
     assert B.llama3_set_kernel_path(0) == 1
     old = B.llama3_set_wait_limit_ms(500)
     assert B.llama3_set_wait_limit_ms(old) == 500
+
+
+def test_sample_top_p_rejects_bad_arguments_before_launch():
+    lib = B.lib()
+    f = ctypes.c_float
+    s = lambda **k: lib.llama3_sample_top_p(k.get("logits", FAKE), k.get("rows", 4), k.get("ld", 100),
+                                            k.get("vocab", 100), f(k.get("t", 0.7)), f(k.get("p", 0.9)),
+                                            1, 0, k.get("ids", FAKE), None)
+    assert s(rows=0) == 1
+    assert s(vocab=0) == 1
+    assert s(ld=99) == 1
+    assert s(p=-0.1) == 1
+    assert s(p=float("nan")) == 1
+    assert s(t=float("nan")) == 1
+    assert s(logits=None) == 1
+    assert s(ids=ctypes.c_void_p(18)) == 2   # ids not 4-byte aligned
+    assert B.KERNEL_KINDS["sample"] == 11
+
+
+def test_flash_variant_switch():
+    old = B.llama3_set_flash_variant(1)
+    assert B.llama3_set_flash_variant(7) == 1      # values other than 1 select the second design
+    assert B.llama3_set_flash_variant(old) == 2
