@@ -348,14 +348,15 @@ int llama3_set_wait_limit_ms(int ms);
  * 0: ordinary launches.  Returns the previous value. */
 int llama3_set_programmatic_launch(int on);
 
-/* Prefill attention kernel design (bf16, tcgen05 path): 2 (default) = two
- * softmax threads per query row (each over half the keys of a tile) with P
- * written back into tensor memory; 1 = one softmax thread per row with P
- * staged in shared memory; 3 = one softmax thread per row holding the whole
- * row of a tile in registers (warpgroup register reallocation) with P in
- * tensor memory.  All compute the same attention.  Values other than 1 and 3
- * select 2.  Variant 3 returns LLAMA3_ERR_UNSUPPORTED if the compiled kernel's
- * register count cannot fund its register split.  Returns the previous value. */
+/* Prefill attention kernel design (bf16, tcgen05 path): 3 (default) = one
+ * softmax thread per query row holding the whole row of a tile in registers
+ * (warpgroup register reallocation) with P in tensor memory; 1 = one softmax
+ * thread per row with P staged in shared memory; 2 = two softmax threads per
+ * row (each over half the keys of a tile) with P in tensor memory; 4 = as 3
+ * with P staged in shared memory.  All compute the same attention.  Values
+ * outside 1..4 select 3.  Variants 3 and 4 return LLAMA3_ERR_UNSUPPORTED if
+ * the compiled kernel's register count cannot fund their register split.
+ * Returns the previous value. */
 int llama3_set_flash_variant(int variant);
 
 #ifdef __cplusplus

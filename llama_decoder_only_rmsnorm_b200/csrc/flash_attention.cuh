@@ -71,6 +71,14 @@ __device__ __forceinline__ void flash_unit(const FlashShape& fs, int u, int& b, 
   g = r % fs.KV;
   b = r / fs.KV;
 }
+// The k-th unit of this CTA.  Units are numbered longest first; taking them
+// in rows of gridDim.x, alternately left to right and right to left, evens out
+// the per-CTA totals (for the 8B prefill the busiest CTA gets 229 key tiles
+// instead of 256 with a plain stride, against a mean of 225).
+__device__ __forceinline__ int flash_snake(int k) {
+  const int G = gridDim.x, c = blockIdx.x;
+  return k * G + ((k & 1) ? G - 1 - c : c);
+}
 __device__ __forceinline__ int flash_ntiles(const FlashShape& fs, int qt) {
   const int last_key = min(fs.P + qt * 128 + 127, fs.P + fs.S - 1);
   return last_key / 128 + 1;
@@ -137,7 +145,7 @@ __global__ void __launch_bounds__(384, 1)
       uint32_t kph = 0, vph = 0, qph[2] = {0, 0};
       bool ok = true;
       uint32_t kiss = 0, kpar = 0, viss = 0, vpar = 0, qiss = 0, qpar = 0;
-      for (int u = blockIdx.x; u < fs.units && ok; u += gridDim.x) {
+      for (int k_ = 0, u = flash_snake(0); u < fs.units && ok; u = flash_snake(++k_)) {
         int b, g, pair, qt;
         flash_unit(fs, u, b, g, pair, qt);
         const int nt = flash_ntiles(fs, qt);
@@ -210,7 +218,7 @@ __global__ void __launch_bounds__(384, 1)
         }
         tc_commit(&o_done[s]);
       };
-      for (int u = blockIdx.x; u < fs.units && ok; u += gridDim.x) {
+      for (int k_ = 0, u = flash_snake(0); u < fs.units && ok; u = flash_snake(++k_)) {
         int b, g, pair, qt;
         flash_unit(fs, u, b, g, pair, qt);
         const int nt = flash_ntiles(fs, qt);
@@ -266,7 +274,7 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t o_tmem = s_tmem + 128;
     uint8_t* p_smem = smem + C::OFF_P + slot * C::P_BYTES;
     uint32_t sph = 0, oph = 0;
-    for (int u = blockIdx.x; u < fs.units; u += gridDim.x) {
+    for (int k_ = 0, u = flash_snake(0); u < fs.units; u = flash_snake(++k_)) {
       int b, g, pair, qt;
       flash_unit(fs, u, b, g, pair, qt);
       if (slot == 1 && !(pair * 2 + 1 < fs.n_rep)) continue;

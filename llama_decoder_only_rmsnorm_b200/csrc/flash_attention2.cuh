@@ -103,7 +103,7 @@ __global__ void __launch_bounds__(640, 1)
       uint32_t kph = 0, vph = 0, qph[2] = {0, 0};
       bool ok = true;
       uint32_t kiss = 0, kpar = 0, viss = 0, vpar = 0, qiss = 0, qpar = 0;
-      for (int u = blockIdx.x; u < fs.units && ok; u += gridDim.x) {
+      for (int k_ = 0, u = flash_snake(0); u < fs.units && ok; u = flash_snake(++k_)) {
         int b, g, pair, qt;
         flash_unit(fs, u, b, g, pair, qt);
         const int nt = flash_ntiles(fs, qt);
@@ -189,7 +189,7 @@ __global__ void __launch_bounds__(640, 1)
         tc_commit(&o_done[s]);
         opend[s] = true;
       };
-      for (int u = blockIdx.x; u < fs.units && ok; u += gridDim.x) {
+      for (int k_ = 0, u = flash_snake(0); u < fs.units && ok; u = flash_snake(++k_)) {
         int b, g, pair, qt;
         flash_unit(fs, u, b, g, pair, qt);
         const int nt = flash_ntiles(fs, qt);
@@ -260,7 +260,7 @@ __global__ void __launch_bounds__(640, 1)
       xpar ^= 1;
       return done;
     };
-    for (int u = blockIdx.x; u < fs.units; u += gridDim.x) {
+    for (int k_ = 0, u = flash_snake(0); u < fs.units; u = flash_snake(++k_)) {
       int b, g, pair, qt;
       flash_unit(fs, u, b, g, pair, qt);
       if (slot == 1 && !(pair * 2 + 1 < fs.n_rep)) continue;

@@ -51,31 +51,26 @@ __device__ __forceinline__ void flash3_load_row(uint32_t taddr, uint32_t (&a)[32
 }
 
 // p = 2^(s*scale - m) for 32 scores, their sum, and the bf16 pairs stored
-// to the 16 TMEM columns at taddr.
-// (Masked scores were already set to -inf by flash3_row_max; on masked tiles
-// every exponent takes the MUFU path, which gives exactly 0 there.)
-template <bool MASKED>
+// to the 16 TMEM columns at taddr.  The exponent is rounded to bf16 and two
+// exponentials come from one packed MUFU operation, already in the bf16 pair
+// form P.V consumes; the row sum adds those same rounded values, so the
+// normaliser matches what the MMA multiplies.  (Masked scores are -inf: 0.)
 __device__ __forceinline__ void flash3_exp_chunk(const uint32_t (&r)[32], float scl, float neg_m, float& sum_a,
                                                  float& sum_b, uint32_t taddr) {
   uint32_t pk[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    float x0, x1, p0, p1;
+    float x0, x1;
     fma2(x0, x1, __uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), scl, scl, neg_m, neg_m);
-    if (!MASKED && (i & 7) < 3) {   // 6 of every 16 pairs on the FMA pipe (unmasked tiles only)
-      exp2_poly2(x0, x1, p0, p1);
-    } else {
-      p0 = ex2_approx(x0);
-      p1 = ex2_approx(x1);
-    }
-    add2(sum_a, sum_b, p0, p1);
-    pk[i] = pack_bf16x2(p0, p1);
+    pk[i] = ex2_bf16x2(pack_bf16x2(x0, x1));
+    add2(sum_a, sum_b, bf16lo(pk[i]), bf16hi(pk[i]));
   }
   tmem_st16(taddr, pk);
 }
 
 template <bool MASKED>
-__device__ __forceinline__ float flash3_row_max(uint32_t (&r)[32], int key0, int qpos, int lo, float mx) {
+__device__ __forceinline__ float flash3_row_max(uint32_t (&r)[32], int key0, int qpos, int lo) {
+  float mx = -INFINITY;
   if (MASKED) {
 #pragma unroll
     for (int i = 0; i < 32; ++i)
@@ -140,7 +135,7 @@ __global__ void __launch_bounds__(kFlash3Threads, 1)
       uint32_t kph = 0, vph = 0, qph = 0;   // qph: phase bit per Q slot
       bool ok = true;
       uint32_t kiss = 0, kpar = 0, viss = 0, vpar = 0, qiss = 0, qpar = 0;
-      for (int u = blockIdx.x; u < fs.units && ok; u += gridDim.x) {
+      for (int k_ = 0, u = flash_snake(0); u < fs.units && ok; u = flash_snake(++k_)) {
         int b, g, pair, qt;
         flash_unit(fs, u, b, g, pair, qt);
         const int nt = flash_ntiles(fs, qt);
@@ -223,7 +218,7 @@ __global__ void __launch_bounds__(kFlash3Threads, 1)
         tc_commit(&o_done[s]);
         opend |= 1u << s;
       };
-      for (int u = blockIdx.x; u < fs.units && ok; u += gridDim.x) {
+      for (int k_ = 0, u = flash_snake(0); u < fs.units && ok; u = flash_snake(++k_)) {
         int b, g, pair, qt;
         flash_unit(fs, u, b, g, pair, qt);
         const int nt = flash_ntiles(fs, qt);
@@ -283,7 +278,7 @@ __global__ void __launch_bounds__(kFlash3Threads, 1)
     const uint32_t s_tmem = tmem_base + lane_off + slot * 256;
     const uint32_t o_tmem = s_tmem + 128;
     uint32_t sph = 0, oph = 0;
-    for (int u = blockIdx.x; u < fs.units; u += gridDim.x) {
+    for (int k_ = 0, u = flash_snake(0); u < fs.units; u = flash_snake(++k_)) {
       int b, g, pair, qt;
       flash_unit(fs, u, b, g, pair, qt);
       if (slot == 1 && !(pair * 2 + 1 < fs.n_rep)) continue;
@@ -302,18 +297,19 @@ __global__ void __launch_bounds__(kFlash3Threads, 1)
         const int key0 = j * 128;
         uint32_t ra[32], rb[32], rc[32], rd[32];
         flash3_load_row(s_tmem, ra, rb, rc, rd);
-        float mx = -INFINITY;
+        float m0, m1, m2, m3;   // four independent chains
         if (need_mask) {
-          mx = flash3_row_max<true>(ra, key0, qpos, lo, mx);
-          mx = flash3_row_max<true>(rb, key0 + 32, qpos, lo, mx);
-          mx = flash3_row_max<true>(rc, key0 + 64, qpos, lo, mx);
-          mx = flash3_row_max<true>(rd, key0 + 96, qpos, lo, mx);
+          m0 = flash3_row_max<true>(ra, key0, qpos, lo);
+          m1 = flash3_row_max<true>(rb, key0 + 32, qpos, lo);
+          m2 = flash3_row_max<true>(rc, key0 + 64, qpos, lo);
+          m3 = flash3_row_max<true>(rd, key0 + 96, qpos, lo);
         } else {
-          mx = flash3_row_max<false>(ra, key0, qpos, lo, mx);
-          mx = flash3_row_max<false>(rb, key0 + 32, qpos, lo, mx);
-          mx = flash3_row_max<false>(rc, key0 + 64, qpos, lo, mx);
-          mx = flash3_row_max<false>(rd, key0 + 96, qpos, lo, mx);
+          m0 = flash3_row_max<false>(ra, key0, qpos, lo);
+          m1 = flash3_row_max<false>(rb, key0 + 32, qpos, lo);
+          m2 = flash3_row_max<false>(rc, key0 + 64, qpos, lo);
+          m3 = flash3_row_max<false>(rd, key0 + 96, qpos, lo);
         }
+        const float mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
         const float m_tile = mx * fs.scale_log2;   // scale_log2 > 0: max commutes with the scale
         // the previous tile's P.V must be complete before O is rescaled (and
         // before P is rewritten: the MMA issuer also waits for it before S)
@@ -344,17 +340,10 @@ __global__ void __launch_bounds__(kFlash3Threads, 1)
         const float scl = fs.scale_log2;
         const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;   // a row with no visible key yet: p = 0
         float sum_a = 0.f, sum_b = 0.f;
-        if (need_mask) {
-          flash3_exp_chunk<true>(ra, scl, neg_m, sum_a, sum_b, s_tmem);
-          flash3_exp_chunk<true>(rb, scl, neg_m, sum_a, sum_b, s_tmem + 16);
-          flash3_exp_chunk<true>(rc, scl, neg_m, sum_a, sum_b, s_tmem + 32);
-          flash3_exp_chunk<true>(rd, scl, neg_m, sum_a, sum_b, s_tmem + 48);
-        } else {
-          flash3_exp_chunk<false>(ra, scl, neg_m, sum_a, sum_b, s_tmem);
-          flash3_exp_chunk<false>(rb, scl, neg_m, sum_a, sum_b, s_tmem + 16);
-          flash3_exp_chunk<false>(rc, scl, neg_m, sum_a, sum_b, s_tmem + 32);
-          flash3_exp_chunk<false>(rd, scl, neg_m, sum_a, sum_b, s_tmem + 48);
-        }
+        flash3_exp_chunk(ra, scl, neg_m, sum_a, sum_b, s_tmem);
+        flash3_exp_chunk(rb, scl, neg_m, sum_a, sum_b, s_tmem + 16);
+        flash3_exp_chunk(rc, scl, neg_m, sum_a, sum_b, s_tmem + 32);
+        flash3_exp_chunk(rd, scl, neg_m, sum_a, sum_b, s_tmem + 48);
         l += sum_a + sum_b;
         tc_wait_st();
         tc_fence_before();

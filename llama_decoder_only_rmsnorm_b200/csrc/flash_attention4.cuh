@@ -1,0 +1,352 @@
+// flash_attention4.cuh -- causal GQA prefill attention, tcgen05, fourth design.
+//
+// Computes the same thing as flash_attention.cuh ("Build your own Llama 3 from
+// scratch" §3.4; document mask of 附 1).  Softmax as in the third design (one
+// thread per query row, the whole 128-score row of a tile in registers after
+// a setmaxnreg register split, packed bf16 exponentials), but P goes to shared
+// memory as in the first design: the next tile's S can then be issued right
+// behind P.V (they touch different TMEM columns), so the tensor pipe does not
+// drain while P.V finishes.  The softmax waits for the previous P.V before it
+// overwrites P.  Shared memory: Q for two heads, one K stage, two V stages,
+// P for two heads.
+#pragma once
+#include "flash_attention3.cuh"
+
+namespace l3 {
+
+
+template <int HD>
+struct Flash4Cfg {
+  static constexpr int CHUNKS = (HD + 63) / 64;
+  static constexpr int TILE_BYTES = 128 * 128;
+  static constexpr int Q_BYTES = CHUNKS * TILE_BYTES;
+  static constexpr int KV_BYTES = CHUNKS * TILE_BYTES;
+  static constexpr int P_BYTES = 2 * TILE_BYTES;    // 128 rows x 128 keys, two 64-key slabs
+  static constexpr int KST = 1, VST = 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
+  static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
+  static constexpr int OFF_P = OFF_V + VST * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
+  static constexpr int N_BARS = 2 + 2 + 2 * KST + 2 * VST + 2 + 2 + 2;
+  static constexpr int SMEM_BYTES = 1024 + OFF_BAR + N_BARS * 8 + 16;
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
+  static_assert(HD % 32 == 0 && HD <= 128, "head_dim");
+};
+
+// p = 2^(s*scale - m) for keys 32c .. 32c+31 of this row, their sum, and
+// the bf16 pairs stored into the row's P line in shared memory, in the
+// 128-byte-swizzled K-major layout the MMA reads (two 64-key slabs).
+__device__ __forceinline__ void flash4_exp_chunk(const uint32_t (&r)[32], float scl, float neg_m, float& sum_a,
+                                                 float& sum_b, uint8_t* p_smem, int row, int c) {
+  uint32_t pk[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    float x0, x1;
+    fma2(x0, x1, __uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), scl, scl, neg_m, neg_m);
+    pk[i] = ex2_bf16x2(pack_bf16x2(x0, x1));
+    add2(sum_a, sum_b, bf16lo(pk[i]), bf16hi(pk[i]));
+  }
+  uint8_t* slab = p_smem + (c >> 1) * (128 * 128) + row * 128;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int piece = (c & 1) * 4 + q;
+    *reinterpret_cast<uint4*>(slab + ((piece ^ (row & 7)) << 4)) =
+        make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+  }
+}
+
+template <int HD>
+__global__ void __launch_bounds__(kFlash3Threads, 1)
+    flash_attention4_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
+                            const __grid_constant__ CUtensorMap mapV, bf16* __restrict__ out, const FlashShape fs,
+                            const unsigned long long wait_ns) {
+  using C = Flash4Cfg<HD>;
+  constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, 0, 0);
+  constexpr uint32_t IDESC_O = idesc_bf16_f32(128, HD, 0, 1);   // A = P (smem), B = V MN-major
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* q_full = bars;
+  uint64_t* q_empty = q_full + 2;
+  uint64_t* k_full = q_empty + 2;
+  uint64_t* k_empty = k_full + C::KST;
+  uint64_t* v_full = k_empty + C::KST;
+  uint64_t* v_empty = v_full + C::VST;
+  uint64_t* s_full = v_empty + C::VST;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* o_done = p_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_done + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&q_full[s], 1); mbar_init(&q_empty[s], 1);
+      mbar_init(&s_full[s], 1); mbar_init(&p_full[s], 128); mbar_init(&o_done[s], 1);
+    }
+    for (int s = 0; s < C::KST; ++s) { mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1); }
+    for (int s = 0; s < C::VST; ++s) { mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1); }
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&mapQ); prefetch_tensormap(&mapK); prefetch_tensormap(&mapV);
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  // Each warpgroup takes its register share (all threads of a warpgroup
+  // execute it).  The two roles stay in separate branches up to the final
+  // barrier, so the register limit of one never applies to the other's code.
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kFlash3LowRegs));
+    griddep_wait_and_release();
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      int ks = 0, vs = 0;
+      uint32_t kph = 0, vph = 0, qph = 0;   // qph: phase bit per Q slot
+      bool ok = true;
+      uint32_t kiss = 0, kpar = 0, viss = 0, vpar = 0, qiss = 0, qpar = 0;
+      for (int k_ = 0, u = flash_snake(0); u < fs.units && ok; u = flash_snake(++k_)) {
+        int b, g, pair, qt;
+        flash_unit(fs, u, b, g, pair, qt);
+        const int nt = flash_ntiles(fs, qt);
+        const bool has1 = pair * 2 + 1 < fs.n_rep;
+        for (int s = 0; s < 2 && ok; ++s) {
+          if (s == 1 && !has1) break;
+          if (!mbar_wait(&q_empty[s], ((qph >> s) & 1u) ^ 1u, wait_ns)) { ok = false; break; }
+          mbar_arrive_expect_tx(&q_full[s], C::Q_BYTES);
+          const int h = g * fs.n_rep + pair * 2 + s;
+          for (int c = 0; c < C::CHUNKS; ++c)
+            tma_load_4d(smem + C::OFF_Q + s * C::Q_BYTES + c * C::TILE_BYTES, &mapQ, &q_full[s], c * 64, h,
+                        qt * 128, b);
+          qiss |= 1u << s; qpar = (qpar & ~(1u << s)) | (qph & (1u << s));
+          qph ^= 1u << s;
+        }
+        const int jt0 = flash_first_tile(fs, b, qt);
+        for (int j = jt0; j < nt && ok; ++j) {
+          if (!mbar_wait(&k_empty[ks], kph ^ 1u, wait_ns)) { ok = false; break; }
+          mbar_arrive_expect_tx(&k_full[ks], C::KV_BYTES);
+          for (int c = 0; c < C::CHUNKS; ++c)
+            tma_load_4d(smem + C::OFF_K + ks * C::KV_BYTES + c * C::TILE_BYTES, &mapK, &k_full[ks], c * 64, g,
+                        j * 128, b);
+          kiss |= 1u << ks; kpar = (kpar & ~(1u << ks)) | (kph << ks);
+          if (++ks == C::KST) { ks = 0; kph ^= 1u; }
+          if (!mbar_wait(&v_empty[vs], vph ^ 1u, wait_ns)) { ok = false; break; }
+          mbar_arrive_expect_tx(&v_full[vs], C::KV_BYTES);
+          for (int c = 0; c < C::CHUNKS; ++c)
+            tma_load_4d(smem + C::OFF_V + vs * C::KV_BYTES + c * C::TILE_BYTES, &mapV, &v_full[vs], c * 64, g,
+                        j * 128, b);
+          viss |= 1u << vs; vpar = (vpar & ~(1u << vs)) | (vph << vs);
+          if (++vs == C::VST) { vs = 0; vph ^= 1u; }
+        }
+      }
+      for (int s = 0; s < 2; ++s)
+        if (qiss & (1u << s)) mbar_wait(&q_full[s], (qpar >> s) & 1u, wait_ns);
+      for (int s = 0; s < C::KST; ++s)
+        if (kiss & (1u << s)) mbar_wait(&k_full[s], (kpar >> s) & 1u, wait_ns);
+      for (int s = 0; s < C::VST; ++s)
+        if (viss & (1u << s)) mbar_wait(&v_full[s], (vpar >> s) & 1u, wait_ns);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      int ks = 0, vs = 0;
+      // phase bits per slot (bit s) of the Q and P barriers as this thread sees them
+      uint32_t kph = 0, vph = 0, qph = 0, pph = 0;
+      bool ok = true;
+      const uint32_t q_addr = smem_u32(smem + C::OFF_Q);
+      const uint32_t p_addr = smem_u32(smem + C::OFF_P);
+      auto issue_s = [&](int s, int kst) {
+        const uint32_t d = tmem_base + s * 256;
+        const uint32_t qa = q_addr + s * C::Q_BYTES;
+        const uint32_t ka = smem_u32(smem + C::OFF_K + kst * C::KV_BYTES);
+#pragma unroll
+        for (int k = 0; k < HD / 16; ++k) {
+          const uint32_t off = (k >> 2) * C::TILE_BYTES + (k & 3) * 32;
+          tc_mma_f16_ss(d, sw128_desc(qa + off, 1024, 16), sw128_desc(ka + off, 1024, 16), IDESC_S, k > 0);
+        }
+        tc_commit(&s_full[s]);
+      };
+      auto issue_pv = [&](int s, int vst, bool accumulate) {
+        const uint32_t d = tmem_base + s * 256 + 128;
+        const uint32_t pa = p_addr + s * C::P_BYTES;
+        const uint32_t va = smem_u32(smem + C::OFF_V + vst * C::KV_BYTES);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {   // 128 keys, 16 per MMA
+          const uint64_t adesc = sw128_desc(pa + (k >> 2) * C::TILE_BYTES + (k & 3) * 32, 1024, 16);
+          tc_mma_f16_ss(d, adesc, sw128_desc(va + k * 2048, 1024, C::TILE_BYTES), IDESC_O,
+                        (accumulate || k > 0) ? 1u : 0u);
+        }
+        tc_commit(&o_done[s]);
+      };
+      for (int k_ = 0, u = flash_snake(0); u < fs.units && ok; u = flash_snake(++k_)) {
+        int b, g, pair, qt;
+        flash_unit(fs, u, b, g, pair, qt);
+        const int nt = flash_ntiles(fs, qt);
+        const int nslots = (pair * 2 + 1 < fs.n_rep) ? 2 : 1;
+        for (int s = 0; s < nslots; ++s) {
+          if (!mbar_wait(&q_full[s], (qph >> s) & 1u, wait_ns)) ok = false;
+          qph ^= 1u << s;
+        }
+        if (!ok) break;
+        tc_fence_after();
+        const int jt0 = flash_first_tile(fs, b, qt);
+        if (!mbar_wait(&k_full[ks], kph, wait_ns)) break;
+        tc_fence_after();
+        for (int s = 0; s < nslots; ++s) issue_s(s, ks);
+        tc_commit(&k_empty[ks]);
+        if (++ks == C::KST) { ks = 0; kph ^= 1u; }
+        for (int j = jt0; j < nt && ok; ++j) {
+          if (!mbar_wait(&v_full[vs], vph, wait_ns)) { ok = false; break; }
+          const bool more = j + 1 < nt;
+          bool k_ready = false;
+          for (int s = 0; s < nslots; ++s) {
+            if (!mbar_wait(&p_full[s], (pph >> s) & 1u, wait_ns)) { ok = false; break; }
+            pph ^= 1u << s;
+            tc_fence_after();
+            issue_pv(s, vs, j > jt0);
+            if (more) {
+              if (!k_ready && !mbar_wait(&k_full[ks], kph, wait_ns)) { ok = false; break; }
+              k_ready = true;
+              tc_fence_after();
+              issue_s(s, ks);   // S and P.V use different TMEM columns: no wait
+            }
+          }
+          if (!ok) break;
+          tc_commit(&v_empty[vs]);
+          if (++vs == C::VST) { vs = 0; vph ^= 1u; }
+          if (more) {
+            tc_commit(&k_empty[ks]);
+            if (++ks == C::KST) { ks = 0; kph ^= 1u; }
+          }
+        }
+        for (int s = 0; s < nslots; ++s) tc_commit(&q_empty[s]);
+      }
+    }
+  }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kFlash3HighRegs));
+    griddep_wait_and_release();
+    // ---------------------------------------------------------------- softmax (one thread per row)
+    const int slot = (warp - 4) >> 2;
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;            // query row in the tile == TMEM lane
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t s_tmem = tmem_base + lane_off + slot * 256;
+    const uint32_t o_tmem = s_tmem + 128;
+    uint8_t* p_smem = smem + C::OFF_P + slot * C::P_BYTES;
+    uint32_t sph = 0, oph = 0;
+    for (int k_ = 0, u = flash_snake(0); u < fs.units; u = flash_snake(++k_)) {
+      int b, g, pair, qt;
+      flash_unit(fs, u, b, g, pair, qt);
+      if (slot == 1 && !(pair * 2 + 1 < fs.n_rep)) continue;
+      const int nt = flash_ntiles(fs, qt);
+      const int jt0 = flash_first_tile(fs, b, qt);
+      const int qpos = fs.P + qt * 128 + row;
+      const int lo = flash_row_lo(fs, b, qt * 128 + row);
+      const int lo_last = flash_row_lo(fs, b, qt * 128 + 127);   // largest lower bound in the tile
+      float m_ref = -INFINITY, l = 0.f;
+      bool ok = true;
+      for (int j = jt0; j < nt; ++j) {
+        if (!mbar_wait(&s_full[slot], sph, wait_ns)) { ok = false; break; }
+        sph ^= 1u;
+        tc_fence_after();
+        const bool need_mask = j * 128 + 127 > fs.P + qt * 128 || j * 128 < lo_last;
+        const int key0 = j * 128;
+        uint32_t ra[32], rb[32], rc[32], rd[32];
+        flash3_load_row(s_tmem, ra, rb, rc, rd);
+        float m0, m1, m2, m3;   // four independent chains
+        if (need_mask) {
+          m0 = flash3_row_max<true>(ra, key0, qpos, lo);
+          m1 = flash3_row_max<true>(rb, key0 + 32, qpos, lo);
+          m2 = flash3_row_max<true>(rc, key0 + 64, qpos, lo);
+          m3 = flash3_row_max<true>(rd, key0 + 96, qpos, lo);
+        } else {
+          m0 = flash3_row_max<false>(ra, key0, qpos, lo);
+          m1 = flash3_row_max<false>(rb, key0 + 32, qpos, lo);
+          m2 = flash3_row_max<false>(rc, key0 + 64, qpos, lo);
+          m3 = flash3_row_max<false>(rd, key0 + 96, qpos, lo);
+        }
+        const float mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+        const float m_tile = mx * fs.scale_log2;   // scale_log2 > 0: max commutes with the scale
+        // the previous tile's P.V must be complete before O is rescaled and
+        // before P (one buffer per head) is overwritten
+        if (j > jt0) {
+          if (!mbar_wait(&o_done[slot], oph, wait_ns)) { ok = false; break; }
+          oph ^= 1u;
+          tc_fence_after();
+        }
+        const bool grow = m_tile > m_ref + 8.0f;
+        float alpha = 1.f;
+        if (grow) {
+          alpha = exp2f(m_ref - m_tile);   // 0 on the first tile
+          l *= alpha;
+          m_ref = m_tile;
+        }
+        if (j > jt0 && __any_sync(0xffffffffu, grow)) {
+#pragma unroll 1
+          for (int c = 0; c < HD / 16; ++c) {
+            uint32_t o[16];
+            tmem_ld16(o_tmem + c * 16, o);
+            tc_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st16(o_tmem + c * 16, o);
+          }
+          tc_wait_st();
+        }
+        const float scl = fs.scale_log2;
+        const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;   // a row with no visible key yet: p = 0
+        float sum_a = 0.f, sum_b = 0.f;
+        flash4_exp_chunk(ra, scl, neg_m, sum_a, sum_b, p_smem, row, 0);
+        flash4_exp_chunk(rb, scl, neg_m, sum_a, sum_b, p_smem, row, 1);
+        flash4_exp_chunk(rc, scl, neg_m, sum_a, sum_b, p_smem, row, 2);
+        flash4_exp_chunk(rd, scl, neg_m, sum_a, sum_b, p_smem, row, 3);
+        l += sum_a + sum_b;
+        fence_proxy_async_smem();   // P (generic stores) before the MMA reads it
+        tc_fence_before();
+        mbar_arrive(&p_full[slot]);
+      }
+      if (!ok) break;
+      // epilogue: wait for the last P.V, out = O / l
+      if (!mbar_wait(&o_done[slot], oph, wait_ns)) break;
+      oph ^= 1u;
+      tc_fence_after();
+      const int t = qt * 128 + row;
+      const int h = g * fs.n_rep + pair * 2 + slot;
+      const float inv = 1.f / l;
+      bf16* orow = out + ((size_t)b * fs.S + t) * fs.ldo + (size_t)h * HD;
+#pragma unroll 1
+      for (int c = 0; c < HD / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(o_tmem + c * 32, r);
+        tc_wait_ld();
+        if (t < fs.S) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 o;
+            o.x = pack_bf16x2(__uint_as_float(r[8 * q + 0]) * inv, __uint_as_float(r[8 * q + 1]) * inv);
+            o.y = pack_bf16x2(__uint_as_float(r[8 * q + 2]) * inv, __uint_as_float(r[8 * q + 3]) * inv);
+            o.z = pack_bf16x2(__uint_as_float(r[8 * q + 4]) * inv, __uint_as_float(r[8 * q + 5]) * inv);
+            o.w = pack_bf16x2(__uint_as_float(r[8 * q + 6]) * inv, __uint_as_float(r[8 * q + 7]) * inv);
+            *reinterpret_cast<uint4*>(orow + c * 32 + q * 8) = o;
+          }
+        }
+      }
+      tc_fence_before();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+}  // namespace l3

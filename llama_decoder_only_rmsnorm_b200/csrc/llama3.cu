@@ -18,6 +18,7 @@
 #include "flash_attention.cuh"
 #include "flash_attention2.cuh"
 #include "flash_attention3.cuh"
+#include "flash_attention4.cuh"
 #include "sampling.cuh"
 #include "simt.cuh"
 #include "tc_gemm.cuh"
@@ -92,9 +93,11 @@ void timer_end(int kind, cudaStream_t st) {
 // touches memory.  g_pdl = false launches them the ordinary way.
 bool g_pdl = true;
 
-// Prefill attention kernel design: 1 = one softmax thread per query row, P
-// through shared memory; 2 = two softmax threads per row, P kept in TMEM.
-int g_flash_variant = 2;
+// Prefill attention kernel design (see the flash_attention*.cuh headers):
+// 1 = one softmax thread per row, P through shared memory; 2 = two softmax
+// threads per row, P in TMEM; 3 = one thread per row with the whole tile row in
+// registers (register split), P in TMEM; 4 = as 3 with P in shared memory.
+int g_flash_variant = 3;
 
 template <typename... KArgs, typename... Args>
 cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
@@ -244,10 +247,12 @@ int run_flash_attention_t(int H, int KV, const void* q, const void* kc, const vo
   fs.ldo = H * HD;
   fs.scale_log2 = (float)(1.4426950408889634 / sqrt((double)HD));
   fs.doc_start = doc_start;
-  constexpr int smem = VARIANT == 3 ? Flash3Cfg<HD>::SMEM_BYTES
+  constexpr int smem = VARIANT == 4 ? Flash4Cfg<HD>::SMEM_BYTES
+                     : VARIANT == 3 ? Flash3Cfg<HD>::SMEM_BYTES
                      : VARIANT == 2 ? Flash2Cfg<HD>::SMEM_BYTES : FlashCfg<HD>::SMEM_BYTES;
-  constexpr int threads = VARIANT == 3 ? kFlash3Threads : VARIANT == 2 ? 640 : 384;
-  auto kern = VARIANT == 3 ? flash_attention3_kernel<HD>
+  constexpr int threads = VARIANT >= 3 ? kFlash3Threads : VARIANT == 2 ? 640 : 384;
+  auto kern = VARIANT == 4 ? flash_attention4_kernel<HD>
+            : VARIANT == 3 ? flash_attention3_kernel<HD>
             : VARIANT == 2 ? flash_attention2_kernel<HD> : flash_attention_kernel<HD>;
   int dev = 0;
   L3_TRY(current_device(&dev));
@@ -255,7 +260,7 @@ int run_flash_attention_t(int H, int KV, const void* q, const void* kc, const vo
   static bool regs_ok[kMaxDevices];
   if (!attr_done[dev]) {
     L3_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-    if (VARIANT == 3) {
+    if (VARIANT >= 3) {
       // The warpgroups' setmaxnreg shares must fit the registers the block is
       // launched with, or the raising warpgroups would wait for ever.
       cudaFuncAttributes fa;
@@ -264,7 +269,7 @@ int run_flash_attention_t(int H, int KV, const void* q, const void* kc, const vo
     }
     attr_done[dev] = true;
   }
-  if (VARIANT == 3 && !regs_ok[dev]) return LLAMA3_ERR_UNSUPPORTED;
+  if (VARIANT >= 3 && !regs_ok[dev]) return LLAMA3_ERR_UNSUPPORTED;
   const int grid = std::min(fs.units, sms);
   L3_LAUNCH(LLAMA3_KERNEL_ATTENTION, st, launch_k(kern, grid, threads, smem, st, mq, mk, mv, (bf16*)out, fs, wns));
   return launch_check();
@@ -274,6 +279,8 @@ template <int HD>
 int run_flash_attention_v(int H, int KV, const void* q, const void* kc, const void* vc, int cap, int B, int S,
                           int P, void* out, const int32_t* doc_start, int sms, unsigned long long wns,
                           cudaStream_t st) {
+  if (g_flash_variant == 4)
+    return run_flash_attention_t<HD, 4>(H, KV, q, kc, vc, cap, B, S, P, out, doc_start, sms, wns, st);
   if (g_flash_variant == 3)
     return run_flash_attention_t<HD, 3>(H, KV, q, kc, vc, cap, B, S, P, out, doc_start, sms, wns, st);
   if (g_flash_variant == 2)
@@ -337,6 +344,9 @@ T* ws_at(void* ws, size_t off) {
 // ---------------------------------------------------------------------------
 // tcgen05 GEMM launch helpers
 // ---------------------------------------------------------------------------
+#ifndef L3_GROUP_M
+#define L3_GROUP_M 16
+#endif
 GemmShape make_shape(int rows_a, int rows_a2, int rows_b, int k, int bn, int splits) {
   GemmShape s;
   s.rows_a = rows_a;
@@ -351,10 +361,11 @@ GemmShape make_shape(int rows_a, int rows_a2, int rows_b, int k, int bn, int spl
   s.kb_per_split = (s.kblocks + splits - 1) / splits;
   s.splits = (s.kblocks + s.kb_per_split - 1) / s.kb_per_split;
   s.units = s.splits * s.tiles_m * s.tiles_n;
-  // Groups of 16 m-tiles: with a 148-CTA persistent grid the tiles in flight
-  // span 16 A row-blocks x ~9 B column-blocks.  The swapped (weight-streaming)
-  // launches have one n-tile, where grouping changes nothing.
-  s.group_m = std::max(1, std::min(16, s.tiles_m));
+  // Groups of L3_GROUP_M m-tiles: with a 148-CTA persistent grid the tiles in
+  // flight span that many A row-blocks x ~148/L3_GROUP_M B column-blocks.  The
+  // swapped (weight-streaming) launches have one n-tile, where grouping
+  // changes nothing.
+  s.group_m = std::max(1, std::min(L3_GROUP_M, s.tiles_m));
   return s;
 }
 
@@ -900,7 +911,7 @@ int llama3_sample_top_p(const float* logits, int rows, long long ld, int vocab, 
 
 int llama3_set_flash_variant(int variant) {
   const int old = g_flash_variant;
-  g_flash_variant = (variant == 1 || variant == 3) ? variant : 2;
+  g_flash_variant = (variant >= 1 && variant <= 4) ? variant : 3;
   return old;
 }
 

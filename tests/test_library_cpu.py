@@ -126,5 +126,5 @@ def test_sample_top_p_rejects_bad_arguments_before_launch():
 
 def test_flash_variant_switch():
     old = B.llama3_set_flash_variant(1)
-    assert B.llama3_set_flash_variant(7) == 1      # values other than 1 select the second design
-    assert B.llama3_set_flash_variant(old) == 2
+    assert B.llama3_set_flash_variant(7) == 1      # values outside 1..4 select the third design
+    assert B.llama3_set_flash_variant(old) == 3
