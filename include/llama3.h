@@ -247,19 +247,35 @@ int llama3_lm_head_argmax_noalloc(const llama3_config* cfg, const void* norm_w, 
  *   (ties: lower index first) are kept while the probability ranked before
  *   them is <= top_p (top_p >= 1 keeps all, top_p = 0 keeps the top token);
  *   one kept token is drawn with probability proportional to p.
- * The draw is deterministic in (seed, offset, row): the first 64-bit word of
+ * The draw is deterministic in (seed, counter, row): the first 64-bit word of
  * Philox-4x64-10 (Salmon et al., SC 2011) with key (seed, 0) and counter
- * (offset, r, 0, 0) selects the token by the inverse CDF of the kept law
- * taken in index order.  Probabilities are evaluated in fp32 and summed
- * exactly as integers in units of 2^-40 of the largest one.  Pass the
- * decoding step as `offset` to get a fresh draw per step.
+ * (offset + positions[r], r, 0, 0) -- just offset when positions is NULL --
+ * selects the token by the inverse CDF of the kept law taken in index order.
+ * Probabilities are evaluated in fp32 and summed exactly as integers in units
+ * of 2^-40 of the largest one.  Pass each sequence's current position (device
+ * int32 [rows]) or the step number as offset to get a fresh draw per step.
  * Errors: LLAMA3_ERR_ARG (null pointers, rows < 1, vocab < 1, ld < vocab,
  * top_p < 0 or NaN, temperature NaN), LLAMA3_ERR_ALIGN (pointers not 4-byte
  * aligned), LLAMA3_ERR_CUDA.  Allocates nothing; asynchronous on `stream`.
  */
 int llama3_sample_top_p(const float* logits, int rows, long long ld, int vocab, float temperature,
                         float top_p, unsigned long long seed, unsigned long long offset,
-                        int32_t* ids_out, llama3_stream_t stream);
+                        const int32_t* positions, int32_t* ids_out, llama3_stream_t stream);
+
+/*
+ * Device-side bookkeeping of one generation step, so that a whole step
+ * (embed -> llama3_layer_decode_ragged per block -> LM head / draw -> this
+ * call) can be captured once in a CUDA graph and replayed: every argument is
+ * a device pointer whose contents change, none is a host value.
+ * history[*step][b] = ids[b] for b < batch (skipped once *step >= history_rows;
+ * row stride history_stride >= batch), positions[b] += 1, *step += 1.
+ * No counterpart on the pages, which run this loop on the host ([S2] 六).
+ * Errors: LLAMA3_ERR_ARG (null pointers, batch < 1, history_rows < 1,
+ * history_stride < batch), LLAMA3_ERR_ALIGN (pointers not 4-byte aligned).
+ */
+int llama3_generation_advance(int32_t* positions, const int32_t* ids, int32_t* history, int32_t* step,
+                              int batch, int history_rows, long long history_stride,
+                              llama3_stream_t stream);
 
 /* ---- building blocks (the steps of the calls above, exposed for tests) ---- */
 

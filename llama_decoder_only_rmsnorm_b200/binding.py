@@ -66,7 +66,8 @@ _SIGNATURES = {
     "llama3_set_wait_limit_ms": [_i],
     "llama3_set_programmatic_launch": [_i],
     "llama3_set_flash_variant": [_i],
-    "llama3_sample_top_p": [_p, _i, _ll, _i, ctypes.c_float, ctypes.c_float, ctypes.c_ulonglong, ctypes.c_ulonglong, _p, _p],
+    "llama3_sample_top_p": [_p, _i, _ll, _i, ctypes.c_float, ctypes.c_float, ctypes.c_ulonglong, ctypes.c_ulonglong, _p, _p, _p],
+    "llama3_generation_advance": [_p, _p, _p, _p, _i, _i, _ll, _p],
     "llama3_set_launch_timer": [_i, _p, _p, _i],
     "llama3_launch_timer_used": [],
     "llama3_launch_count": [],
@@ -195,11 +196,20 @@ def llama3_lm_head_argmax(cfg, norm_w, w_out, h, rows, row_stride, ids_out, logi
         _ptr(logits_out), _ptr(ws), ws_bytes, _stream(stream)))
 
 
-def llama3_sample_top_p(logits, rows, ld, vocab, temperature, top_p, seed, offset, ids_out, stream=None):
-    """Temperature / top-p draw of one token per row of fp32 logits."""
+def llama3_sample_top_p(logits, rows, ld, vocab, temperature, top_p, seed, offset, ids_out, stream=None,
+                        positions=None):
+    """Temperature / top-p draw of one token per row of fp32 logits (the
+    draw counter of row r is offset, plus positions[r] when given)."""
     _check("llama3_sample_top_p", lib().llama3_sample_top_p(
         _ptr(logits), rows, ld, vocab, float(temperature), float(top_p), int(seed) & (2 ** 64 - 1),
-        int(offset) & (2 ** 64 - 1), _ptr(ids_out), _stream(stream)))
+        int(offset) & (2 ** 64 - 1), _ptr(positions), _ptr(ids_out), _stream(stream)))
+
+
+def llama3_generation_advance(positions, ids, history, step, batch, history_rows, history_stride, stream=None):
+    """history[step] = ids, positions += 1, step += 1, all on the device."""
+    _check("llama3_generation_advance", lib().llama3_generation_advance(
+        _ptr(positions), _ptr(ids), _ptr(history), _ptr(step), batch, history_rows, history_stride,
+        _stream(stream)))
 
 
 NOALLOC_SCRATCH_BYTES = 4 << 20

@@ -51,19 +51,25 @@ __device__ __forceinline__ void flash3_load_row(uint32_t taddr, uint32_t (&a)[32
 }
 
 // p = 2^(s*scale - m) for 32 scores, their sum, and the bf16 pairs stored
-// to the 16 TMEM columns at taddr.  The exponent is rounded to bf16 and two
-// exponentials come from one packed MUFU operation, already in the bf16 pair
-// form P.V consumes; the row sum adds those same rounded values, so the
-// normaliser matches what the MMA multiplies.  (Masked scores are -inf: 0.)
+// to the 16 TMEM columns at taddr.  Exponentials in fp32: on unmasked tiles 6
+// of every 16 pairs go to the FMA pipe (exp2_poly2), the rest to the MUFU;
+// masked tiles use the MUFU only, which gives exactly 0 for the -inf scores.
+template <bool MASKED>
 __device__ __forceinline__ void flash3_exp_chunk(const uint32_t (&r)[32], float scl, float neg_m, float& sum_a,
                                                  float& sum_b, uint32_t taddr) {
   uint32_t pk[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    float x0, x1;
+    float x0, x1, p0, p1;
     fma2(x0, x1, __uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), scl, scl, neg_m, neg_m);
-    pk[i] = ex2_bf16x2(pack_bf16x2(x0, x1));
-    add2(sum_a, sum_b, bf16lo(pk[i]), bf16hi(pk[i]));
+    if (!MASKED && (i & 7) < 3) {
+      exp2_poly2(x0, x1, p0, p1);
+    } else {
+      p0 = ex2_approx(x0);
+      p1 = ex2_approx(x1);
+    }
+    add2(sum_a, sum_b, p0, p1);
+    pk[i] = pack_bf16x2(p0, p1);
   }
   tmem_st16(taddr, pk);
 }
@@ -340,10 +346,17 @@ __global__ void __launch_bounds__(kFlash3Threads, 1)
         const float scl = fs.scale_log2;
         const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;   // a row with no visible key yet: p = 0
         float sum_a = 0.f, sum_b = 0.f;
-        flash3_exp_chunk(ra, scl, neg_m, sum_a, sum_b, s_tmem);
-        flash3_exp_chunk(rb, scl, neg_m, sum_a, sum_b, s_tmem + 16);
-        flash3_exp_chunk(rc, scl, neg_m, sum_a, sum_b, s_tmem + 32);
-        flash3_exp_chunk(rd, scl, neg_m, sum_a, sum_b, s_tmem + 48);
+        if (need_mask) {
+          flash3_exp_chunk<true>(ra, scl, neg_m, sum_a, sum_b, s_tmem);
+          flash3_exp_chunk<true>(rb, scl, neg_m, sum_a, sum_b, s_tmem + 16);
+          flash3_exp_chunk<true>(rc, scl, neg_m, sum_a, sum_b, s_tmem + 32);
+          flash3_exp_chunk<true>(rd, scl, neg_m, sum_a, sum_b, s_tmem + 48);
+        } else {
+          flash3_exp_chunk<false>(ra, scl, neg_m, sum_a, sum_b, s_tmem);
+          flash3_exp_chunk<false>(rb, scl, neg_m, sum_a, sum_b, s_tmem + 16);
+          flash3_exp_chunk<false>(rc, scl, neg_m, sum_a, sum_b, s_tmem + 32);
+          flash3_exp_chunk<false>(rd, scl, neg_m, sum_a, sum_b, s_tmem + 48);
+        }
         l += sum_a + sum_b;
         tc_wait_st();
         tc_fence_before();

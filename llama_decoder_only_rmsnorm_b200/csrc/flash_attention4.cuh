@@ -3,7 +3,7 @@
 // Computes the same thing as flash_attention.cuh ("Build your own Llama 3 from
 // scratch" §3.4; document mask of 附 1).  Softmax as in the third design (one
 // thread per query row, the whole 128-score row of a tile in registers after
-// a setmaxnreg register split, packed bf16 exponentials), but P goes to shared
+// a setmaxnreg register split), but P goes to shared
 // memory as in the first design: the next tile's S can then be issued right
 // behind P.V (they touch different TMEM columns), so the tensor pipe does not
 // drain while P.V finishes.  The softmax waits for the previous P.V before it
@@ -34,18 +34,26 @@ struct Flash4Cfg {
   static_assert(HD % 32 == 0 && HD <= 128, "head_dim");
 };
 
-// p = 2^(s*scale - m) for keys 32c .. 32c+31 of this row, their sum, and
-// the bf16 pairs stored into the row's P line in shared memory, in the
-// 128-byte-swizzled K-major layout the MMA reads (two 64-key slabs).
+// p = 2^(s*scale - m) for keys 32c .. 32c+31 of this row (fp32, as the
+// third design), their sum, and the bf16 pairs stored into the row's P line
+// in shared memory, in the 128-byte-swizzled K-major layout the MMA reads
+// (two 64-key slabs).
+template <bool MASKED>
 __device__ __forceinline__ void flash4_exp_chunk(const uint32_t (&r)[32], float scl, float neg_m, float& sum_a,
                                                  float& sum_b, uint8_t* p_smem, int row, int c) {
   uint32_t pk[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    float x0, x1;
+    float x0, x1, p0, p1;
     fma2(x0, x1, __uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), scl, scl, neg_m, neg_m);
-    pk[i] = ex2_bf16x2(pack_bf16x2(x0, x1));
-    add2(sum_a, sum_b, bf16lo(pk[i]), bf16hi(pk[i]));
+    if (!MASKED && (i & 7) < 3) {
+      exp2_poly2(x0, x1, p0, p1);
+    } else {
+      p0 = ex2_approx(x0);
+      p1 = ex2_approx(x1);
+    }
+    add2(sum_a, sum_b, p0, p1);
+    pk[i] = pack_bf16x2(p0, p1);
   }
   uint8_t* slab = p_smem + (c >> 1) * (128 * 128) + row * 128;
 #pragma unroll
@@ -302,10 +310,17 @@ __global__ void __launch_bounds__(kFlash3Threads, 1)
         const float scl = fs.scale_log2;
         const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;   // a row with no visible key yet: p = 0
         float sum_a = 0.f, sum_b = 0.f;
-        flash4_exp_chunk(ra, scl, neg_m, sum_a, sum_b, p_smem, row, 0);
-        flash4_exp_chunk(rb, scl, neg_m, sum_a, sum_b, p_smem, row, 1);
-        flash4_exp_chunk(rc, scl, neg_m, sum_a, sum_b, p_smem, row, 2);
-        flash4_exp_chunk(rd, scl, neg_m, sum_a, sum_b, p_smem, row, 3);
+        if (need_mask) {
+          flash4_exp_chunk<true>(ra, scl, neg_m, sum_a, sum_b, p_smem, row, 0);
+          flash4_exp_chunk<true>(rb, scl, neg_m, sum_a, sum_b, p_smem, row, 1);
+          flash4_exp_chunk<true>(rc, scl, neg_m, sum_a, sum_b, p_smem, row, 2);
+          flash4_exp_chunk<true>(rd, scl, neg_m, sum_a, sum_b, p_smem, row, 3);
+        } else {
+          flash4_exp_chunk<false>(ra, scl, neg_m, sum_a, sum_b, p_smem, row, 0);
+          flash4_exp_chunk<false>(rb, scl, neg_m, sum_a, sum_b, p_smem, row, 1);
+          flash4_exp_chunk<false>(rc, scl, neg_m, sum_a, sum_b, p_smem, row, 2);
+          flash4_exp_chunk<false>(rd, scl, neg_m, sum_a, sum_b, p_smem, row, 3);
+        }
         l += sum_a + sum_b;
         fence_proxy_async_smem();   // P (generic stores) before the MMA reads it
         tc_fence_before();

@@ -882,11 +882,12 @@ int llama3_set_kernel_path(int path) {
 }
 
 int llama3_sample_top_p(const float* logits, int rows, long long ld, int vocab, float temperature, float top_p,
-                        unsigned long long seed, unsigned long long offset, int32_t* ids_out,
-                        llama3_stream_t stream) {
+                        unsigned long long seed, unsigned long long offset, const int32_t* positions,
+                        int32_t* ids_out, llama3_stream_t stream) {
   if (!logits || !ids_out || rows < 1 || vocab < 1 || ld < vocab) return LLAMA3_ERR_ARG;
   if (std::isnan(temperature) || std::isnan(top_p) || top_p < 0.f) return LLAMA3_ERR_ARG;
-  if ((reinterpret_cast<uintptr_t>(logits) & 3) || (reinterpret_cast<uintptr_t>(ids_out) & 3))
+  if ((reinterpret_cast<uintptr_t>(logits) & 3) || (reinterpret_cast<uintptr_t>(ids_out) & 3) ||
+      (reinterpret_cast<uintptr_t>(positions) & 3))
     return LLAMA3_ERR_ALIGN;
   cudaStream_t st = (cudaStream_t)stream;
   int dev = 0;
@@ -904,8 +905,22 @@ int llama3_sample_top_p(const float* logits, int rows, long long ld, int vocab, 
   sp.top_p = top_p;
   sp.seed = seed;
   sp.offset = offset;
+  sp.positions = positions;
   sp.ids = ids_out;
   L3_LAUNCH(LLAMA3_KERNEL_SAMPLE, st, launch_k(sample_top_p_kernel, rows, kSampleThreads, kSampleSmem, st, sp));
+  return launch_check();
+}
+
+int llama3_generation_advance(int32_t* positions, const int32_t* ids, int32_t* history, int32_t* step, int batch,
+                              int history_rows, long long history_stride, llama3_stream_t stream) {
+  if (!positions || !ids || !history || !step || batch < 1 || history_rows < 1 || history_stride < batch)
+    return LLAMA3_ERR_ARG;
+  const uintptr_t any = reinterpret_cast<uintptr_t>(positions) | reinterpret_cast<uintptr_t>(ids) |
+                        reinterpret_cast<uintptr_t>(history) | reinterpret_cast<uintptr_t>(step);
+  if (any & 3) return LLAMA3_ERR_ALIGN;
+  cudaStream_t st = (cudaStream_t)stream;
+  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k(generation_advance_kernel, 1, 256, 0, st, positions, ids, history,
+                                                    step, batch, history_rows, history_stride));
   return launch_check();
 }
 

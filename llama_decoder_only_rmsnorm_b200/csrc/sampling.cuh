@@ -20,7 +20,7 @@
 //    are kept up to the needed count in index order.
 //  * The draw: word = first output of Philox-4x64-10 (Salmon et al., "Parallel
 //    random numbers: as easy as 1, 2, 3", SC 2011) with key (seed, 0) and
-//    counter (offset, row, 0, 0); target = floor(word * K / 2^64) for the kept
+//    counter (offset [+ positions[row]], row, 0, 0); target = floor(word * K / 2^64) for the kept
 //    mass K; the token is the first kept one, in index order, whose running
 //    kept mass exceeds target (the inverse CDF of the renormalised kept law).
 #pragma once
@@ -34,6 +34,7 @@ struct SampleParams {
   int V;
   float temperature, top_p;
   unsigned long long seed, offset;
+  const int32_t* positions;   // optional: row r's draw counts from offset + positions[r]
   int32_t* ids;
 };
 
@@ -204,7 +205,8 @@ __global__ void __launch_bounds__(kSampleThreads) sample_top_p_kernel(const Samp
     n_tie = fb ? (thr - above) / fb + 1 : 0;
     kept_mass = above + n_tie * fb;
   }
-  const uint64_t word = philox4x64_10_word0(sp.offset, (uint64_t)row, 0, 0, sp.seed, 0);
+  const uint64_t ctr = sp.offset + (sp.positions ? (uint64_t)(int64_t)sp.positions[row] : 0ull);
+  const uint64_t word = philox4x64_10_word0(ctr, (uint64_t)row, 0, 0, sp.seed, 0);
   const uint64_t target = __umul64hi(word, kept_mass);
 
   // ---- pass A: per-warp segment totals (warp w owns indices [w*seg, (w+1)*seg))

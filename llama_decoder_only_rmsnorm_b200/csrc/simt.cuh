@@ -30,6 +30,25 @@ __global__ void embed_kernel(const int32_t* __restrict__ ids, const T* __restric
   }
 }
 
+// ---- generation bookkeeping ("Build your own Llama 3 from scratch" 六) -------
+// After a step has written the next token of every sequence into ids:
+// history[step][b] = ids[b] (while step < rows), positions[b] += 1, step += 1.
+// One CTA, so the step counter is read once and advanced after every write.
+__global__ void generation_advance_kernel(int32_t* __restrict__ positions, const int32_t* __restrict__ ids,
+                                          int32_t* __restrict__ history, int32_t* __restrict__ step, int batch,
+                                          int rows, long long stride) {
+  griddep_wait_and_release();
+  __shared__ int t;
+  if (threadIdx.x == 0) t = *step;
+  __syncthreads();
+  for (int b = threadIdx.x; b < batch; b += blockDim.x) {
+    if (t >= 0 && t < rows) history[(size_t)t * stride + b] = ids[b];
+    positions[b] += 1;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) *step = t + 1;
+}
+
 // ---- RMSNorm ("Build your own Llama 3 from scratch" §3.1) -------------------
 // One CTA per row; fp32 sum of squares, one rounding on output.
 template <typename T>

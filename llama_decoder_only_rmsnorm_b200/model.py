@@ -71,46 +71,73 @@ class Llama3Stack:
 
     # -- generation ("Build your own Llama 3 from scratch" 六 generate)
     def generate(self, prompt_ids, n_new, eos_id=None, stream=None, temperature=0.0, top_p=0.9, seed=0,
-                 return_logits=False):
+                 return_logits=False, cuda_graph=False):
         """Prefill the prompts (int32 [batch, S] on the device), then decode
         n_new tokens.  temperature <= 0 is greedy (the LM head's argmax);
-        otherwise each step's fp32 logits go through llama3_sample_top_p with
-        the step number as the draw's counter offset.  Each step writes its
-        tokens straight into row `step` of a [n_new, batch] device buffer,
-        which the next step's embedding reads, so no token leaves the device
-        in the loop.  Returns the [batch, n_new] tokens as a host array (and,
-        with return_logits, the [n_new, batch, vocab] fp32 logits); after a
-        sequence's first eos_id the rest of its row is eos_id (the page stops
-        the loop there)."""
+        otherwise each step's fp32 logits go through llama3_sample_top_p,
+        whose draw for sequence b is keyed by the position of the token that
+        produced the logits (S - 1 for the first new token, then S, S+1, ...).
+
+        Every decode step is the same sequence of launches with device-side
+        state only -- embed the current ids, llama3_layer_decode_ragged per
+        block at the device positions, LM head (+ draw) into the current ids,
+        llama3_generation_advance -- so with cuda_graph=True it is captured once
+        and replayed.  Returns the [batch, n_new] tokens as a host array (and,
+        with return_logits, the [n_new, batch, vocab] fp32 logits, not with
+        cuda_graph); after a sequence's first eos_id the rest of its row is
+        eos_id (the page stops the loop there)."""
         import torch
         Bn, S = prompt_ids.shape
         assert Bn == self.batch and S + n_new - 1 <= self.cache_cap
+        assert not (cuda_graph and (return_logits or stream is not None))
         D, V = self.cfg_dict["dim"], self.cfg_dict["vocab"]
+        dev = self.device
         sampling = temperature > 0
-        x = torch.empty((Bn, S, D), dtype=self.dtype, device=self.device)
+        x = torch.empty((Bn, S, D), dtype=self.dtype, device=dev)
         self.embed(prompt_ids, x, stream)
         self.forward_layers(x, S, 0, stream)
-        row = (Bn + 3) // 4 * 4            # keeps every step's ids 16-byte aligned
-        out = torch.empty((n_new, row), dtype=torch.int32, device=self.device)
+        row = (Bn + 3) // 4 * 4            # keeps every history row 16-byte aligned
+        hist = torch.empty((n_new, row), dtype=torch.int32, device=dev)
+        cur = torch.empty((row,), dtype=torch.int32, device=dev)
+        pos = torch.full((Bn,), S - 1, dtype=torch.int32, device=dev)   # position behind the logits
+        step = torch.zeros((1,), dtype=torch.int32, device=dev)
+        pick = torch.empty((row,), dtype=torch.int32, device=dev)
         keep = return_logits or sampling
         logits = torch.empty((n_new if return_logits else 1, Bn, V), dtype=torch.float32,
-                             device=self.device) if keep else None
-        pick = torch.empty((row,), dtype=torch.int32, device=self.device) if sampling else None
+                             device=dev) if keep else None
 
-        def head(h, stride, step):
-            lg = logits[step if return_logits else 0] if keep else None
+        def head(h, stride, k):
+            lg = logits[k if return_logits else 0] if keep else None
             B.llama3_lm_head_argmax(self.cfg, self.out["norm"], self.out["output"], h, Bn, stride,
-                                    pick if sampling else out[step], lg, self.ws, self.ws_bytes, stream)
+                                    pick if sampling else cur, lg, self.ws, self.ws_bytes, stream)
             if sampling:
-                B.llama3_sample_top_p(lg, Bn, V, V, temperature, top_p, seed, step, out[step], stream)
+                B.llama3_sample_top_p(lg, Bn, V, V, temperature, top_p, seed, 0, cur, stream, positions=pos)
+            B.llama3_generation_advance(pos, cur, hist, step, Bn, n_new, row, stream)
 
-        head(x[:, -1], S * D, 0)
-        xd = torch.empty((Bn, 1, D), dtype=self.dtype, device=self.device)
-        for step in range(1, n_new):
-            B.llama3_embed(self.cfg, out[step - 1], self.out["tok_embeddings"], xd, Bn, stream)
-            self.decode_layers(xd, S + step - 1, stream)
-            head(xd, D, step)
-        toks = out[:, :Bn].t().cpu().numpy()
+        head(x[:, -1], S * D, 0)           # first new token; pos -> S, step -> 1
+        xd = torch.empty((Bn, 1, D), dtype=self.dtype, device=dev)
+        max_pos = self.cache_cap - 1
+
+        def decode_step(k):
+            B.llama3_embed(self.cfg, cur, self.out["tok_embeddings"], xd, Bn, stream)
+            self.decode_layers_ragged(xd, pos, max_pos, stream)
+            head(xd, D, k)
+
+        if cuda_graph and n_new > 1:
+            g = torch.cuda.CUDAGraph()
+            side = torch.cuda.Stream()
+            side.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(side):
+                decode_step(1)             # warm-up step (also token 1)
+            torch.cuda.current_stream().wait_stream(side)
+            with torch.cuda.graph(g):
+                decode_step(2)
+            for _ in range(2, n_new):
+                g.replay()
+        else:
+            for k in range(1, n_new):
+                decode_step(k)
+        toks = hist[:, :Bn].t().cpu().numpy()
         if eos_id is not None:   # host-side: hold the end token once emitted
             for b in range(Bn):
                 hits = (toks[b] == eos_id).nonzero()[0]

@@ -290,6 +290,8 @@ def test_greedy_generation_matches_oracle():
     st = Llama3Stack(w.cfg(), layers, outw, w.batch, w.seq + n_new, w.seq, lm_rows=w.batch)
     prompt = I.token_ids(w, DEV)
     got = st.generate(prompt, n_new)
+    st2 = Llama3Stack(w.cfg(), layers, outw, w.batch, w.seq + n_new, w.seq, lm_rows=w.batch)
+    np.testing.assert_array_equal(st2.generate(prompt, n_new, cuda_graph=True), got)   # graph replay, same tokens
     toks, gaps = O.generate_greedy(prompt.cpu().numpy(), f64(outw["tok_embeddings"]),
                                    [oracle_layer(l) for l in layers], f64(outw["norm"]), f64(outw["output"]),
                                    oracle_cfg(w), n_new)

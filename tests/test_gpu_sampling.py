@@ -134,7 +134,7 @@ def test_sampled_generation_draws_from_the_models_logits():
     for step in range(n_new):
         for b in range(w.batch):
             want, (cut, draw) = O.top_p_sample(logits[step, b].astype(np.float64), T32, p32,
-                                               O.sampling_word(seed, step, b))
+                                               O.sampling_word(seed, w.seq - 1 + step, b))
             if cut > MARGIN and draw > MARGIN:
                 assert toks[b, step] == want, (step, b)
                 decided += 1
@@ -147,3 +147,7 @@ def test_sampled_generation_draws_from_the_models_logits():
     want_logits, _ = O.lm_head(rows, f64(outw["norm"]), f64(outw["output"]), w.norm_eps)
     got = logits.transpose(1, 0, 2).reshape(-1, w.vocab)
     assert_close(got, want_logits, "bf16", "generation logits")
+    # the same loop captured once in a CUDA graph and replayed draws the same tokens
+    st2 = Llama3Stack(w.cfg(), layers, outw, w.batch, w.seq + n_new, w.seq, lm_rows=w.batch)
+    toks_graph = st2.generate(prompt, n_new, temperature=T, top_p=top_p, seed=seed, cuda_graph=True)
+    np.testing.assert_array_equal(toks_graph, toks)

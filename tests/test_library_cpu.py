@@ -112,7 +112,7 @@ def test_sample_top_p_rejects_bad_arguments_before_launch():
     f = ctypes.c_float
     s = lambda **k: lib.llama3_sample_top_p(k.get("logits", FAKE), k.get("rows", 4), k.get("ld", 100),
                                             k.get("vocab", 100), f(k.get("t", 0.7)), f(k.get("p", 0.9)),
-                                            1, 0, k.get("ids", FAKE), None)
+                                            1, 0, k.get("pos", None), k.get("ids", FAKE), None)
     assert s(rows=0) == 1
     assert s(vocab=0) == 1
     assert s(ld=99) == 1
@@ -121,6 +121,14 @@ def test_sample_top_p_rejects_bad_arguments_before_launch():
     assert s(t=float("nan")) == 1
     assert s(logits=None) == 1
     assert s(ids=ctypes.c_void_p(18)) == 2   # ids not 4-byte aligned
+    assert s(pos=ctypes.c_void_p(FAKE + 2)) == 2
+    adv = lambda **k: lib.llama3_generation_advance(k.get("pos", FAKE), FAKE, FAKE, FAKE, k.get("batch", 4),
+                                                    k.get("rows", 8), k.get("stride", 4), None)
+    assert adv(batch=0) == 1
+    assert adv(rows=0) == 1
+    assert adv(stride=3) == 1
+    assert adv(pos=None) == 1
+    assert adv(pos=ctypes.c_void_p(FAKE + 1)) == 2
     assert B.KERNEL_KINDS["sample"] == 11
 
 
