@@ -263,6 +263,21 @@ int llama3_sample_top_p(const float* logits, int rows, long long ld, int vocab, 
                         const int32_t* positions, int32_t* ids_out, llama3_stream_t stream);
 
 /*
+ * out[r] = x[row_index[r]] for r < rows: copies `dim` elements per row (x rows
+ * n_rows of them, row_stride elements apart; out dense [rows, dim]).  With a
+ * batch of prompts of different lengths padded to a common S, the LM head of
+ * the first new token reads row b*S + len[b] - 1 of every sequence this way
+ * (the padded prefill is exact on each sequence's own rows: causal attention
+ * never lets a real token see a padding row).  No counterpart on the pages.
+ * An index outside [0, n_rows) zeroes that row and reports LLAMA3_ERR_ARG
+ * through llama3_device_status.  Errors: LLAMA3_ERR_ARG, LLAMA3_ERR_ALIGN
+ * (x, out not 16-byte aligned, rows not 16-byte multiples, row_index not
+ * 4-byte aligned).
+ */
+int llama3_gather_rows(const llama3_config* cfg, const void* x, long long row_stride, int n_rows,
+                       const int32_t* row_index, int rows, void* out, llama3_stream_t stream);
+
+/*
  * Device-side bookkeeping of one generation step, so that a whole step
  * (embed -> llama3_layer_decode_ragged per block -> LM head / draw -> this
  * call) can be captured once in a CUDA graph and replayed: every argument is

@@ -68,6 +68,7 @@ _SIGNATURES = {
     "llama3_set_flash_variant": [_i],
     "llama3_sample_top_p": [_p, _i, _ll, _i, ctypes.c_float, ctypes.c_float, ctypes.c_ulonglong, ctypes.c_ulonglong, _p, _p, _p],
     "llama3_generation_advance": [_p, _p, _p, _p, _i, _i, _ll, _p],
+    "llama3_gather_rows": [_cfgp, _p, _ll, _i, _p, _i, _p, _p],
     "llama3_set_launch_timer": [_i, _p, _p, _i],
     "llama3_launch_timer_used": [],
     "llama3_launch_count": [],
@@ -203,6 +204,12 @@ def llama3_sample_top_p(logits, rows, ld, vocab, temperature, top_p, seed, offse
     _check("llama3_sample_top_p", lib().llama3_sample_top_p(
         _ptr(logits), rows, ld, vocab, float(temperature), float(top_p), int(seed) & (2 ** 64 - 1),
         int(offset) & (2 ** 64 - 1), _ptr(positions), _ptr(ids_out), _stream(stream)))
+
+
+def llama3_gather_rows(cfg, x, row_stride, n_rows, row_index, rows, out, stream=None):
+    """out[r] = x[row_index[r]] (dim elements per row)."""
+    _check("llama3_gather_rows", lib().llama3_gather_rows(
+        ctypes.byref(cfg), _ptr(x), row_stride, n_rows, _ptr(row_index), rows, _ptr(out), _stream(stream)))
 
 
 def llama3_generation_advance(positions, ids, history, step, batch, history_rows, history_stride, stream=None):

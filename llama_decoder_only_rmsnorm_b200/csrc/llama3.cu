@@ -911,6 +911,21 @@ int llama3_sample_top_p(const float* logits, int rows, long long ld, int vocab, 
   return launch_check();
 }
 
+int llama3_gather_rows(const llama3_config* cfg, const void* x, long long row_stride, int n_rows,
+                       const int32_t* row_index, int rows, void* out, llama3_stream_t stream) {
+  L3_TRY(check_config(cfg));
+  if (!x || !row_index || !out || rows < 1 || n_rows < 1 || row_stride < cfg->dim) return LLAMA3_ERR_ARG;
+  const long long es = esize(cfg);
+  if (!aligned16(x) || !aligned16(out) || (reinterpret_cast<uintptr_t>(row_index) & 3) ||
+      (row_stride * es) % 16 || ((long long)cfg->dim * es) % 16)
+    return LLAMA3_ERR_ALIGN;
+  cudaStream_t st = (cudaStream_t)stream;
+  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st,
+            launch_k(gather_rows_kernel, rows, 128, 0, st, (const uint4*)x, row_stride * es / 16, row_index, n_rows,
+                     (uint4*)out, (int)((long long)cfg->dim * es / 16)));
+  return launch_check();
+}
+
 int llama3_generation_advance(int32_t* positions, const int32_t* ids, int32_t* history, int32_t* step, int batch,
                               int history_rows, long long history_stride, llama3_stream_t stream) {
   if (!positions || !ids || !history || !step || batch < 1 || history_rows < 1 || history_stride < batch)

@@ -30,6 +30,19 @@ __global__ void embed_kernel(const int32_t* __restrict__ ids, const T* __restric
   }
 }
 
+// ---- row gather: out[r] = x[idx[r]] (rows of D elements, 16-byte chunks) -----
+// An index outside [0, n_rows) is reported and its output row zeroed.
+__global__ void gather_rows_kernel(const uint4* __restrict__ x, long long row_stride16, const int32_t* __restrict__ idx,
+                                   int n_rows, uint4* __restrict__ out, int row16) {
+  griddep_wait_and_release();
+  const int r = blockIdx.x;
+  const int i = idx[r];
+  const bool ok = i >= 0 && i < n_rows;
+  if (!ok && threadIdx.x == 0) record_error(LLAMA3_ERR_ARG);
+  const uint4* src = x + (size_t)(ok ? i : 0) * row_stride16;
+  for (int c = threadIdx.x; c < row16; c += blockDim.x) out[(size_t)r * row16 + c] = ok ? src[c] : make_uint4(0, 0, 0, 0);
+}
+
 // ---- generation bookkeeping ("Build your own Llama 3 from scratch" 六) -------
 // After a step has written the next token of every sequence into ids:
 // history[step][b] = ids[b] (while step < rows), positions[b] += 1, step += 1.

@@ -250,6 +250,8 @@ __global__ void __launch_bounds__(192, 1)
                    const GemmShape sh, const EpiParams ep, const unsigned long long wait_ns) {
   using C = TcGemmCfg<BN, STAGES, DUAL>;
   constexpr uint32_t IDESC = idesc_bf16_f32(128, BN, 0, 0);
+  constexpr uint32_t IDESC_DUAL = idesc_bf16_f32(128, DUAL ? 2 * BN : BN, 0, 0);
+  static_assert(!DUAL || 2 * BN <= 256, "one MMA covers both B tiles");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -369,11 +371,10 @@ __global__ void __launch_bounds__(192, 1)
             const uint64_t adesc = sw128_desc(a_addr + k * 32, 1024, 16);
             const uint64_t bdesc = sw128_desc(b_addr + k * 32, 1024, 16);
             const uint32_t accum = (kb > kb0 || k > 0) ? 1u : 0u;
-            tc_mma_f16_ss(d, adesc, bdesc, IDESC, accum);
-            if constexpr (DUAL) {
-              const uint64_t bdesc2 = sw128_desc(b_addr + C::B_BYTES + k * 32, 1024, 16);
-              tc_mma_f16_ss(d + BN, adesc, bdesc2, IDESC, accum);
-            }
+            // DUAL: the two B tiles sit back to back in shared memory (same
+            // swizzle atoms), so one N = 2*BN MMA covers both and writes the
+            // first operand's columns at d and the second's at d + BN.
+            tc_mma_f16_ss(d, adesc, bdesc, DUAL ? IDESC_DUAL : IDESC, accum);
           }
           tc_commit(&empty[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }

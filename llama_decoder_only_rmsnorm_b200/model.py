@@ -71,7 +71,7 @@ class Llama3Stack:
 
     # -- generation ("Build your own Llama 3 from scratch" 六 generate)
     def generate(self, prompt_ids, n_new, eos_id=None, stream=None, temperature=0.0, top_p=0.9, seed=0,
-                 return_logits=False, cuda_graph=False):
+                 return_logits=False, cuda_graph=False, prompt_lens=None):
         """Prefill the prompts (int32 [batch, S] on the device), then decode
         n_new tokens.  temperature <= 0 is greedy (the LM head's argmax);
         otherwise each step's fp32 logits go through llama3_sample_top_p,
@@ -85,7 +85,15 @@ class Llama3Stack:
         and replayed.  Returns the [batch, n_new] tokens as a host array (and,
         with return_logits, the [n_new, batch, vocab] fp32 logits, not with
         cuda_graph); after a sequence's first eos_id the rest of its row is
-        eos_id (the page stops the loop there)."""
+        eos_id (the page stops the loop there).
+
+        prompt_lens (host ints, one per sequence, each <= S): prompts of
+        different lengths, left-aligned and padded to S.  The padded prefill
+        is exact on each sequence's own rows (causal attention never lets a
+        real token see a later padding row); the first LM head reads row
+        len[b] - 1 of each sequence, and decoding continues at position
+        len[b] (padding K/V in the cache are overwritten before they are
+        ever visible)."""
         import torch
         Bn, S = prompt_ids.shape
         assert Bn == self.batch and S + n_new - 1 <= self.cache_cap
@@ -99,7 +107,9 @@ class Llama3Stack:
         row = (Bn + 3) // 4 * 4            # keeps every history row 16-byte aligned
         hist = torch.empty((n_new, row), dtype=torch.int32, device=dev)
         cur = torch.empty((row,), dtype=torch.int32, device=dev)
-        pos = torch.full((Bn,), S - 1, dtype=torch.int32, device=dev)   # position behind the logits
+        lens = [S] * Bn if prompt_lens is None else [int(v) for v in prompt_lens]
+        assert len(lens) == Bn and all(1 <= v <= S for v in lens)
+        pos = torch.tensor([v - 1 for v in lens], dtype=torch.int32, device=dev)   # position behind the logits
         step = torch.zeros((1,), dtype=torch.int32, device=dev)
         pick = torch.empty((row,), dtype=torch.int32, device=dev)
         keep = return_logits or sampling
@@ -114,7 +124,13 @@ class Llama3Stack:
                 B.llama3_sample_top_p(lg, Bn, V, V, temperature, top_p, seed, 0, cur, stream, positions=pos)
             B.llama3_generation_advance(pos, cur, hist, step, Bn, n_new, row, stream)
 
-        head(x[:, -1], S * D, 0)           # first new token; pos -> S, step -> 1
+        if prompt_lens is None:
+            head(x[:, -1], S * D, 0)       # first new token; pos -> S, step -> 1
+        else:
+            idx = torch.tensor([b * S + v - 1 for b, v in enumerate(lens)], dtype=torch.int32, device=dev)
+            last = torch.empty((Bn, D), dtype=self.dtype, device=dev)
+            B.llama3_gather_rows(self.cfg, x, D, Bn * S, idx, Bn, last, stream)
+            head(last, D, 0)
         xd = torch.empty((Bn, 1, D), dtype=self.dtype, device=dev)
         max_pos = self.cache_cap - 1
 

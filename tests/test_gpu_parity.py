@@ -305,6 +305,33 @@ def test_greedy_generation_matches_oracle():
     assert compared >= n_new  # the check covered a real stretch of tokens
 
 
+def test_greedy_generation_with_prompts_of_different_lengths():
+    """Prompts of lengths 20, 7 and 13 padded to 20: each sequence's tokens
+    equal the oracle's greedy generation from its own prompt alone (at every
+    step whose top-2 gap exceeds 1e-2), with and without the CUDA graph."""
+    w = small_bf16(batch=3, seq=20, vocab=1000)
+    layers = [I.layer_weights(w, i, DEV, "random") for i in range(w.n_layers)]
+    outw = I.output_weights(w, DEV, "random")
+    n_new, lens = 10, [20, 7, 13]
+    st = Llama3Stack(w.cfg(), layers, outw, w.batch, w.seq + n_new, w.seq, lm_rows=w.batch)
+    prompt = I.token_ids(w, DEV)
+    got = st.generate(prompt, n_new, prompt_lens=lens)
+    st2 = Llama3Stack(w.cfg(), layers, outw, w.batch, w.seq + n_new, w.seq, lm_rows=w.batch)
+    np.testing.assert_array_equal(st2.generate(prompt, n_new, prompt_lens=lens, cuda_graph=True), got)
+    host = prompt.cpu().numpy()
+    compared = 0
+    for b, L in enumerate(lens):
+        toks, gaps = O.generate_greedy(host[b:b + 1, :L], f64(outw["tok_embeddings"]),
+                                       [oracle_layer(l) for l in layers], f64(outw["norm"]), f64(outw["output"]),
+                                       oracle_cfg(w), n_new)
+        for t in range(n_new):
+            if gaps[0, t] <= 1e-2:
+                break
+            assert got[b, t] == toks[0, t], (b, t, got[b], toks[0])
+            compared += 1
+    assert compared >= n_new
+
+
 # ------------------------------------------------------------ document mask
 def _doc_starts(Bn, S, P, seed):
     """Per-token document start positions: random document lengths packed

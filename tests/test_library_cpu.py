@@ -122,6 +122,13 @@ def test_sample_top_p_rejects_bad_arguments_before_launch():
     assert s(logits=None) == 1
     assert s(ids=ctypes.c_void_p(18)) == 2   # ids not 4-byte aligned
     assert s(pos=ctypes.c_void_p(FAKE + 2)) == 2
+    c = cfg8b()
+    gat = lambda **k: lib.llama3_gather_rows(ctypes.byref(c), FAKE, k.get("stride", 4096), k.get("n", 8), FAKE,
+                                             k.get("rows", 2), FAKE, None)
+    assert gat(rows=0) == 1
+    assert gat(n=0) == 1
+    assert gat(stride=100) == 1
+    assert gat(stride=4100) == 2
     adv = lambda **k: lib.llama3_generation_advance(k.get("pos", FAKE), FAKE, FAKE, FAKE, k.get("batch", 4),
                                                     k.get("rows", 8), k.get("stride", 4), None)
     assert adv(batch=0) == 1
