@@ -103,7 +103,7 @@ def _attn_case(Bn, S, P, H, KV, hd, seed):
     (2, 200, 0, 8, 2, 64), (2, 129, 37, 8, 2, 96), (1, 300, 0, 32, 8, 128), (3, 64, 500, 4, 4, 128),
     (1, 1, 0, 8, 2, 128), (4, 1, 1, 8, 1, 64), (3, 1, 1000, 32, 8, 128), (2, 1, 300, 8, 2, 96),
     (2, 1, 777, 16, 16, 64), (2, 1, 500, 12, 4, 64), (1, 150, 20, 12, 4, 64), (2, 1, 130, 16, 1, 128),
-    (1, 1, 8192, 32, 8, 128), (2, 300, 0, 6, 2, 96)])
+    (1, 1, 8192, 32, 8, 128), (2, 300, 0, 6, 2, 96), (1, 200, 10, 12, 4, 128), (2, 129, 0, 16, 2, 128)])
 @pytest.mark.parametrize("variant", [1, 2, 3, 4])
 def test_attention(Bn, S, P, H, KV, hd, variant):
     if variant != 3 and S == 1:
