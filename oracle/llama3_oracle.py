@@ -17,8 +17,7 @@ Sources (the five web pages on the Llama-3 decoder; cited by title + section):
   [S3] "llama3-from-scratch：输出层与预测" (agent.csdn.net), "预测流程的完整实现".
   [S4] "Llama3 architecture" blog (joto.ai), GQA and RoPE paragraphs.
 
-Readings taken where the pages are silent or disagree (each also listed in
-DESIGN.md):
+Readings taken where the pages are silent or disagree:
   * RoPE pairs adjacent elements (2i, 2i+1) as one complex number, real part
     first ([S1] §6.6-6.9, [S2] §3.2); the exponent uses head_dim ([S2] §3.2,
     frequencies built for dim=head_dim); angles are evaluated exactly in fp64.
