@@ -4,8 +4,8 @@
 // scratch" §3.4; document mask of 附 1).  One softmax thread per query row as
 // in the first design, but:
 //  * the warpgroups trade registers at start-up (setmaxnreg): the producer /
-//    MMA warpgroup drops to 40 per thread and the two softmax warpgroups rise
-//    to 232, so a thread holds its row's 128 scores of a tile at once and
+//    MMA warpgroup drops to 104 per thread and the two softmax warpgroups rise
+//    to 200, so a thread holds its row's 128 scores of a tile at once and
 //    reads them from TMEM a single time (one max pass, one exponent pass, both
 //    from registers);
 //  * P (bf16, two per 32-bit column) is written back into TMEM over the
@@ -13,7 +13,7 @@
 //    from TMEM, so P never goes through shared memory;
 //  * K and V are both double-buffered in the shared memory P no longer uses.
 // The split of registers is only valid for a launch of 384 threads at 168
-// registers each (128*40 + 256*232 = 384*168); the host checks the compiled
+// registers each (128*104 + 256*200 = 384*168); the host checks the compiled
 // register count before every launch.
 #pragma once
 #include "flash_attention2.cuh"
@@ -186,21 +186,14 @@ __global__ void __launch_bounds__(kFlash3Threads, 1)
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       int ks = 0, vs = 0;
-      // phase bits per slot (bit s) of the Q, P and O barriers as this thread sees them
+      // phase bits per slot (bit s) of the Q and P barriers as this thread sees them
       uint32_t kph = 0, vph = 0, qph = 0, pph = 0;
-      // S of the next tile overwrites the TMEM columns that hold P: the P.V
-      // that reads them must be complete first (this thread's view of o_done,
-      // which the softmax warps also wait on; opend: a P.V not yet waited for)
-      uint32_t oph = 0, opend = 0;
       bool ok = true;
-      auto pv_retired = [&](int s) -> bool {
-        if (!(opend & (1u << s))) return true;
-        opend &= ~(1u << s);
-        const bool r = mbar_wait(&o_done[s], (oph >> s) & 1u, wait_ns);
-        oph ^= 1u << s;
-        tc_fence_after();
-        return r;
-      };
+      // S of the next tile overwrites the TMEM columns that hold P.  It is
+      // issued right behind the P.V that reads them, without waiting for that
+      // P.V to complete: the MMAs one thread issues execute in issue order, so
+      // every read of P precedes the first write of the next S (the tcgen05
+      // attention mainloops of CUTLASS rely on the same order).
       const uint32_t q_addr = smem_u32(smem + C::OFF_Q);
       auto issue_s = [&](int s, int kst) {
         const uint32_t d = tmem_base + s * 256;
@@ -222,7 +215,6 @@ __global__ void __launch_bounds__(kFlash3Threads, 1)
           tc_mma_f16_ts(d, pa + k * 8, sw128_desc(va + k * 2048, 1024, C::TILE_BYTES), IDESC_O,
                         (accumulate || k > 0) ? 1u : 0u);
         tc_commit(&o_done[s]);
-        opend |= 1u << s;
       };
       for (int k_ = 0, u = flash_snake(0); u < fs.units && ok; u = flash_snake(++k_)) {
         int b, g, pair, qt;
@@ -238,11 +230,7 @@ __global__ void __launch_bounds__(kFlash3Threads, 1)
         const int jt0 = flash_first_tile(fs, b, qt);
         if (!mbar_wait(&k_full[ks], kph, wait_ns)) break;
         tc_fence_after();
-        for (int s = 0; s < nslots; ++s) {
-          if (!pv_retired(s)) { ok = false; break; }
-          issue_s(s, ks);
-        }
-        if (!ok) break;
+        for (int s = 0; s < nslots; ++s) issue_s(s, ks);
         tc_commit(&k_empty[ks]);
         if (++ks == C::KST) { ks = 0; kph ^= 1u; }
         for (int j = jt0; j < nt && ok; ++j) {
@@ -257,7 +245,6 @@ __global__ void __launch_bounds__(kFlash3Threads, 1)
             if (more) {
               if (!k_ready && !mbar_wait(&k_full[ks], kph, wait_ns)) { ok = false; break; }
               k_ready = true;
-              if (!pv_retired(s)) { ok = false; break; }
               issue_s(s, ks);
             }
           }
