@@ -150,20 +150,11 @@ __global__ void __launch_bounds__(640, 1)
       int ks = 0, vs = 0;
       uint32_t kph = 0, vph = 0, qph[2] = {0, 0};
       uint32_t pph[2] = {0, 0};
-      // S of the next tile overwrites the TMEM columns that hold P: the P.V
-      // that reads them must be complete first (oph/opend: this thread's view
-      // of o_done, which the softmax warps also wait on)
-      uint32_t oph[2] = {0, 0};
-      bool opend[2] = {false, false};
       bool ok = true;
-      auto pv_retired = [&](int s) -> bool {
-        if (!opend[s]) return true;
-        opend[s] = false;
-        const bool r = mbar_wait(&o_done[s], oph[s], wait_ns);
-        oph[s] ^= 1u;
-        tc_fence_after();
-        return r;
-      };
+      // S of the next tile overwrites the TMEM columns that hold P.  It is
+      // issued right behind the P.V that reads them, without waiting for that
+      // P.V to complete: the MMAs one thread issues execute in issue order, so
+      // every read of P precedes the first write of the next S.
       const uint32_t q_addr = smem_u32(smem + C::OFF_Q);
       auto issue_s = [&](int s, int kst) {
         const uint32_t d = tmem_base + s * 256;
@@ -187,7 +178,6 @@ __global__ void __launch_bounds__(640, 1)
           tc_mma_f16_ts(d, a, bdesc, IDESC_O, (accumulate || k > 0) ? 1u : 0u);
         }
         tc_commit(&o_done[s]);
-        opend[s] = true;
       };
       for (int k_ = 0, u = flash_snake(0); u < fs.units && ok; u = flash_snake(++k_)) {
         int b, g, pair, qt;
@@ -203,11 +193,7 @@ __global__ void __launch_bounds__(640, 1)
         const int jt0 = flash_first_tile(fs, b, qt);
         if (!mbar_wait(&k_full[ks], kph, wait_ns)) break;
         tc_fence_after();
-        for (int s = 0; s < nslots; ++s) {
-          if (!pv_retired(s)) { ok = false; break; }
-          issue_s(s, ks);
-        }
-        if (!ok) break;
+        for (int s = 0; s < nslots; ++s) issue_s(s, ks);
         tc_commit(&k_empty[ks]);
         if (++ks == C::KST) { ks = 0; kph ^= 1u; }
         for (int j = jt0; j < nt && ok; ++j) {
@@ -222,7 +208,6 @@ __global__ void __launch_bounds__(640, 1)
             if (more) {
               if (!k_ready && !mbar_wait(&k_full[ks], kph, wait_ns)) { ok = false; break; }
               k_ready = true;
-              if (!pv_retired(s)) { ok = false; break; }
               issue_s(s, ks);
             }
           }

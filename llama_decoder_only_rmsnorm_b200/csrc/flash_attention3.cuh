@@ -50,28 +50,49 @@ __device__ __forceinline__ void flash3_load_row(uint32_t taddr, uint32_t (&a)[32
   tc_wait_ld();
 }
 
-// p = 2^(s*scale - m) for 32 scores, their sum, and the bf16 pairs stored
-// to the 16 TMEM columns at taddr.  Exponentials in fp32: on unmasked tiles 6
-// of every 16 pairs go to the FMA pipe (exp2_poly2), the rest to the MUFU;
-// masked tiles use the MUFU only, which gives exactly 0 for the -inf scores.
+// p = 2^(s*scl - m) for 32 scores of the row, in place (as fp32 bits), and
+// their sum in (sa, sb).  Exponentials in fp32: on unmasked tiles 4 of every
+// 16 pairs go to the FMA pipe (exp2_poly2), the rest to the MUFU; masked tiles
+// use the MUFU only, which gives exactly 0 for the -inf scores.
 template <bool MASKED>
-__device__ __forceinline__ void flash3_exp_chunk(const uint32_t (&r)[32], float scl, float neg_m, float& sum_a,
-                                                 float& sum_b, uint32_t taddr) {
-  uint32_t pk[16];
+__device__ __forceinline__ void flash3_exp_inplace(uint32_t (&r)[32], float scl, float neg_m, float& sa, float& sb) {
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     float x0, x1, p0, p1;
     fma2(x0, x1, __uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), scl, scl, neg_m, neg_m);
-    if (!MASKED && (i & 7) < 3) {
+    if (!MASKED && (i & 7) < 2) {
       exp2_poly2(x0, x1, p0, p1);
     } else {
       p0 = ex2_approx(x0);
       p1 = ex2_approx(x1);
     }
-    add2(sum_a, sum_b, p0, p1);
-    pk[i] = pack_bf16x2(p0, p1);
+    add2(sa, sb, p0, p1);
+    r[2 * i] = __float_as_uint(p0);
+    r[2 * i + 1] = __float_as_uint(p1);
   }
+}
+__device__ __forceinline__ void flash3_pack_store(uint32_t (&r)[32], uint32_t taddr) {
+  uint32_t pk[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
   tmem_st16(taddr, pk);
+}
+// The whole row: all 128 exponentials before any pack or store, so that the
+// four chunks overlap; then the bf16 pairs go to the 64 TMEM columns at taddr
+// (keys 0-127 -> columns 0-63).  Returns the row's sum over the tile.
+template <bool MASKED>
+__device__ __forceinline__ float flash3_exp_row(uint32_t (&ra)[32], uint32_t (&rb)[32], uint32_t (&rc)[32],
+                                                uint32_t (&rd)[32], float scl, float neg_m, uint32_t taddr) {
+  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f, s4 = 0.f, s5 = 0.f, s6 = 0.f, s7 = 0.f;
+  flash3_exp_inplace<MASKED>(ra, scl, neg_m, s0, s1);
+  flash3_exp_inplace<MASKED>(rb, scl, neg_m, s2, s3);
+  flash3_exp_inplace<MASKED>(rc, scl, neg_m, s4, s5);
+  flash3_exp_inplace<MASKED>(rd, scl, neg_m, s6, s7);
+  flash3_pack_store(ra, taddr);
+  flash3_pack_store(rb, taddr + 16);
+  flash3_pack_store(rc, taddr + 32);
+  flash3_pack_store(rd, taddr + 48);
+  return ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
 }
 
 template <bool MASKED>
@@ -110,7 +131,10 @@ __global__ void __launch_bounds__(kFlash3Threads, 1)
   uint64_t* o_done = p_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_done + 2);
 
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // warp index through a shuffle: the compiler then treats it as uniform
+  // across the warp, so the whole-warp MMA issuer below keeps its addresses
+  // and descriptors in uniform registers
+  const int warp = __shfl_sync(0xffffffffu, (int)(threadIdx.x >> 5), 0), lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
       mbar_init(&q_full[s], 1); mbar_init(&q_empty[s], 1);
@@ -127,7 +151,7 @@ __global__ void __launch_bounds__(kFlash3Threads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
+  const uint32_t tmem_base = __shfl_sync(0xffffffffu, *tmem_slot, 0);
   // Each warpgroup takes its register share (all threads of a warpgroup
   // execute it).  The two roles stay in separate branches up to the final
   // barrier, so the register limit of one never applies to the other's code.
@@ -184,7 +208,10 @@ __global__ void __launch_bounds__(kFlash3Threads, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the loop and waits; one elected lane issues the
+    // MMAs and commits, from warp-uniform addresses.
+    {
+      const bool leader = elect_one_sync();
       int ks = 0, vs = 0;
       // phase bits per slot (bit s) of the Q and P barriers as this thread sees them
       uint32_t kph = 0, vph = 0, qph = 0, pph = 0;
@@ -199,22 +226,28 @@ __global__ void __launch_bounds__(kFlash3Threads, 1)
         const uint32_t d = tmem_base + s * 256;
         const uint32_t qa = q_addr + s * C::Q_BYTES;
         const uint32_t ka = smem_u32(smem + C::OFF_K + kst * C::KV_BYTES);
+        if (leader) {
 #pragma unroll
-        for (int k = 0; k < HD / 16; ++k) {
-          const uint32_t off = (k >> 2) * C::TILE_BYTES + (k & 3) * 32;
-          tc_mma_f16_ss(d, sw128_desc(qa + off, 1024, 16), sw128_desc(ka + off, 1024, 16), IDESC_S, k > 0);
+          for (int k = 0; k < HD / 16; ++k) {
+            const uint32_t off = (k >> 2) * C::TILE_BYTES + (k & 3) * 32;
+            tc_mma_f16_ss(d, sw128_desc(qa + off, 1024, 16), sw128_desc(ka + off, 1024, 16), IDESC_S, k > 0);
+          }
+          tc_commit(&s_full[s]);
         }
-        tc_commit(&s_full[s]);
+        __syncwarp();
       };
       auto issue_pv = [&](int s, int vst, bool accumulate) {
         const uint32_t d = tmem_base + s * 256 + 128;
         const uint32_t pa = tmem_base + s * 256;   // P: keys 16k.. in columns 8k..
         const uint32_t va = smem_u32(smem + C::OFF_V + vst * C::KV_BYTES);
+        if (leader) {
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-          tc_mma_f16_ts(d, pa + k * 8, sw128_desc(va + k * 2048, 1024, C::TILE_BYTES), IDESC_O,
-                        (accumulate || k > 0) ? 1u : 0u);
-        tc_commit(&o_done[s]);
+          for (int k = 0; k < 8; ++k)
+            tc_mma_f16_ts(d, pa + k * 8, sw128_desc(va + k * 2048, 1024, C::TILE_BYTES), IDESC_O,
+                          (accumulate || k > 0) ? 1u : 0u);
+          tc_commit(&o_done[s]);
+        }
+        __syncwarp();
       };
       for (int k_ = 0, u = flash_snake(0); u < fs.units && ok; u = flash_snake(++k_)) {
         int b, g, pair, qt;
@@ -222,41 +255,43 @@ __global__ void __launch_bounds__(kFlash3Threads, 1)
         const int nt = flash_ntiles(fs, qt);
         const int nslots = (pair * 2 + 1 < fs.n_rep) ? 2 : 1;
         for (int s = 0; s < nslots; ++s) {
-          if (!mbar_wait(&q_full[s], (qph >> s) & 1u, wait_ns)) ok = false;
+          if (!mbar_wait_warp(&q_full[s], (qph >> s) & 1u, wait_ns)) ok = false;
           qph ^= 1u << s;
         }
         if (!ok) break;
         tc_fence_after();
         const int jt0 = flash_first_tile(fs, b, qt);
-        if (!mbar_wait(&k_full[ks], kph, wait_ns)) break;
+        if (!mbar_wait_warp(&k_full[ks], kph, wait_ns)) break;
         tc_fence_after();
         for (int s = 0; s < nslots; ++s) issue_s(s, ks);
-        tc_commit(&k_empty[ks]);
+        if (leader) tc_commit(&k_empty[ks]);
         if (++ks == C::KST) { ks = 0; kph ^= 1u; }
         for (int j = jt0; j < nt && ok; ++j) {
-          if (!mbar_wait(&v_full[vs], vph, wait_ns)) { ok = false; break; }
+          if (!mbar_wait_warp(&v_full[vs], vph, wait_ns)) { ok = false; break; }
           const bool more = j + 1 < nt;
           bool k_ready = false;
           for (int s = 0; s < nslots; ++s) {
-            if (!mbar_wait(&p_full[s], (pph >> s) & 1u, wait_ns)) { ok = false; break; }
+            if (!mbar_wait_warp(&p_full[s], (pph >> s) & 1u, wait_ns)) { ok = false; break; }
             pph ^= 1u << s;
             tc_fence_after();
             issue_pv(s, vs, j > jt0);
             if (more) {
-              if (!k_ready && !mbar_wait(&k_full[ks], kph, wait_ns)) { ok = false; break; }
+              if (!k_ready && !mbar_wait_warp(&k_full[ks], kph, wait_ns)) { ok = false; break; }
               k_ready = true;
               issue_s(s, ks);
             }
           }
           if (!ok) break;
-          tc_commit(&v_empty[vs]);
+          if (leader) tc_commit(&v_empty[vs]);
           if (++vs == C::VST) { vs = 0; vph ^= 1u; }
           if (more) {
-            tc_commit(&k_empty[ks]);
+            if (leader) tc_commit(&k_empty[ks]);
             if (++ks == C::KST) { ks = 0; kph ^= 1u; }
           }
         }
-        for (int s = 0; s < nslots; ++s) tc_commit(&q_empty[s]);
+        if (leader)
+          for (int s = 0; s < nslots; ++s) tc_commit(&q_empty[s]);
+        __syncwarp();
       }
     }
   }
@@ -304,13 +339,11 @@ __global__ void __launch_bounds__(kFlash3Threads, 1)
         }
         const float mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
         const float m_tile = mx * fs.scale_log2;   // scale_log2 > 0: max commutes with the scale
-        // the previous tile's P.V must be complete before O is rescaled (and
-        // before P is rewritten: the MMA issuer also waits for it before S)
-        if (j > jt0) {
-          if (!mbar_wait(&o_done[slot], oph, wait_ns)) { ok = false; break; }
-          oph ^= 1u;
-          tc_fence_after();
-        }
+        // The previous tile's P.V is complete here: the s_full commit just
+        // waited for tracks every MMA issued before it, that P.V included.
+        // So O may be rescaled without waiting on o_done; only its phase is
+        // counted (one per P.V), for the epilogue's wait on the last one.
+        if (j > jt0) oph ^= 1u;
         const bool grow = m_tile > m_ref + 8.0f;
         float alpha = 1.f;
         if (grow) {
@@ -332,19 +365,10 @@ __global__ void __launch_bounds__(kFlash3Threads, 1)
         }
         const float scl = fs.scale_log2;
         const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;   // a row with no visible key yet: p = 0
-        float sum_a = 0.f, sum_b = 0.f;
-        if (need_mask) {
-          flash3_exp_chunk<true>(ra, scl, neg_m, sum_a, sum_b, s_tmem);
-          flash3_exp_chunk<true>(rb, scl, neg_m, sum_a, sum_b, s_tmem + 16);
-          flash3_exp_chunk<true>(rc, scl, neg_m, sum_a, sum_b, s_tmem + 32);
-          flash3_exp_chunk<true>(rd, scl, neg_m, sum_a, sum_b, s_tmem + 48);
-        } else {
-          flash3_exp_chunk<false>(ra, scl, neg_m, sum_a, sum_b, s_tmem);
-          flash3_exp_chunk<false>(rb, scl, neg_m, sum_a, sum_b, s_tmem + 16);
-          flash3_exp_chunk<false>(rc, scl, neg_m, sum_a, sum_b, s_tmem + 32);
-          flash3_exp_chunk<false>(rd, scl, neg_m, sum_a, sum_b, s_tmem + 48);
-        }
-        l += sum_a + sum_b;
+        if (need_mask)
+          l += flash3_exp_row<true>(ra, rb, rc, rd, scl, neg_m, s_tmem);
+        else
+          l += flash3_exp_row<false>(ra, rb, rc, rd, scl, neg_m, s_tmem);
         tc_wait_st();
         tc_fence_before();
         mbar_arrive(&p_full[slot]);
