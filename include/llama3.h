@@ -384,10 +384,11 @@ int llama3_set_programmatic_launch(int on);
  * (warpgroup register reallocation) with P in tensor memory; 1 = one softmax
  * thread per row with P staged in shared memory; 2 = two softmax threads per
  * row (each over half the keys of a tile) with P in tensor memory; 4 = as 3
- * with P staged in shared memory.  All compute the same attention.  Values
- * outside 1..4 select 3.  Variants 3 and 4 return LLAMA3_ERR_UNSUPPORTED if
- * the compiled kernel's register count cannot fund their register split.
- * Returns the previous value. */
+ * with P staged in shared memory; 5 = as 3, but both softmax warpgroups work
+ * on each tile (half the keys each) and then on the other head's tile.  All
+ * compute the same attention.  Values outside 1..5 select 3.  Variants 3, 4
+ * and 5 return LLAMA3_ERR_UNSUPPORTED if the compiled kernel's register count
+ * cannot fund their register split.  Returns the previous value. */
 int llama3_set_flash_variant(int variant);
 
 #ifdef __cplusplus

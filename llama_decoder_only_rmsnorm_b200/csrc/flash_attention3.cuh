@@ -108,15 +108,167 @@ __device__ __forceinline__ float flash3_row_max(uint32_t (&r)[32], int key0, int
   return mx;
 }
 
+// The barriers the three roles share (all in shared memory).
+struct Flash3Bars {
+  uint64_t *q_full, *q_empty, *k_full, *k_empty, *v_full, *v_empty, *s_full, *p_full, *o_done;
+};
+
+// Producer (one thread): per work unit the Q tiles of its one or two heads,
+// then K and V of every visible key tile, through the K and V rings.
+template <int HD>
+__device__ __forceinline__ void flash3_produce(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
+                                               uint8_t* smem, const Flash3Bars& B, const FlashShape& fs,
+                                               unsigned long long wait_ns) {
+  using C = Flash3Cfg<HD>;
+  uint64_t *q_full = B.q_full, *q_empty = B.q_empty, *k_full = B.k_full, *k_empty = B.k_empty;
+  uint64_t *v_full = B.v_full, *v_empty = B.v_empty;
+  int ks = 0, vs = 0;
+  uint32_t kph = 0, vph = 0, qph = 0;   // qph: phase bit per Q slot
+  bool ok = true;
+  uint32_t kiss = 0, kpar = 0, viss = 0, vpar = 0, qiss = 0, qpar = 0;
+  for (int k_ = 0, u = flash_snake(0); u < fs.units && ok; u = flash_snake(++k_)) {
+    int b, g, pair, qt;
+    flash_unit(fs, u, b, g, pair, qt);
+    const int nt = flash_ntiles(fs, qt);
+    const bool has1 = pair * 2 + 1 < fs.n_rep;
+    for (int s = 0; s < 2 && ok; ++s) {
+      if (s == 1 && !has1) break;
+      if (!mbar_wait(&q_empty[s], ((qph >> s) & 1u) ^ 1u, wait_ns)) { ok = false; break; }
+      mbar_arrive_expect_tx(&q_full[s], C::Q_BYTES);
+      const int h = g * fs.n_rep + pair * 2 + s;
+      for (int c = 0; c < C::CHUNKS; ++c)
+        tma_load_4d(smem + C::OFF_Q + s * C::Q_BYTES + c * C::TILE_BYTES, &mapQ, &q_full[s], c * 64, h,
+                    qt * 128, b);
+      qiss |= 1u << s; qpar = (qpar & ~(1u << s)) | (qph & (1u << s));
+      qph ^= 1u << s;
+    }
+    const int jt0 = flash_first_tile(fs, b, qt);
+    for (int j = jt0; j < nt && ok; ++j) {
+      if (!mbar_wait(&k_empty[ks], kph ^ 1u, wait_ns)) { ok = false; break; }
+      mbar_arrive_expect_tx(&k_full[ks], C::KV_BYTES);
+      for (int c = 0; c < C::CHUNKS; ++c)
+        tma_load_4d(smem + C::OFF_K + ks * C::KV_BYTES + c * C::TILE_BYTES, &mapK, &k_full[ks], c * 64, g,
+                    j * 128, b);
+      kiss |= 1u << ks; kpar = (kpar & ~(1u << ks)) | (kph << ks);
+      if (++ks == C::KST) { ks = 0; kph ^= 1u; }
+      if (!mbar_wait(&v_empty[vs], vph ^ 1u, wait_ns)) { ok = false; break; }
+      mbar_arrive_expect_tx(&v_full[vs], C::KV_BYTES);
+      for (int c = 0; c < C::CHUNKS; ++c)
+        tma_load_4d(smem + C::OFF_V + vs * C::KV_BYTES + c * C::TILE_BYTES, &mapV, &v_full[vs], c * 64, g,
+                    j * 128, b);
+      viss |= 1u << vs; vpar = (vpar & ~(1u << vs)) | (vph << vs);
+      if (++vs == C::VST) { vs = 0; vph ^= 1u; }
+    }
+  }
+  for (int s = 0; s < 2; ++s)
+    if (qiss & (1u << s)) mbar_wait(&q_full[s], (qpar >> s) & 1u, wait_ns);
+  for (int s = 0; s < C::KST; ++s)
+    if (kiss & (1u << s)) mbar_wait(&k_full[s], (kpar >> s) & 1u, wait_ns);
+  for (int s = 0; s < C::VST; ++s)
+    if (viss & (1u << s)) mbar_wait(&v_full[s], (vpar >> s) & 1u, wait_ns);
+}
+
+// MMA issuer (one whole warp; one elected lane issues).  Per key tile and head:
+// S = Q K^T into the head's S columns, and, once the softmax has written P over
+// them, O += P V (P from TMEM, V MN-major from shared memory).
+template <int HD>
+__device__ __forceinline__ void flash3_issue_mma(uint8_t* smem, const Flash3Bars& B, uint32_t tmem_base,
+                                                 const FlashShape& fs, unsigned long long wait_ns) {
+  using C = Flash3Cfg<HD>;
+  constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, 0, 0);
+  constexpr uint32_t IDESC_O = idesc_bf16_f32(128, HD, 0, 1);   // A = P (TMEM), B = V MN-major
+  uint64_t *q_full = B.q_full, *q_empty = B.q_empty, *k_full = B.k_full, *k_empty = B.k_empty;
+  uint64_t *v_full = B.v_full, *v_empty = B.v_empty, *s_full = B.s_full, *p_full = B.p_full, *o_done = B.o_done;
+  const bool leader = elect_one_sync();
+  int ks = 0, vs = 0;
+  // phase bits per slot (bit s) of the Q and P barriers as this thread sees them
+  uint32_t kph = 0, vph = 0, qph = 0, pph = 0;
+  bool ok = true;
+  // S of the next tile overwrites the TMEM columns that hold P.  It is
+  // issued right behind the P.V that reads them, without waiting for that
+  // P.V to complete: the MMAs one thread issues execute in issue order, so
+  // every read of P precedes the first write of the next S (the tcgen05
+  // attention mainloops of CUTLASS rely on the same order).
+  const uint32_t q_addr = smem_u32(smem + C::OFF_Q);
+  auto issue_s = [&](int s, int kst) {
+    const uint32_t d = tmem_base + s * 256;
+    const uint32_t qa = q_addr + s * C::Q_BYTES;
+    const uint32_t ka = smem_u32(smem + C::OFF_K + kst * C::KV_BYTES);
+    if (leader) {
+#pragma unroll
+      for (int k = 0; k < HD / 16; ++k) {
+        const uint32_t off = (k >> 2) * C::TILE_BYTES + (k & 3) * 32;
+        tc_mma_f16_ss(d, sw128_desc(qa + off, 1024, 16), sw128_desc(ka + off, 1024, 16), IDESC_S, k > 0);
+      }
+      tc_commit(&s_full[s]);
+    }
+    __syncwarp();
+  };
+  auto issue_pv = [&](int s, int vst, bool accumulate) {
+    const uint32_t d = tmem_base + s * 256 + 128;
+    const uint32_t pa = tmem_base + s * 256;   // P: keys 16k.. in columns 8k..
+    const uint32_t va = smem_u32(smem + C::OFF_V + vst * C::KV_BYTES);
+    if (leader) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        tc_mma_f16_ts(d, pa + k * 8, sw128_desc(va + k * 2048, 1024, C::TILE_BYTES), IDESC_O,
+                      (accumulate || k > 0) ? 1u : 0u);
+      tc_commit(&o_done[s]);
+    }
+    __syncwarp();
+  };
+  for (int k_ = 0, u = flash_snake(0); u < fs.units && ok; u = flash_snake(++k_)) {
+    int b, g, pair, qt;
+    flash_unit(fs, u, b, g, pair, qt);
+    const int nt = flash_ntiles(fs, qt);
+    const int nslots = (pair * 2 + 1 < fs.n_rep) ? 2 : 1;
+    for (int s = 0; s < nslots; ++s) {
+      if (!mbar_wait_warp(&q_full[s], (qph >> s) & 1u, wait_ns)) ok = false;
+      qph ^= 1u << s;
+    }
+    if (!ok) break;
+    tc_fence_after();
+    const int jt0 = flash_first_tile(fs, b, qt);
+    if (!mbar_wait_warp(&k_full[ks], kph, wait_ns)) break;
+    tc_fence_after();
+    for (int s = 0; s < nslots; ++s) issue_s(s, ks);
+    if (leader) tc_commit(&k_empty[ks]);
+    if (++ks == C::KST) { ks = 0; kph ^= 1u; }
+    for (int j = jt0; j < nt && ok; ++j) {
+      if (!mbar_wait_warp(&v_full[vs], vph, wait_ns)) { ok = false; break; }
+      const bool more = j + 1 < nt;
+      bool k_ready = false;
+      for (int s = 0; s < nslots; ++s) {
+        if (!mbar_wait_warp(&p_full[s], (pph >> s) & 1u, wait_ns)) { ok = false; break; }
+        pph ^= 1u << s;
+        tc_fence_after();
+        issue_pv(s, vs, j > jt0);
+        if (more) {
+          if (!k_ready && !mbar_wait_warp(&k_full[ks], kph, wait_ns)) { ok = false; break; }
+          k_ready = true;
+          issue_s(s, ks);
+        }
+      }
+      if (!ok) break;
+      if (leader) tc_commit(&v_empty[vs]);
+      if (++vs == C::VST) { vs = 0; vph ^= 1u; }
+      if (more) {
+        if (leader) tc_commit(&k_empty[ks]);
+        if (++ks == C::KST) { ks = 0; kph ^= 1u; }
+      }
+    }
+    if (leader)
+      for (int s = 0; s < nslots; ++s) tc_commit(&q_empty[s]);
+    __syncwarp();
+  }
+}
+
 template <int HD>
 __global__ void __launch_bounds__(kFlash3Threads, 1)
     flash_attention3_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
                             const __grid_constant__ CUtensorMap mapV, bf16* __restrict__ out, const FlashShape fs,
                             const unsigned long long wait_ns) {
   using C = Flash3Cfg<HD>;
-  constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, 0, 0);
-  constexpr uint32_t IDESC_O = idesc_bf16_f32(128, HD, 0, 1);   // A = P (TMEM), B = V MN-major
-
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
@@ -130,6 +282,7 @@ __global__ void __launch_bounds__(kFlash3Threads, 1)
   uint64_t* p_full = s_full + 2;
   uint64_t* o_done = p_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_done + 2);
+  const Flash3Bars bars3{q_full, q_empty, k_full, k_empty, v_full, v_empty, s_full, p_full, o_done};
 
   // warp index through a shuffle: the compiler then treats it as uniform
   // across the warp, so the whole-warp MMA issuer below keeps its addresses
@@ -160,140 +313,10 @@ __global__ void __launch_bounds__(kFlash3Threads, 1)
     griddep_wait_and_release();
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
-    if (lane == 0) {
-      int ks = 0, vs = 0;
-      uint32_t kph = 0, vph = 0, qph = 0;   // qph: phase bit per Q slot
-      bool ok = true;
-      uint32_t kiss = 0, kpar = 0, viss = 0, vpar = 0, qiss = 0, qpar = 0;
-      for (int k_ = 0, u = flash_snake(0); u < fs.units && ok; u = flash_snake(++k_)) {
-        int b, g, pair, qt;
-        flash_unit(fs, u, b, g, pair, qt);
-        const int nt = flash_ntiles(fs, qt);
-        const bool has1 = pair * 2 + 1 < fs.n_rep;
-        for (int s = 0; s < 2 && ok; ++s) {
-          if (s == 1 && !has1) break;
-          if (!mbar_wait(&q_empty[s], ((qph >> s) & 1u) ^ 1u, wait_ns)) { ok = false; break; }
-          mbar_arrive_expect_tx(&q_full[s], C::Q_BYTES);
-          const int h = g * fs.n_rep + pair * 2 + s;
-          for (int c = 0; c < C::CHUNKS; ++c)
-            tma_load_4d(smem + C::OFF_Q + s * C::Q_BYTES + c * C::TILE_BYTES, &mapQ, &q_full[s], c * 64, h,
-                        qt * 128, b);
-          qiss |= 1u << s; qpar = (qpar & ~(1u << s)) | (qph & (1u << s));
-          qph ^= 1u << s;
-        }
-        const int jt0 = flash_first_tile(fs, b, qt);
-        for (int j = jt0; j < nt && ok; ++j) {
-          if (!mbar_wait(&k_empty[ks], kph ^ 1u, wait_ns)) { ok = false; break; }
-          mbar_arrive_expect_tx(&k_full[ks], C::KV_BYTES);
-          for (int c = 0; c < C::CHUNKS; ++c)
-            tma_load_4d(smem + C::OFF_K + ks * C::KV_BYTES + c * C::TILE_BYTES, &mapK, &k_full[ks], c * 64, g,
-                        j * 128, b);
-          kiss |= 1u << ks; kpar = (kpar & ~(1u << ks)) | (kph << ks);
-          if (++ks == C::KST) { ks = 0; kph ^= 1u; }
-          if (!mbar_wait(&v_empty[vs], vph ^ 1u, wait_ns)) { ok = false; break; }
-          mbar_arrive_expect_tx(&v_full[vs], C::KV_BYTES);
-          for (int c = 0; c < C::CHUNKS; ++c)
-            tma_load_4d(smem + C::OFF_V + vs * C::KV_BYTES + c * C::TILE_BYTES, &mapV, &v_full[vs], c * 64, g,
-                        j * 128, b);
-          viss |= 1u << vs; vpar = (vpar & ~(1u << vs)) | (vph << vs);
-          if (++vs == C::VST) { vs = 0; vph ^= 1u; }
-        }
-      }
-      for (int s = 0; s < 2; ++s)
-        if (qiss & (1u << s)) mbar_wait(&q_full[s], (qpar >> s) & 1u, wait_ns);
-      for (int s = 0; s < C::KST; ++s)
-        if (kiss & (1u << s)) mbar_wait(&k_full[s], (kpar >> s) & 1u, wait_ns);
-      for (int s = 0; s < C::VST; ++s)
-        if (viss & (1u << s)) mbar_wait(&v_full[s], (vpar >> s) & 1u, wait_ns);
-    }
+    if (lane == 0) flash3_produce<HD>(mapQ, mapK, mapV, smem, bars3, fs, wait_ns);
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    // The whole warp runs the loop and waits; one elected lane issues the
-    // MMAs and commits, from warp-uniform addresses.
-    {
-      const bool leader = elect_one_sync();
-      int ks = 0, vs = 0;
-      // phase bits per slot (bit s) of the Q and P barriers as this thread sees them
-      uint32_t kph = 0, vph = 0, qph = 0, pph = 0;
-      bool ok = true;
-      // S of the next tile overwrites the TMEM columns that hold P.  It is
-      // issued right behind the P.V that reads them, without waiting for that
-      // P.V to complete: the MMAs one thread issues execute in issue order, so
-      // every read of P precedes the first write of the next S (the tcgen05
-      // attention mainloops of CUTLASS rely on the same order).
-      const uint32_t q_addr = smem_u32(smem + C::OFF_Q);
-      auto issue_s = [&](int s, int kst) {
-        const uint32_t d = tmem_base + s * 256;
-        const uint32_t qa = q_addr + s * C::Q_BYTES;
-        const uint32_t ka = smem_u32(smem + C::OFF_K + kst * C::KV_BYTES);
-        if (leader) {
-#pragma unroll
-          for (int k = 0; k < HD / 16; ++k) {
-            const uint32_t off = (k >> 2) * C::TILE_BYTES + (k & 3) * 32;
-            tc_mma_f16_ss(d, sw128_desc(qa + off, 1024, 16), sw128_desc(ka + off, 1024, 16), IDESC_S, k > 0);
-          }
-          tc_commit(&s_full[s]);
-        }
-        __syncwarp();
-      };
-      auto issue_pv = [&](int s, int vst, bool accumulate) {
-        const uint32_t d = tmem_base + s * 256 + 128;
-        const uint32_t pa = tmem_base + s * 256;   // P: keys 16k.. in columns 8k..
-        const uint32_t va = smem_u32(smem + C::OFF_V + vst * C::KV_BYTES);
-        if (leader) {
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            tc_mma_f16_ts(d, pa + k * 8, sw128_desc(va + k * 2048, 1024, C::TILE_BYTES), IDESC_O,
-                          (accumulate || k > 0) ? 1u : 0u);
-          tc_commit(&o_done[s]);
-        }
-        __syncwarp();
-      };
-      for (int k_ = 0, u = flash_snake(0); u < fs.units && ok; u = flash_snake(++k_)) {
-        int b, g, pair, qt;
-        flash_unit(fs, u, b, g, pair, qt);
-        const int nt = flash_ntiles(fs, qt);
-        const int nslots = (pair * 2 + 1 < fs.n_rep) ? 2 : 1;
-        for (int s = 0; s < nslots; ++s) {
-          if (!mbar_wait_warp(&q_full[s], (qph >> s) & 1u, wait_ns)) ok = false;
-          qph ^= 1u << s;
-        }
-        if (!ok) break;
-        tc_fence_after();
-        const int jt0 = flash_first_tile(fs, b, qt);
-        if (!mbar_wait_warp(&k_full[ks], kph, wait_ns)) break;
-        tc_fence_after();
-        for (int s = 0; s < nslots; ++s) issue_s(s, ks);
-        if (leader) tc_commit(&k_empty[ks]);
-        if (++ks == C::KST) { ks = 0; kph ^= 1u; }
-        for (int j = jt0; j < nt && ok; ++j) {
-          if (!mbar_wait_warp(&v_full[vs], vph, wait_ns)) { ok = false; break; }
-          const bool more = j + 1 < nt;
-          bool k_ready = false;
-          for (int s = 0; s < nslots; ++s) {
-            if (!mbar_wait_warp(&p_full[s], (pph >> s) & 1u, wait_ns)) { ok = false; break; }
-            pph ^= 1u << s;
-            tc_fence_after();
-            issue_pv(s, vs, j > jt0);
-            if (more) {
-              if (!k_ready && !mbar_wait_warp(&k_full[ks], kph, wait_ns)) { ok = false; break; }
-              k_ready = true;
-              issue_s(s, ks);
-            }
-          }
-          if (!ok) break;
-          if (leader) tc_commit(&v_empty[vs]);
-          if (++vs == C::VST) { vs = 0; vph ^= 1u; }
-          if (more) {
-            if (leader) tc_commit(&k_empty[ks]);
-            if (++ks == C::KST) { ks = 0; kph ^= 1u; }
-          }
-        }
-        if (leader)
-          for (int s = 0; s < nslots; ++s) tc_commit(&q_empty[s]);
-        __syncwarp();
-      }
-    }
+    flash3_issue_mma<HD>(smem, bars3, tmem_base, fs, wait_ns);
   }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kFlash3HighRegs));
@@ -318,7 +341,7 @@ __global__ void __launch_bounds__(kFlash3Threads, 1)
       float m_ref = -INFINITY, l = 0.f;
       bool ok = true;
       for (int j = jt0; j < nt; ++j) {
-        if (!mbar_wait(&s_full[slot], sph, wait_ns)) { ok = false; break; }
+        if (!mbar_wait_warp(&s_full[slot], sph, wait_ns)) { ok = false; break; }
         sph ^= 1u;
         tc_fence_after();
         const bool need_mask = j * 128 + 127 > fs.P + qt * 128 || j * 128 < lo_last;
@@ -375,7 +398,7 @@ __global__ void __launch_bounds__(kFlash3Threads, 1)
       }
       if (!ok) break;
       // epilogue: wait for the last P.V, out = O / l
-      if (!mbar_wait(&o_done[slot], oph, wait_ns)) break;
+      if (!mbar_wait_warp(&o_done[slot], oph, wait_ns)) break;
       oph ^= 1u;
       tc_fence_after();
       const int t = qt * 128 + row;

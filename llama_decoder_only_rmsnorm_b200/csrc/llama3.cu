@@ -19,6 +19,7 @@
 #include "flash_attention2.cuh"
 #include "flash_attention3.cuh"
 #include "flash_attention4.cuh"
+#include "flash_attention5.cuh"
 #include "sampling.cuh"
 #include "simt.cuh"
 #include "tc_gemm.cuh"
@@ -247,11 +248,13 @@ int run_flash_attention_t(int H, int KV, const void* q, const void* kc, const vo
   fs.ldo = H * HD;
   fs.scale_log2 = (float)(1.4426950408889634 / sqrt((double)HD));
   fs.doc_start = doc_start;
-  constexpr int smem = VARIANT == 4 ? Flash4Cfg<HD>::SMEM_BYTES
+  constexpr int smem = VARIANT == 5 ? Flash5Cfg<HD>::SMEM_BYTES
+                     : VARIANT == 4 ? Flash4Cfg<HD>::SMEM_BYTES
                      : VARIANT == 3 ? Flash3Cfg<HD>::SMEM_BYTES
                      : VARIANT == 2 ? Flash2Cfg<HD>::SMEM_BYTES : FlashCfg<HD>::SMEM_BYTES;
   constexpr int threads = VARIANT >= 3 ? kFlash3Threads : VARIANT == 2 ? 640 : 384;
-  auto kern = VARIANT == 4 ? flash_attention4_kernel<HD>
+  auto kern = VARIANT == 5 ? flash_attention5_kernel<HD>
+            : VARIANT == 4 ? flash_attention4_kernel<HD>
             : VARIANT == 3 ? flash_attention3_kernel<HD>
             : VARIANT == 2 ? flash_attention2_kernel<HD> : flash_attention_kernel<HD>;
   int dev = 0;
@@ -279,6 +282,8 @@ template <int HD>
 int run_flash_attention_v(int H, int KV, const void* q, const void* kc, const void* vc, int cap, int B, int S,
                           int P, void* out, const int32_t* doc_start, int sms, unsigned long long wns,
                           cudaStream_t st) {
+  if (g_flash_variant == 5)
+    return run_flash_attention_t<HD, 5>(H, KV, q, kc, vc, cap, B, S, P, out, doc_start, sms, wns, st);
   if (g_flash_variant == 4)
     return run_flash_attention_t<HD, 4>(H, KV, q, kc, vc, cap, B, S, P, out, doc_start, sms, wns, st);
   if (g_flash_variant == 3)
@@ -941,7 +946,7 @@ int llama3_generation_advance(int32_t* positions, const int32_t* ids, int32_t* h
 
 int llama3_set_flash_variant(int variant) {
   const int old = g_flash_variant;
-  g_flash_variant = (variant >= 1 && variant <= 4) ? variant : 3;
+  g_flash_variant = (variant >= 1 && variant <= 5) ? variant : 3;
   return old;
 }
 

@@ -104,7 +104,7 @@ def _attn_case(Bn, S, P, H, KV, hd, seed):
     (1, 1, 0, 8, 2, 128), (4, 1, 1, 8, 1, 64), (3, 1, 1000, 32, 8, 128), (2, 1, 300, 8, 2, 96),
     (2, 1, 777, 16, 16, 64), (2, 1, 500, 12, 4, 64), (1, 150, 20, 12, 4, 64), (2, 1, 130, 16, 1, 128),
     (1, 1, 8192, 32, 8, 128), (2, 300, 0, 6, 2, 96), (1, 200, 10, 12, 4, 128), (2, 129, 0, 16, 2, 128)])
-@pytest.mark.parametrize("variant", [1, 2, 3, 4])
+@pytest.mark.parametrize("variant", [1, 2, 3, 4, 5])
 def test_attention(Bn, S, P, H, KV, hd, variant):
     if variant != 3 and S == 1:
         pytest.skip("single-token steps take the decode kernel")
@@ -170,7 +170,7 @@ def test_gqa_768_layer(path):
     _run_layers_vs_oracle(wl("gqa_768"), path=path)
 
 
-@pytest.mark.parametrize("variant", [1, 2, 4])
+@pytest.mark.parametrize("variant", [1, 2, 4, 5])
 def test_gqa_768_layer_other_attention_designs(variant):
     B.llama3_set_flash_variant(variant)
     _run_layers_vs_oracle(wl("gqa_768"))
@@ -351,7 +351,7 @@ def _doc_starts(Bn, S, P, seed):
 
 @pytest.mark.parametrize("Bn,S,P,H,KV,hd,path", [
     (2, 300, 0, 8, 2, 128, 0), (2, 200, 37, 8, 2, 64, 0), (1, 257, 0, 12, 4, 96, 0), (2, 130, 5, 8, 2, 64, 1)])
-@pytest.mark.parametrize("variant", [1, 2, 3, 4])
+@pytest.mark.parametrize("variant", [1, 2, 3, 4, 5])
 def test_attention_document_mask(Bn, S, P, H, KV, hd, path, variant):
     if variant != 3 and path != 0:
         pytest.skip("the SIMT path has one attention kernel")

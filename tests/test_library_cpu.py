@@ -141,5 +141,6 @@ def test_sample_top_p_rejects_bad_arguments_before_launch():
 
 def test_flash_variant_switch():
     old = B.llama3_set_flash_variant(1)
-    assert B.llama3_set_flash_variant(7) == 1      # values outside 1..4 select the third design
+    assert B.llama3_set_flash_variant(5) == 1
+    assert B.llama3_set_flash_variant(7) == 5      # values outside 1..5 select the third design
     assert B.llama3_set_flash_variant(old) == 3
