@@ -371,6 +371,7 @@ GemmShape make_shape(int rows_a, int rows_a2, int rows_b, int k, int bn, int spl
   // swapped (weight-streaming) launches have one n-tile, where grouping
   // changes nothing.
   s.group_m = std::max(1, std::min(L3_GROUP_M, s.tiles_m));
+  s.sk_per = 0;
   return s;
 }
 
@@ -382,6 +383,36 @@ GemmShape make_shape(int rows_a, int rows_a2, int rows_b, int k, int bn, int spl
 #ifndef L3_SPLIT_UNIT_COST
 #define L3_SPLIT_UNIT_COST 2
 #endif
+// Stream-K plan for `tiles` tiles of `kblocks` k-blocks on `sms` CTAs: per =
+// k-blocks per CTA, ctas = CTAs with work, slabs = most CTAs sharing a tile,
+// cost = the busiest CTA's k-blocks plus L3_SPLIT_UNIT_COST per tile it
+// touches (the same units as choose_splits).
+struct StreamK {
+  bool ok;
+  int per, ctas, slabs;
+  long long cost;
+};
+StreamK plan_stream_k(int tiles, int kblocks, int sms) {
+  StreamK p{};
+  const long long total = (long long)tiles * kblocks;
+  if (total <= 0 || sms <= 0) return p;
+  p.per = (int)((total + sms - 1) / sms);
+  p.ctas = (int)((total + p.per - 1) / p.per);
+  int slabs = 0, most_units = 0;
+  for (int t = 0; t < tiles; ++t) {
+    const long long t0 = (long long)t * kblocks;
+    slabs = std::max(slabs, (int)((t0 + kblocks - 1) / p.per - t0 / p.per + 1));
+  }
+  for (int c = 0; c < p.ctas; ++c) {
+    const long long a = (long long)c * p.per, b = std::min(a + p.per, total);
+    most_units = std::max(most_units, (int)((b - 1) / kblocks - a / kblocks + 1));
+  }
+  p.slabs = slabs;
+  p.cost = p.per + (long long)most_units * L3_SPLIT_UNIT_COST;
+  p.ok = slabs <= kMaxSplitK;
+  return p;
+}
+
 int choose_splits(int tiles, int kblocks, int sms) {
   int best = 1;
   long long best_t = -1;
@@ -474,8 +505,23 @@ int swapped_partial_gemm(const void* w, int rows_w, const void* w_second, int ro
   if (w_second) L3_TRY(make_map(&ma2, w_second, rows_w2, k, 128)); else ma2 = ma;
   L3_TRY(make_map(&mb, x, rows_x, k, bn));
   const int tiles = ((rows_w + 127) / 128 + (rows_w2 + 127) / 128) * ((rows_x + bn - 1) / bn);
-  const int splits = choose_splits(tiles, (k + 63) / 64, num_sms());
+  const int kblocks = (k + 63) / 64;
+  const int splits = choose_splits(tiles, kblocks, num_sms());
   GemmShape sh = make_shape(rows_w, w_second ? rows_w2 : 0, rows_x, k, bn, splits);
+  // Stream-K over (m-tile, k-block) when it beats the best even split: every
+  // CTA streams an equal share of the weights, and a tile shared by several
+  // CTAs gets one partial slab per CTA (the tile's last CTA zeroes the slabs
+  // its tile does not use, so the reductions still sum `splits` slabs).
+  if (sh.tiles_n == 1) {
+    const StreamK sk = plan_stream_k(sh.tiles_m, kblocks, num_sms());
+    const long long t_split = (((long long)sh.units + num_sms() - 1) / num_sms()) *
+                              (sh.kb_per_split + L3_SPLIT_UNIT_COST);
+    if (sk.ok && sk.cost < t_split) {
+      sh.sk_per = sk.per;
+      sh.units = sk.ctas;
+      sh.splits = sk.slabs;
+    }
+  }
   EpiParams ep = empty_epi();
   ep.out = P;
   ep.ldo = ldo;

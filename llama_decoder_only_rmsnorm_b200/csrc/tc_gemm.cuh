@@ -47,8 +47,11 @@ struct GemmShape {
   int kblocks;         // ceil(k / 64)
   int kb_per_split;
   int splits;
-  int units;           // splits * tiles_m * tiles_n
+  int units;           // splits * tiles_m * tiles_n (stream-K: the CTAs of the schedule)
   int group_m;         // raster: m-tiles per group (tiles of a group share A rows and B columns)
+  // Stream-K (one n-tile only): CTA c takes k-blocks [c*sk_per, (c+1)*sk_per)
+  // of the (m-tile, k-block) space in m-major order; 0 = split-K units.
+  int sk_per;
 };
 
 // Work unit -> (split, m-tile, n-tile).  Within a split, tiles are visited in
@@ -66,6 +69,42 @@ __device__ __forceinline__ void gemm_unit(const GemmShape& sh, int u, int& split
   const int q = r % per_group;
   mt = first_m + q % gm;
   nt = q / gm;
+}
+
+// One unit of a CTA's work: an output tile and a k-block range of it.  slab:
+// the partial-sum slab it writes (EPI_PARTIAL).  zero_from > 0: this CTA is the
+// tile's last contributor and also zeroes slabs [zero_from, splits).
+struct GemmUnit {
+  int mt, nt, kb0, kb1, slab, zero_from;
+};
+
+// Unit `it` of CTA `c` (of `ctas`); false once the CTA has no more.
+__device__ __forceinline__ bool cta_unit(const GemmShape& sh, int c, int ctas, int it, GemmUnit& g) {
+  if (sh.sk_per == 0) {
+    const int u = c + it * ctas;
+    if (u >= sh.units) return false;
+    int split;
+    gemm_unit(sh, u, split, g.mt, g.nt);
+    g.kb0 = split * sh.kb_per_split;
+    g.kb1 = min(g.kb0 + sh.kb_per_split, sh.kblocks);
+    g.slab = split;
+    g.zero_from = 0;
+    return true;
+  }
+  const int total = sh.tiles_m * sh.kblocks;
+  const int start = c * sh.sk_per, end = min(start + sh.sk_per, total);
+  const int tile = start / sh.kblocks + it;
+  const int tstart = tile * sh.kblocks;
+  if (tstart >= end) return false;
+  g.mt = tile;
+  g.nt = 0;
+  g.kb0 = max(start - tstart, 0);
+  g.kb1 = min(end - tstart, sh.kblocks);
+  const int first = tstart / sh.sk_per;                     // CTAs that share the tile, in k order
+  const int last = (tstart + sh.kblocks - 1) / sh.sk_per;
+  g.slab = c - first;
+  g.zero_from = c == last ? last - first + 1 : 0;
+  return true;
 }
 
 struct EpiParams {
@@ -133,7 +172,7 @@ template <int EPI, int CW>
 __device__ __forceinline__ void epilogue_chunk(const EpiParams& ep, const GemmShape& sh,
                                                const float (&acc)[32], const float (&acc3)[32],
                                                int arow, bool arow_ok, int out_row, int bcol0,
-                                               int split, int lane) {
+                                               int split, int lane, int zero_from = 0) {
   if constexpr (EPI == EPI_STORE || EPI == EPI_RESIDUAL || EPI == EPI_SWIGLU) {
     if (!arow_ok) return;
     bf16* out = reinterpret_cast<bf16*>(ep.out) + (size_t)arow * ep.ldo + bcol0;
@@ -222,6 +261,15 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams& ep, const GemmSh
 #pragma unroll
     for (int j = 0; j < CW; ++j)
       if (bcol0 + j < sh.rows_b) P[(size_t)(bcol0 + j) * ep.ldo] = acc[j];
+    // stream-K: the tile's last contributor zeroes the slabs no CTA writes
+    if (zero_from > 0) {
+      for (int z = zero_from; z < sh.splits; ++z) {
+        float* Z = reinterpret_cast<float*>(ep.out) + (size_t)z * ep.split_stride + out_row;
+#pragma unroll
+        for (int j = 0; j < CW; ++j)
+          if (bcol0 + j < sh.rows_b) Z[(size_t)(bcol0 + j) * ep.ldo] = 0.f;
+      }
+    }
   } else if constexpr (EPI == EPI_ARGMAX) {
     // Swapped: A rows are vocabulary entries, B rows are hidden rows.
     float v[32];
@@ -297,13 +345,13 @@ __global__ void __launch_bounds__(192, 1)
       bool ok = true;
       int pre = 0;   // k-blocks of the first unit whose A tile went out before the dependency wait
       if constexpr (kEarlyA) {
-        if ((int)blockIdx.x < sh.units) {
-          int split, mt, nt;
-          gemm_unit(sh, blockIdx.x, split, mt, nt);
+        GemmUnit g0;
+        if (cta_unit(sh, blockIdx.x, gridDim.x, 0, g0)) {
+          const int mt = g0.mt, nt = g0.nt;
           const bool second = mt >= sh.tiles_m1;
           const int arow = (second ? mt - sh.tiles_m1 : mt) * C::BM;
-          const int kb0 = split * sh.kb_per_split;
-          pre = min(STAGES, min(kb0 + sh.kb_per_split, sh.kblocks) - kb0);
+          const int kb0 = g0.kb0;
+          pre = min(STAGES, g0.kb1 - kb0);
           for (int i = 0; i < pre; ++i) {   // fresh ring: these stages are free
             mbar_arrive_expect_tx(&full[i], C::STAGE_BYTES);
             tma_load_2d(sA + i * C::A_BYTES, second ? &mapA2 : &mapA, &full[i], (kb0 + i) * C::BK, arow);
@@ -321,14 +369,14 @@ __global__ void __launch_bounds__(192, 1)
           griddep_wait_and_release();
         }
       }
-      for (int u = blockIdx.x; u < sh.units && ok; u += gridDim.x) {
-        int split, mt, nt;
-        gemm_unit(sh, u, split, mt, nt);
+      GemmUnit g;
+      for (int it = 0; ok && cta_unit(sh, blockIdx.x, gridDim.x, it, g); ++it) {
+        const int mt = g.mt, nt = g.nt;
         const bool second = mt >= sh.tiles_m1;
         const CUtensorMap* ma = second ? &mapA2 : &mapA;
         const int arow = (second ? mt - sh.tiles_m1 : mt) * C::BM;
-        const int kb0 = split * sh.kb_per_split + (u == (int)blockIdx.x ? pre : 0);
-        const int kb1 = min(split * sh.kb_per_split + sh.kb_per_split, sh.kblocks);
+        const int kb0 = g.kb0 + (it == 0 ? pre : 0);
+        const int kb1 = g.kb1;
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, wait_ns)) { ok = false; break; }
           mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
@@ -353,11 +401,9 @@ __global__ void __launch_bounds__(192, 1)
       int last_buf = -1;
       uint32_t last_parity = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < sh.units && ok; u += gridDim.x) {
-        int split, mt_unused, nt_unused;
-        gemm_unit(sh, u, split, mt_unused, nt_unused);
-        const int kb0 = split * sh.kb_per_split;
-        const int kb1 = min(kb0 + sh.kb_per_split, sh.kblocks);
+      GemmUnit g;
+      for (int it = 0; ok && cta_unit(sh, blockIdx.x, gridDim.x, it, g); ++it) {
+        const int kb0 = g.kb0, kb1 = g.kb1;
         if (!mbar_wait(&acc_empty[abuf], aphase ^ 1u, wait_ns)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + abuf * C::ACC_COLS;
@@ -394,9 +440,9 @@ __global__ void __launch_bounds__(192, 1)
     const int row_in_tile = quarter * 32 + lane;
     int abuf = 0;
     uint32_t aphase = 0;
-    for (int u = blockIdx.x; u < sh.units; u += gridDim.x) {
-      int split, mt, nt;
-      gemm_unit(sh, u, split, mt, nt);
+    GemmUnit g;
+    for (int it = 0; cta_unit(sh, blockIdx.x, gridDim.x, it, g); ++it) {
+      const int mt = g.mt, nt = g.nt, split = g.slab;
       const bool second = mt >= sh.tiles_m1;
       const int local_row = (second ? mt - sh.tiles_m1 : mt) * C::BM + row_in_tile;
       const bool arow_ok = local_row < (second ? sh.rows_a2 : sh.rows_a);
@@ -431,7 +477,7 @@ __global__ void __launch_bounds__(192, 1)
           }
         }
         epilogue_chunk<EPI, C::CW>(ep, sh, acc, acc3, local_row, arow_ok, out_row,
-                                   nt * BN + c * C::CW, split, lane);
+                                   nt * BN + c * C::CW, split, lane, g.zero_from);
       }
       tc_fence_before();
       __syncwarp();
