@@ -215,6 +215,28 @@ def test_decode_step_matches_prefill_path_for_large_batch():
     assert_close(torch.cat([a.cpu(), d.cpu()], 1), want, "bf16", "batch-300 decode")
 
 
+def test_decode_stream_k_gemm_with_garbage_workspace():
+    """dim 512, FFN 5632, 32 sequences: the w1|w3 decode GEMM takes the
+    stream-K schedule (3 partial slabs, some tiles written by fewer CTAs, whose
+    unused slabs the tile's last CTA zeroes).  The workspace starts as NaN, so a
+    slab left unwritten poisons the block output."""
+    w = small_bf16(batch=32, n_layers=1, dim=512, n_heads=8, n_kv_heads=2, ffn_hidden=5632)
+    layers = [I.layer_weights(w, 0, DEV, "random")]
+    st = Llama3Stack(w.cfg(), layers, I.output_weights(w, DEV), w.batch, 48, 40)
+    st.ws.view(torch.float32).fill_(float("nan"))
+    g = torch.Generator(device="cpu").manual_seed(17)
+    xs = torch.randn((w.batch, 42, w.dim), generator=g).to(torch.bfloat16)
+    a = xs[:, :40].contiguous().to(DEV)
+    st.forward_layers(a, 40, 0)
+    outs = [a]
+    for t in (40, 41):
+        d = xs[:, t:t + 1].contiguous().to(DEV)
+        st.decode_layers(d, t)
+        outs.append(d)
+    want, _, _ = O.forward_stack(f64(xs), [oracle_layer(l) for l in layers], oracle_cfg(w))
+    assert_close(torch.cat([o.cpu() for o in outs], 1), want, "bf16", "stream-K decode")
+
+
 # -------------------------------------------------------------- LM head
 @pytest.mark.parametrize("rows", [1, 5, 32, 300])
 def test_lm_head_8b_vocab(rows):
