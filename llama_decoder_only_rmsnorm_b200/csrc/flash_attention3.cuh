@@ -11,7 +11,12 @@
 //  * P (bf16, two per 32-bit column) is written back into TMEM over the
 //    scores just read (keys 0-127 -> columns 0-63) and P.V takes its A operand
 //    from TMEM, so P never goes through shared memory;
-//  * K and V are both double-buffered in the shared memory P no longer uses.
+//  * K and V are both double-buffered in the shared memory P no longer uses;
+//  * a whole warp runs the MMA loop (warp-uniform addresses and descriptors)
+//    and one elected lane issues; a head's next S goes right behind the P.V
+//    that reads its columns, since the MMAs of one thread run in issue order;
+//  * the softmax never waits for a P.V before its exponentials: the S commit
+//    it waits for covers every MMA issued before that S, the P.V included.
 // The split of registers is only valid for a launch of 384 threads at 168
 // registers each (128*104 + 256*200 = 384*168); the host checks the compiled
 // register count before every launch.
