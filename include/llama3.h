@@ -195,6 +195,32 @@ int llama3_layer_decode_ragged(const llama3_config* cfg, const llama3_layer_weig
                                llama3_stream_t stream);
 
 /*
+ * One decode step of one block, as llama3_layer_decode (positions == NULL:
+ * every sequence at start_pos) or llama3_layer_decode_ragged (positions !=
+ * NULL, start_pos then being max_position), for a loop over the blocks that
+ * hands the normalised input from one block to the next instead of
+ * normalising it again ([S2] 三 TransformerBlock: the next block's first step
+ * is RMSNorm of this block's output).
+ *   next_attention_norm (nullable, bf16 [D], 16-byte aligned): the next
+ *     block's attention-norm weight; the block's last residual step then also
+ *     leaves RMSNorm(x_out, next_attention_norm) in the workspace.
+ *   input_normalised: nonzero when the previous call on this workspace, for
+ *     the same batch, was given this block's attention_norm as its
+ *     next_attention_norm; the block then skips its first RMSNorm.
+ * Only the tcgen05 decode path (bf16, batch <= 256 or ragged) hands the
+ * normalised input on; the other paths ignore both arguments and normalise x
+ * themselves, so the result is the same either way.  Errors as
+ * llama3_layer_decode / llama3_layer_decode_ragged, plus LLAMA3_ERR_ALIGN for
+ * a misaligned next_attention_norm.
+ */
+int llama3_layer_decode_chained(const llama3_config* cfg, const llama3_layer_weights* w,
+                                const float* rope, int rope_len, void* x, void* k_cache,
+                                void* v_cache, int cache_cap, int batch, int start_pos,
+                                const int32_t* positions, const void* next_attention_norm,
+                                int input_normalised, void* ws, size_t ws_bytes,
+                                llama3_stream_t stream);
+
+/*
  * Output block ([S1] §11-12, [S3] 预测流程): for each of `rows` hidden rows
  * h[r] = h + r*row_stride (elements), compute logits = RMSNorm(h[r], norm_w)
  * W_out^T over the vocabulary and ids_out[r] = argmax (lowest index on ties).

@@ -52,6 +52,7 @@ _SIGNATURES = {
     "llama3_layer_forward": [_cfgp, _wp, _p, _i, _p, _p, _p, _i, _i, _i, _i, _p, _sz, _p],
     "llama3_layer_decode": [_cfgp, _wp, _p, _i, _p, _p, _p, _i, _i, _i, _p, _sz, _p],
     "llama3_layer_decode_ragged": [_cfgp, _wp, _p, _i, _p, _p, _p, _i, _i, _p, _i, _p, _sz, _p],
+    "llama3_layer_decode_chained": [_cfgp, _wp, _p, _i, _p, _p, _p, _i, _i, _i, _p, _p, _i, _p, _sz, _p],
     "llama3_layer_forward_docs": [_cfgp, _wp, _p, _i, _p, _p, _p, _i, _i, _i, _i, _p, _p, _sz, _p],
     "llama3_attention_docs": [_cfgp, _p, _p, _p, _i, _i, _i, _i, _p, _p, _p, _sz, _p],
     "llama3_lm_head_argmax": [_cfgp, _p, _p, _p, _i, _ll, _p, _p, _p, _sz, _p],
@@ -188,6 +189,16 @@ def llama3_layer_decode_ragged(cfg, w, rope, rope_len, x, k_cache, v_cache, cach
     _check("llama3_layer_decode_ragged", lib().llama3_layer_decode_ragged(
         ctypes.byref(cfg), ctypes.byref(w), _ptr(rope), rope_len, _ptr(x), _ptr(k_cache), _ptr(v_cache),
         cache_cap, batch, _ptr(positions), max_position, _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def llama3_layer_decode_chained(cfg, w, rope, rope_len, x, k_cache, v_cache, cache_cap, batch, start_pos, positions,
+                                next_attention_norm, input_normalised, ws, ws_bytes, stream=None):
+    """One decode step of one block that can take its normalised input from the
+    previous block's call and leave the next block's in the workspace."""
+    _check("llama3_layer_decode_chained", lib().llama3_layer_decode_chained(
+        ctypes.byref(cfg), ctypes.byref(w), _ptr(rope), rope_len, _ptr(x), _ptr(k_cache), _ptr(v_cache),
+        cache_cap, batch, start_pos, _ptr(positions), _ptr(next_attention_norm), 1 if input_normalised else 0,
+        _ptr(ws), ws_bytes, _stream(stream)))
 
 
 def llama3_lm_head_argmax(cfg, norm_w, w_out, h, rows, row_stride, ids_out, logits_out, ws, ws_bytes,

@@ -816,9 +816,13 @@ int layer_tc_prefill(const llama3_config* c, const llama3_layer_weights* w, cons
 // Layer: tcgen05 decode path (bf16, few tokens): weight-streaming split-K
 // GEMMs + SIMT epilogues over the fp32 partials.
 // ---------------------------------------------------------------------------
+// next_norm: also leave RMSNorm(x_out, next_norm) in the workspace's normalised-
+// input buffer for the next block; input_normalised: that buffer already holds
+// this block's RMSNorm(x, attention_norm) (left by the previous block).
 int layer_tc_decode(const llama3_config* c, const llama3_layer_weights* w, const float* rope, void* x, void* kc,
                     void* vc, int cap, int B, int P, const Workspace& L, void* ws, cudaStream_t st,
-                    const int32_t* positions = nullptr) {
+                    const int32_t* positions = nullptr, const void* next_norm = nullptr,
+                    bool input_normalised = false) {
   const int M = B, D = c->dim, H = c->n_heads, KV = c->n_kv_heads, hd = c->head_dim, F = c->ffn_hidden;
   const int nqkv = (H + 2 * KV) * hd;
   bf16* xn = ws_at<bf16>(ws, L.xn);
@@ -828,39 +832,45 @@ int layer_tc_decode(const llama3_config* c, const llama3_layer_weights* w, const
   float* Pp = ws_at<float>(ws, L.part);
   float* Ap = ws_at<float>(ws, L.attn_part);
   int splits = 1;
-  L3_TRY(rmsnorm_any(c, x, D, w->attention_norm, xn, M, st));
+  if (!input_normalised) L3_TRY(rmsnorm_any(c, x, D, w->attention_norm, xn, M, st));
   L3_TRY(swapped_partial_gemm(w->wqkv, nqkv, nullptr, 0, 0, xn, M, D, Pp, nqkv, &splits, st));
   L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_qkv_rope_kernel<bf16>), blocks_for((long long)M * nqkv / 4, 256), 256, 0, st,
       Pp, splits, (long long)M * nqkv, M, 1, P, H, KV, hd, rope, q, (bf16*)kc, (bf16*)vc, cap, positions, P));
   L3_TRY(launch_check());
   L3_TRY(attention_dispatch(c, q, kc, vc, cap, B, 1, P, o, Ap, st, nullptr, positions));
-  L3_TRY(swapped_partial_gemm(w->wo, D, nullptr, 0, 0, o, M, H * hd, Pp, D, &splits, st));
-  // h = x + o Wo^T and hn = RMSNorm(h) in one pass over each row
-  if (D <= 4 * 4 * 1024) {
-    const int G = (D + 4095) / 4096;
-    const long long sstride = (long long)M * D;
-    if (G <= 1)
-      L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_residual_rmsnorm_kernel<1>), M, 1024, 0, st, Pp, splits,
-                                                        sstride, (bf16*)x, (const bf16*)w->ffn_norm, xn, D, c->norm_eps));
-    else if (G <= 2)
-      L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_residual_rmsnorm_kernel<2>), M, 1024, 0, st, Pp, splits,
-                                                        sstride, (bf16*)x, (const bf16*)w->ffn_norm, xn, D, c->norm_eps));
-    else
-      L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_residual_rmsnorm_kernel<4>), M, 1024, 0, st, Pp, splits,
-                                                        sstride, (bf16*)x, (const bf16*)w->ffn_norm, xn, D, c->norm_eps));
-    L3_TRY(launch_check());
-  } else {
+  // x += the split sums (row-wise), then xn = RMSNorm(x, norm_w), in one pass
+  // over each row where the row fits one CTA
+  auto residual_then_norm = [&](const void* norm_w) -> int {
+    if (D <= 4 * 4 * 1024) {
+      const int G = (D + 4095) / 4096;
+      const long long sstride = (long long)M * D;
+      if (G <= 1)
+        L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_residual_rmsnorm_kernel<1>), M, 1024, 0, st, Pp, splits,
+                                                          sstride, (bf16*)x, (const bf16*)norm_w, xn, D, c->norm_eps));
+      else if (G <= 2)
+        L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_residual_rmsnorm_kernel<2>), M, 1024, 0, st, Pp, splits,
+                                                          sstride, (bf16*)x, (const bf16*)norm_w, xn, D, c->norm_eps));
+      else
+        L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_residual_rmsnorm_kernel<4>), M, 1024, 0, st, Pp, splits,
+                                                          sstride, (bf16*)x, (const bf16*)norm_w, xn, D, c->norm_eps));
+      return launch_check();
+    }
     L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_residual_kernel<bf16>), blocks_for((long long)M * D / 4, 256),
                                                       256, 0, st, Pp, splits, (long long)M * D, D, (const bf16*)x,
                                                       (bf16*)x, M, D));
     L3_TRY(launch_check());
-    L3_TRY(rmsnorm_any(c, x, D, w->ffn_norm, xn, M, st));
-  }
+    return rmsnorm_any(c, x, D, norm_w, xn, M, st);
+  };
+  L3_TRY(swapped_partial_gemm(w->wo, D, nullptr, 0, 0, o, M, H * hd, Pp, D, &splits, st));
+  // h = x + o Wo^T and hn = RMSNorm(h)
+  L3_TRY(residual_then_norm(w->ffn_norm));
   L3_TRY(swapped_partial_gemm(w->w1, F, w->w3, F, F, xn, M, D, Pp, 2 * F, &splits, st));
   L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_swiglu_kernel<bf16>), blocks_for((long long)M * F / 4, 256), 256, 0, st, Pp, splits, (long long)M * 2 * F, g,
                                                                                 M, F));
   L3_TRY(launch_check());
   L3_TRY(swapped_partial_gemm(w->w2, D, nullptr, 0, 0, g, M, F, Pp, D, &splits, st));
+  // out = h + g W2^T, and with next_norm the next block's normalised input
+  if (next_norm) return residual_then_norm(next_norm);
   L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((epi_residual_kernel<bf16>), blocks_for((long long)M * D / 4, 256), 256, 0, st,
       Pp, splits, (long long)M * D, D, (const bf16*)x, (bf16*)x, M, D));
   return launch_check();
@@ -1168,6 +1178,28 @@ int llama3_layer_decode_ragged(const llama3_config* cfg, const llama3_layer_weig
                              nullptr, positions);
   return layer_simt<bf16>(cfg, w, rope, x, k_cache, v_cache, cache_cap, batch, 1, max_position, L, ws, st,
                           nullptr, positions);
+}
+
+int llama3_layer_decode_chained(const llama3_config* cfg, const llama3_layer_weights* w, const float* rope,
+                                int rope_len, void* x, void* k_cache, void* v_cache, int cache_cap, int batch,
+                                int start_pos, const int32_t* positions, const void* next_attention_norm,
+                                int input_normalised, void* ws, size_t ws_bytes, llama3_stream_t stream) {
+  if (positions && (reinterpret_cast<uintptr_t>(positions) & 3)) return LLAMA3_ERR_ALIGN;
+  if (next_attention_norm && !aligned16(next_attention_norm)) return LLAMA3_ERR_ALIGN;
+  Workspace L;
+  L3_TRY(check_layer_args(cfg, w, rope, rope_len, x, k_cache, v_cache, cache_cap, batch, 1, start_pos, ws,
+                          ws_bytes, &L));
+  cudaStream_t st = (cudaStream_t)stream;
+  // Only the tcgen05 decode path hands the normalised input from block to
+  // block; every other path ignores both flags and normalises x itself.
+  if (use_tc(cfg) && (positions || batch <= 256))
+    return layer_tc_decode(cfg, w, rope, x, k_cache, v_cache, cache_cap, batch, start_pos, L, ws, st, positions,
+                           next_attention_norm, input_normalised != 0);
+  if (positions)
+    return llama3_layer_decode_ragged(cfg, w, rope, rope_len, x, k_cache, v_cache, cache_cap, batch, positions,
+                                      start_pos, ws, ws_bytes, stream);
+  return llama3_layer_decode(cfg, w, rope, rope_len, x, k_cache, v_cache, cache_cap, batch, start_pos, ws, ws_bytes,
+                             stream);
 }
 
 int llama3_layer_forward_docs(const llama3_config* cfg, const llama3_layer_weights* w, const float* rope,

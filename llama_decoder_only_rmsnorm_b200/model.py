@@ -49,20 +49,27 @@ class Llama3Stack:
             B.llama3_layer_forward(self.cfg, self.wstructs[i], self.rope, self.rope_len, x, kc, vc,
                                    self.cache_cap, self.batch, seq, start_pos, self.ws, self.ws_bytes, stream)
 
-    def decode_layers(self, x, start_pos, stream=None, layers=None):
-        for i in (range(len(self.layers)) if layers is None else layers):
+    def _decode_chain(self, x, start_pos, positions, stream, layers):
+        # Each block leaves the next block's normalised input in the workspace
+        # (llama3_layer_decode_chained); a block is told so only when the call
+        # before it, on the same workspace, was the block right before it.
+        idx = list(range(len(self.layers)) if layers is None else layers)
+        for n, i in enumerate(idx):
             kc, vc = self.caches[i]
-            B.llama3_layer_decode(self.cfg, self.wstructs[i], self.rope, self.rope_len, x, kc, vc,
-                                  self.cache_cap, self.batch, start_pos, self.ws, self.ws_bytes, stream)
+            nxt = idx[n + 1] if n + 1 < len(idx) else None
+            next_norm = self.layers[nxt]["attention_norm"] if nxt is not None and nxt == i + 1 else None
+            chained_in = n > 0 and idx[n - 1] == i - 1
+            B.llama3_layer_decode_chained(self.cfg, self.wstructs[i], self.rope, self.rope_len, x, kc, vc,
+                                          self.cache_cap, self.batch, start_pos, positions, next_norm, chained_in,
+                                          self.ws, self.ws_bytes, stream)
+
+    def decode_layers(self, x, start_pos, stream=None, layers=None):
+        self._decode_chain(x, start_pos, None, stream, layers)
 
     def decode_layers_ragged(self, x, positions, max_position, stream=None, layers=None):
         """One decode step where sequence b's token sits at positions[b]
         (int32 device tensor); max_position bounds them all."""
-        for i in (range(len(self.layers)) if layers is None else layers):
-            kc, vc = self.caches[i]
-            B.llama3_layer_decode_ragged(self.cfg, self.wstructs[i], self.rope, self.rope_len, x, kc, vc,
-                                         self.cache_cap, self.batch, positions, max_position, self.ws,
-                                         self.ws_bytes, stream)
+        self._decode_chain(x, max_position, positions, stream, layers)
 
     def lm_head(self, h, rows, row_stride, logits=None, stream=None):
         B.llama3_lm_head_argmax(self.cfg, self.out["norm"], self.out["output"], h, rows, row_stride,

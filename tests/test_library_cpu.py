@@ -80,6 +80,12 @@ def test_layer_calls_reject_bad_arguments_before_launch():
     dec = lib.llama3_layer_decode(ctypes.byref(c), ctypes.byref(w), FAKE, 64, FAKE, FAKE, FAKE, 64, 2, 64,
                                   FAKE, ws_bytes, None)
     assert dec == 1                       # position 64 does not fit a 64-entry cache
+    chained = lambda **k: lib.llama3_layer_decode_chained(
+        ctypes.byref(c), ctypes.byref(w), FAKE, 64, FAKE, FAKE, FAKE, 64, 2, k.get("start", 10),
+        k.get("positions", None), k.get("next_norm", None), 1, FAKE, ws_bytes, None)
+    assert chained(start=64) == 1         # max position 64 does not fit a 64-entry cache
+    assert chained(next_norm=FAKE + 2) == 2
+    assert chained(positions=FAKE + 2) == 2
 
 
 def test_lm_head_and_helpers_reject_bad_arguments():
