@@ -350,7 +350,7 @@ enum llama3_kernel_kind {
   LLAMA3_KERNEL_GEMM_W13 = 3,          /* prefill w1|w3 GEMM + SwiGLU              */
   LLAMA3_KERNEL_GEMM_W2 = 4,           /* prefill w2 GEMM + residual               */
   LLAMA3_KERNEL_ATTENTION = 5,         /* prefill causal GQA attention             */
-  LLAMA3_KERNEL_DECODE_GEMM = 6,       /* weight-streaming split-K GEMMs (decode)  */
+  LLAMA3_KERNEL_DECODE_GEMM = 6,       /* weight-streaming GEMMs (decode)          */
   LLAMA3_KERNEL_DECODE_ATTENTION = 7,  /* split-KV decode attention (main kernel)  */
   LLAMA3_KERNEL_LM_HEAD = 8,           /* LM-head GEMM + argmax                    */
   LLAMA3_KERNEL_NORM = 9,              /* RMSNorm                                  */
