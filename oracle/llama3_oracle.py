@@ -27,6 +27,18 @@ Readings taken where the pages are silent or disagree:
   * RMSNorm is not rounded between normalising and weighting.
   * argmax breaks ties toward the lowest vocabulary index.
 
+Precision variant (``rounding="bf16"``): the pages' own bf16 model holds
+every activation passed between steps as a bf16 tensor (the RMSNorm output
+cast back to the input type, [S2] §3.1; q, k, v and the attention
+probabilities cast to the activation type, [S2] §3.4 and [S1] §7; the block
+output and the residual stream in the model dtype).  With that option the
+oracle rounds to bf16 (8 significant bits, ties to even) at exactly those
+step boundaries -- normalised rows, rotated q/k and v, probabilities before
+the P.V product, attention output, residual stream after each residual add,
+SwiGLU product -- and keeps every sum, the softmax statistics and the RoPE
+angles exact.  It measures how far bf16 storage alone takes a result from the
+exact answer, which is what the full-size tests calibrate their bound with.
+
 Parity status: every function below is pinned by ``tests/test_oracle_pins.py``
 except ``forward_stack`` on real checkpoints (parity unpinned for real Meta
 weights: the checkpoint and tokenizer are not available, so the worked
@@ -37,7 +49,7 @@ from __future__ import annotations
 import numpy as np
 
 __all__ = [
-    "rms_norm", "ffn_hidden_dim", "rope_inverse_frequencies", "rope_angles",
+    "bf16_round", "rms_norm", "ffn_hidden_dim", "rope_inverse_frequencies", "rope_angles",
     "apply_rope", "causal_mask", "gqa_attention", "silu", "swiglu_ffn",
     "decoder_block", "decoder_block_rows", "lm_head", "embed", "forward_stack",
     "generate_greedy", "philox4x64", "sampling_word", "top_p_sample",
@@ -46,6 +58,29 @@ __all__ = [
 
 def _f64(a):
     return np.asarray(a, dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------
+# bf16 storage (the precision variant; see the module docstring)
+# ---------------------------------------------------------------------------
+def bf16_round(x):
+    """Round to the nearest bfloat16 value (8 significant bits, ties to even),
+    returned as float64.  Written out from the format: x = m * 2^e with
+    m in [0.5, 1); keep m to 8 bits by rounding m * 2^8 to the nearest
+    integer, ties to even.  (Values below 2^-126, where bf16 turns
+    subnormal, never occur here and are not treated specially.)"""
+    x = _f64(x)
+    m, e = np.frexp(x)
+    return np.ldexp(np.rint(m * 256.0), e - 8)
+
+
+def _store(x, rounding):
+    """An activation as the path stores it between steps."""
+    if rounding is None:
+        return x
+    if rounding == "bf16":
+        return bf16_round(x)
+    raise ValueError(f"unknown rounding {rounding!r}")
 
 
 # ---------------------------------------------------------------------------
@@ -124,12 +159,14 @@ def causal_mask(n_queries, n_keys, start_pos=0, doc_start=None):
     return np.where(ok, 0.0, -np.inf)
 
 
-def gqa_attention(q, k, v, start_pos=0, return_probs=False, doc_start=None):
+def gqa_attention(q, k, v, start_pos=0, return_probs=False, doc_start=None, rounding=None):
     """softmax(q k^T / sqrt(hd) + mask) v for one sequence.
 
     q: [S, H, hd] (rotated); k, v: [T, KV, hd] with T = start_pos + S.
     Query head h reads KV head h // (H // KV).  Returns [S, H, hd]
     (and the [H, S, T] probabilities when ``return_probs``).
+    rounding="bf16": the probabilities are stored in bf16 before the
+    product with v (the softmax sum itself stays exact).
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
     S, H, hd = q.shape
@@ -143,9 +180,13 @@ def gqa_attention(q, k, v, start_pos=0, return_probs=False, doc_start=None):
         g = h // n_rep
         scores = q[:, h, :] @ k[:, g, :].T / np.sqrt(hd) + mask
         scores = scores - scores.max(axis=1, keepdims=True)
-        p = np.exp(scores)
-        p = p / p.sum(axis=1, keepdims=True)
-        out[:, h, :] = p @ v[:, g, :]
+        e = np.exp(scores)
+        total = e.sum(axis=1, keepdims=True)
+        p = e / total
+        if rounding is None:
+            out[:, h, :] = p @ v[:, g, :]
+        else:
+            out[:, h, :] = (_store(e, rounding) @ v[:, g, :]) / total
         if return_probs:
             probs[h] = p
     return (out, probs) if return_probs else out
@@ -168,7 +209,7 @@ def swiglu_ffn(x, w1, w2, w3):
 # ---------------------------------------------------------------------------
 # One pre-norm decoder block  ([S2] §3.6 TransformerBlock; [S1] §6-10)
 # ---------------------------------------------------------------------------
-def decoder_block(x, layer, cfg, k_cache, v_cache, start_pos=0, doc_start=None):
+def decoder_block(x, layer, cfg, k_cache, v_cache, start_pos=0, doc_start=None, rounding=None):
     """h = x + Attn(RMSNorm(x)); out = h + FFN(RMSNorm(h)).
 
     x: [B, S, D].  ``layer`` maps the page's weight names (attention_norm, wq,
@@ -177,7 +218,8 @@ def decoder_block(x, layer, cfg, k_cache, v_cache, start_pos=0, doc_start=None):
     [start_pos, start_pos+S) are overwritten with this call's rotated k and v
     ([S2] §3.3 / §3.4 inference branch).  ``doc_start`` [B, S] (optional):
     the position where each token's document begins (document mask).
-    Returns out [B, S, D].
+    ``rounding``: None (exact) or "bf16" (activations stored in bf16 between
+    steps; module docstring).  Returns out [B, S, D].
     """
     x = _f64(x)
     B, S, D = x.shape
@@ -185,25 +227,36 @@ def decoder_block(x, layer, cfg, k_cache, v_cache, start_pos=0, doc_start=None):
     eps, theta = cfg["norm_eps"], cfg["rope_theta"]
     pos = start_pos + np.arange(S)
 
-    xn = rms_norm(x, layer["attention_norm"], eps)
+    r = lambda a: _store(a, rounding)
+    xn = r(rms_norm(x, layer["attention_norm"], eps))
     q = (xn @ _f64(layer["wq"]).T).reshape(B, S, H, hd)
     k = (xn @ _f64(layer["wk"]).T).reshape(B, S, KV, hd)
-    v = (xn @ _f64(layer["wv"]).T).reshape(B, S, KV, hd)
-    q = apply_rope(q, pos, theta)
-    k = apply_rope(k, pos, theta)
+    v = r((xn @ _f64(layer["wv"]).T).reshape(B, S, KV, hd))
+    q = r(apply_rope(q, pos, theta))
+    k = r(apply_rope(k, pos, theta))
     k_cache[:B, start_pos:start_pos + S] = k
     v_cache[:B, start_pos:start_pos + S] = v
 
     o = np.empty((B, S, H, hd))
     for b in range(B):
         o[b] = gqa_attention(q[b], k_cache[b, :start_pos + S], v_cache[b, :start_pos + S], start_pos,
-                             doc_start=None if doc_start is None else np.asarray(doc_start)[b])
-    h = x + o.reshape(B, S, H * hd) @ _f64(layer["wo"]).T
-    hn = rms_norm(h, layer["ffn_norm"], eps)
-    return h + swiglu_ffn(hn, layer["w1"], layer["w2"], layer["w3"])
+                             doc_start=None if doc_start is None else np.asarray(doc_start)[b],
+                             rounding=rounding)
+    h = r(x + r(o.reshape(B, S, H * hd)) @ _f64(layer["wo"]).T)
+    hn = r(rms_norm(h, layer["ffn_norm"], eps))
+    return r(h + _swiglu_rounded(hn, layer, rounding))
 
 
-def decoder_block_rows(x, layer, cfg, rows, k_prefix=None, v_prefix=None, start_pos=0):
+def _swiglu_rounded(hn, layer, rounding):
+    """swiglu_ffn with the SwiGLU product stored as the path stores it."""
+    if rounding is None:
+        return swiglu_ffn(hn, layer["w1"], layer["w2"], layer["w3"])
+    hn = _f64(hn)
+    g = _store(silu(hn @ _f64(layer["w1"]).T) * (hn @ _f64(layer["w3"]).T), rounding)
+    return g @ _f64(layer["w2"]).T
+
+
+def decoder_block_rows(x, layer, cfg, rows, k_prefix=None, v_prefix=None, start_pos=0, rounding=None):
     """Selected output rows of ``decoder_block`` for ONE sequence.
 
     x: [S, D] (tokens at positions start_pos..start_pos+S-1); k_prefix /
@@ -212,43 +265,46 @@ def decoder_block_rows(x, layer, cfg, rows, k_prefix=None, v_prefix=None, start_
     attends to all earlier ones); queries, attention, wo, the FFN and both
     residuals only for the tokens in ``rows``.  Returns (out [len(rows), D],
     k [S, KV, hd], v [S, KV, hd]) with k rotated, i.e. what the cache receives.
+    ``rounding`` as in ``decoder_block``.
     """
     x = _f64(x)
     S, D = x.shape
     H, KV, hd = cfg["n_heads"], cfg["n_kv_heads"], cfg["head_dim"]
     eps, theta = cfg["norm_eps"], cfg["rope_theta"]
     rows = list(rows)
-    xn = rms_norm(x, layer["attention_norm"], eps)
+    r = lambda a: _store(a, rounding)
+    xn = r(rms_norm(x, layer["attention_norm"], eps))
     pos = start_pos + np.arange(S)
-    k = apply_rope((xn @ _f64(layer["wk"]).T).reshape(S, KV, hd), pos, theta)
-    v = (xn @ _f64(layer["wv"]).T).reshape(S, KV, hd)
+    k = r(apply_rope((xn @ _f64(layer["wk"]).T).reshape(S, KV, hd), pos, theta))
+    v = r((xn @ _f64(layer["wv"]).T).reshape(S, KV, hd))
     if start_pos:
         k_all = np.concatenate([_f64(k_prefix), k], 0)
         v_all = np.concatenate([_f64(v_prefix), v], 0)
     else:
         k_all, v_all = k, v
     xr = x[rows]
-    q = apply_rope((xn[rows] @ _f64(layer["wq"]).T).reshape(len(rows), H, hd),
-                   start_pos + np.asarray(rows), theta)
+    q = r(apply_rope((xn[rows] @ _f64(layer["wq"]).T).reshape(len(rows), H, hd),
+                     start_pos + np.asarray(rows), theta))
     o = np.empty((len(rows), H, hd))
     for i, t in enumerate(rows):
         n_keys = start_pos + t + 1
-        o[i] = gqa_attention(q[i:i + 1], k_all[:n_keys], v_all[:n_keys], n_keys - 1)[0]
-    h = xr + o.reshape(len(rows), H * hd) @ _f64(layer["wo"]).T
-    hn = rms_norm(h, layer["ffn_norm"], eps)
-    return h + swiglu_ffn(hn, layer["w1"], layer["w2"], layer["w3"]), k, v
+        o[i] = gqa_attention(q[i:i + 1], k_all[:n_keys], v_all[:n_keys], n_keys - 1, rounding=rounding)[0]
+    h = r(xr + r(o.reshape(len(rows), H * hd)) @ _f64(layer["wo"]).T)
+    hn = r(rms_norm(h, layer["ffn_norm"], eps))
+    return r(h + _swiglu_rounded(hn, layer, rounding)), k, v
 
 
 # ---------------------------------------------------------------------------
 # Output block  ([S1] §11-12; [S2] 四; [S3] 预测流程)
 # ---------------------------------------------------------------------------
-def lm_head(h_rows, norm_weight, w_out, eps):
+def lm_head(h_rows, norm_weight, w_out, eps, rounding=None):
     """RMSNorm the rows, project onto the vocabulary, take argmax.
 
     h_rows: [R, D].  Returns (logits [R, V], ids [R]); ids pick the lowest
-    index among equal maxima.
+    index among equal maxima.  rounding="bf16": the normalised rows are
+    stored in bf16 before the projection.
     """
-    hn = rms_norm(h_rows, norm_weight, eps)
+    hn = _store(rms_norm(h_rows, norm_weight, eps), rounding)
     logits = hn @ _f64(w_out).T
     return logits, np.argmax(logits, axis=-1).astype(np.int64)
 
@@ -259,7 +315,7 @@ def embed(ids, table):
 
 
 def forward_stack(x, layers, cfg, k_caches=None, v_caches=None, start_pos=0,
-                  cache_len=None, doc_start=None):
+                  cache_len=None, doc_start=None, rounding=None):
     """Run x through every block in ``layers`` (the layer loop of [S2] 四).
 
     Creates fp64 caches of length ``cache_len`` (default start_pos+S) when none
@@ -273,7 +329,7 @@ def forward_stack(x, layers, cfg, k_caches=None, v_caches=None, start_pos=0,
         k_caches = [np.zeros((B, cap, KV, hd)) for _ in layers]
         v_caches = [np.zeros((B, cap, KV, hd)) for _ in layers]
     for layer, kc, vc in zip(layers, k_caches, v_caches):
-        x = decoder_block(x, layer, cfg, kc, vc, start_pos, doc_start)
+        x = decoder_block(x, layer, cfg, kc, vc, start_pos, doc_start, rounding)
     return x, k_caches, v_caches
 
 

@@ -237,15 +237,26 @@ def test_block_with_zero_projections_is_identity():
     np.testing.assert_array_equal(O.decoder_block(x, layer, cfg, kc, vc), x)
 
 
-def brute_force_block(x, layer, cfg, start_pos, k_hist, v_hist):
-    """Scalar-loop restatement of one block for a single sequence [S, D]."""
+def bf16_scalar(a):
+    """One value rounded to bfloat16 (8 significant bits, ties to even), in
+    plain Python: Python's round() of a float ties to even."""
+    if a == 0.0:
+        return 0.0
+    m, e = math.frexp(a)
+    return math.ldexp(round(m * 256.0), e - 8)
+
+
+def brute_force_block(x, layer, cfg, start_pos, k_hist, v_hist, store=lambda a: a):
+    """Scalar-loop restatement of one block for a single sequence [S, D].
+    ``store`` is applied to every activation the bf16 variant holds in bf16
+    (identity: the exact block)."""
     S, D = x.shape
     H, KV, hd = cfg["n_heads"], cfg["n_kv_heads"], cfg["head_dim"]
     eps, theta = cfg["norm_eps"], cfg["rope_theta"]
 
     def norm(row, w):
         r = math.sqrt(sum(a * a for a in row) / len(row) + eps)
-        return [a / r * wi for a, wi in zip(row, w)]
+        return [store(a / r * wi) for a, wi in zip(row, w)]
 
     def lin(row, W):
         return [sum(W[o_, i] * row[i] for i in range(len(row))) for o_ in range(W.shape[0])]
@@ -263,10 +274,10 @@ def brute_force_block(x, layer, cfg, start_pos, k_hist, v_hist):
     qs = []
     for t in range(S):
         xn = norm(x[t], layer["attention_norm"])
-        q, k, v = lin(xn, layer["wq"]), lin(xn, layer["wk"]), lin(xn, layer["wv"])
+        q, k, v = lin(xn, layer["wq"]), lin(xn, layer["wk"]), [store(a) for a in lin(xn, layer["wv"])]
         m = start_pos + t
-        q = sum((rot(q[h * hd:(h + 1) * hd], m) for h in range(H)), [])
-        k = sum((rot(k[g * hd:(g + 1) * hd], m) for g in range(KV)), [])
+        q = [store(a) for a in sum((rot(q[h * hd:(h + 1) * hd], m) for h in range(H)), [])]
+        k = [store(a) for a in sum((rot(k[g * hd:(g + 1) * hd], m) for g in range(KV)), [])]
         qs.append(q); ks.append(k); vs.append(v)
     out = np.zeros((S, D))
     for t in range(S):
@@ -276,12 +287,13 @@ def brute_force_block(x, layer, cfg, start_pos, k_hist, v_hist):
             sc = [sum(qs[t][h * hd + d] * ks[j][g * hd + d] for d in range(hd)) / math.sqrt(hd)
                   for j in range(start_pos + t + 1)]
             mx = max(sc); e = [math.exp(s - mx) for s in sc]; z = sum(e)
-            att += [sum(e[j] * vs[j][g * hd + d] for j in range(len(e))) / z for d in range(hd)]
-        hrow = [a + b for a, b in zip(x[t], lin(att, layer["wo"]))]
+            e = [store(a) for a in e]      # probabilities stored; their sum stays exact
+            att += [store(sum(e[j] * vs[j][g * hd + d] for j in range(len(e))) / z) for d in range(hd)]
+        hrow = [store(a + b) for a, b in zip(x[t], lin(att, layer["wo"]))]
         hn = norm(hrow, layer["ffn_norm"])
         g1, g3 = lin(hn, layer["w1"]), lin(hn, layer["w3"])
-        gate = [a / (1 + math.exp(-a)) * b for a, b in zip(g1, g3)]
-        out[t] = [a + b for a, b in zip(hrow, lin(gate, layer["w2"]))]
+        gate = [store(a / (1 + math.exp(-a)) * b) for a, b in zip(g1, g3)]
+        out[t] = [store(a + b) for a, b in zip(hrow, lin(gate, layer["w2"]))]
     return out, ks, vs
 
 
@@ -298,6 +310,50 @@ def test_block_brute_force_with_cache_offset():
     np.testing.assert_allclose(got[0], want, rtol=1e-11, atol=1e-12)
     np.testing.assert_allclose(kc[0].reshape(P + S, 8), np.array(ks), rtol=1e-12, atol=1e-13)
     np.testing.assert_allclose(vc[0].reshape(P + S, 8), np.array(vs), rtol=1e-12, atol=1e-13)
+
+
+def test_bf16_round_hand_values_and_library_conversion():
+    # ties go to the even neighbour; 1/3 = 1.0101010|101..b x 2^-2 rounds up
+    cases = {1 + 2 ** -8: 1.0, 1 + 3 * 2 ** -8: 1 + 2 ** -6, -(1 + 2 ** -8): -1.0, 0.0: 0.0,
+             1 + 2 ** -7: 1 + 2 ** -7, 3.140625: 3.140625, 1 / 3: 0.333984375, 255.5: 256.0, 254.5: 254.0}
+    for a, want in cases.items():
+        assert O.bf16_round(np.array([a]))[0] == want, a
+        assert bf16_scalar(a) == want, a
+    # float32 inputs against torch's float32 -> bfloat16 conversion (round to nearest even)
+    import torch
+    g = torch.Generator().manual_seed(3)
+    x = torch.randn(200_000, generator=g) * torch.exp(torch.randn(200_000, generator=g) * 6)
+    want = x.to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(O.bf16_round(x.to(torch.float64).numpy()), want)
+
+
+def test_bf16_storage_variant_matches_brute_force():
+    """The bf16 precision variant rounds at exactly the step boundaries the
+    scalar restatement rounds at (a skipped or extra rounding shows as a
+    2^-9-sized difference)."""
+    cfg = tiny_cfg()
+    layer = tiny_layer(cfg)
+    P, S = 3, 4
+    k_hist = O.bf16_round(rand(P, 8)); v_hist = O.bf16_round(rand(P, 8))
+    x = O.bf16_round(rand(1, S, 16))
+    kc = np.zeros((1, P + S, 2, 4)); vc = np.zeros((1, P + S, 2, 4))
+    kc[0, :P] = k_hist.reshape(P, 2, 4); vc[0, :P] = v_hist.reshape(P, 2, 4)
+    got = O.decoder_block(x, layer, cfg, kc, vc, start_pos=P, rounding="bf16")
+    want, ks, vs = brute_force_block(x[0], layer, cfg, P, k_hist, v_hist, store=bf16_scalar)
+    np.testing.assert_allclose(got[0], want, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(kc[0].reshape(P + S, 8), np.array(ks), rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(vc[0].reshape(P + S, 8), np.array(vs), rtol=1e-12, atol=1e-14)
+    assert np.array_equal(O.bf16_round(got), got)            # the block output is stored in bf16
+    exact = O.decoder_block(x, layer, cfg, kc.copy(), vc.copy(), start_pos=P)
+    rel = np.abs(got - exact).max() / np.abs(exact).max()
+    assert 1e-4 < rel < 2e-2                                  # rounding noise, not a different function
+    rows, k, v = O.decoder_block_rows(x[0], layer, cfg, [0, 2, 3], k_hist.reshape(P, 2, 4),
+                                      v_hist.reshape(P, 2, 4), P, rounding="bf16")
+    np.testing.assert_allclose(rows, want[[0, 2, 3]], rtol=1e-12, atol=1e-14)
+    # the LM head of the variant stores the normalised rows
+    w_out = rand(11, 16)
+    lg, _ = O.lm_head(got[0], np.ones(16), w_out, 1e-5, rounding="bf16")
+    np.testing.assert_allclose(lg, O.bf16_round(O.rms_norm(got[0], np.ones(16), 1e-5)) @ w_out.T, rtol=1e-13)
 
 
 def test_block_rows_matches_brute_force_block():
