@@ -11,8 +11,11 @@ ids uniform; everything is resident in HBM before the timed region, and the
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-Under torchrun (N > 1) every rank runs its own replica (no collective on the
-data path; `scaling: weak`); times are the max over ranks.
+Under torchrun (N > 1) every rank runs its own replica of the prefill (no
+collective on the data path; `scaling: weak`), and the decode step's 32
+sequences are split over the ranks (each holds the model and its own
+sequences' caches; the next-token ids are gathered on the host); times are the
+max over ranks.
 """
 import argparse
 import datetime
@@ -34,12 +37,17 @@ import torch  # noqa: E402
 from llama_decoder_only_rmsnorm_b200 import binding as B  # noqa: E402
 from llama_decoder_only_rmsnorm_b200 import inputs as I  # noqa: E402
 from llama_decoder_only_rmsnorm_b200.model import Llama3Stack  # noqa: E402
+from llama_decoder_only_rmsnorm_b200.sharding import gather_ids, shard  # noqa: E402
 
 METRIC = "prefill & decode tokens/s on 1 B200; % of bf16 tensor / HBM roofline"
 PREFILL, DECODE = I.WORKLOADS["llama3_8b_prefill"], I.WORKLOADS["llama3_8b_decode"]
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_PATH = os.path.join(ROOT, "profiles", "traffic.json")
-FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# Used only when MEASURED_PEAKS.json is absent: the pool's earlier measurement
+# of a plain copy (HBM) and of a cuBLAS bf16 GEMM burst.  No sustained figure
+# exists for the fallback, so a kernel inside a long step is compared with the
+# burst one (reported as such).
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 
 
 def parse():
@@ -52,8 +60,6 @@ def parse():
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--layers", type=int, default=None, help=argparse.SUPPRESS)  # profiling captures only
     p.add_argument("--no-pdl", action="store_true", help=argparse.SUPPRESS)   # A/B of programmatic launch
-    p.add_argument("--kernel-path", type=int, default=0, help=argparse.SUPPRESS)  # A/B of GEMM variants
-    p.add_argument("--flash-variant", type=int, default=None, help=argparse.SUPPRESS)  # A/B of attention designs
     return p.parse_args()
 
 
@@ -189,22 +195,17 @@ def build(dev, n_layers):
     return layers, outw
 
 
-def decode_caches(dev, n_layers):
-    wd = DECODE
-    return [I.kv_cache(wd, i, wd.cache_len + 1, dev) for i in range(n_layers)]
-
-
-def time_steps(fn, steps, warmup, world, timer=None, name="timed"):
+def time_steps(fn, steps, warmup, world, name="timed"):
+    """W untimed warm-up steps, then K steps between CUDA events on the
+    current stream, bracketed by a barrier and a synchronize on both sides.
+    Returns (max over ranks of ms per step, library launches in the region)."""
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize()
     if B.llama3_device_status() != 0:
         raise RuntimeError("device status word set during warm-up")
     barrier(world)
-    if timer:
-        kind, n = timer
-        starts, stops = event_pairs(n)
-        B.llama3_set_launch_timer(kind, starts, stops)
+    torch.cuda.synchronize()
     l0 = B.llama3_launch_count()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.nvtx.range_push(name)
@@ -219,13 +220,45 @@ def time_steps(fn, steps, warmup, world, timer=None, name="timed"):
         raise RuntimeError("device status word set during the timed region")
     barrier(world)
     ms = t0.elapsed_time(t1) / steps
-    kernel_ms = None
-    if timer:
+    return max_over_ranks(ms, world), launches
+
+
+def kernel_times(fn, kind, n_pairs, steps=1):
+    """Per-launch times (ms) of the first n_pairs launches of kernel family
+    `kind` during `steps` eager calls of fn, from CUDA events the library
+    records on the launching stream.  Run apart from the timed region: an
+    event between two kernels ends their programmatic overlap."""
+    starts, stops = event_pairs(n_pairs)
+    B.llama3_set_launch_timer(kind, starts, stops)
+    try:
+        for _ in range(steps):
+            fn()
+        torch.cuda.synchronize()
         used = B.llama3_launch_timer_used()
+    finally:
         B.llama3_set_launch_timer(kind, [], [])
-        if used:
-            kernel_ms = sum(s.elapsed_time(e) for s, e in zip(starts[:used], stops[:used])) / used
-    return max_over_ranks(ms, world), kernel_ms, launches
+    return [s.elapsed_time(e) for s, e in zip(starts[:used], stops[:used])]
+
+
+def graph_kernel_times(step, kind, n_pairs, replays=3):
+    """As kernel_times, for a step captured in its own CUDA graph: the events
+    become graph nodes and every replay re-records them; the last replay's
+    times are returned."""
+    starts, stops = event_pairs(n_pairs)
+    B.llama3_set_launch_timer(kind, starts, stops)
+    g = torch.cuda.CUDAGraph()
+    try:
+        with torch.cuda.graph(g):
+            step()
+        used = B.llama3_launch_timer_used()
+    finally:
+        B.llama3_set_launch_timer(kind, [], [])
+    for _ in range(replays):
+        g.replay()
+    torch.cuda.synchronize()
+    out = [s.elapsed_time(e) for s, e in zip(starts[:used], stops[:used])]
+    del g
+    return out
 
 
 # ------------------------------------------------------- oracle baseline ---
@@ -282,21 +315,27 @@ def oracle_sample(layers, outw, caches, prefix, decode_seq=True):
 
 
 # ------------------------------------------------------------- our arm ---
+DECODE_GEMMS = (("wqkv", 6144 * 4096 * 2), ("wo", 4096 * 4096 * 2), ("w1|w3", 2 * 14336 * 4096 * 2),
+                ("w2", 4096 * 14336 * 2))   # weight bytes each decode GEMM streams (8B shapes)
+
+
 def run_ours(args):
     world, rank, local = dist_setup()
     dev = f"cuda:{local}"
     if args.no_pdl:
         B.llama3_set_programmatic_launch(False)
-    B.llama3_set_kernel_path(args.kernel_path)
-    if args.flash_variant is not None:
-        B.llama3_set_flash_variant(args.flash_variant)
+    B.llama3_set_kernel_path(0)
     peaks, peak_kind = load_peaks()
     n_layers = args.layers or PREFILL.n_layers
     layers, outw = build(dev, n_layers)
     cfg = PREFILL.cfg()
     S, D = PREFILL.seq, PREFILL.dim
+    if "bf16_tflops_sustained" in peaks:
+        peak, peak_src = peaks["bf16_tflops_sustained"], f"{peak_kind} bf16_tflops_sustained"
+    else:
+        peak, peak_src = peaks["bf16_tflops"], f"{peak_kind} bf16_tflops (burst; no sustained figure)"
 
-    # ---------------- prefill
+    # ---------------- prefill (every rank a full replica)
     pst = Llama3Stack(cfg, layers, outw, batch=1, cache_cap=S, max_seq=S, lm_rows=DECODE.batch, device=dev)
     ids = I.token_ids(PREFILL, dev)
     x = torch.empty((1, S, D), dtype=torch.bfloat16, device=dev)
@@ -307,31 +346,30 @@ def run_ours(args):
         return pst.lm_head(x[:, -1], 1, S * D)
 
     with ClockSampler(torch.cuda.current_device()) as clk:
-        ms, k_ms, launches = time_steps(prefill_step, args.steps, args.warmup, world,
-                                        timer=("gemm_w13", args.steps * n_layers), name="prefill_timed")
+        ms, launches = time_steps(prefill_step, args.steps, args.warmup, world, name="prefill_timed")
     clocks = clk.summary()
     value = world * S / (ms / 1e3)
+    # Kernel times in separate passes with the launch timer on (never inside
+    # the timed region above).  Algorithmic flops: the w1|w3 GEMM's 2*M*N*K;
+    # attention's QK^T and PV over the visible (causal) keys only.
+    k_steps = max(1, min(3, args.steps))
+    w13 = kernel_times(prefill_step, "gemm_w13", k_steps * n_layers, k_steps)
+    k_ms = sum(w13) / len(w13) if w13 else None
     F = PREFILL.ffn_hidden
     w13_flop = 2.0 * S * (2 * F) * D
     achieved = w13_flop / (k_ms / 1e3) / 1e12 if k_ms else None
-    peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
     roofline = {"bound": "tensor", "kernel": "tc_gemm w1|w3 + SwiGLU (M=8192, N=2x14336, K=4096)",
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": (achieved / peak) if achieved else None,
-                "peak_source": f"{peak_kind} bf16_tflops_sustained",
+                "frac": (achieved / peak) if achieved else None, "peak_source": peak_src,
                 "traffic": recorded_traffic("gemm_w13", ["llama_decoder_only_rmsnorm_b200/csrc/tc_gemm.cuh"]),
-                "kernel_ms": k_ms}
+                "kernel_ms": k_ms, "timed_launches": len(w13)}
     total_flop = n_layers * (2.0 * S * 6.979e9 / 32) + 2.0 * D * PREFILL.vocab  # linear layers + LM head row
     attn_flop = n_layers * PREFILL.n_heads * 2.0 * S * (S + 1) * PREFILL.head_dim
     whole = {"flop_per_step": total_flop + attn_flop,
              "tflops": (total_flop + attn_flop) / (ms / 1e3) / 1e12}
     whole["frac_of_peak"] = whole["tflops"] / peak
-    # the causal attention kernel, timed in a second, shorter pass (its own
-    # events; one timer family at a time).  Algorithmic flops: QK^T and PV over
-    # the visible (causal) keys only.
-    a_steps = max(1, min(3, args.steps))
-    _, a_ms, _ = time_steps(prefill_step, a_steps, 1, world, timer=("attention", a_steps * n_layers),
-                            name="prefill_attention")
+    at = kernel_times(prefill_step, "attention", k_steps * n_layers, k_steps)
+    a_ms = sum(at) / len(at) if at else None
     a_flop = PREFILL.n_heads * 2.0 * 2.0 * (S * (S + 1) / 2) * PREFILL.head_dim
     attention = {"kernel": "causal GQA flash attention (S=8192, 32 q heads, 8 kv heads, hd 128)",
                  "kernel_ms": a_ms, "flop_per_launch": a_flop,
@@ -339,29 +377,32 @@ def run_ours(args):
     if attention["tflops"]:
         attention["frac_of_peak"] = attention["tflops"] / peak
 
-    # e2e through the public API with host buffers
+    # e2e through the public API with host buffers: ids in, next id out, read
+    # on the host every step
     ids_h = ids.cpu().pin_memory()
     out_h = torch.empty((1,), dtype=torch.int32).pin_memory()
 
     def prefill_e2e():
         ids.copy_(ids_h, non_blocking=True)
         out_h.copy_(prefill_step(), non_blocking=True)
+        torch.cuda.current_stream().synchronize()
 
-    e2e_ms, _, _ = time_steps(prefill_e2e, args.steps, 1, world, name="prefill_e2e")
+    e2e_ms, _ = time_steps(prefill_e2e, args.steps, 1, world, name="prefill_e2e")
     e2e = {"value": world * S / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": ids_h.numel() * 4,
            "d2h_bytes_per_step": 4}
     del pst, x
     torch.cuda.empty_cache()
 
-    # ---------------- decode
+    # ---------------- decode (the batch of 32 sequences split over the ranks)
     decode = None
     caches = None
     if not args.no_decode:
-        caches = decode_caches(dev, n_layers)
-        Bd, P = DECODE.batch, DECODE.cache_len
+        Bt, P = DECODE.batch, DECODE.cache_len
+        first, Bd = shard(Bt, world, rank)
+        caches = [I.kv_cache(DECODE, i, P + 1, dev, first, Bd) for i in range(n_layers)]
         dst = Llama3Stack(cfg, layers, outw, batch=Bd, cache_cap=P + 1, max_seq=1, lm_rows=Bd, device=dev,
                           caches=caches)
-        dids = I.token_ids(DECODE, dev)
+        dids = I.token_ids(DECODE, dev)[first:first + Bd].contiguous()
         xd = torch.empty((Bd, 1, D), dtype=torch.bfloat16, device=dev)
 
         def decode_step():
@@ -370,63 +411,87 @@ def run_ours(args):
             return dst.lm_head(xd, Bd, D)
 
         # The decode step (about a dozen launches per block) is captured once
-        # in a CUDA graph after eager warm-up and replayed; the library records
-        # the decode-attention launch events inside the graph, so every replay
-        # of the timed region timestamps them.  Only the first few blocks'
-        # launches carry events: an event between two kernels ends their
-        # programmatic overlap, so timing all 32 would slow the step itself.
+        # in a CUDA graph after eager warm-up and replayed.
         for _ in range(args.warmup):
             decode_step()
         torch.cuda.synchronize()
-        starts, stops = event_pairs(min(4, n_layers))
-        B.llama3_set_launch_timer("decode_attention", starts, stops)
         graph = torch.cuda.CUDAGraph()
         l0 = B.llama3_launch_count()
         with torch.cuda.graph(graph):
             nxt_dev = decode_step()
         per_step_launches = B.llama3_launch_count() - l0
-        B.llama3_set_launch_timer("decode_attention", [], [])
         with ClockSampler(torch.cuda.current_device()) as clk2:
-            dms, _, _ = time_steps(graph.replay, args.steps, args.warmup, world, name="decode_timed")
-        dk_ms = sum(a.elapsed_time(b) for a, b in zip(starts, stops)) / len(starts)
-        dlaunch = per_step_launches * args.steps
+            dms, _ = time_steps(graph.replay, args.steps, args.warmup, world, name="decode_timed")
+        # kernel times from separately captured graphs: the first 4 blocks'
+        # attention launches, and their 4 weight-streaming GEMMs each
+        nb = min(4, n_layers)
+        att = graph_kernel_times(decode_step, "decode_attention", nb)
+        gem = graph_kernel_times(decode_step, "decode_gemm", 4 * nb)
+        dk_ms = sum(att) / len(att) if att else None
         kv_bytes = Bd * (P + 1) * DECODE.n_kv_heads * DECODE.head_dim * 2 * 2
         dach = kv_bytes / (dk_ms / 1e3) / 1e9 if dk_ms else None
         hbm = peaks.get("hbm_gbs")
+        gemms = {}
+        for j, (name, wbytes) in enumerate(DECODE_GEMMS):
+            t = [gem[i] for i in range(j, len(gem), 4)]
+            if t:
+                tm = sum(t) / len(t)
+                gemms[name] = {"kernel_ms": tm, "weight_bytes": wbytes, "gbs": wbytes / (tm / 1e3) / 1e9,
+                               "frac_of_hbm": wbytes / (tm / 1e3) / 1e9 / hbm}
         step_bytes = n_layers * (kv_bytes + 2 * 6.979e9 / 32) + 2.0 * DECODE.vocab * D
         dids_h = dids.cpu().pin_memory()
         dout_h = torch.empty((Bd,), dtype=torch.int32).pin_memory()
+        gloo = torch.distributed.new_group(backend="gloo") if world > 1 else None
 
         def decode_e2e():
             dids.copy_(dids_h, non_blocking=True)
             graph.replay()
             dout_h.copy_(nxt_dev, non_blocking=True)
+            torch.cuda.current_stream().synchronize()
+            gather_ids(dout_h, Bt, world, rank, gloo)   # the 32 next ids on rank 0's host
 
-        de2e_ms, _, _ = time_steps(decode_e2e, args.steps, 1, world, name="decode_e2e")
-        decode = {"metric": "decode tokens/s", "value": world * Bd / (dms / 1e3), "unit": "tokens/s",
+        de2e_ms, _ = time_steps(decode_e2e, args.steps, 1, world, name="decode_e2e")
+        decode = {"metric": "decode tokens/s", "value": Bt / (dms / 1e3), "unit": "tokens/s",
                   "ms_per_step": dms, "steps": args.steps, "warmup": args.warmup,
-                  "config": {"workload": "llama3_8b_decode", "batch": Bd, "cached_positions": P,
-                             "new_token_position": P},
-                  "roofline": {"bound": "hbm", "kernel": "split-KV decode attention (1.07 GB K/V per launch)",
+                  "scaling": "strong" if world > 1 else "weak",
+                  "config": {"workload": "llama3_8b_decode", "batch": Bt, "cached_positions": P,
+                             "new_token_position": P,
+                             "parallelism": f"batch split over {world} ranks ({Bd} sequences on rank {rank}); "
+                                            "ids gathered on the host"},
+                  "roofline": {"bound": "hbm", "kernel": "split-KV decode attention (K/V of this rank's "
+                                                          f"{Bd} sequences per launch)",
                                "achieved": dach, "peak": hbm, "unit": "GB/s",
                                "frac": (dach / hbm) if dach else None, "peak_source": f"{peak_kind} hbm_gbs",
                                "traffic": recorded_traffic("decode_attention", [
-                                   "llama_decoder_only_rmsnorm_b200/csrc/decode_attention.cuh"]),
+                                   "llama_decoder_only_rmsnorm_b200/csrc/decode_attention.cuh"])
+                               if Bd == Bt else None,
                                "kernel_ms": dk_ms},
+                  "decode_gemms": gemms,
                   "whole_step": {"bytes_per_step": step_bytes, "gbs": step_bytes / (dms / 1e3) / 1e9,
                                  "frac_of_hbm": step_bytes / (dms / 1e3) / 1e9 / hbm},
-                  "e2e": {"value": world * Bd / (de2e_ms / 1e3), "unit": "tokens/s",
+                  "e2e": {"value": Bt / (de2e_ms / 1e3), "unit": "tokens/s",
                           "h2d_bytes_per_step": Bd * 4, "d2h_bytes_per_step": Bd * 4},
-                  "gpu_launches": dlaunch, "cuda_graph": True, "clocks": clk2.summary()}
+                  "gpu_launches": per_step_launches * args.steps, "cuda_graph": True, "clocks": clk2.summary()}
+        del graph
+        if gloo is not None:
+            torch.distributed.destroy_process_group(gloo)
 
     # ---------------- oracle on the host cores
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         prefix = 64
         t_pre, t_dec, cores = oracle_sample(layers, outw, caches, prefix, decode_seq=caches is not None)
+        # per-token work of the 64-token prefix against the whole 8192-token
+        # prefill (linear layers per token, plus causal attention over ~t keys)
+        lin = 2.0 * 6.979e9 * n_layers / 32
+        att_tok = lambda n: n_layers * PREFILL.n_heads * 2.0 * (n + 1) * PREFILL.head_dim
+        ratio = (lin + att_tok(prefix)) / (lin + att_tok(S))
         cpu = {"value": prefix / t_pre, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                "sample": f"fp64 oracle, first {prefix} tokens of the prefill through all {n_layers} blocks + "
-                         "final norm + LM head on the last position (weight fp64 conversion not timed)"}
+                         "final norm + LM head on the last position (weight fp64 conversion not timed); the "
+                         "whole 8192-token prefill does more attention work per token, so at the same rate "
+                         f"of work the oracle would reach about {ratio:.2f} of this value there",
+               "full_sequence_estimate": prefix / t_pre * ratio}
         if decode is not None and t_dec > 0:
             decode["cpu_baseline"] = {"value": 1.0 / t_dec, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                                       "sample": "fp64 oracle, one sequence's decode step at position 8192 "

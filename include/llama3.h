@@ -206,7 +206,11 @@ int llama3_layer_decode_ragged(const llama3_config* cfg, const llama3_layer_weig
  *     leaves RMSNorm(x_out, next_attention_norm) in the workspace.
  *   input_normalised: nonzero when the previous call on this workspace, for
  *     the same batch, was given this block's attention_norm as its
- *     next_attention_norm; the block then skips its first RMSNorm.
+ *     next_attention_norm; the block then skips its first RMSNorm.  The
+ *     library cannot check this: any other call on the same workspace in
+ *     between (an LM head, a prefill, a decode of another batch or block)
+ *     overwrites the normalised rows, and the flag then gives a wrong block
+ *     output.
  * Only the tcgen05 decode path (bf16, batch <= 256 or ragged) hands the
  * normalised input on; the other paths ignore both arguments and normalise x
  * themselves, so the result is the same either way.  Errors as
@@ -251,13 +255,14 @@ int llama3_lm_head_argmax(const llama3_config* cfg, const void* norm_w, const vo
  * the process exits.  The call needs  roundup(rows * 8, 256) +
  * rows * dim * sizeof(element)  bytes of it and returns LLAMA3_ERR_WORKSPACE
  * when that exceeds the array (for dim 4096 in bf16: at most 511 rows).
- * The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture.  All calls share the one array and find the
- * previous call's contents there (the argmax keys are re-initialised by each
- * call): calls whose executions overlap on the GPU (other streams, other
- * host threads) race on it and must be serialised by the caller.  The
- * library allocates nothing for this call.
+ * Set-up: each call made outside a stream capture looks up the array's
+ * device address (cudaGetSymbolAddress) in the current device's context, so
+ * a context torn down and created again gets its own address; make the first
+ * call on a device before any stream capture.  All calls share the one array
+ * and find the previous call's contents there (the argmax keys are
+ * re-initialised by each call): calls whose executions overlap on the GPU
+ * (other streams, other host threads) race on it and must be serialised by
+ * the caller.  The library allocates nothing for this call.
  */
 #define LLAMA3_NOALLOC_SCRATCH_BYTES (4u << 20)
 int llama3_lm_head_argmax_noalloc(const llama3_config* cfg, const void* norm_w, const void* w_out,
@@ -310,13 +315,21 @@ int llama3_gather_rows(const llama3_config* cfg, const void* x, long long row_st
  * a device pointer whose contents change, none is a host value.
  * history[*step][b] = ids[b] for b < batch (skipped once *step >= history_rows;
  * row stride history_stride >= batch), positions[b] += 1, *step += 1.
- * No counterpart on the pages, which run this loop on the host ([S2] 六).
- * Errors: LLAMA3_ERR_ARG (null pointers, batch < 1, history_rows < 1,
- * history_stride < batch), LLAMA3_ERR_ALIGN (pointers not 4-byte aligned).
+ * End token ([S2] 六 generate stops a sequence at its end token and the loop
+ * once every sequence has stopped): with eos_id >= 0, done is device int32
+ * [batch + 1] (zeroed by the caller before the first step).  A sequence whose
+ * done[b] is set has ids[b] replaced by eos_id before it is recorded (so it
+ * keeps emitting the end token and feeds it to the next step); a sequence
+ * whose ids[b] == eos_id gets done[b] = 1; done[batch] is set to 1 once every
+ * sequence is done, for the host to end the loop.  eos_id < 0: done is not
+ * used (may be NULL) and ids is not written.
+ * Errors: LLAMA3_ERR_ARG (null pointers, done NULL with eos_id >= 0,
+ * batch < 1, history_rows < 1, history_stride < batch), LLAMA3_ERR_ALIGN
+ * (pointers not 4-byte aligned).
  */
-int llama3_generation_advance(int32_t* positions, const int32_t* ids, int32_t* history, int32_t* step,
-                              int batch, int history_rows, long long history_stride,
-                              llama3_stream_t stream);
+int llama3_generation_advance(int32_t* positions, int32_t* ids, int32_t* history, int32_t* step,
+                              int32_t* done, int eos_id, int batch, int history_rows,
+                              long long history_stride, llama3_stream_t stream);
 
 /* ---- building blocks (the steps of the calls above, exposed for tests) ---- */
 
@@ -391,9 +404,8 @@ int llama3_device_status(int* out);
 int llama3_last_cuda_error(void);
 
 /* Kernel selection: 0 (default) = tcgen05/TMA kernels for bf16, 1 = the plain
- * SIMT kernels for every dtype, 2 = as 0 but the prefill GEMMs (m >= 256) run
- * on CTA pairs (tcgen05 cta_group::2, 256-row tiles).  Returns the previous
- * value. */
+ * SIMT kernels for every dtype (any other value selects 0).  Returns the
+ * previous value. */
 int llama3_set_kernel_path(int path);
 
 /* Limit, in milliseconds, of every bounded device-side wait (default 2000). */
@@ -404,18 +416,6 @@ int llama3_set_wait_limit_ms(int ms);
  * the stream (each kernel waits for its predecessor before touching memory);
  * 0: ordinary launches.  Returns the previous value. */
 int llama3_set_programmatic_launch(int on);
-
-/* Prefill attention kernel design (bf16, tcgen05 path): 3 (default) = one
- * softmax thread per query row holding the whole row of a tile in registers
- * (warpgroup register reallocation) with P in tensor memory; 1 = one softmax
- * thread per row with P staged in shared memory; 2 = two softmax threads per
- * row (each over half the keys of a tile) with P in tensor memory; 4 = as 3
- * with P staged in shared memory; 5 = as 3, but both softmax warpgroups work
- * on each tile (half the keys each) and then on the other head's tile.  All
- * compute the same attention.  Values outside 1..5 select 3.  Variants 3, 4
- * and 5 return LLAMA3_ERR_UNSUPPORTED if the compiled kernel's register count
- * cannot fund their register split.  Returns the previous value. */
-int llama3_set_flash_variant(int variant);
 
 #ifdef __cplusplus
 }

@@ -66,9 +66,8 @@ _SIGNATURES = {
     "llama3_set_kernel_path": [_i],
     "llama3_set_wait_limit_ms": [_i],
     "llama3_set_programmatic_launch": [_i],
-    "llama3_set_flash_variant": [_i],
     "llama3_sample_top_p": [_p, _i, _ll, _i, ctypes.c_float, ctypes.c_float, ctypes.c_ulonglong, ctypes.c_ulonglong, _p, _p, _p],
-    "llama3_generation_advance": [_p, _p, _p, _p, _i, _i, _ll, _p],
+    "llama3_generation_advance": [_p, _p, _p, _p, _p, _i, _i, _i, _ll, _p],
     "llama3_gather_rows": [_cfgp, _p, _ll, _i, _p, _i, _p, _p],
     "llama3_set_launch_timer": [_i, _p, _p, _i],
     "llama3_launch_timer_used": [],
@@ -223,11 +222,13 @@ def llama3_gather_rows(cfg, x, row_stride, n_rows, row_index, rows, out, stream=
         ctypes.byref(cfg), _ptr(x), row_stride, n_rows, _ptr(row_index), rows, _ptr(out), _stream(stream)))
 
 
-def llama3_generation_advance(positions, ids, history, step, batch, history_rows, history_stride, stream=None):
-    """history[step] = ids, positions += 1, step += 1, all on the device."""
+def llama3_generation_advance(positions, ids, history, step, batch, history_rows, history_stride, stream=None,
+                              done=None, eos_id=-1):
+    """history[step] = ids, positions += 1, step += 1, all on the device; with
+    eos_id >= 0 and done (int32 [batch + 1]), sequences stop at the end token."""
     _check("llama3_generation_advance", lib().llama3_generation_advance(
-        _ptr(positions), _ptr(ids), _ptr(history), _ptr(step), batch, history_rows, history_stride,
-        _stream(stream)))
+        _ptr(positions), _ptr(ids), _ptr(history), _ptr(step), _ptr(done), int(eos_id), batch, history_rows,
+        history_stride, _stream(stream)))
 
 
 NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -281,10 +282,6 @@ def llama3_set_wait_limit_ms(ms):
 
 def llama3_set_programmatic_launch(on):
     return lib().llama3_set_programmatic_launch(1 if on else 0)
-
-
-def llama3_set_flash_variant(variant):
-    return lib().llama3_set_flash_variant(int(variant))
 
 
 KERNEL_KINDS = {"gemm_qkv": 1, "gemm_wo": 2, "gemm_w13": 3, "gemm_w2": 4, "attention": 5, "decode_gemm": 6,

@@ -4,7 +4,9 @@
 // "从0开发大模型—译llama3-from-scratch" §6.11-§8): for the token at position
 // p = start_pos + t and query head h,
 //     o[t, h] = sum_{j <= p} softmax_j(q[t,h] . k[j, h/n_rep] / sqrt(hd)) v[j, h/n_rep]
-// with k, v read from the caller's cache [B, cap, KV, hd] (rotated keys).
+// with k, v read from the caller's cache [B, cap, KV, hd] (rotated keys), and
+// optionally the document mask of 附 1 (keys before the token's document start
+// are invisible).
 //
 // Design (B200):
 //  * A CTA owns one KV group g of one sequence b, 128 query positions, and TWO
@@ -12,21 +14,33 @@
 //    and used by both heads' MMAs, so repeat_kv is never formed and a KV head
 //    is read ceil(n_rep/2) times per query tile instead of n_rep times.
 //  * S = Q K^T (M=128 queries, N=128 keys, K=hd) and O += P V (M=128, N=hd,
-//    K=128 keys) run on tcgen05 with fp32 accumulators in TMEM:
-//    slot s uses columns [256s, 256s+128) for S and [256s+128, 256s+128+hd) for O.
-//  * One warpgroup per slot does the online softmax, one thread per query row
-//    (its TMEM lane).  While one slot's warpgroup exponentiates, the tensor
-//    core runs the other slot's MMAs (ping-pong).  Scores are kept in the
-//    log2 domain; O is rescaled in TMEM only when a row maximum grows by more
-//    than 2^8 (exact: the same reference maximum is used for numerator and
-//    denominator).
-//  * P (bf16) is written to shared memory in the 128-byte-swizzled K-major
-//    layout the MMA reads; V is consumed directly as an MN-major operand.
+//    K=128 keys) run on tcgen05 with fp32 accumulators in TMEM: slot s uses
+//    columns [256s, 256s+128) for S and [256s+128, 256s+128+hd) for O.
+//  * One softmax thread per query row (its TMEM lane), one warpgroup per slot.
+//    The warpgroups trade registers at start-up (setmaxnreg): the producer /
+//    MMA warpgroup drops to 104 per thread and the two softmax warpgroups rise
+//    to 200, so a thread holds its row's 128 scores of a tile at once and
+//    reads them from TMEM a single time (one max pass, one exponent pass, both
+//    from registers).  Scores stay in the log2 domain; O is rescaled in TMEM
+//    only when a row maximum grows by more than 2^8 (exact: the same reference
+//    maximum serves numerator and denominator).
+//  * P (bf16, two per 32-bit column) is written back into TMEM over the
+//    scores just read (keys 0-127 -> columns 0-63) and P.V takes its A operand
+//    from TMEM, so P never goes through shared memory; K and V are both
+//    double-buffered in shared memory.
+//  * A whole warp runs the MMA loop (warp-uniform addresses and descriptors)
+//    and one elected lane issues; a head's next S goes right behind the P.V
+//    that reads its columns, since the MMAs of one thread run in issue order.
+//  * The softmax never waits for a P.V before its exponentials: the S commit
+//    it waits for covers every MMA issued before that S, the P.V included.
 //  * Q and K/V tiles come through 4-D TMA maps whose extents stop at `seq`
 //    and `start_pos + seq`, so rows past the valid range read as zeros and no
 //    unwritten cache entry is ever touched.
 //  * Causal tile skipping: a query tile visits only key tiles up to its last
-//    position; work units are issued longest first.
+//    position; work units are issued longest first, in snake order.
+// The split of registers is only valid for a launch of 384 threads at 168
+// registers each (128*104 + 256*200 = 384*168); the host checks the compiled
+// register count before every launch.
 #pragma once
 #include "common.cuh"
 
@@ -40,27 +54,6 @@ struct FlashShape {
   // document of token t begins (non-decreasing in t, <= start_pos + t); keys
   // before it are invisible ("Build your own Llama 3 from scratch" 附 1).
   const int32_t* doc_start;
-};
-
-template <int HD>
-struct FlashCfg {
-  static constexpr int CHUNKS = (HD + 63) / 64;     // 64-element (128-byte) slabs of a head
-  static constexpr int TILE_BYTES = 128 * 128;      // one [128 rows x 64 elems] bf16 slab
-  static constexpr int Q_BYTES = CHUNKS * TILE_BYTES;
-  static constexpr int KV_BYTES = CHUNKS * TILE_BYTES;
-  static constexpr int P_BYTES = 2 * TILE_BYTES;    // 128 rows x 128 keys
-  static constexpr int KST = 1, VST = 2;
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
-  static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
-  static constexpr int OFF_P = OFF_V + VST * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
-  static constexpr int N_BARS = 2 /*q_full*/ + 2 /*q_empty*/ + 2 * KST + 2 * VST + 2 /*s_full*/ +
-                                2 /*p_full*/ + 2 /*o_done*/;
-  static constexpr int SMEM_BYTES = 1024 + OFF_BAR + N_BARS * 8 + 16;
-  static constexpr int KSTEPS_QK = HD / 16;   // MMA K-steps over the head dimension
-  static_assert(SMEM_BYTES <= 232448, "shared memory");
-  static_assert(HD % 32 == 0 && HD <= 128, "head_dim");
 };
 
 __device__ __forceinline__ void flash_unit(const FlashShape& fs, int u, int& b, int& g, int& pair, int& qt) {
@@ -95,15 +88,267 @@ __device__ __forceinline__ int flash_first_tile(const FlashShape& fs, int b, int
   return flash_row_lo(fs, b, qt * 128) / 128;
 }
 
+// D[tmem] (+)= A[tmem] * B[smem desc]^T, kind::f16; A is K-major in TMEM
+// (row m in lane m, two bf16 per 32-bit column).
+__device__ __forceinline__ void tc_mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+constexpr int kFlashThreads = 384;
+constexpr int kFlashLowRegs = 104, kFlashHighRegs = 200;
+
 template <int HD>
-__global__ void __launch_bounds__(384, 1)
-    flash_attention_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
-                           const __grid_constant__ CUtensorMap mapV, bf16* __restrict__ out, const FlashShape fs,
-                           const unsigned long long wait_ns) {
+struct FlashCfg {
+  static constexpr int CHUNKS = (HD + 63) / 64;
+  static constexpr int TILE_BYTES = 128 * 128;
+  static constexpr int Q_BYTES = CHUNKS * TILE_BYTES;
+  static constexpr int KV_BYTES = CHUNKS * TILE_BYTES;
+  static constexpr int KST = 2, VST = 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
+  static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_V + VST * KV_BYTES;
+  static constexpr int N_BARS = 2 + 2 + 2 * KST + 2 * VST + 2 + 2 + 2;
+  static constexpr int SMEM_BYTES = 1024 + OFF_BAR + N_BARS * 8 + 16;
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
+  static_assert(HD % 32 == 0 && HD <= 128, "head_dim");
+};
+
+// The 128 scores of one row (this thread's TMEM lane), 32 columns at a time.
+__device__ __forceinline__ void flash_load_row(uint32_t taddr, uint32_t (&a)[32], uint32_t (&b)[32],
+                                                uint32_t (&c)[32], uint32_t (&d)[32]) {
+  tmem_ld32(taddr, a);
+  tmem_ld32(taddr + 32, b);
+  tmem_ld32(taddr + 64, c);
+  tmem_ld32(taddr + 96, d);
+  tc_wait_ld();
+}
+
+// p = 2^(s*scl - m) for 32 scores of the row, in place (as fp32 bits), and
+// their sum in (sa, sb).  Exponentials in fp32: on unmasked tiles 4 of every
+// 16 pairs go to the FMA pipe (exp2_poly2), the rest to the MUFU; masked tiles
+// use the MUFU only, which gives exactly 0 for the -inf scores.
+template <bool MASKED>
+__device__ __forceinline__ void flash_exp_inplace(uint32_t (&r)[32], float scl, float neg_m, float& sa, float& sb) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    float x0, x1, p0, p1;
+    fma2(x0, x1, __uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), scl, scl, neg_m, neg_m);
+    if (!MASKED && (i & 7) < 2) {
+      exp2_poly2(x0, x1, p0, p1);
+    } else {
+      p0 = ex2_approx(x0);
+      p1 = ex2_approx(x1);
+    }
+    add2(sa, sb, p0, p1);
+    r[2 * i] = __float_as_uint(p0);
+    r[2 * i + 1] = __float_as_uint(p1);
+  }
+}
+__device__ __forceinline__ void flash_pack_store(uint32_t (&r)[32], uint32_t taddr) {
+  uint32_t pk[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+  tmem_st16(taddr, pk);
+}
+// The whole row: all 128 exponentials before any pack or store, so that the
+// four chunks overlap; then the bf16 pairs go to the 64 TMEM columns at taddr
+// (keys 0-127 -> columns 0-63).  Returns the row's sum over the tile.
+template <bool MASKED>
+__device__ __forceinline__ float flash_exp_row(uint32_t (&ra)[32], uint32_t (&rb)[32], uint32_t (&rc)[32],
+                                                uint32_t (&rd)[32], float scl, float neg_m, uint32_t taddr) {
+  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f, s4 = 0.f, s5 = 0.f, s6 = 0.f, s7 = 0.f;
+  flash_exp_inplace<MASKED>(ra, scl, neg_m, s0, s1);
+  flash_exp_inplace<MASKED>(rb, scl, neg_m, s2, s3);
+  flash_exp_inplace<MASKED>(rc, scl, neg_m, s4, s5);
+  flash_exp_inplace<MASKED>(rd, scl, neg_m, s6, s7);
+  flash_pack_store(ra, taddr);
+  flash_pack_store(rb, taddr + 16);
+  flash_pack_store(rc, taddr + 32);
+  flash_pack_store(rd, taddr + 48);
+  return ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
+}
+
+template <bool MASKED>
+__device__ __forceinline__ float flash_row_max(uint32_t (&r)[32], int key0, int qpos, int lo) {
+  float mx = -INFINITY;
+  if (MASKED) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (key0 + i > qpos || key0 + i < lo) r[i] = __float_as_uint(-INFINITY);
+  }
+#pragma unroll
+  for (int i = 0; i < 32; i += 2) mx = max3f(mx, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
+  return mx;
+}
+
+// The barriers the three roles share (all in shared memory).
+struct FlashBars {
+  uint64_t *q_full, *q_empty, *k_full, *k_empty, *v_full, *v_empty, *s_full, *p_full, *o_done;
+};
+
+// Producer (one thread): per work unit the Q tiles of its one or two heads,
+// then K and V of every visible key tile, through the K and V rings.
+template <int HD>
+__device__ __forceinline__ void flash_produce(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
+                                               uint8_t* smem, const FlashBars& B, const FlashShape& fs,
+                                               unsigned long long wait_ns) {
+  using C = FlashCfg<HD>;
+  uint64_t *q_full = B.q_full, *q_empty = B.q_empty, *k_full = B.k_full, *k_empty = B.k_empty;
+  uint64_t *v_full = B.v_full, *v_empty = B.v_empty;
+  int ks = 0, vs = 0;
+  uint32_t kph = 0, vph = 0, qph = 0;   // qph: phase bit per Q slot
+  bool ok = true;
+  uint32_t kiss = 0, kpar = 0, viss = 0, vpar = 0, qiss = 0, qpar = 0;
+  for (int k_ = 0, u = flash_snake(0); u < fs.units && ok; u = flash_snake(++k_)) {
+    int b, g, pair, qt;
+    flash_unit(fs, u, b, g, pair, qt);
+    const int nt = flash_ntiles(fs, qt);
+    const bool has1 = pair * 2 + 1 < fs.n_rep;
+    for (int s = 0; s < 2 && ok; ++s) {
+      if (s == 1 && !has1) break;
+      if (!mbar_wait(&q_empty[s], ((qph >> s) & 1u) ^ 1u, wait_ns)) { ok = false; break; }
+      mbar_arrive_expect_tx(&q_full[s], C::Q_BYTES);
+      const int h = g * fs.n_rep + pair * 2 + s;
+      for (int c = 0; c < C::CHUNKS; ++c)
+        tma_load_4d(smem + C::OFF_Q + s * C::Q_BYTES + c * C::TILE_BYTES, &mapQ, &q_full[s], c * 64, h,
+                    qt * 128, b);
+      qiss |= 1u << s; qpar = (qpar & ~(1u << s)) | (qph & (1u << s));
+      qph ^= 1u << s;
+    }
+    const int jt0 = flash_first_tile(fs, b, qt);
+    for (int j = jt0; j < nt && ok; ++j) {
+      if (!mbar_wait(&k_empty[ks], kph ^ 1u, wait_ns)) { ok = false; break; }
+      mbar_arrive_expect_tx(&k_full[ks], C::KV_BYTES);
+      for (int c = 0; c < C::CHUNKS; ++c)
+        tma_load_4d(smem + C::OFF_K + ks * C::KV_BYTES + c * C::TILE_BYTES, &mapK, &k_full[ks], c * 64, g,
+                    j * 128, b);
+      kiss |= 1u << ks; kpar = (kpar & ~(1u << ks)) | (kph << ks);
+      if (++ks == C::KST) { ks = 0; kph ^= 1u; }
+      if (!mbar_wait(&v_empty[vs], vph ^ 1u, wait_ns)) { ok = false; break; }
+      mbar_arrive_expect_tx(&v_full[vs], C::KV_BYTES);
+      for (int c = 0; c < C::CHUNKS; ++c)
+        tma_load_4d(smem + C::OFF_V + vs * C::KV_BYTES + c * C::TILE_BYTES, &mapV, &v_full[vs], c * 64, g,
+                    j * 128, b);
+      viss |= 1u << vs; vpar = (vpar & ~(1u << vs)) | (vph << vs);
+      if (++vs == C::VST) { vs = 0; vph ^= 1u; }
+    }
+  }
+  for (int s = 0; s < 2; ++s)
+    if (qiss & (1u << s)) mbar_wait(&q_full[s], (qpar >> s) & 1u, wait_ns);
+  for (int s = 0; s < C::KST; ++s)
+    if (kiss & (1u << s)) mbar_wait(&k_full[s], (kpar >> s) & 1u, wait_ns);
+  for (int s = 0; s < C::VST; ++s)
+    if (viss & (1u << s)) mbar_wait(&v_full[s], (vpar >> s) & 1u, wait_ns);
+}
+
+// MMA issuer (one whole warp; one elected lane issues).  Per key tile and head:
+// S = Q K^T into the head's S columns, and, once the softmax has written P over
+// them, O += P V (P from TMEM, V MN-major from shared memory).
+template <int HD>
+__device__ __forceinline__ void flash_issue_mma(uint8_t* smem, const FlashBars& B, uint32_t tmem_base,
+                                                 const FlashShape& fs, unsigned long long wait_ns) {
   using C = FlashCfg<HD>;
   constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, 0, 0);
-  constexpr uint32_t IDESC_O = idesc_bf16_f32(128, HD, 0, 1);   // V is MN-major (hd contiguous)
+  constexpr uint32_t IDESC_O = idesc_bf16_f32(128, HD, 0, 1);   // A = P (TMEM), B = V MN-major
+  uint64_t *q_full = B.q_full, *q_empty = B.q_empty, *k_full = B.k_full, *k_empty = B.k_empty;
+  uint64_t *v_full = B.v_full, *v_empty = B.v_empty, *s_full = B.s_full, *p_full = B.p_full, *o_done = B.o_done;
+  const bool leader = elect_one_sync();
+  int ks = 0, vs = 0;
+  // phase bits per slot (bit s) of the Q and P barriers as this thread sees them
+  uint32_t kph = 0, vph = 0, qph = 0, pph = 0;
+  bool ok = true;
+  // S of the next tile overwrites the TMEM columns that hold P.  It is
+  // issued right behind the P.V that reads them, without waiting for that
+  // P.V to complete: the MMAs one thread issues execute in issue order, so
+  // every read of P precedes the first write of the next S (the tcgen05
+  // attention mainloops of CUTLASS rely on the same order).
+  const uint32_t q_addr = smem_u32(smem + C::OFF_Q);
+  auto issue_s = [&](int s, int kst) {
+    const uint32_t d = tmem_base + s * 256;
+    const uint32_t qa = q_addr + s * C::Q_BYTES;
+    const uint32_t ka = smem_u32(smem + C::OFF_K + kst * C::KV_BYTES);
+    if (leader) {
+#pragma unroll
+      for (int k = 0; k < HD / 16; ++k) {
+        const uint32_t off = (k >> 2) * C::TILE_BYTES + (k & 3) * 32;
+        tc_mma_f16_ss(d, sw128_desc(qa + off, 1024, 16), sw128_desc(ka + off, 1024, 16), IDESC_S, k > 0);
+      }
+      tc_commit(&s_full[s]);
+    }
+    __syncwarp();
+  };
+  auto issue_pv = [&](int s, int vst, bool accumulate) {
+    const uint32_t d = tmem_base + s * 256 + 128;
+    const uint32_t pa = tmem_base + s * 256;   // P: keys 16k.. in columns 8k..
+    const uint32_t va = smem_u32(smem + C::OFF_V + vst * C::KV_BYTES);
+    if (leader) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        tc_mma_f16_ts(d, pa + k * 8, sw128_desc(va + k * 2048, 1024, C::TILE_BYTES), IDESC_O,
+                      (accumulate || k > 0) ? 1u : 0u);
+      tc_commit(&o_done[s]);
+    }
+    __syncwarp();
+  };
+  for (int k_ = 0, u = flash_snake(0); u < fs.units && ok; u = flash_snake(++k_)) {
+    int b, g, pair, qt;
+    flash_unit(fs, u, b, g, pair, qt);
+    const int nt = flash_ntiles(fs, qt);
+    const int nslots = (pair * 2 + 1 < fs.n_rep) ? 2 : 1;
+    for (int s = 0; s < nslots; ++s) {
+      if (!mbar_wait_warp(&q_full[s], (qph >> s) & 1u, wait_ns)) ok = false;
+      qph ^= 1u << s;
+    }
+    if (!ok) break;
+    tc_fence_after();
+    const int jt0 = flash_first_tile(fs, b, qt);
+    if (!mbar_wait_warp(&k_full[ks], kph, wait_ns)) break;
+    tc_fence_after();
+    for (int s = 0; s < nslots; ++s) issue_s(s, ks);
+    if (leader) tc_commit(&k_empty[ks]);
+    if (++ks == C::KST) { ks = 0; kph ^= 1u; }
+    for (int j = jt0; j < nt && ok; ++j) {
+      if (!mbar_wait_warp(&v_full[vs], vph, wait_ns)) { ok = false; break; }
+      const bool more = j + 1 < nt;
+      bool k_ready = false;
+      for (int s = 0; s < nslots; ++s) {
+        if (!mbar_wait_warp(&p_full[s], (pph >> s) & 1u, wait_ns)) { ok = false; break; }
+        pph ^= 1u << s;
+        tc_fence_after();
+        issue_pv(s, vs, j > jt0);
+        if (more) {
+          if (!k_ready && !mbar_wait_warp(&k_full[ks], kph, wait_ns)) { ok = false; break; }
+          k_ready = true;
+          issue_s(s, ks);
+        }
+      }
+      if (!ok) break;
+      if (leader) tc_commit(&v_empty[vs]);
+      if (++vs == C::VST) { vs = 0; vph ^= 1u; }
+      if (more) {
+        if (leader) tc_commit(&k_empty[ks]);
+        if (++ks == C::KST) { ks = 0; kph ^= 1u; }
+      }
+    }
+    if (leader)
+      for (int s = 0; s < nslots; ++s) tc_commit(&q_empty[s]);
+    __syncwarp();
+  }
+}
 
+template <int HD>
+__global__ void __launch_bounds__(kFlashThreads, 1)
+    flash_attention_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
+                            const __grid_constant__ CUtensorMap mapV, bf16* __restrict__ out, const FlashShape fs,
+                            const unsigned long long wait_ns) {
+  using C = FlashCfg<HD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
@@ -117,8 +362,12 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* p_full = s_full + 2;
   uint64_t* o_done = p_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_done + 2);
+  const FlashBars fbars{q_full, q_empty, k_full, k_empty, v_full, v_empty, s_full, p_full, o_done};
 
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // warp index through a shuffle: the compiler then treats it as uniform
+  // across the warp, so the whole-warp MMA issuer below keeps its addresses
+  // and descriptors in uniform registers
+  const int warp = __shfl_sync(0xffffffffu, (int)(threadIdx.x >> 5), 0), lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
       mbar_init(&q_full[s], 1); mbar_init(&q_empty[s], 1);
@@ -135,144 +384,30 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
-  griddep_wait_and_release();
-
+  const uint32_t tmem_base = __shfl_sync(0xffffffffu, *tmem_slot, 0);
+  // Each warpgroup takes its register share (all threads of a warpgroup
+  // execute it).  The two roles stay in separate branches up to the final
+  // barrier, so the register limit of one never applies to the other's code.
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kFlashLowRegs));
+    griddep_wait_and_release();
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
-    if (lane == 0) {
-      int ks = 0, vs = 0;
-      uint32_t kph = 0, vph = 0, qph[2] = {0, 0};
-      bool ok = true;
-      uint32_t kiss = 0, kpar = 0, viss = 0, vpar = 0, qiss = 0, qpar = 0;
-      for (int k_ = 0, u = flash_snake(0); u < fs.units && ok; u = flash_snake(++k_)) {
-        int b, g, pair, qt;
-        flash_unit(fs, u, b, g, pair, qt);
-        const int nt = flash_ntiles(fs, qt);
-        const bool has1 = pair * 2 + 1 < fs.n_rep;
-        for (int s = 0; s < 2 && ok; ++s) {
-          if (s == 1 && !has1) break;
-          if (!mbar_wait(&q_empty[s], qph[s] ^ 1u, wait_ns)) { ok = false; break; }
-          mbar_arrive_expect_tx(&q_full[s], C::Q_BYTES);
-          const int h = g * fs.n_rep + pair * 2 + s;
-          for (int c = 0; c < C::CHUNKS; ++c)
-            tma_load_4d(smem + C::OFF_Q + s * C::Q_BYTES + c * C::TILE_BYTES, &mapQ, &q_full[s], c * 64, h,
-                        qt * 128, b);
-          qiss |= 1u << s; qpar = (qpar & ~(1u << s)) | (qph[s] << s);
-          qph[s] ^= 1u;
-        }
-        const int jt0 = flash_first_tile(fs, b, qt);
-        for (int j = jt0; j < nt && ok; ++j) {
-          if (!mbar_wait(&k_empty[ks], kph ^ 1u, wait_ns)) { ok = false; break; }
-          mbar_arrive_expect_tx(&k_full[ks], C::KV_BYTES);
-          for (int c = 0; c < C::CHUNKS; ++c)
-            tma_load_4d(smem + C::OFF_K + ks * C::KV_BYTES + c * C::TILE_BYTES, &mapK, &k_full[ks], c * 64, g,
-                        j * 128, b);
-          kiss |= 1u << ks; kpar = (kpar & ~(1u << ks)) | (kph << ks);
-          if (++ks == C::KST) { ks = 0; kph ^= 1u; }
-          if (!mbar_wait(&v_empty[vs], vph ^ 1u, wait_ns)) { ok = false; break; }
-          mbar_arrive_expect_tx(&v_full[vs], C::KV_BYTES);
-          for (int c = 0; c < C::CHUNKS; ++c)
-            tma_load_4d(smem + C::OFF_V + vs * C::KV_BYTES + c * C::TILE_BYTES, &mapV, &v_full[vs], c * 64, g,
-                        j * 128, b);
-          viss |= 1u << vs; vpar = (vpar & ~(1u << vs)) | (vph << vs);
-          if (++vs == C::VST) { vs = 0; vph ^= 1u; }
-        }
-      }
-      for (int s = 0; s < 2; ++s)
-        if (qiss & (1u << s)) mbar_wait(&q_full[s], (qpar >> s) & 1u, wait_ns);
-      for (int s = 0; s < C::KST; ++s)
-        if (kiss & (1u << s)) mbar_wait(&k_full[s], (kpar >> s) & 1u, wait_ns);
-      for (int s = 0; s < C::VST; ++s)
-        if (viss & (1u << s)) mbar_wait(&v_full[s], (vpar >> s) & 1u, wait_ns);
-    }
+    if (lane == 0) flash_produce<HD>(mapQ, mapK, mapV, smem, fbars, fs, wait_ns);
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      int ks = 0, vs = 0;
-      uint32_t kph = 0, vph = 0, qph[2] = {0, 0};
-      uint32_t pph[2] = {0, 0};
-      bool ok = true;
-      const uint32_t q_addr = smem_u32(smem + C::OFF_Q);
-      const uint32_t p_addr = smem_u32(smem + C::OFF_P);
-      auto issue_s = [&](int s, int kst) {
-        const uint32_t d = tmem_base + s * 256;
-        const uint32_t qa = q_addr + s * C::Q_BYTES;
-        const uint32_t ka = smem_u32(smem + C::OFF_K + kst * C::KV_BYTES);
-#pragma unroll
-        for (int k = 0; k < C::KSTEPS_QK; ++k) {
-          const uint32_t off = (k >> 2) * C::TILE_BYTES + (k & 3) * 32;
-          tc_mma_f16_ss(d, sw128_desc(qa + off, 1024, 16), sw128_desc(ka + off, 1024, 16), IDESC_S, k > 0);
-        }
-        tc_commit(&s_full[s]);
-      };
-      auto issue_pv = [&](int s, int vst, bool accumulate) {
-        const uint32_t d = tmem_base + s * 256 + 128;
-        const uint32_t pa = p_addr + s * C::P_BYTES;
-        const uint32_t va = smem_u32(smem + C::OFF_V + vst * C::KV_BYTES);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {   // 128 keys, 16 per MMA
-          const uint64_t adesc = sw128_desc(pa + (k >> 2) * C::TILE_BYTES + (k & 3) * 32, 1024, 16);
-          const uint64_t bdesc = sw128_desc(va + k * 2048, 1024, C::TILE_BYTES);
-          tc_mma_f16_ss(d, adesc, bdesc, IDESC_O, (accumulate || k > 0) ? 1u : 0u);
-        }
-        tc_commit(&o_done[s]);
-      };
-      for (int k_ = 0, u = flash_snake(0); u < fs.units && ok; u = flash_snake(++k_)) {
-        int b, g, pair, qt;
-        flash_unit(fs, u, b, g, pair, qt);
-        const int nt = flash_ntiles(fs, qt);
-        const int nslots = (pair * 2 + 1 < fs.n_rep) ? 2 : 1;
-        for (int s = 0; s < nslots; ++s) {
-          if (!mbar_wait(&q_full[s], qph[s], wait_ns)) ok = false;
-          qph[s] ^= 1u;
-        }
-        if (!ok) break;
-        tc_fence_after();
-        const int jt0 = flash_first_tile(fs, b, qt);
-        // S of the first key tile for every slot
-        if (!mbar_wait(&k_full[ks], kph, wait_ns)) break;
-        tc_fence_after();
-        for (int s = 0; s < nslots; ++s) issue_s(s, ks);
-        tc_commit(&k_empty[ks]);
-        if (++ks == C::KST) { ks = 0; kph ^= 1u; }
-        for (int j = jt0; j < nt && ok; ++j) {
-          if (!mbar_wait(&v_full[vs], vph, wait_ns)) { ok = false; break; }
-          const bool more = j + 1 < nt;
-          bool k_ready = false;
-          for (int s = 0; s < nslots; ++s) {
-            if (!mbar_wait(&p_full[s], pph[s], wait_ns)) { ok = false; break; }
-            pph[s] ^= 1u;
-            tc_fence_after();
-            issue_pv(s, vs, j > jt0);
-            if (more) {
-              // K of the next tile is only needed from here on: P.V above does not wait for it
-              if (!k_ready && !mbar_wait(&k_full[ks], kph, wait_ns)) { ok = false; break; }
-              k_ready = true;
-              tc_fence_after();
-              issue_s(s, ks);
-            }
-          }
-          if (!ok) break;
-          tc_commit(&v_empty[vs]);
-          if (++vs == C::VST) { vs = 0; vph ^= 1u; }
-          if (more) {
-            tc_commit(&k_empty[ks]);
-            if (++ks == C::KST) { ks = 0; kph ^= 1u; }
-          }
-        }
-        for (int s = 0; s < nslots; ++s) tc_commit(&q_empty[s]);
-      }
-    }
-  } else if (warp >= 4) {
-    // ---------------------------------------------------------------- softmax
+    flash_issue_mma<HD>(smem, fbars, tmem_base, fs, wait_ns);
+  }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kFlashHighRegs));
+    griddep_wait_and_release();
+    // ---------------------------------------------------------------- softmax (one thread per row)
     const int slot = (warp - 4) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;            // query row in the tile == TMEM lane
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t s_tmem = tmem_base + lane_off + slot * 256;
     const uint32_t o_tmem = s_tmem + 128;
-    uint8_t* p_smem = smem + C::OFF_P + slot * C::P_BYTES;
     uint32_t sph = 0, oph = 0;
     for (int k_ = 0, u = flash_snake(0); u < fs.units; u = flash_snake(++k_)) {
       int b, g, pair, qt;
@@ -286,40 +421,32 @@ __global__ void __launch_bounds__(384, 1)
       float m_ref = -INFINITY, l = 0.f;
       bool ok = true;
       for (int j = jt0; j < nt; ++j) {
-        if (!mbar_wait(&s_full[slot], sph, wait_ns)) { ok = false; break; }
+        if (!mbar_wait_warp(&s_full[slot], sph, wait_ns)) { ok = false; break; }
         sph ^= 1u;
         tc_fence_after();
         const bool need_mask = j * 128 + 127 > fs.P + qt * 128 || j * 128 < lo_last;
-        // pass 1: row maximum of the raw scores (the next chunk's TMEM load is
-        // in flight while the current one is reduced)
-        float mx = -INFINITY;
-        {
-          uint32_t ra[32], rb[32];
-          tmem_ld32(s_tmem, ra);
-          tc_wait_ld();
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t(&cur)[32] = (c & 1) ? rb : ra;
-            uint32_t(&nxt)[32] = (c & 1) ? ra : rb;
-            if (c + 1 < 4) tmem_ld32(s_tmem + (c + 1) * 32, nxt);
-            if (need_mask) {
-#pragma unroll
-              for (int i = 0; i < 32; ++i)
-                if (j * 128 + c * 32 + i > qpos || j * 128 + c * 32 + i < lo) cur[i] = __float_as_uint(-INFINITY);
-            }
-#pragma unroll
-            for (int i = 0; i < 32; i += 2) mx = max3f(mx, __uint_as_float(cur[i]), __uint_as_float(cur[i + 1]));
-            if (c + 1 < 4) tc_wait_ld();
-          }
+        const int key0 = j * 128;
+        uint32_t ra[32], rb[32], rc[32], rd[32];
+        flash_load_row(s_tmem, ra, rb, rc, rd);
+        float m0, m1, m2, m3;   // four independent chains
+        if (need_mask) {
+          m0 = flash_row_max<true>(ra, key0, qpos, lo);
+          m1 = flash_row_max<true>(rb, key0 + 32, qpos, lo);
+          m2 = flash_row_max<true>(rc, key0 + 64, qpos, lo);
+          m3 = flash_row_max<true>(rd, key0 + 96, qpos, lo);
+        } else {
+          m0 = flash_row_max<false>(ra, key0, qpos, lo);
+          m1 = flash_row_max<false>(rb, key0 + 32, qpos, lo);
+          m2 = flash_row_max<false>(rc, key0 + 64, qpos, lo);
+          m3 = flash_row_max<false>(rd, key0 + 96, qpos, lo);
         }
+        const float mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
         const float m_tile = mx * fs.scale_log2;   // scale_log2 > 0: max commutes with the scale
-        // the O written by the previous tile's P.V must be complete before P
-        // (single buffer) is overwritten or O is rescaled
-        if (j > jt0) {
-          if (!mbar_wait(&o_done[slot], oph, wait_ns)) { ok = false; break; }
-          oph ^= 1u;
-          tc_fence_after();
-        }
+        // The previous tile's P.V is complete here: the s_full commit just
+        // waited for tracks every MMA issued before it, that P.V included.
+        // So O may be rescaled without waiting on o_done; only its phase is
+        // counted (one per P.V), for the epilogue's wait on the last one.
+        if (j > jt0) oph ^= 1u;
         const bool grow = m_tile > m_ref + 8.0f;
         float alpha = 1.f;
         if (grow) {
@@ -327,84 +454,31 @@ __global__ void __launch_bounds__(384, 1)
           l *= alpha;
           m_ref = m_tile;
         }
-        // rescale this warp's rows of O in TMEM when any of them grew (the
-        // TMEM accesses are warp-collective; rows that did not grow use 1)
         if (j > jt0 && __any_sync(0xffffffffu, grow)) {
 #pragma unroll 1
           for (int c = 0; c < HD / 16; ++c) {
-            uint32_t r[16];
-            tmem_ld16(o_tmem + c * 16, r);
+            uint32_t o[16];
+            tmem_ld16(o_tmem + c * 16, o);
             tc_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            tmem_st16(o_tmem + c * 16, r);
+            for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st16(o_tmem + c * 16, o);
           }
           tc_wait_st();
         }
-        // pass 2: p = 2^(s*scale - m_ref), row sum, bf16 P into shared memory
-        // (again with the next chunk's TMEM load overlapping this chunk's math)
         const float scl = fs.scale_log2;
         const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;   // a row with no visible key yet: p = 0
-        float sum_a = 0.f, sum_b = 0.f;
-        {
-          uint32_t ra[32], rb[32];
-          tmem_ld32(s_tmem, ra);
-          tc_wait_ld();
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t(&r)[32] = (c & 1) ? rb : ra;
-            uint32_t(&nxt)[32] = (c & 1) ? ra : rb;
-            if (c + 1 < 4) tmem_ld32(s_tmem + (c + 1) * 32, nxt);
-            if (need_mask) {
-#pragma unroll
-              for (int i = 0; i < 32; ++i)
-                if (j * 128 + c * 32 + i > qpos || j * 128 + c * 32 + i < lo) r[i] = __float_as_uint(-INFINITY);
-            }
-            uint32_t pk[16];
-            if (need_mask) {   // masked keys must give exactly 0: MUFU path only
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                float x0, x1;
-                fma2(x0, x1, __uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), scl, scl, neg_m, neg_m);
-                const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-                add2(sum_a, sum_b, p0, p1);
-                pk[i] = pack_bf16x2(p0, p1);
-              }
-            } else {           // 6 of every 16 pairs on the FMA pipe, the rest on MUFU
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                float x0, x1, p0, p1;
-                fma2(x0, x1, __uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), scl, scl, neg_m, neg_m);
-                if ((i & 7) < 3) {
-                  exp2_poly2(x0, x1, p0, p1);
-                } else {
-                  p0 = ex2_approx(x0);
-                  p1 = ex2_approx(x1);
-                }
-                add2(sum_a, sum_b, p0, p1);
-                pk[i] = pack_bf16x2(p0, p1);
-              }
-            }
-            // chunk c covers keys 32c..32c+31: slab c/2, 16-byte pieces (c%2)*4 .. +3
-            uint8_t* slab = p_smem + (c >> 1) * C::TILE_BYTES + row * 128;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int piece = (c & 1) * 4 + q;
-              *reinterpret_cast<uint4*>(slab + ((piece ^ (row & 7)) << 4)) =
-                  make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-            }
-            if (c + 1 < 4) tc_wait_ld();
-          }
-        }
-        const float sum = sum_a + sum_b;
-        l += sum;
-        fence_proxy_async_smem();
+        if (need_mask)
+          l += flash_exp_row<true>(ra, rb, rc, rd, scl, neg_m, s_tmem);
+        else
+          l += flash_exp_row<false>(ra, rb, rc, rd, scl, neg_m, s_tmem);
+        tc_wait_st();
         tc_fence_before();
         mbar_arrive(&p_full[slot]);
       }
       if (!ok) break;
       // epilogue: wait for the last P.V, out = O / l
-      if (!mbar_wait(&o_done[slot], oph, wait_ns)) break;
+      if (!mbar_wait_warp(&o_done[slot], oph, wait_ns)) break;
       oph ^= 1u;
       tc_fence_after();
       const int t = qt * 128 + row;

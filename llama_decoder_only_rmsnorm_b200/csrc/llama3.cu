@@ -16,22 +16,16 @@
 #include "common.cuh"
 #include "decode_attention.cuh"
 #include "flash_attention.cuh"
-#include "flash_attention2.cuh"
-#include "flash_attention3.cuh"
-#include "flash_attention4.cuh"
-#include "flash_attention5.cuh"
 #include "sampling.cuh"
 #include "simt.cuh"
 #include "tc_gemm.cuh"
-#include "tc_gemm_pair.cuh"
 
 using namespace l3;
 
 namespace {
 
 thread_local int t_last_cuda = 0;
-int g_kernel_path = 0;       // 0 = tcgen05 for bf16, 1 = SIMT everywhere,
-                             // 2 = tcgen05 with CTA-pair prefill GEMMs
+int g_kernel_path = 0;       // 0 = tcgen05 for bf16, 1 = SIMT everywhere
 int g_wait_ms = 2000;        // bounded device waits
 constexpr int kMaxDevices = 64;
 int g_num_sms[kMaxDevices];
@@ -94,12 +88,6 @@ void timer_end(int kind, cudaStream_t st) {
 // touches memory.  g_pdl = false launches them the ordinary way.
 bool g_pdl = true;
 
-// Prefill attention kernel design (see the flash_attention*.cuh headers):
-// 1 = one softmax thread per row, P through shared memory; 2 = two softmax
-// threads per row, P in TMEM; 3 = one thread per row with the whole tile row in
-// registers (register split), P in TMEM; 4 = as 3 with P in shared memory.
-int g_flash_variant = 3;
-
 template <typename... KArgs, typename... Args>
 cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
                      Args... args) {
@@ -141,7 +129,6 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 size_t esize(const llama3_config* c) { return c->dtype == LLAMA3_DTYPE_F32 ? 4 : 2; }
 
 bool use_tc(const llama3_config* c) { return c->dtype == LLAMA3_DTYPE_BF16 && g_kernel_path != 1; }
-bool use_pair_gemm(int m) { return g_kernel_path == 2 && m >= 256; }
 
 int check_config(const llama3_config* c) {
   if (!c) return LLAMA3_ERR_ARG;
@@ -230,7 +217,7 @@ bool flash_attention_supported(int hd, int H, int KV) {
   return hd == 64 || hd == 96 || hd == 128;
 }
 
-template <int HD, int VARIANT>
+template <int HD>
 int run_flash_attention_t(int H, int KV, const void* q, const void* kc, const void* vc, int cap, int B, int S,
                           int P, void* out, const int32_t* doc_start, int sms, unsigned long long wns,
                           cudaStream_t st) {
@@ -248,58 +235,35 @@ int run_flash_attention_t(int H, int KV, const void* q, const void* kc, const vo
   fs.ldo = H * HD;
   fs.scale_log2 = (float)(1.4426950408889634 / sqrt((double)HD));
   fs.doc_start = doc_start;
-  constexpr int smem = VARIANT == 5 ? Flash5Cfg<HD>::SMEM_BYTES
-                     : VARIANT == 4 ? Flash4Cfg<HD>::SMEM_BYTES
-                     : VARIANT == 3 ? Flash3Cfg<HD>::SMEM_BYTES
-                     : VARIANT == 2 ? Flash2Cfg<HD>::SMEM_BYTES : FlashCfg<HD>::SMEM_BYTES;
-  constexpr int threads = VARIANT >= 3 ? kFlash3Threads : VARIANT == 2 ? 640 : 384;
-  auto kern = VARIANT == 5 ? flash_attention5_kernel<HD>
-            : VARIANT == 4 ? flash_attention4_kernel<HD>
-            : VARIANT == 3 ? flash_attention3_kernel<HD>
-            : VARIANT == 2 ? flash_attention2_kernel<HD> : flash_attention_kernel<HD>;
+  constexpr int smem = FlashCfg<HD>::SMEM_BYTES;
+  auto kern = flash_attention_kernel<HD>;
   int dev = 0;
   L3_TRY(current_device(&dev));
   static bool attr_done[kMaxDevices];
   static bool regs_ok[kMaxDevices];
   if (!attr_done[dev]) {
     L3_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-    if (VARIANT >= 3) {
-      // The warpgroups' setmaxnreg shares must fit the registers the block is
-      // launched with, or the raising warpgroups would wait for ever.
-      cudaFuncAttributes fa;
-      L3_CUDA(cudaFuncGetAttributes(&fa, kern));
-      regs_ok[dev] = (long long)fa.numRegs * kFlash3Threads >= 128LL * kFlash3LowRegs + 256LL * kFlash3HighRegs;
-    }
+    // The warpgroups' setmaxnreg shares must fit the registers the block is
+    // launched with, or the raising warpgroups would wait for ever.
+    cudaFuncAttributes fa;
+    L3_CUDA(cudaFuncGetAttributes(&fa, kern));
+    regs_ok[dev] = (long long)fa.numRegs * kFlashThreads >= 128LL * kFlashLowRegs + 256LL * kFlashHighRegs;
     attr_done[dev] = true;
   }
-  if (VARIANT >= 3 && !regs_ok[dev]) return LLAMA3_ERR_UNSUPPORTED;
+  if (!regs_ok[dev]) return LLAMA3_ERR_UNSUPPORTED;
   const int grid = std::min(fs.units, sms);
-  L3_LAUNCH(LLAMA3_KERNEL_ATTENTION, st, launch_k(kern, grid, threads, smem, st, mq, mk, mv, (bf16*)out, fs, wns));
+  L3_LAUNCH(LLAMA3_KERNEL_ATTENTION, st,
+            launch_k(kern, grid, kFlashThreads, smem, st, mq, mk, mv, (bf16*)out, fs, wns));
   return launch_check();
-}
-
-template <int HD>
-int run_flash_attention_v(int H, int KV, const void* q, const void* kc, const void* vc, int cap, int B, int S,
-                          int P, void* out, const int32_t* doc_start, int sms, unsigned long long wns,
-                          cudaStream_t st) {
-  if (g_flash_variant == 5)
-    return run_flash_attention_t<HD, 5>(H, KV, q, kc, vc, cap, B, S, P, out, doc_start, sms, wns, st);
-  if (g_flash_variant == 4)
-    return run_flash_attention_t<HD, 4>(H, KV, q, kc, vc, cap, B, S, P, out, doc_start, sms, wns, st);
-  if (g_flash_variant == 3)
-    return run_flash_attention_t<HD, 3>(H, KV, q, kc, vc, cap, B, S, P, out, doc_start, sms, wns, st);
-  if (g_flash_variant == 2)
-    return run_flash_attention_t<HD, 2>(H, KV, q, kc, vc, cap, B, S, P, out, doc_start, sms, wns, st);
-  return run_flash_attention_t<HD, 1>(H, KV, q, kc, vc, cap, B, S, P, out, doc_start, sms, wns, st);
 }
 
 int run_flash_attention(int hd, int H, int KV, const void* q, const void* kc, const void* vc, int cap, int B, int S,
                         int P, void* out, const int32_t* doc_start, int sms, unsigned long long wns,
                         cudaStream_t st) {
   switch (hd) {
-    case 64: return run_flash_attention_v<64>(H, KV, q, kc, vc, cap, B, S, P, out, doc_start, sms, wns, st);
-    case 96: return run_flash_attention_v<96>(H, KV, q, kc, vc, cap, B, S, P, out, doc_start, sms, wns, st);
-    case 128: return run_flash_attention_v<128>(H, KV, q, kc, vc, cap, B, S, P, out, doc_start, sms, wns, st);
+    case 64: return run_flash_attention_t<64>(H, KV, q, kc, vc, cap, B, S, P, out, doc_start, sms, wns, st);
+    case 96: return run_flash_attention_t<96>(H, KV, q, kc, vc, cap, B, S, P, out, doc_start, sms, wns, st);
+    case 128: return run_flash_attention_t<128>(H, KV, q, kc, vc, cap, B, S, P, out, doc_start, sms, wns, st);
     default: return LLAMA3_ERR_UNSUPPORTED;
   }
 }
@@ -441,48 +405,6 @@ int launch_gemm(int kind, const CUtensorMap& a, const CUtensorMap& a2, const CUt
   if (sh.units <= 0) return LLAMA3_OK;
   const int grid = std::min(sh.units, num_sms());
   L3_LAUNCH(kind, st, launch_k(kern, grid, 192, Cfg::SMEM_BYTES, st, a, a2, b, b2, sh, ep, wait_ns()));
-  return launch_check();
-}
-
-// Prefill GEMM tile shape for CTA pairs: 256-row tiles of A.
-GemmShape make_shape_pair(int rows_a, int rows_b, int k, int bn) {
-  GemmShape s = make_shape(rows_a, 0, rows_b, k, bn, 1);
-  s.tiles_m1 = s.tiles_m = (rows_a + 255) / 256;
-  s.units = s.tiles_m * s.tiles_n;
-  s.group_m = std::max(1, std::min(8, s.tiles_m));
-  return s;
-}
-
-template <int BN, int STAGES, int EPI, bool DUAL>
-int launch_gemm_pair(int kind, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2,
-                     const GemmShape& sh, const EpiParams& ep, cudaStream_t st) {
-  using Cfg = TcGemmPairCfg<BN, STAGES, DUAL>;
-  auto kern = tc_gemm_pair_kernel<BN, STAGES, EPI, DUAL>;
-  int dev = 0;
-  L3_TRY(current_device(&dev));
-  static bool attr_done[kMaxDevices];
-  if (!attr_done[dev]) {
-    L3_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES));
-    attr_done[dev] = true;
-  }
-  if (sh.units <= 0) return LLAMA3_OK;
-  const int pairs = std::min(sh.units, std::max(1, num_sms() / 2));
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * pairs);
-  cfg.blockDim = dim3(192);
-  cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = g_pdl ? 2 : 1;
-  const unsigned long long wns = wait_ns();
-  L3_LAUNCH(kind, st, cudaLaunchKernelEx(&cfg, kern, a, b, b2, sh, ep, wns));
   return launch_check();
 }
 
@@ -749,19 +671,15 @@ int layer_tc_prefill(const llama3_config* c, const llama3_layer_weights* w, cons
   bf16* o = ws_at<bf16>(ws, L.o);
   bf16* g = ws_at<bf16>(ws, L.g);
   float* Ap = ws_at<float>(ws, L.attn_part);
-  // CTA-pair GEMMs take B in halves per CTA (box rows BN/2); single-CTA ones whole.
-  const bool pair = use_pair_gemm(M);
-  const int bb = pair ? kPrefillBN / 2 : kPrefillBN;
-  const int bd = pair ? 64 : 128;
   CUtensorMap mxn, mo, mg, mwqkv, mwo, mw1, mw3, mw2;
   L3_TRY(make_map(&mxn, xn, M, D, 128));
   L3_TRY(make_map(&mo, o, M, H * hd, 128));
   L3_TRY(make_map(&mg, g, M, F, 128));
-  L3_TRY(make_map(&mwqkv, w->wqkv, nqkv, D, bb));
-  L3_TRY(make_map(&mwo, w->wo, D, H * hd, bb));
-  L3_TRY(make_map(&mw1, w->w1, F, D, bd));
-  L3_TRY(make_map(&mw3, w->w3, F, D, bd));
-  L3_TRY(make_map(&mw2, w->w2, D, F, bb));
+  L3_TRY(make_map(&mwqkv, w->wqkv, nqkv, D, kPrefillBN));
+  L3_TRY(make_map(&mwo, w->wo, D, H * hd, kPrefillBN));
+  L3_TRY(make_map(&mw1, w->w1, F, D, 128));
+  L3_TRY(make_map(&mw3, w->w3, F, D, 128));
+  L3_TRY(make_map(&mw2, w->w2, D, F, kPrefillBN));
 
   // attention half
   L3_TRY(rmsnorm_any(c, x, D, w->attention_norm, xn, M, st));
@@ -769,45 +687,29 @@ int layer_tc_prefill(const llama3_config* c, const llama3_layer_weights* w, cons
     EpiParams ep = empty_epi();
     ep.seq = S; ep.start_pos = P; ep.n_heads = H; ep.n_kv = KV; ep.head_dim = hd; ep.cache_cap = cap;
     ep.rope = rope; ep.q_out = q; ep.k_cache = kc; ep.v_cache = vc;
-    if (pair)
-      L3_TRY((launch_gemm_pair<kPrefillBN, 6, EPI_QKV_ROPE, false>(
-          LLAMA3_KERNEL_GEMM_QKV, mxn, mwqkv, mwqkv, make_shape_pair(M, nqkv, D, kPrefillBN), ep, st)));
-    else
-      L3_TRY((launch_gemm<kPrefillBN, 4, EPI_QKV_ROPE, false>(LLAMA3_KERNEL_GEMM_QKV, mxn, mxn, mwqkv, mwqkv,
-                                                               make_shape(M, 0, nqkv, D, kPrefillBN, 1), ep, st)));
+    L3_TRY((launch_gemm<kPrefillBN, 4, EPI_QKV_ROPE, false>(LLAMA3_KERNEL_GEMM_QKV, mxn, mxn, mwqkv, mwqkv,
+                                                             make_shape(M, 0, nqkv, D, kPrefillBN, 1), ep, st)));
   }
   L3_TRY(attention_dispatch(c, q, kc, vc, cap, B, S, P, o, Ap, st, doc_start));
   {
     EpiParams ep = empty_epi();
     ep.out = x; ep.res = x; ep.ldo = D;
-    if (pair)
-      L3_TRY((launch_gemm_pair<kPrefillBN, 6, EPI_RESIDUAL, false>(
-          LLAMA3_KERNEL_GEMM_WO, mo, mwo, mwo, make_shape_pair(M, D, H * hd, kPrefillBN), ep, st)));
-    else
-      L3_TRY((launch_gemm<kPrefillBN, 4, EPI_RESIDUAL, false>(LLAMA3_KERNEL_GEMM_WO, mo, mo, mwo, mwo,
-                                                               make_shape(M, 0, D, H * hd, kPrefillBN, 1), ep, st)));
+    L3_TRY((launch_gemm<kPrefillBN, 4, EPI_RESIDUAL, false>(LLAMA3_KERNEL_GEMM_WO, mo, mo, mwo, mwo,
+                                                             make_shape(M, 0, D, H * hd, kPrefillBN, 1), ep, st)));
   }
   // FFN half
   L3_TRY(rmsnorm_any(c, x, D, w->ffn_norm, xn, M, st));
   {
     EpiParams ep = empty_epi();
     ep.out = g; ep.ldo = F;
-    if (pair)
-      L3_TRY((launch_gemm_pair<128, 6, EPI_SWIGLU, true>(LLAMA3_KERNEL_GEMM_W13, mxn, mw1, mw3,
-                                                          make_shape_pair(M, F, D, 128), ep, st)));
-    else
-      L3_TRY((launch_gemm<128, 4, EPI_SWIGLU, true>(LLAMA3_KERNEL_GEMM_W13, mxn, mxn, mw1, mw3,
-                                                     make_shape(M, 0, F, D, 128, 1), ep, st)));
+    L3_TRY((launch_gemm<128, 4, EPI_SWIGLU, true>(LLAMA3_KERNEL_GEMM_W13, mxn, mxn, mw1, mw3,
+                                                   make_shape(M, 0, F, D, 128, 1), ep, st)));
   }
   {
     EpiParams ep = empty_epi();
     ep.out = x; ep.res = x; ep.ldo = D;
-    if (pair)
-      L3_TRY((launch_gemm_pair<kPrefillBN, 6, EPI_RESIDUAL, false>(
-          LLAMA3_KERNEL_GEMM_W2, mg, mw2, mw2, make_shape_pair(M, D, F, kPrefillBN), ep, st)));
-    else
-      L3_TRY((launch_gemm<kPrefillBN, 4, EPI_RESIDUAL, false>(LLAMA3_KERNEL_GEMM_W2, mg, mg, mw2, mw2,
-                                                               make_shape(M, 0, D, F, kPrefillBN, 1), ep, st)));
+    L3_TRY((launch_gemm<kPrefillBN, 4, EPI_RESIDUAL, false>(LLAMA3_KERNEL_GEMM_W2, mg, mg, mw2, mw2,
+                                                             make_shape(M, 0, D, F, kPrefillBN, 1), ep, st)));
   }
   return LLAMA3_OK;
 }
@@ -895,6 +797,64 @@ int check_layer_args(const llama3_config* c, const llama3_layer_weights* w, cons
   return LLAMA3_OK;
 }
 
+// Argument checks shared by both LM-head entry points.
+int check_lm_head_args(const llama3_config* cfg, const void* norm_w, const void* w_out, const void* h, int rows,
+                       long long row_stride, const int32_t* ids_out, const float* logits_out) {
+  L3_TRY(check_config(cfg));
+  if (!norm_w || !w_out || !h || !ids_out || rows < 1 || cfg->vocab < 1 || row_stride < cfg->dim)
+    return LLAMA3_ERR_ARG;
+  if (!aligned16(norm_w) || !aligned16(w_out) || !aligned16(h) || !aligned16(ids_out) ||
+      (logits_out && !aligned16(logits_out)))
+    return LLAMA3_ERR_ALIGN;
+  if ((row_stride * (long long)esize(cfg)) % 16) return LLAMA3_ERR_ALIGN;
+  return LLAMA3_OK;
+}
+
+// Final RMSNorm -> logits -> argmax of `rows` rows, with its scratch where the
+// caller of this helper chose: hn (rows x dim elements, 16-byte aligned) for
+// the normalised rows and keys (rows 64-bit words) for the packed per-row
+// maxima.  The keys are re-initialised here on every call.
+int lm_head_run(const llama3_config* cfg, const void* norm_w, const void* w_out, const void* h, int rows,
+                long long row_stride, int32_t* ids_out, float* logits_out, void* hn, unsigned long long* keys,
+                cudaStream_t st) {
+  const int V = cfg->vocab, D = cfg->dim;
+  L3_TRY(rmsnorm_any(cfg, h, row_stride, norm_w, hn, rows, st));
+  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st,
+            launch_k((argmax_init_kernel), blocks_for(rows, 256), 256, 0, st, keys, rows));
+  L3_TRY(launch_check());
+  if (use_tc(cfg)) {
+    const int bn = rows <= 16 ? 16 : rows <= 32 ? 32 : rows <= 64 ? 64 : rows <= 128 ? 128 : 256;
+    CUtensorMap ma, mb;
+    L3_TRY(make_map(&ma, w_out, V, D, 128));
+    L3_TRY(make_map(&mb, hn, rows, D, bn));
+    GemmShape sh = make_shape(V, 0, rows, D, bn, 1);
+    EpiParams ep = empty_epi();
+    ep.logits = logits_out;
+    ep.keys = keys;
+    switch (bn) {
+      case 16: L3_TRY((launch_gemm<16, 8, EPI_ARGMAX, false>(LLAMA3_KERNEL_LM_HEAD, ma, ma, mb, mb, sh, ep, st))); break;
+      case 32: L3_TRY((launch_gemm<32, 8, EPI_ARGMAX, false>(LLAMA3_KERNEL_LM_HEAD, ma, ma, mb, mb, sh, ep, st))); break;
+      case 64: L3_TRY((launch_gemm<64, 6, EPI_ARGMAX, false>(LLAMA3_KERNEL_LM_HEAD, ma, ma, mb, mb, sh, ep, st))); break;
+      case 128: L3_TRY((launch_gemm<128, 5, EPI_ARGMAX, false>(LLAMA3_KERNEL_LM_HEAD, ma, ma, mb, mb, sh, ep, st))); break;
+      default: L3_TRY((launch_gemm<256, 4, EPI_ARGMAX, false>(LLAMA3_KERNEL_LM_HEAD, ma, ma, mb, mb, sh, ep, st))); break;
+    }
+  } else {
+    const long long warps = (long long)rows * ((V + 31) / 32);
+    if (cfg->dtype == LLAMA3_DTYPE_F32)
+      L3_LAUNCH(LLAMA3_KERNEL_LM_HEAD, st,
+                launch_k((lm_head_simt_kernel<float>), blocks_for(warps * 32, 256), 256, 0, st, (const float*)hn,
+                         (const float*)w_out, logits_out, keys, rows, V, D));
+    else
+      L3_LAUNCH(LLAMA3_KERNEL_LM_HEAD, st,
+                launch_k((lm_head_simt_kernel<bf16>), blocks_for(warps * 32, 256), 256, 0, st, (const bf16*)hn,
+                         (const bf16*)w_out, logits_out, keys, rows, V, D));
+    L3_TRY(launch_check());
+  }
+  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st,
+            launch_k((argmax_finalize_kernel), blocks_for(rows, 256), 256, 0, st, keys, ids_out, rows));
+  return launch_check();
+}
+
 }  // namespace
 
 // ===========================================================================
@@ -938,7 +898,7 @@ unsigned long long llama3_launch_count(void) { return g_launches.load(); }
 
 int llama3_set_kernel_path(int path) {
   int old = g_kernel_path;
-  g_kernel_path = (path >= 0 && path <= 2) ? path : 0;
+  g_kernel_path = (path == 1) ? 1 : 0;
   return old;
 }
 
@@ -987,23 +947,21 @@ int llama3_gather_rows(const llama3_config* cfg, const void* x, long long row_st
   return launch_check();
 }
 
-int llama3_generation_advance(int32_t* positions, const int32_t* ids, int32_t* history, int32_t* step, int batch,
-                              int history_rows, long long history_stride, llama3_stream_t stream) {
+int llama3_generation_advance(int32_t* positions, int32_t* ids, int32_t* history, int32_t* step, int32_t* done,
+                              int eos_id, int batch, int history_rows, long long history_stride,
+                              llama3_stream_t stream) {
   if (!positions || !ids || !history || !step || batch < 1 || history_rows < 1 || history_stride < batch)
     return LLAMA3_ERR_ARG;
+  if (eos_id >= 0 && !done) return LLAMA3_ERR_ARG;
   const uintptr_t any = reinterpret_cast<uintptr_t>(positions) | reinterpret_cast<uintptr_t>(ids) |
-                        reinterpret_cast<uintptr_t>(history) | reinterpret_cast<uintptr_t>(step);
+                        reinterpret_cast<uintptr_t>(history) | reinterpret_cast<uintptr_t>(step) |
+                        reinterpret_cast<uintptr_t>(done);
   if (any & 3) return LLAMA3_ERR_ALIGN;
   cudaStream_t st = (cudaStream_t)stream;
+  int32_t* d = eos_id >= 0 ? done : nullptr;
   L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k(generation_advance_kernel, 1, 256, 0, st, positions, ids, history,
-                                                    step, batch, history_rows, history_stride));
+                                                    step, d, eos_id, batch, history_rows, history_stride));
   return launch_check();
-}
-
-int llama3_set_flash_variant(int variant) {
-  const int old = g_flash_variant;
-  g_flash_variant = (variant >= 1 && variant <= 5) ? variant : 3;
-  return old;
 }
 
 int llama3_set_programmatic_launch(int on) {
@@ -1087,14 +1045,6 @@ int llama3_linear(const llama3_config* cfg, const void* x, const void* w, const 
     CUtensorMap ma, mb;
     EpiParams ep = empty_epi();
     ep.out = y; ep.res = residual; ep.ldo = n;
-    if (use_pair_gemm(m)) {
-      L3_TRY(make_map(&ma, x, m, k, 128));
-      L3_TRY(make_map(&mb, w, n, k, kPrefillBN / 2));
-      const GemmShape sp = make_shape_pair(m, n, k, kPrefillBN);
-      if (residual)
-        return launch_gemm_pair<kPrefillBN, 6, EPI_RESIDUAL, false>(LLAMA3_KERNEL_GEMM_WO, ma, mb, mb, sp, ep, st);
-      return launch_gemm_pair<kPrefillBN, 6, EPI_STORE, false>(LLAMA3_KERNEL_GEMM_WO, ma, mb, mb, sp, ep, st);
-    }
     L3_TRY(make_map(&ma, x, m, k, 128));
     L3_TRY(make_map(&mb, w, n, k, kPrefillBN));
     GemmShape sh = make_shape(m, 0, n, k, kPrefillBN, 1);
@@ -1240,51 +1190,12 @@ int llama3_attention_docs(const llama3_config* cfg, const void* q, const void* k
 int llama3_lm_head_argmax(const llama3_config* cfg, const void* norm_w, const void* w_out, const void* h, int rows,
                           long long row_stride, int32_t* ids_out, float* logits_out, void* ws, size_t ws_bytes,
                           llama3_stream_t stream) {
-  L3_TRY(check_config(cfg));
-  if (!norm_w || !w_out || !h || !ids_out || rows < 1 || cfg->vocab < 1 || row_stride < cfg->dim)
-    return LLAMA3_ERR_ARG;
-  if (!aligned16(norm_w) || !aligned16(w_out) || !aligned16(h) || !aligned16(ids_out) ||
-      (logits_out && !aligned16(logits_out)))
-    return LLAMA3_ERR_ALIGN;
-  if ((row_stride * (long long)esize(cfg)) % 16) return LLAMA3_ERR_ALIGN;
+  L3_TRY(check_lm_head_args(cfg, norm_w, w_out, h, rows, row_stride, ids_out, logits_out));
   Workspace L = layout(cfg, 1, 1, rows);
   if (!ws || ws_bytes < L.total) return LLAMA3_ERR_WORKSPACE;
   if (!aligned16(ws)) return LLAMA3_ERR_ALIGN;
-  cudaStream_t st = (cudaStream_t)stream;
-  void* hn = ws_at<void>(ws, L.lm_rows);
-  unsigned long long* keys = ws_at<unsigned long long>(ws, L.keys);
-  const int V = cfg->vocab, D = cfg->dim;
-  L3_TRY(rmsnorm_any(cfg, h, row_stride, norm_w, hn, rows, st));
-  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((argmax_init_kernel), blocks_for(rows, 256), 256, 0, st, keys, rows));
-  L3_TRY(launch_check());
-  if (use_tc(cfg)) {
-    const int bn = rows <= 16 ? 16 : rows <= 32 ? 32 : rows <= 64 ? 64 : rows <= 128 ? 128 : 256;
-    CUtensorMap ma, mb;
-    L3_TRY(make_map(&ma, w_out, V, D, 128));
-    L3_TRY(make_map(&mb, hn, rows, D, bn));
-    GemmShape sh = make_shape(V, 0, rows, D, bn, 1);
-    EpiParams ep = empty_epi();
-    ep.logits = logits_out;
-    ep.keys = keys;
-    switch (bn) {
-      case 16: L3_TRY((launch_gemm<16, 8, EPI_ARGMAX, false>(LLAMA3_KERNEL_LM_HEAD, ma, ma, mb, mb, sh, ep, st))); break;
-      case 32: L3_TRY((launch_gemm<32, 8, EPI_ARGMAX, false>(LLAMA3_KERNEL_LM_HEAD, ma, ma, mb, mb, sh, ep, st))); break;
-      case 64: L3_TRY((launch_gemm<64, 6, EPI_ARGMAX, false>(LLAMA3_KERNEL_LM_HEAD, ma, ma, mb, mb, sh, ep, st))); break;
-      case 128: L3_TRY((launch_gemm<128, 5, EPI_ARGMAX, false>(LLAMA3_KERNEL_LM_HEAD, ma, ma, mb, mb, sh, ep, st))); break;
-      default: L3_TRY((launch_gemm<256, 4, EPI_ARGMAX, false>(LLAMA3_KERNEL_LM_HEAD, ma, ma, mb, mb, sh, ep, st))); break;
-    }
-  } else {
-    const long long warps = (long long)rows * ((V + 31) / 32);
-    if (cfg->dtype == LLAMA3_DTYPE_F32)
-      L3_LAUNCH(LLAMA3_KERNEL_LM_HEAD, st, launch_k((lm_head_simt_kernel<float>), blocks_for(warps * 32, 256), 256, 0, st, (const float*)hn, (const float*)w_out,
-                                                                               logits_out, keys, rows, V, D));
-    else
-      L3_LAUNCH(LLAMA3_KERNEL_LM_HEAD, st, launch_k((lm_head_simt_kernel<bf16>), blocks_for(warps * 32, 256), 256, 0, st, (const bf16*)hn, (const bf16*)w_out,
-                                                                              logits_out, keys, rows, V, D));
-    L3_TRY(launch_check());
-  }
-  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((argmax_finalize_kernel), blocks_for(rows, 256), 256, 0, st, keys, ids_out, rows));
-  return launch_check();
+  return lm_head_run(cfg, norm_w, w_out, h, rows, row_stride, ids_out, logits_out, ws_at<void>(ws, L.lm_rows),
+                     ws_at<unsigned long long>(ws, L.keys), (cudaStream_t)stream);
 }
 
 }  // extern "C"
@@ -1292,28 +1203,67 @@ int llama3_lm_head_argmax(const llama3_config* cfg, const void* norm_w, const vo
 // ===========================================================================
 // LM head without a caller workspace: scratch in a fixed device global.
 // ===========================================================================
-// Callers that cannot supply device memory use this 4 MiB array instead of a
-// workspace.  It exists on every device that loads the library.  Host code
-// must not use the symbol as a pointer: its device address is looked up once
-// per device with cudaGetSymbolAddress and cached in g_noalloc_addr.
+// For callers that cannot hand the library device memory, this 4 MiB array
+// takes the place of the workspace.  It exists on every device that loads the
+// library.  Host code must not use the symbol as a pointer: its device
+// address belongs to the current context and is looked up with
+// cudaGetSymbolAddress.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[LLAMA3_NOALLOC_SCRATCH_BYTES];
 
 namespace {
-void* g_noalloc_addr[kMaxDevices];
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+struct NoallocSlot {
+  CUcontext ctx;   // context the address was looked up in
+  void* addr;
+};
+NoallocSlot g_noalloc[kMaxDevices];
 std::mutex g_noalloc_mu;
 
-// Device address of g_noalloc_scratch on the current device (set-up on first use).
-int noalloc_scratch(void** out) {
+int current_context(CUcontext* ctx) {
+  static CtxGetCurrentFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return (CtxGetCurrentFn) nullptr;
+    return reinterpret_cast<CtxGetCurrentFn>(p);
+  }();
+  if (!fn) return LLAMA3_ERR_CUDA;
+  CUresult r = fn(ctx);
+  if (r != CUDA_SUCCESS) {
+    t_last_cuda = (int)r;
+    return LLAMA3_ERR_CUDA;
+  }
+  return LLAMA3_OK;
+}
+
+// Device address of g_noalloc_scratch in the current context.  Outside a
+// stream capture it is looked up on every call, so a context that was torn
+// down and created again (cudaDeviceReset) gets its own address.  Inside a
+// capture the address cached by an earlier call in the same context is used;
+// without one the call fails instead of looking it up mid-capture.
+int noalloc_scratch(cudaStream_t st, void** out) {
   int dev = 0;
   L3_TRY(current_device(&dev));
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  L3_CUDA(cudaStreamIsCapturing(st, &cs));
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_addr[dev]) {
-    void* p = nullptr;
-    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) return cuda_fail(e);
-    g_noalloc_addr[dev] = p;
+  NoallocSlot& slot = g_noalloc[dev];
+  if (cs != cudaStreamCaptureStatusNone) {
+    CUcontext ctx = nullptr;
+    L3_TRY(current_context(&ctx));
+    if (!slot.addr || slot.ctx != ctx) return LLAMA3_ERR_ARG;
+    *out = slot.addr;
+    return LLAMA3_OK;
   }
-  *out = g_noalloc_addr[dev];
+  // the lookup also makes the device's primary context current
+  void* p = nullptr;
+  L3_CUDA(cudaGetSymbolAddress(&p, g_noalloc_scratch));
+  CUcontext ctx = nullptr;
+  L3_TRY(current_context(&ctx));
+  slot.ctx = ctx;
+  slot.addr = p;
+  *out = p;
   return LLAMA3_OK;
 }
 }  // namespace
@@ -1321,52 +1271,16 @@ int noalloc_scratch(void** out) {
 extern "C" int llama3_lm_head_argmax_noalloc(const llama3_config* cfg, const void* norm_w, const void* w_out,
                                              const void* h, int rows, long long row_stride, int32_t* ids_out,
                                              float* logits_out, llama3_stream_t stream) {
-  L3_TRY(check_config(cfg));
-  if (!norm_w || !w_out || !h || !ids_out || rows < 1 || cfg->vocab < 1 || row_stride < cfg->dim)
-    return LLAMA3_ERR_ARG;
-  if (!aligned16(norm_w) || !aligned16(w_out) || !aligned16(h) || !aligned16(ids_out) ||
-      (logits_out && !aligned16(logits_out)))
-    return LLAMA3_ERR_ALIGN;
-  if ((row_stride * (long long)esize(cfg)) % 16) return LLAMA3_ERR_ALIGN;
+  L3_TRY(check_lm_head_args(cfg, norm_w, w_out, h, rows, row_stride, ids_out, logits_out));
   const size_t keys_bytes = up256((size_t)rows * 8);
   const size_t rows_bytes = (size_t)rows * cfg->dim * esize(cfg);
   if (keys_bytes + rows_bytes > (size_t)LLAMA3_NOALLOC_SCRATCH_BYTES) return LLAMA3_ERR_WORKSPACE;
+  cudaStream_t st = (cudaStream_t)stream;
   void* base = nullptr;
-  L3_TRY(noalloc_scratch(&base));
+  L3_TRY(noalloc_scratch(st, &base));
+  // keys first (the previous call's maxima are overwritten by lm_head_run's
+  // initialisation), then the normalised rows, 256-byte aligned
   unsigned long long* keys = reinterpret_cast<unsigned long long*>(base);
   void* hn = static_cast<char*>(base) + keys_bytes;
-  cudaStream_t st = (cudaStream_t)stream;
-  const int V = cfg->vocab, D = cfg->dim;
-  L3_TRY(rmsnorm_any(cfg, h, row_stride, norm_w, hn, rows, st));
-  // the keys hold the previous call's maxima: start from zero every call
-  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((argmax_init_kernel), blocks_for(rows, 256), 256, 0, st, keys, rows));
-  L3_TRY(launch_check());
-  if (use_tc(cfg)) {
-    const int bn = rows <= 16 ? 16 : rows <= 32 ? 32 : rows <= 64 ? 64 : rows <= 128 ? 128 : 256;
-    CUtensorMap ma, mb;
-    L3_TRY(make_map(&ma, w_out, V, D, 128));
-    L3_TRY(make_map(&mb, hn, rows, D, bn));
-    GemmShape sh = make_shape(V, 0, rows, D, bn, 1);
-    EpiParams ep = empty_epi();
-    ep.logits = logits_out;
-    ep.keys = keys;
-    switch (bn) {
-      case 16: L3_TRY((launch_gemm<16, 8, EPI_ARGMAX, false>(LLAMA3_KERNEL_LM_HEAD, ma, ma, mb, mb, sh, ep, st))); break;
-      case 32: L3_TRY((launch_gemm<32, 8, EPI_ARGMAX, false>(LLAMA3_KERNEL_LM_HEAD, ma, ma, mb, mb, sh, ep, st))); break;
-      case 64: L3_TRY((launch_gemm<64, 6, EPI_ARGMAX, false>(LLAMA3_KERNEL_LM_HEAD, ma, ma, mb, mb, sh, ep, st))); break;
-      case 128: L3_TRY((launch_gemm<128, 5, EPI_ARGMAX, false>(LLAMA3_KERNEL_LM_HEAD, ma, ma, mb, mb, sh, ep, st))); break;
-      default: L3_TRY((launch_gemm<256, 4, EPI_ARGMAX, false>(LLAMA3_KERNEL_LM_HEAD, ma, ma, mb, mb, sh, ep, st))); break;
-    }
-  } else {
-    const long long warps = (long long)rows * ((V + 31) / 32);
-    if (cfg->dtype == LLAMA3_DTYPE_F32)
-      L3_LAUNCH(LLAMA3_KERNEL_LM_HEAD, st, launch_k((lm_head_simt_kernel<float>), blocks_for(warps * 32, 256), 256, 0, st, 
-                                               (const float*)hn, (const float*)w_out, logits_out, keys, rows, V, D));
-    else
-      L3_LAUNCH(LLAMA3_KERNEL_LM_HEAD, st, launch_k((lm_head_simt_kernel<bf16>), blocks_for(warps * 32, 256), 256, 0, st, 
-                                               (const bf16*)hn, (const bf16*)w_out, logits_out, keys, rows, V, D));
-    L3_TRY(launch_check());
-  }
-  L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st, launch_k((argmax_finalize_kernel), blocks_for(rows, 256), 256, 0, st, keys, ids_out, rows));
-  return launch_check();
+  return lm_head_run(cfg, norm_w, w_out, h, rows, row_stride, ids_out, logits_out, hn, keys, st);
 }

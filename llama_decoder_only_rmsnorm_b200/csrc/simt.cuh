@@ -46,20 +46,40 @@ __global__ void gather_rows_kernel(const uint4* __restrict__ x, long long row_st
 // ---- generation bookkeeping ("Build your own Llama 3 from scratch" 六) -------
 // After a step has written the next token of every sequence into ids:
 // history[step][b] = ids[b] (while step < rows), positions[b] += 1, step += 1.
-// One CTA, so the step counter is read once and advanced after every write.
-__global__ void generation_advance_kernel(int32_t* __restrict__ positions, const int32_t* __restrict__ ids,
-                                          int32_t* __restrict__ history, int32_t* __restrict__ step, int batch,
-                                          int rows, long long stride) {
+// With done (eos_id >= 0): a sequence whose done flag is set has its token
+// replaced by eos_id (the page stops a sequence at its end token), a sequence
+// emitting eos_id gets its flag set, and done[batch] = 1 once every sequence
+// is done.  One CTA, so the step counter is read once and advanced after every
+// write.
+__global__ void generation_advance_kernel(int32_t* __restrict__ positions, int32_t* __restrict__ ids,
+                                          int32_t* __restrict__ history, int32_t* __restrict__ step,
+                                          int32_t* __restrict__ done, int eos_id, int batch, int rows,
+                                          long long stride) {
   griddep_wait_and_release();
   __shared__ int t;
   if (threadIdx.x == 0) t = *step;
   __syncthreads();
+  int all = 1;
   for (int b = threadIdx.x; b < batch; b += blockDim.x) {
-    if (t >= 0 && t < rows) history[(size_t)t * stride + b] = ids[b];
+    int id = ids[b];
+    if (done) {
+      // a sequence that has emitted the end token keeps emitting it
+      if (done[b]) {
+        id = eos_id;
+        ids[b] = id;
+      } else if (id == eos_id) {
+        done[b] = 1;
+      }
+      all &= done[b] != 0;
+    }
+    if (t >= 0 && t < rows) history[(size_t)t * stride + b] = id;
     positions[b] += 1;
   }
-  __syncthreads();
-  if (threadIdx.x == 0) *step = t + 1;
+  all = __syncthreads_and(all);
+  if (threadIdx.x == 0) {
+    *step = t + 1;
+    if (done) done[batch] = all;
+  }
 }
 
 // ---- RMSNorm ("Build your own Llama 3 from scratch" §3.1) -------------------

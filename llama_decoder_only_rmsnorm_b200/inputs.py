@@ -139,6 +139,28 @@ def layer_weights(w: Workload, layer: int, device="cpu", norm_weight="ones"):
     return out
 
 
+def stack_weights(w: Workload, device="cpu", norm_weight="ones", threads: int = 8):
+    """All ``w.n_layers`` blocks' weights and the output weights, drawn on the
+    host by the CPU generators (the same draws on every machine for a given
+    torch build) in ``threads`` parallel threads, then moved to ``device``.
+    Returns (layers, output_weights)."""
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(max(1, threads)) as ex:
+        layers = list(ex.map(lambda i: layer_weights(w, i, "cpu", norm_weight), range(w.n_layers)))
+    out = output_weights(w, "cpu", norm_weight)
+    if str(device) != "cpu":
+        def move(d):
+            m = {k: v.to(device) for k, v in d.items() if k not in ("wq", "wk", "wv")}
+            if "wqkv" in m:
+                H, KV, hd = w.n_heads, w.n_kv_heads, w.head_dim
+                m["wq"], m["wk"], m["wv"] = (m["wqkv"][:H * hd], m["wqkv"][H * hd:(H + KV) * hd],
+                                             m["wqkv"][(H + KV) * hd:])
+            return m
+        layers = [move(l) for l in layers]
+        out = move(out)
+    return layers, out
+
+
 def _norm_weight(w: Workload, device, kind, seed):
     t = torch.empty((w.dim,), dtype=w.torch_dtype, device=device)
     if kind == "ones":
@@ -179,15 +201,18 @@ def hidden_rows(w: Workload, rows: int, device="cpu", std=1.0, step=0):
     return _normal_into(x, std, _seed(w.seed, "hidden", rows, step))
 
 
-def kv_cache(w: Workload, layer: int, capacity: int, device="cpu"):
-    """Per-layer caches [batch, capacity, KV, hd]; the first ``cache_len``
-    positions hold N(0,1) entries (already-rotated keys and values), the rest
-    zeros."""
-    shape = (w.batch, capacity, w.n_kv_heads, w.head_dim)
+def kv_cache(w: Workload, layer: int, capacity: int, device="cpu", first: int = 0, count: Optional[int] = None):
+    """Per-layer caches [count, capacity, KV, hd] of sequences first ..
+    first+count-1 (default: the whole batch); the first ``cache_len`` positions
+    hold N(0,1) entries (already-rotated keys and values), the rest zeros.
+    Each sequence has its own seed, so a shard of the batch draws exactly the
+    rows the whole batch would hold."""
+    count = w.batch - first if count is None else count
+    shape = (count, capacity, w.n_kv_heads, w.head_dim)
     k = torch.zeros(shape, dtype=w.torch_dtype, device=device)
     v = torch.zeros(shape, dtype=w.torch_dtype, device=device)
     if w.cache_len:
         for name, t in (("k", k), ("v", v)):
-            for b in range(w.batch):
-                _normal_into(t[b, :w.cache_len], 1.0, _seed(w.seed, "cache", layer, name, b))
+            for i in range(count):
+                _normal_into(t[i, :w.cache_len], 1.0, _seed(w.seed, "cache", layer, name, first + i))
     return k, v

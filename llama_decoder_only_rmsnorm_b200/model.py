@@ -80,7 +80,7 @@ class Llama3Stack:
     def generate(self, prompt_ids, n_new, eos_id=None, stream=None, temperature=0.0, top_p=0.9, seed=0,
                  return_logits=False, cuda_graph=False, prompt_lens=None):
         """Prefill the prompts (int32 [batch, S] on the device), then decode
-        n_new tokens.  temperature <= 0 is greedy (the LM head's argmax);
+        up to n_new tokens.  temperature <= 0 is greedy (the LM head's argmax);
         otherwise each step's fp32 logits go through llama3_sample_top_p,
         whose draw for sequence b is keyed by the position of the token that
         produced the logits (S - 1 for the first new token, then S, S+1, ...).
@@ -91,8 +91,11 @@ class Llama3Stack:
         llama3_generation_advance -- so with cuda_graph=True it is captured once
         and replayed.  Returns the [batch, n_new] tokens as a host array (and,
         with return_logits, the [n_new, batch, vocab] fp32 logits, not with
-        cuda_graph); after a sequence's first eos_id the rest of its row is
-        eos_id (the page stops the loop there).
+        cuda_graph).  With eos_id, llama3_generation_advance keeps a done
+        flag per sequence on the device: after a sequence's first eos_id the
+        rest of its row is eos_id, and the loop ends as soon as every
+        sequence is done (the page's generate stops there too); the host
+        reads one flag per step for that.
 
         prompt_lens (host ints, one per sequence, each <= S): prompts of
         different lengths, left-aligned and padded to S.  The padded prefill
@@ -101,7 +104,6 @@ class Llama3Stack:
         len[b] - 1 of each sequence, and decoding continues at position
         len[b] (padding K/V in the cache are overwritten before they are
         ever visible)."""
-        import torch
         Bn, S = prompt_ids.shape
         assert Bn == self.batch and S + n_new - 1 <= self.cache_cap
         assert not (cuda_graph and (return_logits or stream is not None))
@@ -112,7 +114,10 @@ class Llama3Stack:
         self.embed(prompt_ids, x, stream)
         self.forward_layers(x, S, 0, stream)
         row = (Bn + 3) // 4 * 4            # keeps every history row 16-byte aligned
-        hist = torch.empty((n_new, row), dtype=torch.int32, device=dev)
+        stop = eos_id is not None
+        hist = torch.full((n_new, row), eos_id if stop else -1, dtype=torch.int32, device=dev)
+        done = torch.zeros((row + 1,), dtype=torch.int32, device=dev) if stop else None
+        all_done = torch.zeros((1,), dtype=torch.int32).pin_memory() if stop else None
         cur = torch.empty((row,), dtype=torch.int32, device=dev)
         lens = [S] * Bn if prompt_lens is None else [int(v) for v in prompt_lens]
         assert len(lens) == Bn and all(1 <= v <= S for v in lens)
@@ -129,7 +134,8 @@ class Llama3Stack:
                                     pick if sampling else cur, lg, self.ws, self.ws_bytes, stream)
             if sampling:
                 B.llama3_sample_top_p(lg, Bn, V, V, temperature, top_p, seed, 0, cur, stream, positions=pos)
-            B.llama3_generation_advance(pos, cur, hist, step, Bn, n_new, row, stream)
+            B.llama3_generation_advance(pos, cur, hist, step, Bn, n_new, row, stream, done=done,
+                                        eos_id=eos_id if stop else -1)
 
         if prompt_lens is None:
             head(x[:, -1], S * D, 0)       # first new token; pos -> S, step -> 1
@@ -146,26 +152,38 @@ class Llama3Stack:
             self.decode_layers_ragged(xd, pos, max_pos, stream)
             head(xd, D, k)
 
-        if cuda_graph and n_new > 1:
+        def finished():
+            # one int read per step: done[Bn] is set once every sequence has
+            # emitted the end token
+            if not stop:
+                return False
+            all_done.copy_(done[Bn:Bn + 1], non_blocking=True)
+            (torch.cuda.current_stream() if stream is None else stream).synchronize()
+            return bool(all_done.item())
+
+        if finished():
+            pass
+        elif cuda_graph and n_new > 1:
             g = torch.cuda.CUDAGraph()
             side = torch.cuda.Stream()
             side.wait_stream(torch.cuda.current_stream())
             with torch.cuda.stream(side):
                 decode_step(1)             # warm-up step (also token 1)
             torch.cuda.current_stream().wait_stream(side)
-            with torch.cuda.graph(g):
-                decode_step(2)
-            for _ in range(2, n_new):
-                g.replay()
+            if n_new > 2 and not finished():
+                with torch.cuda.graph(g):
+                    decode_step(2)
+                for k in range(2, n_new):   # the capture ran nothing: replay steps 2 .. n_new-1
+                    if k > 2 and finished():
+                        break
+                    g.replay()
         else:
             for k in range(1, n_new):
                 decode_step(k)
+                if finished():
+                    break
+        self.steps_run = int(step.item())
         toks = hist[:, :Bn].t().cpu().numpy()
-        if eos_id is not None:   # host-side: hold the end token once emitted
-            for b in range(Bn):
-                hits = (toks[b] == eos_id).nonzero()[0]
-                if hits.size:
-                    toks[b, hits[0]:] = eos_id
         if return_logits:
             return toks, logits.cpu().numpy()
         return toks

@@ -48,3 +48,61 @@ def oracle_cfg(w):
     c = w.cfg()
     return dict(dim=c["dim"], n_heads=c["n_heads"], n_kv_heads=c["n_kv_heads"], head_dim=c["head_dim"],
                 ffn_hidden=c["ffn_hidden"], norm_eps=c["norm_eps"], rope_theta=c["rope_theta"])
+
+
+# ---------------------------------------------------------------------------
+# Full-size bound.  At the 8B sizes (and any layer of comparable width) the
+# per-element bound above is out of reach for a path that stores its
+# activations in bf16: the fp64 oracle with bf16 storage at the same step
+# boundaries (oracle rounding="bf16") already misses it on a few percent of
+# a block's outputs, and on most elements after 32 blocks.  There the GPU is
+# held to that variant instead: its relative L2 distance from the exact
+# oracle may be at most NOISE_FACTOR times the variant's own distance, and
+# argmax ids must match wherever the exact top-2 gap exceeds ARGMAX_NOISE_K
+# times the variant's logit error (and 1e-2).
+NOISE_FACTOR = 1.5
+ARGMAX_NOISE_K = 6.0
+
+
+def rel_l2(a, b):
+    a, b = np.asarray(a, np.float64), np.asarray(b, np.float64)
+    return float(np.linalg.norm(a - b) / np.linalg.norm(b))
+
+
+def within_bound_fraction(got, want, dtype="bf16"):
+    atol, rtol = TOL[dtype]
+    got, want = np.asarray(got, np.float64), np.asarray(want, np.float64)
+    return float(np.mean(np.abs(got - want) <= atol + rtol * np.abs(want)))
+
+
+def assert_within_bf16_noise(gpu, exact, bf16_variant, what, factor=NOISE_FACTOR):
+    """rel_l2(gpu, exact) <= factor * rel_l2(bf16 variant, exact); returns both
+    (and the fraction of elements each keeps inside the per-element bound)."""
+    g = f64(gpu) if isinstance(gpu, torch.Tensor) else np.asarray(gpu, dtype=np.float64)
+    e = np.asarray(exact, np.float64)
+    r = np.asarray(bf16_variant, np.float64)
+    assert g.shape == e.shape == r.shape, (what, g.shape, e.shape, r.shape)
+    assert np.all(np.isfinite(g)), f"{what}: non-finite values"
+    rg, rr = rel_l2(g, e), rel_l2(r, e)
+    info = dict(rel_gpu=rg, rel_bf16=rr, in_bound_gpu=within_bound_fraction(g, e),
+                in_bound_bf16=within_bound_fraction(r, e))
+    assert rg <= factor * rr, f"{what}: {info}"
+    return info
+
+
+def assert_argmax_beyond_noise(gpu_ids, exact_logits, bf16_logits, what, k=ARGMAX_NOISE_K, need=1):
+    """ids equal the exact argmax on every row whose exact top-2 gap exceeds
+    max(1e-2, k * std(bf16 variant logits - exact logits) of that row); at
+    least `need` rows must be decided that way.  Returns the decided count."""
+    ids = gpu_ids.detach().cpu().numpy().astype(np.int64).reshape(-1)
+    lg = np.asarray(exact_logits, np.float64).reshape(len(ids), -1)
+    lr = np.asarray(bf16_logits, np.float64).reshape(len(ids), -1)
+    noise = np.std(lr - lg, axis=1)
+    top2 = np.sort(lg, axis=1)[:, -2:]
+    decided = (top2[:, 1] - top2[:, 0]) > np.maximum(ARGMAX_GAP, k * noise)
+    want = np.argmax(lg, axis=1)
+    assert decided.sum() >= need, f"{what}: only {decided.sum()} decided rows (noise {noise.mean():.3g})"
+    mism = decided & (ids != want)
+    assert not mism.any(), f"{what}: ids differ at rows {np.nonzero(mism)[0][:10]}"
+    assert np.all((ids >= 0) & (ids < lg.shape[1]))
+    return int(decided.sum())

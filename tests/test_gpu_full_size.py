@@ -1,15 +1,19 @@
-"""Parity at the full Llama-3-8B sizes the benchmark runs, on outputs the fp64
-oracle can compute one by one: one decoder block of the 8192-token prefill
-(sampled output rows, plus every K/V row the block writes to the cache) and
-one block of the 32-sequence decode step at 8192 cached positions (sampled
-sequences, plus their new cache rows).  Same kernels and launch configuration
-as bench.py (tcgen05 GEMMs, the default prefill attention design, split-KV
-decode attention)."""
+"""Parity of single blocks at the full Llama-3-8B sizes the benchmark runs, and
+of layers wider than 8B, against the fp64 oracle: one block of the
+8192-token prefill (64 output rows spread over the sequence, plus every K/V
+row the block writes) and one block of the 32-sequence decode step at 8192
+cached positions (all 32 sequences and their new cache rows).  Same kernels
+and launch configuration as bench.py.
+
+Block outputs at these widths are held to the full-size bound of helpers.py
+(the GPU within 1.5x of the relative L2 error that bf16 storage alone gives,
+measured on the same inputs by the oracle's bf16 variant); the K/V rows,
+one projection deep, keep the per-element bound 2e-2 + 2e-2|oracle|."""
 import numpy as np
 import pytest
 import torch
 
-from helpers import assert_close, f64, oracle_cfg, oracle_layer
+from helpers import assert_close, assert_within_bf16_noise, f64, oracle_cfg, oracle_layer
 from llama_decoder_only_rmsnorm_b200 import binding as B
 from llama_decoder_only_rmsnorm_b200 import inputs as I
 from llama_decoder_only_rmsnorm_b200.model import Llama3Stack
@@ -17,32 +21,6 @@ from oracle import llama3_oracle as O
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
-
-# One full-size bf16 block carries rounding noise from its bf16 intermediates
-# (normalised rows, SwiGLU product, residual stream), each rounded to a
-# relative 2^-9/sqrt(3) ~ 1.1e-3.  With the seeded N(0, 0.02) weights the w2
-# output (K = 14336) has a standard deviation near 1.9, and the rounding of its
-# inputs alone reaches the block output with a standard deviation near 5e-3.
-# Measured, the fp64 arithmetic with bf16 rounding at the GPU's rounding points
-# differs from the exact oracle by a standard deviation of 1.2e-2, as much as
-# the GPU does, so the per-element bound 2e-2 + 2e-2|o| of the smaller
-# workloads is missed on a fraction of a percent of near-zero elements.  At these sizes the tests require the bound on at
-# least 99 % of the elements, 4x the bound on every element, and a relative
-# L2 error below 1e-2; the K/V rows keep the plain bound.
-BULK, SLACK, REL_L2 = 0.99, 4.0, 1e-2
-
-
-def assert_close_bulk(gpu, oracle, what):
-    g = f64(gpu) if isinstance(gpu, torch.Tensor) else np.asarray(gpu, float)
-    o = np.asarray(oracle, float)
-    assert g.shape == o.shape, (what, g.shape, o.shape)
-    err = np.abs(g - o)
-    bound = 2e-2 + 2e-2 * np.abs(o)
-    within = float(np.mean(err <= bound))
-    worst = float(np.max(err / bound))
-    rel = float(np.linalg.norm(g - o) / np.linalg.norm(o))
-    assert np.all(np.isfinite(g)), what
-    assert within >= BULK and worst <= SLACK and rel <= REL_L2, (what, within, worst, rel)
 
 
 @pytest.fixture(autouse=True)
@@ -55,7 +33,15 @@ def _gpu_state():
     assert B.llama3_device_status() == 0, "device status word set"
 
 
-def test_8b_prefill_block_full_sequence_sampled_rows():
+def _spread_rows(S, n, seed):
+    """Tile edges and ends of the sequence plus random rows, sorted."""
+    fixed = {0, 1, 127, 128, 129, 255, 256, S // 2, S - 129, S - 128, S - 2, S - 1}
+    rng = np.random.default_rng(seed)
+    extra = rng.choice(S, size=n - len(fixed), replace=False)
+    return sorted(fixed | {int(r) for r in extra})[:n]
+
+
+def test_8b_prefill_block_full_sequence():
     w = I.WORKLOADS["llama3_8b_prefill"].replace(input_kind="activations")
     layer = I.layer_weights(w, 0, DEV)
     S = w.seq
@@ -64,15 +50,17 @@ def test_8b_prefill_block_full_sequence_sampled_rows():
     x0 = f64(x)[0]
     st.forward_layers(x, S, 0)
     torch.cuda.synchronize()
-    rows = [0, 1, 127, 128, 129, 2047, 4096, 6000, 8190, 8191]
-    want, k, v = O.decoder_block_rows(x0, oracle_layer(layer), oracle_cfg(w), rows)
-    assert_close_bulk(x[0, rows], want, "8B prefill rows")
+    rows = _spread_rows(S, 64, 1)
+    lo, oc = oracle_layer(layer), oracle_cfg(w)
+    want, k, v = O.decoder_block_rows(x0, lo, oc, rows)
+    want_bf, _, _ = O.decoder_block_rows(x0, lo, oc, rows, rounding="bf16")
+    assert_within_bf16_noise(x[0, rows], want, want_bf, "8B prefill block rows")
     kc, vc = st.caches[0]
     assert_close(kc[0, :S], k, "bf16", "8B prefill K cache (all positions)")
     assert_close(vc[0, :S], v, "bf16", "8B prefill V cache (all positions)")
 
 
-def test_8b_decode_step_sampled_sequences():
+def test_8b_decode_block_all_sequences():
     wd = I.WORKLOADS["llama3_8b_decode"]
     w8 = I.WORKLOADS["llama3_8b_prefill"]
     layer = I.layer_weights(w8, 0, DEV)
@@ -82,13 +70,63 @@ def test_8b_decode_step_sampled_sequences():
                      caches=[(kc, vc)])
     g = torch.Generator(device="cpu").manual_seed(31)
     x = torch.randn((wd.batch, 1, wd.dim), generator=g).to(torch.bfloat16)
-    k_prefix = {b: (f64(kc[b, :P]), f64(vc[b, :P])) for b in (0, 17, 31)}
     xd = x.to(DEV)
     st.decode_layers(xd, P)
     torch.cuda.synchronize()
+    # the cache prefix is an input: draw it again (same seeds) for the oracle
+    kp, vp = I.kv_cache(wd, 0, P, DEV)
+    kp, vp = f64(kp), f64(vp)
     lo, oc = oracle_layer(layer), oracle_cfg(w8)
-    for b, (kp, vp) in k_prefix.items():
-        want, k_new, v_new = O.decoder_block_rows(f64(x[b]), lo, oc, [0], kp, vp, start_pos=P)
-        assert_close_bulk(xd[b], want, f"8B decode seq {b}")
+    got, want, want_bf = [], [], []
+    for b in range(wd.batch):
+        o_ex, k_new, v_new = O.decoder_block_rows(f64(x[b]), lo, oc, [0], kp[b], vp[b], start_pos=P)
+        o_bf, _, _ = O.decoder_block_rows(f64(x[b]), lo, oc, [0], kp[b], vp[b], start_pos=P, rounding="bf16")
+        got.append(f64(xd[b])); want.append(o_ex); want_bf.append(o_bf)
         assert_close(kc[b, P], k_new[0], "bf16", f"8B decode new K seq {b}")
         assert_close(vc[b, P], v_new[0], "bf16", f"8B decode new V seq {b}")
+    assert_within_bf16_noise(np.stack(got), np.stack(want), np.stack(want_bf), "8B decode block")
+
+
+@pytest.mark.parametrize("dim,H,KV,F", [(8192, 64, 8, 22016), (8448, 66, 6, 22528)])
+def test_wide_prefill_layer(dim, H, KV, F):
+    """Layers wider than 8B (dim 8192, and 8448 = 33 tiles of 256): all 640
+    output rows of a one-layer prefill.  At these widths the per-element bound
+    is missed by the oracle's own bf16 variant as well."""
+    w = I.Workload("wide", dim=dim, n_layers=1, n_heads=H, n_kv_heads=KV, ffn_hidden=F, vocab=None, batch=1,
+                   seq=640, dtype="bf16", input_kind="activations", seed=dim)
+    layer = I.layer_weights(w, 0, DEV, "random")
+    st = Llama3Stack(w.cfg(), [layer], {}, 1, w.seq, w.seq)
+    x = I.activations(w, DEV)
+    x0 = f64(x)
+    st.forward_layers(x, w.seq, 0)
+    torch.cuda.synchronize()
+    lo, oc = oracle_layer(layer), oracle_cfg(w)
+    kc0 = np.zeros((1, w.seq, KV, dim // H)); vc0 = np.zeros_like(kc0)
+    want = O.decoder_block(x0, lo, oc, kc0, vc0)
+    want_bf = O.decoder_block(x0, lo, oc, np.zeros_like(kc0), np.zeros_like(vc0), rounding="bf16")
+    assert_within_bf16_noise(x, want, want_bf, f"dim-{dim} prefill layer")
+    assert_close(st.caches[0][0], kc0, "bf16", f"dim-{dim} K cache")
+    assert_close(st.caches[0][1], vc0, "bf16", f"dim-{dim} V cache")
+
+
+def test_wide_decode_layer_uses_separate_reductions():
+    """dim 16896 (> 16384): the decode step's residual sums and the RMSNorm
+    after them run as separate kernels instead of the fused one."""
+    w = I.Workload("wide_decode", dim=16896, n_layers=1, n_heads=132, n_kv_heads=12, ffn_hidden=4096, vocab=None,
+                   batch=4, seq=1, dtype="bf16", input_kind="activations", seed=16896, cache_len=300)
+    layer = I.layer_weights(w, 0, DEV, "random")
+    P = w.cache_len
+    kc, vc = I.kv_cache(w, 0, P + 1, DEV)
+    st = Llama3Stack(w.cfg(), [layer], {}, w.batch, P + 1, 1, caches=[(kc, vc)])
+    x = I.activations(w, DEV)
+    x0 = f64(x)
+    st.decode_layers(x, P)
+    torch.cuda.synchronize()
+    kp, vp = I.kv_cache(w, 0, P, DEV)
+    kp, vp = f64(kp), f64(vp)
+    lo, oc = oracle_layer(layer), oracle_cfg(w)
+    want = np.stack([O.decoder_block_rows(x0[b], lo, oc, [0], kp[b], vp[b], start_pos=P)[0]
+                     for b in range(w.batch)])
+    want_bf = np.stack([O.decoder_block_rows(x0[b], lo, oc, [0], kp[b], vp[b], start_pos=P, rounding="bf16")[0]
+                        for b in range(w.batch)])
+    assert_within_bf16_noise(x, want, want_bf, "dim-16896 decode layer")

@@ -109,6 +109,8 @@ def test_lm_head_and_helpers_reject_bad_arguments():
 def test_kernel_path_and_wait_limit_switches():
     assert B.llama3_set_kernel_path(1) == 0
     assert B.llama3_set_kernel_path(0) == 1
+    assert B.llama3_set_kernel_path(2) == 0        # anything but 1 selects the tcgen05 kernels
+    assert B.llama3_set_kernel_path(0) == 0
     old = B.llama3_set_wait_limit_ms(500)
     assert B.llama3_set_wait_limit_ms(old) == 500
 
@@ -135,18 +137,14 @@ def test_sample_top_p_rejects_bad_arguments_before_launch():
     assert gat(n=0) == 1
     assert gat(stride=100) == 1
     assert gat(stride=4100) == 2
-    adv = lambda **k: lib.llama3_generation_advance(k.get("pos", FAKE), FAKE, FAKE, FAKE, k.get("batch", 4),
-                                                    k.get("rows", 8), k.get("stride", 4), None)
+    adv = lambda **k: lib.llama3_generation_advance(k.get("pos", FAKE), FAKE, FAKE, FAKE, k.get("done", None),
+                                                    k.get("eos", -1), k.get("batch", 4), k.get("rows", 8),
+                                                    k.get("stride", 4), None)
+    assert adv(eos=7) == 1                          # an end token needs the done flags
+    assert adv(eos=7, done=ctypes.c_void_p(FAKE + 2)) == 2
     assert adv(batch=0) == 1
     assert adv(rows=0) == 1
     assert adv(stride=3) == 1
     assert adv(pos=None) == 1
     assert adv(pos=ctypes.c_void_p(FAKE + 1)) == 2
     assert B.KERNEL_KINDS["sample"] == 11
-
-
-def test_flash_variant_switch():
-    old = B.llama3_set_flash_variant(1)
-    assert B.llama3_set_flash_variant(5) == 1
-    assert B.llama3_set_flash_variant(7) == 5      # values outside 1..5 select the third design
-    assert B.llama3_set_flash_variant(old) == 3

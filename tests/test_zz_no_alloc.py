@@ -19,18 +19,23 @@ DEV = "cuda"
 
 
 @pytest.mark.gpu
-def test_noalloc_lm_head_matches_workspace_entry_point_on_consecutive_calls():
+@pytest.mark.parametrize("workload,row_counts", [
+    ("llama3_8b_prefill", (32, 7)),     # tcgen05 path, few rows
+    ("llama3_8b_prefill", (511, 300)),  # the most rows the scratch holds at dim 4096 bf16, two n-tiles of hn
+    ("tiny_f32", (64, 5)),              # fp32: the SIMT LM head reading its rows from the scratch
+])
+def test_noalloc_lm_head_matches_workspace_entry_point_on_consecutive_calls(workload, row_counts):
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
     B.llama3_set_kernel_path(0)
-    w = I.WORKLOADS["llama3_8b_prefill"]
+    w = I.WORKLOADS[workload]
     outw = I.output_weights(w, DEV, "random")
-    cfg = B.make_config(w.dim, w.n_heads, w.n_kv_heads, w.ffn_hidden, w.vocab)
-    ws_bytes = B.llama3_workspace_size(cfg, 1, 1, 64)
+    cfg = B.make_config(w.dim, w.n_heads, w.n_kv_heads, w.ffn_hidden, w.vocab, dtype=w.dtype)
+    ws_bytes = B.llama3_workspace_size(cfg, 1, 1, max(row_counts))
     ws = torch.empty((ws_bytes,), dtype=torch.uint8, device=DEV)
     # two calls in a row; the second has fewer rows and new inputs, so any
     # maximum left in the shared scratch by the first call would show
-    for call, rows in enumerate((32, 7)):
+    for call, rows in enumerate(row_counts):
         h = I.hidden_rows(w, rows, DEV, std=2.0, step=100 + call)
         ref_ids = torch.empty((rows,), dtype=torch.int32, device=DEV)
         ref_logits = torch.empty((rows, w.vocab), dtype=torch.float32, device=DEV)
@@ -41,7 +46,7 @@ def test_noalloc_lm_head_matches_workspace_entry_point_on_consecutive_calls():
         B.llama3_lm_head_argmax_noalloc(cfg, outw["norm"], outw["output"], h, rows, w.dim, ids, logits)
         torch.cuda.synchronize()
         assert torch.equal(ids, ref_ids), f"call {call}: ids differ"
-        assert_close(logits, f64(ref_logits), "bf16", f"call {call} logits")
+        assert_close(logits, f64(ref_logits), w.dtype, f"call {call} logits")
     assert B.llama3_device_status() == 0
 
 
