@@ -411,6 +411,21 @@ int llama3_set_kernel_path(int path);
 /* Limit, in milliseconds, of every bounded device-side wait (default 2000). */
 int llama3_set_wait_limit_ms(int ms);
 
+/* Failure-detection test hook, off (0) by default.  Every wait of one role of
+ * a kernel for another is bounded (llama3_set_wait_limit_ms): when it runs
+ * out, the kernel records LLAMA3_ERR_TIMEOUT in the status word, lets its
+ * copies in flight land, frees its tensor memory and returns, and the context
+ * stays usable.  This hook makes such a wait run out on purpose:
+ *   1: in the tcgen05 GEMMs, the first epilogue warp of every CTA leaves out
+ *      its release of the accumulator after the CTA's first tile, so the MMA
+ *      issuer's wait for that buffer gives up (needs three tiles per CTA);
+ *   2: in the prefill attention kernel, one softmax thread of every CTA leaves
+ *      out its P arrival on its first key tile, so the MMA issuer's wait for
+ *      P gives up.
+ * Nothing else changes; results of such a call are undefined.  Returns the
+ * previous value (values other than 1 and 2 select 0). */
+int llama3_set_test_withheld_arrival(int which);
+
 /* 1 (default): kernels are launched with programmatic stream serialization,
  * so a kernel's launch and set-up overlap the end of the previous kernel in
  * the stream (each kernel waits for its predecessor before touching memory);

@@ -65,6 +65,7 @@ _SIGNATURES = {
     "llama3_last_cuda_error": [],
     "llama3_set_kernel_path": [_i],
     "llama3_set_wait_limit_ms": [_i],
+    "llama3_set_test_withheld_arrival": [_i],
     "llama3_set_programmatic_launch": [_i],
     "llama3_sample_top_p": [_p, _i, _ll, _i, ctypes.c_float, ctypes.c_float, ctypes.c_ulonglong, ctypes.c_ulonglong, _p, _p, _p],
     "llama3_generation_advance": [_p, _p, _p, _p, _p, _i, _i, _i, _ll, _p],
@@ -278,6 +279,12 @@ def llama3_set_kernel_path(path):
 
 def llama3_set_wait_limit_ms(ms):
     return lib().llama3_set_wait_limit_ms(ms)
+
+
+def llama3_set_test_withheld_arrival(which):
+    """Failure-detection test hook (0 = off): 1 makes the GEMMs' accumulator
+    wait give up, 2 the prefill attention's wait for P."""
+    return lib().llama3_set_test_withheld_arrival(int(which))
 
 
 def llama3_set_programmatic_launch(on):

@@ -27,6 +27,7 @@ namespace {
 thread_local int t_last_cuda = 0;
 int g_kernel_path = 0;       // 0 = tcgen05 for bf16, 1 = SIMT everywhere
 int g_wait_ms = 2000;        // bounded device waits
+int g_withhold = 0;          // failure-detection test hook (llama3_set_test_withheld_arrival)
 constexpr int kMaxDevices = 64;
 int g_num_sms[kMaxDevices];
 
@@ -235,6 +236,7 @@ int run_flash_attention_t(int H, int KV, const void* q, const void* kc, const vo
   fs.ldo = H * HD;
   fs.scale_log2 = (float)(1.4426950408889634 / sqrt((double)HD));
   fs.doc_start = doc_start;
+  fs.withhold = g_withhold == 2 ? 2 : 0;
   constexpr int smem = FlashCfg<HD>::SMEM_BYTES;
   auto kern = flash_attention_kernel<HD>;
   int dev = 0;
@@ -336,6 +338,7 @@ GemmShape make_shape(int rows_a, int rows_a2, int rows_b, int k, int bn, int spl
   // changes nothing.
   s.group_m = std::max(1, std::min(L3_GROUP_M, s.tiles_m));
   s.sk_per = 0;
+  s.withhold = 0;
   return s;
 }
 
@@ -404,7 +407,9 @@ int launch_gemm(int kind, const CUtensorMap& a, const CUtensorMap& a2, const CUt
   }
   if (sh.units <= 0) return LLAMA3_OK;
   const int grid = std::min(sh.units, num_sms());
-  L3_LAUNCH(kind, st, launch_k(kern, grid, 192, Cfg::SMEM_BYTES, st, a, a2, b, b2, sh, ep, wait_ns()));
+  GemmShape s = sh;
+  s.withhold = g_withhold == 1 ? 1 : 0;
+  L3_LAUNCH(kind, st, launch_k(kern, grid, 192, Cfg::SMEM_BYTES, st, a, a2, b, b2, s, ep, wait_ns()));
   return launch_check();
 }
 
@@ -973,6 +978,12 @@ int llama3_set_programmatic_launch(int on) {
 int llama3_set_wait_limit_ms(int ms) {
   int old = g_wait_ms;
   if (ms > 0) g_wait_ms = ms;
+  return old;
+}
+
+int llama3_set_test_withheld_arrival(int which) {
+  const int old = g_withhold;
+  g_withhold = (which == 1 || which == 2) ? which : 0;
   return old;
 }
 

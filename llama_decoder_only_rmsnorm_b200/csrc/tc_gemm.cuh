@@ -52,6 +52,10 @@ struct GemmShape {
   // Stream-K (one n-tile only): CTA c takes k-blocks [c*sk_per, (c+1)*sk_per)
   // of the (m-tile, k-block) space in m-major order; 0 = split-K units.
   int sk_per;
+  // Failure-detection test hook (0 in every normal launch): 1 = the first
+  // epilogue warp leaves out its release of the accumulator after the CTA's
+  // first unit, so the MMA issuer's bounded wait for that buffer gives up.
+  int withhold;
 };
 
 // Work unit -> (split, m-tile, n-tile).  Within a split, tiles are visited in
@@ -481,7 +485,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[abuf]);
+      if (lane == 0 && !(sh.withhold == 1 && it == 0 && warp == 2)) mbar_arrive(&acc_empty[abuf]);
       if (++abuf == C::ACC_BUFS) { abuf = 0; aphase ^= 1u; }
     }
   }

@@ -15,7 +15,11 @@ from . import binding as B
 
 class Llama3Stack:
     def __init__(self, cfg: dict, layers, out_weights, batch: int, cache_cap: int, max_seq: int,
-                 lm_rows: int = 0, device="cuda", rope_len: int | None = None, caches=None):
+                 lm_rows: int = 0, device="cuda", rope_len: int | None = None, caches=None, alloc=None):
+        """alloc (optional): alloc(shape, dtype, device) -> uninitialised
+        tensor, used instead of torch.empty for every buffer this object
+        allocates (RoPE table, workspace, caches, outputs, generation state)."""
+        self._alloc = alloc
         self.cfg_dict = dict(cfg)
         self.cfg = B.make_config(cfg["dim"], cfg["n_heads"], cfg["n_kv_heads"], cfg["ffn_hidden"],
                                  cfg.get("vocab", 0), cfg["norm_eps"], cfg["rope_theta"], cfg["dtype"])
@@ -27,17 +31,22 @@ class Llama3Stack:
         self.device = device
         hd = cfg["dim"] // cfg["n_heads"]
         self.rope_len = rope_len or max(cache_cap, 1)
-        self.rope = torch.empty((self.rope_len, hd // 2, 2), dtype=torch.float32, device=device)
+        self.rope = self._empty((self.rope_len, hd // 2, 2), torch.float32)
         B.llama3_init_rope_table(self.rope, hd, self.rope_len, cfg["rope_theta"])
         self.lm_rows = max(lm_rows, 1)
         self.ws_bytes = B.llama3_workspace_size(self.cfg, batch, max_seq, self.lm_rows)
-        self.ws = torch.empty((self.ws_bytes,), dtype=torch.uint8, device=device)
+        self.ws = self._empty((self.ws_bytes,), torch.uint8)
         if caches is None:
             shape = (batch, cache_cap, cfg["n_kv_heads"], hd)
-            caches = [(torch.zeros(shape, dtype=self.dtype, device=device),
-                       torch.zeros(shape, dtype=self.dtype, device=device)) for _ in self.layers]
+            caches = [(self._empty(shape, self.dtype).zero_(), self._empty(shape, self.dtype).zero_())
+                      for _ in self.layers]
         self.caches = caches
-        self.ids_out = torch.zeros((self.lm_rows,), dtype=torch.int32, device=device)
+        self.ids_out = self._empty((self.lm_rows,), torch.int32).zero_()
+
+    def _empty(self, shape, dtype):
+        if self._alloc is not None:
+            return self._alloc(tuple(shape), dtype, self.device)
+        return torch.empty(shape, dtype=dtype, device=self.device)
 
     # -- steps --------------------------------------------------------------
     def embed(self, ids, x, stream=None):
@@ -110,23 +119,23 @@ class Llama3Stack:
         D, V = self.cfg_dict["dim"], self.cfg_dict["vocab"]
         dev = self.device
         sampling = temperature > 0
-        x = torch.empty((Bn, S, D), dtype=self.dtype, device=dev)
+        x = self._empty((Bn, S, D), self.dtype)
         self.embed(prompt_ids, x, stream)
         self.forward_layers(x, S, 0, stream)
         row = (Bn + 3) // 4 * 4            # keeps every history row 16-byte aligned
         stop = eos_id is not None
-        hist = torch.full((n_new, row), eos_id if stop else -1, dtype=torch.int32, device=dev)
-        done = torch.zeros((row + 1,), dtype=torch.int32, device=dev) if stop else None
+        hist = self._empty((n_new, row), torch.int32).fill_(eos_id if stop else -1)
+        done = self._empty((row + 1,), torch.int32).zero_() if stop else None
         all_done = torch.zeros((1,), dtype=torch.int32).pin_memory() if stop else None
-        cur = torch.empty((row,), dtype=torch.int32, device=dev)
+        cur = self._empty((row,), torch.int32)
         lens = [S] * Bn if prompt_lens is None else [int(v) for v in prompt_lens]
         assert len(lens) == Bn and all(1 <= v <= S for v in lens)
-        pos = torch.tensor([v - 1 for v in lens], dtype=torch.int32, device=dev)   # position behind the logits
-        step = torch.zeros((1,), dtype=torch.int32, device=dev)
-        pick = torch.empty((row,), dtype=torch.int32, device=dev)
+        pos = self._empty((Bn,), torch.int32)      # position behind the logits
+        pos.copy_(torch.tensor([v - 1 for v in lens], dtype=torch.int32))
+        step = self._empty((1,), torch.int32).zero_()
+        pick = self._empty((row,), torch.int32)
         keep = return_logits or sampling
-        logits = torch.empty((n_new if return_logits else 1, Bn, V), dtype=torch.float32,
-                             device=dev) if keep else None
+        logits = self._empty((n_new if return_logits else 1, Bn, V), torch.float32) if keep else None
 
         def head(h, stride, k):
             lg = logits[k if return_logits else 0] if keep else None
@@ -141,10 +150,10 @@ class Llama3Stack:
             head(x[:, -1], S * D, 0)       # first new token; pos -> S, step -> 1
         else:
             idx = torch.tensor([b * S + v - 1 for b, v in enumerate(lens)], dtype=torch.int32, device=dev)
-            last = torch.empty((Bn, D), dtype=self.dtype, device=dev)
+            last = self._empty((Bn, D), self.dtype)
             B.llama3_gather_rows(self.cfg, x, D, Bn * S, idx, Bn, last, stream)
             head(last, D, 0)
-        xd = torch.empty((Bn, 1, D), dtype=self.dtype, device=dev)
+        xd = self._empty((Bn, 1, D), self.dtype)
         max_pos = self.cache_cap - 1
 
         def decode_step(k):

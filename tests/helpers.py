@@ -106,3 +106,56 @@ def assert_argmax_beyond_noise(gpu_ids, exact_logits, bf16_logits, what, k=ARGMA
     assert not mism.any(), f"{what}: ids differ at rows {np.nonzero(mism)[0][:10]}"
     assert np.all((ids >= 0) & (ids < lg.shape[1]))
     return int(decided.sum())
+
+
+# ---------------------------------------------------------------------------
+# Guard bands: the cheap stand-in for a memory checker.  Every output, cache,
+# workspace and state buffer a GPU test hands the library sits between two
+# bands of a fixed byte pattern; after the test every band must be intact, so
+# a kernel writing past either end of a buffer fails the test that ran it.
+# ---------------------------------------------------------------------------
+class GuardArena:
+    BAND = 4096          # bytes on each side (keeps the payload 256-byte aligned)
+    PATTERN = 0xA5
+
+    def __init__(self, device="cuda"):
+        self.device = device
+        self.bufs = []
+
+    def empty(self, shape, dtype=torch.float32, device=None):
+        shape = tuple(shape) if isinstance(shape, (tuple, list)) else (int(shape),)
+        n = 1
+        for s in shape:
+            n *= int(s)
+        nbytes = n * torch.tensor([], dtype=dtype).element_size()
+        raw = torch.empty((2 * self.BAND + nbytes,), dtype=torch.uint8, device=device or self.device)
+        raw[:self.BAND].fill_(self.PATTERN)
+        raw[self.BAND + nbytes:].fill_(self.PATTERN)
+        self.bufs.append((raw, nbytes))
+        return raw[self.BAND:self.BAND + nbytes].view(dtype).view(shape)
+
+    def zeros(self, shape, dtype=torch.float32, device=None):
+        return self.empty(shape, dtype, device).zero_()
+
+    def full(self, shape, value, dtype=torch.float32, device=None):
+        return self.empty(shape, dtype, device).fill_(value)
+
+    def empty_like(self, t):
+        return self.empty(t.shape, t.dtype, t.device)
+
+    def to(self, t):
+        """A guarded device copy of host tensor t (for buffers a call updates in place)."""
+        return self.empty(t.shape, t.dtype).copy_(t)
+
+    def alloc(self, shape, dtype, device):
+        return self.empty(shape, dtype, device)
+
+    def check(self):
+        bad = []
+        for i, (raw, nbytes) in enumerate(self.bufs):
+            head = raw[:self.BAND]
+            tail = raw[self.BAND + nbytes:]
+            if not (bool(torch.all(head == self.PATTERN)) and bool(torch.all(tail == self.PATTERN))):
+                bad.append((i, nbytes))
+        self.bufs.clear()
+        assert not bad, f"guard band overwritten around buffers (index, bytes): {bad}"

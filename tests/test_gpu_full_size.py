@@ -13,7 +13,7 @@ import numpy as np
 import pytest
 import torch
 
-from helpers import assert_close, assert_within_bf16_noise, f64, oracle_cfg, oracle_layer
+from helpers import GuardArena, assert_close, assert_within_bf16_noise, f64, oracle_cfg, oracle_layer
 from llama_decoder_only_rmsnorm_b200 import binding as B
 from llama_decoder_only_rmsnorm_b200 import inputs as I
 from llama_decoder_only_rmsnorm_b200.model import Llama3Stack
@@ -23,14 +23,25 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
+G = None   # the running test's guard arena: outputs, caches and workspaces sit between guard bands
+
+
 @pytest.fixture(autouse=True)
 def _gpu_state():
+    global G
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
     B.llama3_set_kernel_path(0)
+    G = GuardArena(DEV)
     yield
     torch.cuda.synchronize()
     assert B.llama3_device_status() == 0, "device status word set"
+    G.check()
+
+
+def Stack(*a, **k):
+    """Llama3Stack whose buffers all come from the guard arena."""
+    return Llama3Stack(*a, alloc=G.alloc, **k)
 
 
 def _spread_rows(S, n, seed):
@@ -45,8 +56,8 @@ def test_8b_prefill_block_full_sequence():
     w = I.WORKLOADS["llama3_8b_prefill"].replace(input_kind="activations")
     layer = I.layer_weights(w, 0, DEV)
     S = w.seq
-    st = Llama3Stack(w.cfg(), [layer], I.output_weights(w, DEV), 1, S, S, lm_rows=1)
-    x = I.activations(w, DEV)
+    st = Stack(w.cfg(), [layer], I.output_weights(w, DEV), 1, S, S, lm_rows=1)
+    x = G.to(I.activations(w, DEV))
     x0 = f64(x)[0]
     st.forward_layers(x, S, 0)
     torch.cuda.synchronize()
@@ -65,12 +76,12 @@ def test_8b_decode_block_all_sequences():
     w8 = I.WORKLOADS["llama3_8b_prefill"]
     layer = I.layer_weights(w8, 0, DEV)
     P = wd.cache_len
-    kc, vc = I.kv_cache(wd, 0, P + 1, DEV)
-    st = Llama3Stack(w8.cfg(), [layer], I.output_weights(w8, DEV), wd.batch, P + 1, 1, lm_rows=wd.batch,
-                     caches=[(kc, vc)])
+    kc, vc = (G.to(t) for t in I.kv_cache(wd, 0, P + 1, DEV))
+    st = Stack(w8.cfg(), [layer], I.output_weights(w8, DEV), wd.batch, P + 1, 1, lm_rows=wd.batch,
+               caches=[(kc, vc)])
     g = torch.Generator(device="cpu").manual_seed(31)
     x = torch.randn((wd.batch, 1, wd.dim), generator=g).to(torch.bfloat16)
-    xd = x.to(DEV)
+    xd = G.to(x)
     st.decode_layers(xd, P)
     torch.cuda.synchronize()
     # the cache prefix is an input: draw it again (same seeds) for the oracle
@@ -95,8 +106,8 @@ def test_wide_prefill_layer(dim, H, KV, F):
     w = I.Workload("wide", dim=dim, n_layers=1, n_heads=H, n_kv_heads=KV, ffn_hidden=F, vocab=None, batch=1,
                    seq=640, dtype="bf16", input_kind="activations", seed=dim)
     layer = I.layer_weights(w, 0, DEV, "random")
-    st = Llama3Stack(w.cfg(), [layer], {}, 1, w.seq, w.seq)
-    x = I.activations(w, DEV)
+    st = Stack(w.cfg(), [layer], {}, 1, w.seq, w.seq)
+    x = G.to(I.activations(w, DEV))
     x0 = f64(x)
     st.forward_layers(x, w.seq, 0)
     torch.cuda.synchronize()
@@ -116,9 +127,9 @@ def test_wide_decode_layer_uses_separate_reductions():
                    batch=4, seq=1, dtype="bf16", input_kind="activations", seed=16896, cache_len=300)
     layer = I.layer_weights(w, 0, DEV, "random")
     P = w.cache_len
-    kc, vc = I.kv_cache(w, 0, P + 1, DEV)
-    st = Llama3Stack(w.cfg(), [layer], {}, w.batch, P + 1, 1, caches=[(kc, vc)])
-    x = I.activations(w, DEV)
+    kc, vc = (G.to(t) for t in I.kv_cache(w, 0, P + 1, DEV))
+    st = Stack(w.cfg(), [layer], {}, w.batch, P + 1, 1, caches=[(kc, vc)])
+    x = G.to(I.activations(w, DEV))
     x0 = f64(x)
     st.decode_layers(x, P)
     torch.cuda.synchronize()

@@ -6,7 +6,7 @@ import numpy as np
 import pytest
 import torch
 
-from helpers import assert_argmax, assert_close, f64, oracle_cfg, oracle_layer
+from helpers import GuardArena, assert_argmax, assert_close, f64, oracle_cfg, oracle_layer
 from llama_decoder_only_rmsnorm_b200 import binding as B
 from llama_decoder_only_rmsnorm_b200 import inputs as I
 from llama_decoder_only_rmsnorm_b200.model import Llama3Stack
@@ -16,15 +16,26 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
+G = None   # the running test's guard arena: every output / cache / workspace sits between guard bands
+
+
 @pytest.fixture(autouse=True)
 def _gpu_state():
+    global G
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
     B.llama3_set_kernel_path(0)
+    G = GuardArena(DEV)
     yield
     B.llama3_set_kernel_path(0)
     torch.cuda.synchronize()
     assert B.llama3_device_status() == 0, "device status word set"
+    G.check()
+
+
+def Stack(*a, **k):
+    """Llama3Stack whose buffers all come from the guard arena."""
+    return Llama3Stack(*a, alloc=G.alloc, **k)
 
 
 def wl(name, **kw):
@@ -47,7 +58,7 @@ def test_rmsnorm(dtype, D, H, rows):
     stride = D + 64
     x = (torch.randn((rows, stride), generator=g) * 3).to(tdt).to(DEV)
     nw = (1 + 0.1 * torch.randn((D,), generator=g)).to(tdt).to(DEV)
-    y = torch.empty((rows, D), dtype=tdt, device=DEV)
+    y = G.empty((rows, D), dtype=tdt, device=DEV)
     cfg = B.make_config(D, H, 1, 8 * D, dtype=dtype)
     B.llama3_rmsnorm(cfg, x, stride, nw, y, rows)
     want = O.rms_norm(f64(x)[:, :D], f64(nw), 1e-5)
@@ -67,9 +78,9 @@ def test_linear(m, n, k, residual, path):
     x = torch.randn((m, k), generator=g).to(torch.bfloat16).to(DEV)
     w = (torch.randn((n, k), generator=g) * 0.05).to(torch.bfloat16).to(DEV)
     r = torch.randn((m, n), generator=g).to(torch.bfloat16).to(DEV) if residual else None
-    y = torch.empty((m, n), dtype=torch.bfloat16, device=DEV)
+    y = G.empty((m, n), dtype=torch.bfloat16, device=DEV)
     cfg = B.make_config(512, 8, 8, 1024)
-    ws = torch.empty((m * n * 4,), dtype=torch.uint8, device=DEV)
+    ws = G.empty((m * n * 4,), dtype=torch.uint8, device=DEV)
     B.llama3_linear(cfg, x, w, r, y, m, n, k, ws, ws.numel())
     want = f64(x) @ f64(w).T + (f64(r) if residual else 0.0)
     assert_close(y, want, "bf16", f"linear {m}x{n}x{k}")
@@ -105,8 +116,8 @@ def test_attention(Bn, S, P, H, KV, hd):
     q, kc, vc, cap = _attn_case(Bn, S, P, H, KV, hd, Bn * 1000 + S + P + hd)
     cfg = B.make_config(H * hd, H, KV, 1024)
     ws_bytes = B.llama3_workspace_size(cfg, Bn, S, 1)
-    ws = torch.empty((ws_bytes,), dtype=torch.uint8, device=DEV)
-    out = torch.empty((Bn, S, H * hd), dtype=torch.bfloat16, device=DEV)
+    ws = G.empty((ws_bytes,), dtype=torch.uint8, device=DEV)
+    out = G.empty((Bn, S, H * hd), dtype=torch.bfloat16, device=DEV)
     B.llama3_attention(cfg, q.to(DEV), kc.to(DEV), vc.to(DEV), cap, Bn, S, P, out, ws, ws_bytes)
     for b in range(Bn):
         want = O.gqa_attention(f64(q[b]), f64(kc[b, :P + S]), f64(vc[b, :P + S]), P)
@@ -120,14 +131,14 @@ def _run_layers_vs_oracle(w, norm_weight="random", path=0):
     outw = I.output_weights(w, DEV, norm_weight)
     cfg = w.cfg()
     rows = w.batch * w.seq if w.lm_rows == "all" else w.batch
-    st = Llama3Stack(cfg, layers, outw, w.batch, w.seq, w.seq, lm_rows=rows if w.vocab else 0)
+    st = Stack(cfg, layers, outw, w.batch, w.seq, w.seq, lm_rows=rows if w.vocab else 0)
     if w.input_kind == "ids":
         ids = I.token_ids(w, DEV)
-        x = torch.empty((w.batch, w.seq, w.dim), dtype=w.torch_dtype, device=DEV)
+        x = G.empty((w.batch, w.seq, w.dim), dtype=w.torch_dtype, device=DEV)
         st.embed(ids, x)
         x0 = O.embed(ids.cpu().numpy(), f64(outw["tok_embeddings"]))
     else:
-        x = I.activations(w, DEV)
+        x = G.to(I.activations(w, DEV))
         x0 = f64(x)
     st.forward_layers(x, w.seq)
     torch.cuda.synchronize()
@@ -138,7 +149,7 @@ def _run_layers_vs_oracle(w, norm_weight="random", path=0):
         assert_close(kc, kcs[i], w.dtype, f"{w.name} k cache layer {i}")
         assert_close(vc, vcs[i], w.dtype, f"{w.name} v cache layer {i}")
     if w.vocab:
-        logits = torch.empty((rows, w.vocab), dtype=torch.float32, device=DEV)
+        logits = G.empty((rows, w.vocab), dtype=torch.float32, device=DEV)
         ids_out = st.lm_head(x, rows, w.dim, logits)
         want_logits, _ = O.lm_head(h.reshape(rows, w.dim), f64(outw["norm"]), f64(outw["output"]), w.norm_eps)
         assert_close(logits, want_logits, w.dtype, f"{w.name} logits")
@@ -168,14 +179,14 @@ def test_chunked_prefill_then_decode_steps():
     w = small_bf16()
     layers = [I.layer_weights(w, i, DEV, "random") for i in range(w.n_layers)]
     cap, total = 200, 70 + 50 + 3
-    st = Llama3Stack(w.cfg(), layers, I.output_weights(w, DEV), w.batch, cap, 70)
+    st = Stack(w.cfg(), layers, I.output_weights(w, DEV), w.batch, cap, 70)
     g = torch.Generator(device="cpu").manual_seed(9)
     xs = torch.randn((w.batch, total, w.dim), generator=g).to(torch.bfloat16)
     outs = []
-    a = xs[:, :70].contiguous().to(DEV); st.forward_layers(a, 70, 0); outs.append(a)
-    b = xs[:, 70:120].contiguous().to(DEV); st.forward_layers(b, 50, 70); outs.append(b)
+    a = G.to(xs[:, :70].contiguous()); st.forward_layers(a, 70, 0); outs.append(a)
+    b = G.to(xs[:, 70:120].contiguous()); st.forward_layers(b, 50, 70); outs.append(b)
     for t in range(120, total):
-        d = xs[:, t:t + 1].contiguous().to(DEV)
+        d = G.to(xs[:, t:t + 1].contiguous())
         st.decode_layers(d, t)
         outs.append(d)
     got = torch.cat([o.cpu() for o in outs], 1)
@@ -190,12 +201,12 @@ def test_decode_step_matches_prefill_path_for_large_batch():
     """batch > 256 decode routes to the prefill GEMMs; same answer as the oracle."""
     w = small_bf16(batch=300, n_layers=1, dim=256, n_heads=4, n_kv_heads=2, ffn_hidden=512)
     layers = [I.layer_weights(w, 0, DEV, "random")]
-    st = Llama3Stack(w.cfg(), layers, I.output_weights(w, DEV), w.batch, 8, 3)
+    st = Stack(w.cfg(), layers, I.output_weights(w, DEV), w.batch, 8, 3)
     g = torch.Generator(device="cpu").manual_seed(11)
     xs = torch.randn((w.batch, 4, w.dim), generator=g).to(torch.bfloat16)
-    a = xs[:, :3].contiguous().to(DEV)
+    a = G.to(xs[:, :3].contiguous())
     st.forward_layers(a, 3, 0)
-    d = xs[:, 3:4].contiguous().to(DEV)
+    d = G.to(xs[:, 3:4].contiguous())
     st.decode_layers(d, 3)
     want, _, _ = O.forward_stack(f64(xs), [oracle_layer(l) for l in layers], oracle_cfg(w))
     assert_close(torch.cat([a.cpu(), d.cpu()], 1), want, "bf16", "batch-300 decode")
@@ -208,15 +219,15 @@ def test_decode_stream_k_gemm_with_garbage_workspace():
     slab left unwritten poisons the block output."""
     w = small_bf16(batch=32, n_layers=1, dim=512, n_heads=8, n_kv_heads=2, ffn_hidden=5632)
     layers = [I.layer_weights(w, 0, DEV, "random")]
-    st = Llama3Stack(w.cfg(), layers, I.output_weights(w, DEV), w.batch, 48, 40)
+    st = Stack(w.cfg(), layers, I.output_weights(w, DEV), w.batch, 48, 40)
     st.ws.view(torch.float32).fill_(float("nan"))
     g = torch.Generator(device="cpu").manual_seed(17)
     xs = torch.randn((w.batch, 42, w.dim), generator=g).to(torch.bfloat16)
-    a = xs[:, :40].contiguous().to(DEV)
+    a = G.to(xs[:, :40].contiguous())
     st.forward_layers(a, 40, 0)
     outs = [a]
     for t in (40, 41):
-        d = xs[:, t:t + 1].contiguous().to(DEV)
+        d = G.to(xs[:, t:t + 1].contiguous())
         st.decode_layers(d, t)
         outs.append(d)
     want, _, _ = O.forward_stack(f64(xs), [oracle_layer(l) for l in layers], oracle_cfg(w))
@@ -231,11 +242,11 @@ def test_lm_head_8b_vocab(rows):
     h = I.hidden_rows(w, rows, DEV, std=2.0)
     cfg = B.make_config(w.dim, w.n_heads, w.n_kv_heads, w.ffn_hidden, w.vocab)
     ws_bytes = B.llama3_workspace_size(cfg, 1, 1, rows)
-    ws = torch.empty((ws_bytes,), dtype=torch.uint8, device=DEV)
-    ids = torch.empty((rows,), dtype=torch.int32, device=DEV)
-    logits = torch.empty((rows, w.vocab), dtype=torch.float32, device=DEV)
+    ws = G.empty((ws_bytes,), dtype=torch.uint8, device=DEV)
+    ids = G.empty((rows,), dtype=torch.int32, device=DEV)
+    logits = G.empty((rows, w.vocab), dtype=torch.float32, device=DEV)
     B.llama3_lm_head_argmax(cfg, outw["norm"], outw["output"], h, rows, w.dim, ids, logits, ws, ws_bytes)
-    ids2 = torch.empty_like(ids)
+    ids2 = G.empty_like(ids)
     B.llama3_lm_head_argmax(cfg, outw["norm"], outw["output"], h, rows, w.dim, ids2, None, ws, ws_bytes)
     want, _ = O.lm_head(f64(h), f64(outw["norm"]), f64(outw["output"]), w.norm_eps)
     assert_close(logits, want, "bf16", "8b logits")
@@ -246,12 +257,12 @@ def test_lm_head_8b_vocab(rows):
 def test_lm_head_row_stride_selects_last_positions():
     w = small_bf16()
     outw = I.output_weights(w, DEV, "random")
-    x = I.activations(w, DEV)  # [3, 70, 512]
+    x = G.to(I.activations(w, DEV))  # [3, 70, 512]
     cfg = B.make_config(w.dim, w.n_heads, w.n_kv_heads, w.ffn_hidden, w.vocab)
     ws_bytes = B.llama3_workspace_size(cfg, 1, 1, w.batch)
-    ws = torch.empty((ws_bytes,), dtype=torch.uint8, device=DEV)
-    ids = torch.empty((w.batch,), dtype=torch.int32, device=DEV)
-    logits = torch.empty((w.batch, w.vocab), dtype=torch.float32, device=DEV)
+    ws = G.empty((ws_bytes,), dtype=torch.uint8, device=DEV)
+    ids = G.empty((w.batch,), dtype=torch.int32, device=DEV)
+    logits = G.empty((w.batch, w.vocab), dtype=torch.float32, device=DEV)
     B.llama3_lm_head_argmax(cfg, outw["norm"], outw["output"], x[:, -1], w.batch, w.seq * w.dim, ids, logits,
                             ws, ws_bytes)
     want, _ = O.lm_head(f64(x)[:, -1], f64(outw["norm"]), f64(outw["output"]), w.norm_eps)
@@ -262,13 +273,13 @@ def test_lm_head_row_stride_selects_last_positions():
 def test_lm_head_ties_pick_lowest_index():
     V, D = 300, 512
     cfg = B.make_config(D, 8, 2, 1024, V)
-    wout = torch.zeros((V, D), dtype=torch.bfloat16, device=DEV)
+    wout = G.zeros((V, D), dtype=torch.bfloat16, device=DEV)
     wout[[17, 40, 299]] = 1.0
     h = torch.ones((2, D), dtype=torch.bfloat16, device=DEV)
     nw = torch.ones((D,), dtype=torch.bfloat16, device=DEV)
     ws_bytes = B.llama3_workspace_size(cfg, 1, 1, 2)
-    ws = torch.empty((ws_bytes,), dtype=torch.uint8, device=DEV)
-    ids = torch.empty((2,), dtype=torch.int32, device=DEV)
+    ws = G.empty((ws_bytes,), dtype=torch.uint8, device=DEV)
+    ids = G.empty((2,), dtype=torch.int32, device=DEV)
     for path in (0, 1):
         B.llama3_set_kernel_path(path)
         B.llama3_lm_head_argmax(cfg, nw, wout, h, 2, D, ids, None, ws, ws_bytes)
@@ -280,7 +291,7 @@ def test_embed_out_of_range_id_is_reported():
     outw = I.output_weights(w, DEV)
     cfg = B.make_config(w.dim, w.n_heads, w.n_kv_heads, w.ffn_hidden, w.vocab)
     ids = torch.tensor([0, 5, w.vocab + 3], dtype=torch.int32, device=DEV)
-    x = torch.empty((3, w.dim), dtype=torch.bfloat16, device=DEV)
+    x = G.empty((3, w.dim), dtype=torch.bfloat16, device=DEV)
     B.llama3_embed(cfg, ids, outw["tok_embeddings"], x, 3)
     assert B.llama3_device_status() == 6
     assert torch.equal(x[1], outw["tok_embeddings"][5])
@@ -295,10 +306,10 @@ def test_greedy_generation_matches_oracle():
     layers = [I.layer_weights(w, i, DEV, "random") for i in range(w.n_layers)]
     outw = I.output_weights(w, DEV, "random")
     n_new = 12
-    st = Llama3Stack(w.cfg(), layers, outw, w.batch, w.seq + n_new, w.seq, lm_rows=w.batch)
+    st = Stack(w.cfg(), layers, outw, w.batch, w.seq + n_new, w.seq, lm_rows=w.batch)
     prompt = I.token_ids(w, DEV)
     got = st.generate(prompt, n_new)
-    st2 = Llama3Stack(w.cfg(), layers, outw, w.batch, w.seq + n_new, w.seq, lm_rows=w.batch)
+    st2 = Stack(w.cfg(), layers, outw, w.batch, w.seq + n_new, w.seq, lm_rows=w.batch)
     np.testing.assert_array_equal(st2.generate(prompt, n_new, cuda_graph=True), got)   # graph replay, same tokens
     toks, gaps = O.generate_greedy(prompt.cpu().numpy(), f64(outw["tok_embeddings"]),
                                    [oracle_layer(l) for l in layers], f64(outw["norm"]), f64(outw["output"]),
@@ -321,10 +332,10 @@ def test_greedy_generation_with_prompts_of_different_lengths():
     layers = [I.layer_weights(w, i, DEV, "random") for i in range(w.n_layers)]
     outw = I.output_weights(w, DEV, "random")
     n_new, lens = 10, [20, 7, 13]
-    st = Llama3Stack(w.cfg(), layers, outw, w.batch, w.seq + n_new, w.seq, lm_rows=w.batch)
+    st = Stack(w.cfg(), layers, outw, w.batch, w.seq + n_new, w.seq, lm_rows=w.batch)
     prompt = I.token_ids(w, DEV)
     got = st.generate(prompt, n_new, prompt_lens=lens)
-    st2 = Llama3Stack(w.cfg(), layers, outw, w.batch, w.seq + n_new, w.seq, lm_rows=w.batch)
+    st2 = Stack(w.cfg(), layers, outw, w.batch, w.seq + n_new, w.seq, lm_rows=w.batch)
     np.testing.assert_array_equal(st2.generate(prompt, n_new, prompt_lens=lens, cuda_graph=True), got)
     host = prompt.cpu().numpy()
     compared = 0
@@ -371,7 +382,7 @@ def test_greedy_generation_stops_at_end_token():
     want, wgaps = O.generate_greedy(*args, eos_id=eos)
     assert np.all(want[1, t_end:] == eos)
     for graph in (False, True):
-        st = Llama3Stack(w.cfg(), layers, outw, w.batch, w.seq + n_new, w.seq, lm_rows=w.batch)
+        st = Stack(w.cfg(), layers, outw, w.batch, w.seq + n_new, w.seq, lm_rows=w.batch)
         got = st.generate(prompt, n_new, eos_id=eos, cuda_graph=graph)
         assert np.all(got[1, t_end:] == eos), (graph, got[1])
         for b in range(w.batch):
@@ -398,7 +409,7 @@ def test_generation_ends_when_every_sequence_is_done():
     assert t_end is not None and t_end + 1 < n_new
     eos = int(toks[0, t_end])
     for graph in (False, True):
-        st = Llama3Stack(w.cfg(), layers, outw, w.batch, w.seq + n_new, w.seq, lm_rows=w.batch)
+        st = Stack(w.cfg(), layers, outw, w.batch, w.seq + n_new, w.seq, lm_rows=w.batch)
         got = st.generate(prompt, n_new, eos_id=eos, cuda_graph=graph)
         np.testing.assert_array_equal(got[0, :t_end + 1], toks[0, :t_end + 1])
         assert np.all(got[0, t_end:] == eos)
@@ -413,14 +424,14 @@ def test_decode_blocks_in_any_order(order):
     that order (norm weights random, so a wrong hand-off shows)."""
     w = small_bf16(n_layers=3, batch=4, seq=30)
     layers = [I.layer_weights(w, i, DEV, "random") for i in range(w.n_layers)]
-    st = Llama3Stack(w.cfg(), layers, I.output_weights(w, DEV), w.batch, 40, 30)
+    st = Stack(w.cfg(), layers, I.output_weights(w, DEV), w.batch, 40, 30)
     g = torch.Generator(device="cpu").manual_seed(23)
     xs = torch.randn((w.batch, 32, w.dim), generator=g).to(torch.bfloat16)
-    a = xs[:, :30].contiguous().to(DEV)
+    a = G.to(xs[:, :30].contiguous())
     st.forward_layers(a, 30, 0, layers=order)
     outs = [a]
     for t in (30, 31):
-        d = xs[:, t:t + 1].contiguous().to(DEV)
+        d = G.to(xs[:, t:t + 1].contiguous())
         st.decode_layers(d, t, layers=order)
         outs.append(d)
     want, kcs, vcs = O.forward_stack(f64(xs), [oracle_layer(layers[i]) for i in order], oracle_cfg(w))
@@ -454,8 +465,8 @@ def test_attention_document_mask(Bn, S, P, H, KV, hd, path):
     ds = _doc_starts(Bn, S, P, S + hd)
     cfg = B.make_config(H * hd, H, KV, 1024)
     ws_bytes = B.llama3_workspace_size(cfg, Bn, S, 1)
-    ws = torch.empty((ws_bytes,), dtype=torch.uint8, device=DEV)
-    out = torch.empty((Bn, S, H * hd), dtype=torch.bfloat16, device=DEV)
+    ws = G.empty((ws_bytes,), dtype=torch.uint8, device=DEV)
+    out = G.empty((Bn, S, H * hd), dtype=torch.bfloat16, device=DEV)
     B.llama3_attention_docs(cfg, q.to(DEV), kc.to(DEV), vc.to(DEV), cap, Bn, S, P, torch.from_numpy(ds).to(DEV), out,
                             ws, ws_bytes)
     for b in range(Bn):
@@ -466,10 +477,10 @@ def test_attention_document_mask(Bn, S, P, H, KV, hd, path):
 def test_layer_forward_packed_documents():
     w = small_bf16(n_layers=2, seq=150)
     layers = [I.layer_weights(w, i, DEV, "random") for i in range(w.n_layers)]
-    st = Llama3Stack(w.cfg(), layers, I.output_weights(w, DEV), w.batch, w.seq, w.seq)
+    st = Stack(w.cfg(), layers, I.output_weights(w, DEV), w.batch, w.seq, w.seq)
     ds = _doc_starts(w.batch, w.seq, 0, 11)
     dsd = torch.from_numpy(ds).to(DEV)
-    x = I.activations(w, DEV)
+    x = G.to(I.activations(w, DEV))
     x0 = f64(x)
     for i in range(w.n_layers):
         kc, vc = st.caches[i]
@@ -494,7 +505,7 @@ def test_ragged_decode_step_matches_per_sequence_oracle(dtype, path):
     layer = I.layer_weights(w, 0, DEV, "random")
     cap = 200
     positions = np.array([0, 37, 128, 129, 150], dtype=np.int32)
-    st = Llama3Stack(w.cfg(), [layer], I.output_weights(w, DEV), w.batch, cap, 1)
+    st = Stack(w.cfg(), [layer], I.output_weights(w, DEV), w.batch, cap, 1)
     kc, vc = st.caches[0]
     g = torch.Generator(device="cpu").manual_seed(21)
     k0 = torch.randn(kc.shape, generator=g).to(kc.dtype)

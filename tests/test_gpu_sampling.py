@@ -12,7 +12,7 @@ import numpy as np
 import pytest
 import torch
 
-from helpers import assert_close, f64, oracle_cfg, oracle_layer
+from helpers import GuardArena, assert_close, f64, oracle_cfg, oracle_layer
 from llama_decoder_only_rmsnorm_b200 import binding as B
 from llama_decoder_only_rmsnorm_b200 import inputs as I
 from llama_decoder_only_rmsnorm_b200.model import Llama3Stack
@@ -23,13 +23,24 @@ DEV = "cuda"
 MARGIN = 1e-5
 
 
+G = None   # the running test's guard arena: outputs, caches and workspaces sit between guard bands
+
+
 @pytest.fixture(autouse=True)
 def _gpu_state():
+    global G
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
+    G = GuardArena(DEV)
     yield
     torch.cuda.synchronize()
     assert B.llama3_device_status() == 0, "device status word set"
+    G.check()
+
+
+def Stack(*a, **k):
+    """Llama3Stack whose buffers all come from the guard arena."""
+    return Llama3Stack(*a, alloc=G.alloc, **k)
 
 
 def _sample(lg, T, top_p, seed, offset, ld=None):
@@ -38,7 +49,7 @@ def _sample(lg, T, top_p, seed, offset, ld=None):
     buf = torch.zeros((R, ld), dtype=torch.float32)
     buf[:, :V] = torch.from_numpy(lg)
     d = buf.to(DEV)
-    ids = torch.full((R,), -1, dtype=torch.int32, device=DEV)
+    ids = G.full((R,), -1, dtype=torch.int32, device=DEV)
     B.llama3_sample_top_p(d, R, ld, V, T, top_p, seed, offset, ids)
     return ids.cpu().numpy()
 
@@ -126,7 +137,7 @@ def test_sampled_generation_draws_from_the_models_logits():
     layers = [I.layer_weights(w, i, DEV, "random") for i in range(w.n_layers)]
     outw = I.output_weights(w, DEV, "random")
     n_new, T, top_p, seed = 10, 0.8, 0.9, 2024
-    st = Llama3Stack(w.cfg(), layers, outw, w.batch, w.seq + n_new, w.seq, lm_rows=w.batch)
+    st = Stack(w.cfg(), layers, outw, w.batch, w.seq + n_new, w.seq, lm_rows=w.batch)
     prompt = I.token_ids(w, DEV)
     toks, logits = st.generate(prompt, n_new, temperature=T, top_p=top_p, seed=seed, return_logits=True)
     T32, p32 = float(np.float32(T)), float(np.float32(top_p))
@@ -148,6 +159,6 @@ def test_sampled_generation_draws_from_the_models_logits():
     got = logits.transpose(1, 0, 2).reshape(-1, w.vocab)
     assert_close(got, want_logits, "bf16", "generation logits")
     # the same loop captured once in a CUDA graph and replayed draws the same tokens
-    st2 = Llama3Stack(w.cfg(), layers, outw, w.batch, w.seq + n_new, w.seq, lm_rows=w.batch)
+    st2 = Stack(w.cfg(), layers, outw, w.batch, w.seq + n_new, w.seq, lm_rows=w.batch)
     toks_graph = st2.generate(prompt, n_new, temperature=T, top_p=top_p, seed=seed, cuda_graph=True)
     np.testing.assert_array_equal(toks_graph, toks)

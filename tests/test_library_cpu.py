@@ -113,6 +113,9 @@ def test_kernel_path_and_wait_limit_switches():
     assert B.llama3_set_kernel_path(0) == 0
     old = B.llama3_set_wait_limit_ms(500)
     assert B.llama3_set_wait_limit_ms(old) == 500
+    assert B.llama3_set_test_withheld_arrival(1) == 0      # test hook, off by default
+    assert B.llama3_set_test_withheld_arrival(7) == 1      # unknown values switch it off
+    assert B.llama3_set_test_withheld_arrival(0) == 0
 
 
 def test_sample_top_p_rejects_bad_arguments_before_launch():
