@@ -361,7 +361,8 @@ def run_ours(args):
     roofline = {"bound": "tensor", "kernel": "tc_gemm w1|w3 + SwiGLU (M=8192, N=2x14336, K=4096)",
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": (achieved / peak) if achieved else None, "peak_source": peak_src,
-                "traffic": recorded_traffic("gemm_w13", ["llama_decoder_only_rmsnorm_b200/csrc/tc_gemm.cuh"]),
+                "traffic": recorded_traffic("gemm_w13", ["llama_decoder_only_rmsnorm_b200/csrc/tc_gemm.cuh",
+                                                         "llama_decoder_only_rmsnorm_b200/csrc/llama3.cu"]),
                 "kernel_ms": k_ms, "timed_launches": len(w13)}
     total_flop = n_layers * (2.0 * S * 6.979e9 / 32) + 2.0 * D * PREFILL.vocab  # linear layers + LM head row
     attn_flop = n_layers * PREFILL.n_heads * 2.0 * S * (S + 1) * PREFILL.head_dim

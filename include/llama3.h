@@ -24,8 +24,9 @@
  *  - Row-major, densely packed.  Linear weights are [out, in] and a Linear
  *    computes y = x W^T ([S1] §6.5, [S2] §3.4 nn.Linear(bias=False)).
  *  - Element type of activations, weights and caches is cfg->dtype:
- *    LLAMA3_DTYPE_BF16 (bfloat16, the fast tcgen05 path) or LLAMA3_DTYPE_F32
- *    (float, SIMT kernels, meant for small models).  Accumulation is fp32.
+ *    LLAMA3_DTYPE_BF16 (bfloat16, the fast tcgen05 path for head_dim >= 64;
+ *    head_dim 16 and 32 run on the SIMT kernels) or LLAMA3_DTYPE_F32 (float,
+ *    SIMT kernels, meant for small models).  Accumulation is fp32.
  *  - Every device pointer must be 16-byte aligned (LLAMA3_ERR_ALIGN).
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *    default stream) and may be captured in a CUDA graph.
@@ -64,7 +65,7 @@ enum llama3_status {
  * Model hyper-parameters -- the ModelArgs / params.json fields of [S1] §2 and
  * [S2] §1.2.  Constraints checked by every call:
  *   dim == n_heads * head_dim; n_heads % n_kv_heads == 0; head_dim even and
- *   in {16, 32, 64, 96, 128} (bf16 needs head_dim >= 64); ffn_hidden >= 1;
+ *   in {16, 32, 64, 96, 128}; ffn_hidden >= 1;
  *   norm_eps > 0; rope_theta > 1; dim and ffn_hidden multiples of 8 for bf16,
  *   of 4 for fp32.
  * ffn_hidden is taken as given (the caller applies the hidden-size rule of

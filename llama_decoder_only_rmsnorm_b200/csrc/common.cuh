@@ -148,12 +148,19 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
-// Programmatic dependent launch: wait until the grids this one depends on have
-// completed and flushed their memory; then allow the next grid in the stream
-// to be scheduled (it waits the same way before touching our outputs).
+// Programmatic dependent launch: allow the next grid in the stream to be
+// scheduled (it waits the same way before touching our outputs), then wait
+// until the grids this one depends on have completed and flushed their memory.
+//
+// The release comes first: the next kernel may then be scheduled as soon as
+// this one's CTAs are all resident, so its set-up and weight loads overlap
+// this kernel's whole run, not only its tail.  This cannot deadlock: a
+// dependent grid starts only after every CTA of its predecessor has released
+// (so all of them are resident and will finish), and nothing a kernel does
+// before its wait reads memory an earlier kernel writes.
 __device__ __forceinline__ void griddep_wait_and_release() {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------

@@ -173,6 +173,28 @@ def test_gqa_768_layer():
     _run_layers_vs_oracle(wl("gqa_768"))
 
 
+@pytest.mark.parametrize("hd,H,KV", [(16, 8, 2), (32, 8, 4)])
+def test_bf16_small_head_dims_prefill_decode_lm_head(hd, H, KV):
+    """bf16 models with head_dim 16 or 32 (the SIMT kernels): a 2-block
+    prefill with the LM head on every row, then two decode steps."""
+    w = small_bf16(dim=H * hd, n_heads=H, n_kv_heads=KV, ffn_hidden=4 * H * hd, batch=2, seq=40, vocab=500,
+                   seed=hd)
+    _run_layers_vs_oracle(w)
+    layers = [I.layer_weights(w, i, DEV, "random") for i in range(w.n_layers)]
+    st = Stack(w.cfg(), layers, I.output_weights(w, DEV), w.batch, 48, 40)
+    g = torch.Generator(device="cpu").manual_seed(hd)
+    xs = torch.randn((w.batch, 42, w.dim), generator=g).to(torch.bfloat16)
+    a = G.to(xs[:, :40].contiguous())
+    st.forward_layers(a, 40, 0)
+    outs = [a]
+    for t in (40, 41):
+        d = G.to(xs[:, t:t + 1].contiguous())
+        st.decode_layers(d, t)
+        outs.append(d)
+    want, _, _ = O.forward_stack(f64(xs), [oracle_layer(l) for l in layers], oracle_cfg(w))
+    assert_close(torch.cat([o.cpu() for o in outs], 1), want, "bf16", f"bf16 head_dim {hd}")
+
+
 def test_chunked_prefill_then_decode_steps():
     """Prefill 70 tokens, prefill a second chunk of 50 at start_pos 70, then
     three one-token decode steps -- against the oracle's full causal pass."""

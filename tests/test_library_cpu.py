@@ -40,15 +40,16 @@ def test_workspace_size_and_config_validation():
     assert n >= (3 * 8192 * 4096 + 8192 * 14336) * 2
     assert B.llama3_workspace_size(cfg8b(), 32, 1, 32) < n
     bad = [cfg8b(dim=4000), cfg8b(n_kv_heads=7), cfg8b(dim=4096 + 32, n_heads=33),
-           B.make_config(1024, 32, 8, 4096, 10),            # head_dim 32: bf16 needs >= 64
-           B.make_config(64, 4, 2, 192, 10, dtype="bf16"),  # head_dim 16 in bf16
+           B.make_config(48 * 8, 8, 2, 1024, 10),           # head_dim 48: not a supported size
            cfg8b(ffn_hidden=14337), cfg8b(norm_eps=0.0), cfg8b(rope_theta=1.0)]
     for c in bad:
         with pytest.raises(B.Llama3Error) as e:
             B.llama3_workspace_size(c, 1, 16, 1)
         assert e.value.status == 1
-    # fp32 with head_dim 16 is valid (SIMT kernels)
+    # head_dim 16 and 32 are valid in fp32 and bf16 (SIMT kernels)
     assert B.llama3_workspace_size(B.make_config(64, 4, 2, 192, 3771, dtype="f32"), 4, 16, 64) > 0
+    assert B.llama3_workspace_size(B.make_config(64, 4, 2, 192, 10, dtype="bf16"), 4, 16, 1) > 0
+    assert B.llama3_workspace_size(B.make_config(1024, 32, 8, 4096, 10), 2, 16, 1) > 0
     with pytest.raises(B.Llama3Error):
         B.llama3_workspace_size(cfg8b(), 0, 16, 1)
 
