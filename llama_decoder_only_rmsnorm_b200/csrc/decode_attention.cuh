@@ -12,21 +12,24 @@
 
 namespace l3 {
 
-// Partial record per (b, h, split): m (running max of the scores, log2
-// domain), l (sum of 2^(s - m)), acc[hd] (sum of 2^(s - m) * v).  Stored as
-// floats [B][H][splits][hd + 2] and merged by the combine kernel.
-// out[b, h, :] = sum_s e^(m_s - M) acc_s / sum_s e^(m_s - M) l_s
+// Partial record per (b, h, slot): m (running max of the scores, log2 domain),
+// l (sum of 2^(s - m)), acc[hd] (sum of 2^(s - m) * v).  Stored as floats
+// [B][H][slots][hd + 2] and merged by the combine kernel:
+// out[b, h, :] = sum_s e^(m_s - M) acc_s / sum_s e^(m_s - M) l_s over the
+// first `used` slots of (b, h) (records_used below).
 template <int HD>
 __global__ void decode_attention_combine_kernel(const float* __restrict__ part, bf16* __restrict__ out,
-                                                int splits) {
+                                                int slots, int H, int nrep, int tiles, int per) {
   griddep_wait_and_release();
   const int bh = blockIdx.x;  // b * H + h
-  const float* p = part + (size_t)bh * splits * (HD + 2);
+  const int seg = (bh / H) * (H / nrep) + (bh % H) / nrep;   // (b, KV head h / nrep)
+  const int used = per > 0 ? 2 * ((seg * tiles + tiles - 1) / per - (seg * tiles) / per + 1) : slots;
+  const float* p = part + (size_t)bh * slots * (HD + 2);
   float mx = -INFINITY;
-  for (int s = 0; s < splits; ++s) mx = fmaxf(mx, p[s * (HD + 2)]);
+  for (int s = 0; s < used; ++s) mx = fmaxf(mx, p[s * (HD + 2)]);
   for (int d = threadIdx.x; d < HD; d += blockDim.x) {
     float num = 0.f, den = 0.f;
-    for (int s = 0; s < splits; ++s) {
+    for (int s = 0; s < used; ++s) {
       const float ms = p[s * (HD + 2)];
       const float f = ms == -INFINITY ? 0.f : exp2f(ms - mx);
       den += f * p[s * (HD + 2) + 1];
@@ -44,11 +47,21 @@ __global__ void decode_attention_combine_kernel(const float* __restrict__ part, 
 // Keys sit on the MMA's 128-row side, so the n_rep query heads of a group
 // (padded to 16 columns) share every K/V byte read.  Two softmax warpgroups
 // take alternate tiles, each with its own running (m, l, O^T), so one tile's
-// softmax overlaps the next one's; a work unit therefore yields two partial
-// records (slot 2*split + warpgroup) that the combine kernel merges.
+// softmax overlaps the next one's; a piece of work therefore yields two
+// partial records (slot 2*piece + warpgroup) that the combine kernel merges.
+//
+// Schedule: the key tiles of all (sequence, KV head) segments, laid end to
+// end (segment s = b*KV + g holds tiles s*tiles .. s*tiles + tiles - 1), are
+// cut into equal runs of `per` tiles, one per CTA, so every CTA streams the
+// same number of K/V bytes.  A run that crosses segment boundaries is split
+// there into pieces; piece j of a segment is the part of it that the
+// segment's j-th CTA (in run order) covers.
 // ===========================================================================
 struct DecodeShape {
-  int B, H, KV, nrep, n_keys, tiles, splits, tiles_per_split, units;
+  int B, H, KV, nrep, n_keys;
+  int tiles;      // key tiles per segment: ceil(n_keys / 128)
+  int per;        // tiles per CTA run
+  int slots;      // records per (b, h): 2 x the most pieces any segment has
   float scale_log2;
   // Optional per-sequence positions (device, [B]): sequence b's token sits at
   // positions[b] and sees keys 0..positions[b] (at most n_keys of them).
@@ -77,18 +90,28 @@ struct DecodeTcCfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
-// Unit u -> sequence b, KV head g, key tiles [t0, t1) and the number of keys
-// sequence b sees (n_keys, or positions[b] + 1 clamped to [1, n_keys]); a
-// unit past a short sequence's last tile is empty (t1 == t0).
-__device__ __forceinline__ void decode_unit(const DecodeShape& ds, int u, int& b, int& g, int& split, int& t0,
-                                            int& t1, int& nk) {
-  split = u % ds.splits;
-  const int bg = u / ds.splits;
-  g = bg % ds.KV;
-  b = bg / ds.KV;
+// Piece `it` of CTA c's run -> sequence b, KV head g, piece index j within
+// the segment, key tiles [t0, t1) and the number of keys sequence b sees (nk:
+// n_keys, or positions[b] + 1 clamped to [1, n_keys]); false once the run is
+// exhausted.  Tiles past a short sequence's last one are dropped, so a piece
+// may be empty (t1 == t0): it still writes its (empty) records.
+__device__ __forceinline__ bool decode_piece(const DecodeShape& ds, int c, int it, int& b, int& g, int& j, int& t0,
+                                             int& t1, int& nk) {
+  const long long total = (long long)ds.B * ds.KV * ds.tiles;
+  const long long a = (long long)c * ds.per, e = min(a + ds.per, total);
+  if (a >= e) return false;
+  const long long seg = a / ds.tiles + it;
+  const long long s0 = seg * ds.tiles;
+  if (s0 >= e) return false;
+  g = (int)(seg % ds.KV);
+  b = (int)(seg / ds.KV);
+  j = c - (int)(s0 / ds.per);
   nk = ds.positions ? max(1, min(ds.positions[b] + 1, ds.n_keys)) : ds.n_keys;
-  t0 = split * ds.tiles_per_split;
-  t1 = max(t0, min(t0 + ds.tiles_per_split, (nk + 127) / 128));
+  const int own = (nk + 127) / 128;
+  t0 = (int)max(a - s0, 0LL);
+  t1 = (int)min(e - s0, (long long)ds.tiles);
+  t1 = max(t0, min(t1, own));
+  return true;
 }
 
 template <int HD, int NREP>
@@ -159,9 +182,8 @@ __global__ void __launch_bounds__(384, 1)
       uint32_t ph = 0, qph[2] = {0, 0};
       uint32_t iss = 0, par = 0, qiss = 0, qpar = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < ds.units && ok; u += gridDim.x, ++kq) {
-        int b, g, split, t0, t1, nk;
-        decode_unit(ds, u, b, g, split, t0, t1, nk);
+      int b, g, piece, t0, t1, nk;
+      for (int it = 0; ok && decode_piece(ds, blockIdx.x, it, b, g, piece, t0, t1, nk); ++it, ++kq) {
         const int qb = kq & 1;
         if (!mbar_wait(&q_empty[qb], qph[qb] ^ 1u, wait_ns)) break;
         mbar_arrive_expect_tx(&q_full[qb], C::Q_BYTES);
@@ -194,9 +216,8 @@ __global__ void __launch_bounds__(384, 1)
       uint32_t ph = 0, qph[2] = {0, 0};
       uint32_t pph[2][2] = {{0, 0}, {0, 0}};
       bool ok = true;
-      for (int u = blockIdx.x; u < ds.units && ok; u += gridDim.x, ++kq) {
-        int b, g, split, t0, t1, nk;
-        decode_unit(ds, u, b, g, split, t0, t1, nk);
+      int b, g, piece, t0, t1, nk;
+      for (int it = 0; ok && decode_piece(ds, blockIdx.x, it, b, g, piece, t0, t1, nk); ++it, ++kq) {
         const int qb = kq & 1;
         const uint32_t q_addr = smem_u32(smem + C::OFF_Q + qb * C::Q_BYTES);
         if (!mbar_wait(&q_full[qb], qph[qb], wait_ns)) break;
@@ -265,9 +286,8 @@ __global__ void __launch_bounds__(384, 1)
       rph[rpar] ^= 1u;
       return done;
     };
-    for (int u = blockIdx.x; u < ds.units; u += gridDim.x) {
-      int b, g, split, t0, t1, nk;
-      decode_unit(ds, u, b, g, split, t0, t1, nk);
+    int b, g, piece, t0, t1, nk;
+    for (int it = 0; decode_piece(ds, blockIdx.x, it, b, g, piece, t0, t1, nk); ++it) {
       const int n = t1 - t0;
       const int mine = n > wg ? (n - wg + 1) / 2 : 0;   // tiles wg, wg+2, ...
       float m_ref[NREP], l_part[NREP];
@@ -367,11 +387,11 @@ __global__ void __launch_bounds__(384, 1)
       }
       if (!exchange()) break;
       rpar ^= 1;
-      const int slot = 2 * split + wg;
+      const int slot = 2 * piece + wg;
 #pragma unroll
       for (int h = 0; h < NREP; ++h) {
         if (h >= nrep) break;
-        float* rec = part + (((size_t)b * ds.H + g * nrep + h) * (2 * ds.splits) + slot) * (HD + 2);
+        float* rec = part + (((size_t)b * ds.H + g * nrep + h) * ds.slots + slot) * (HD + 2);
         if (row < HD) rec[2 + row] = o_val[h];
         if (row == 0) {
           rec[0] = m_ref[h];

@@ -540,6 +540,28 @@ int run_attention_simt(const llama3_config* c, const void* q, const void* kc, co
   return launch_check();
 }
 
+// Decode attention schedule: the segs x tiles key tiles, laid end to end, cut
+// into equal runs of *per tiles, one per CTA (*grid of them, at most sms).
+// *slots = 2 x the most runs one segment meets (two records per piece); the
+// run length grows until that fits the workspace's kMaxKvSplits records.
+bool plan_decode_runs(int segs, int tiles, int sms, int* per, int* slots, int* grid) {
+  const long long total = (long long)segs * tiles;
+  if (total <= 0 || sms <= 0) return false;
+  long long p = (total + sms - 1) / sms;
+  for (;; ++p) {
+    int most = 1;
+    for (long long s = 0; s < segs; ++s)
+      most = std::max(most, (int)((s * tiles + tiles - 1) / p - (s * tiles) / p + 1));
+    if (2 * most <= kMaxKvSplits) {
+      *per = (int)p;
+      *slots = 2 * most;
+      *grid = (int)((total + p - 1) / p);
+      return true;
+    }
+    if (p >= tiles) return false;
+  }
+}
+
 // Tensor-core decode attention: TMA-streamed K/V tiles, two tcgen05 MMAs per tile.
 template <int HD, int NREP>
 int run_decode_attention_tc_t(const llama3_config* c, const void* q, const void* kc, const void* vc, int cap,
@@ -555,22 +577,8 @@ int run_decode_attention_tc_t(const llama3_config* c, const void* q, const void*
   DecodeShape ds;
   ds.B = B; ds.H = H; ds.KV = KV; ds.nrep = H / KV; ds.n_keys = n_keys;
   ds.tiles = (n_keys + 127) / 128;
-  // Split count minimising the longest per-CTA stream on a persistent grid,
-  // counting one tile of fixed cost per work unit (Q load, per-warpgroup
-  // epilogue, partial records for the combine kernel); ties go to fewer splits.
-  const int sms = num_sms();
-  int best = 1;
-  long long best_t = -1;
-  for (int sp = 1; sp <= std::min(ds.tiles, kMaxKvSplits / 2); ++sp) {
-    const int per = (ds.tiles + sp - 1) / sp;
-    const int real = (ds.tiles + per - 1) / per;
-    const long long units = (long long)B * KV * real;
-    const long long t = ((units + sms - 1) / sms) * (per + 1);
-    if (best_t < 0 || t < best_t) { best_t = t; best = real; }
-  }
-  ds.tiles_per_split = (ds.tiles + best - 1) / best;
-  ds.splits = (ds.tiles + ds.tiles_per_split - 1) / ds.tiles_per_split;
-  ds.units = B * KV * ds.splits;
+  int grid = 0;
+  if (!plan_decode_runs(B * KV, ds.tiles, num_sms(), &ds.per, &ds.slots, &grid)) return LLAMA3_ERR_UNSUPPORTED;
   ds.scale_log2 = (float)(1.4426950408889634 / sqrt((double)HD));
   ds.positions = positions;
   auto kern = decode_attention_tc_kernel<HD, NREP>;
@@ -581,12 +589,12 @@ int run_decode_attention_tc_t(const llama3_config* c, const void* q, const void*
     L3_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES));
     attr_done[dev] = true;
   }
-  const int grid = std::min(ds.units, sms);
   L3_LAUNCH(LLAMA3_KERNEL_DECODE_ATTENTION, st,
             launch_k(kern, grid, 384, Cfg::SMEM_BYTES, st, mq, mk, mv, part, ds, wait_ns()));
   L3_TRY(launch_check());
   L3_LAUNCH(LLAMA3_KERNEL_ELEMENTWISE, st,
-            launch_k((decode_attention_combine_kernel<HD>), B * H, 128, 0, st, part, (bf16*)out, 2 * ds.splits));
+            launch_k((decode_attention_combine_kernel<HD>), B * H, 128, 0, st, part, (bf16*)out, ds.slots, H,
+                     ds.nrep, ds.tiles, ds.per));
   return launch_check();
 }
 
