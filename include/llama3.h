@@ -226,6 +226,26 @@ int llama3_layer_decode_chained(const llama3_config* cfg, const llama3_layer_wei
                                 llama3_stream_t stream);
 
 /*
+ * One decode step through a whole block stack ([S2] 四 Transformer.forward
+ * with one new token per sequence, 六 generate): block i of n_layers runs with
+ * layers[i] and the caches k_caches[i], v_caches[i] (host arrays of device
+ * pointers, [batch, cache_cap, KV, hd] each), in order, on x [batch, 1, D]
+ * (in: the embedded tokens; out: the last block's output, before the final
+ * norm).  positions == NULL: every token sits at start_pos; otherwise
+ * sequence b's token at positions[b] (device int32 [batch]) and start_pos
+ * bounds them all, as in llama3_layer_decode_ragged.  The same as calling
+ * llama3_layer_decode_chained for i = 0 .. n_layers-1 (each block handing the
+ * next its normalised input), as one call; every argument is checked for
+ * every block before the first launch.
+ * Errors as llama3_layer_decode for each block, plus LLAMA3_ERR_ARG for
+ * n_layers < 1 or NULL arrays.
+ */
+int llama3_decode_step(const llama3_config* cfg, const llama3_layer_weights* layers, int n_layers,
+                       const float* rope, int rope_len, void* x, void* const* k_caches,
+                       void* const* v_caches, int cache_cap, int batch, int start_pos,
+                       const int32_t* positions, void* ws, size_t ws_bytes, llama3_stream_t stream);
+
+/*
  * Output block ([S1] §11-12, [S3] 预测流程): for each of `rows` hidden rows
  * h[r] = h + r*row_stride (elements), compute logits = RMSNorm(h[r], norm_w)
  * W_out^T over the vocabulary and ids_out[r] = argmax (lowest index on ties).

@@ -53,6 +53,7 @@ _SIGNATURES = {
     "llama3_layer_decode": [_cfgp, _wp, _p, _i, _p, _p, _p, _i, _i, _i, _p, _sz, _p],
     "llama3_layer_decode_ragged": [_cfgp, _wp, _p, _i, _p, _p, _p, _i, _i, _p, _i, _p, _sz, _p],
     "llama3_layer_decode_chained": [_cfgp, _wp, _p, _i, _p, _p, _p, _i, _i, _i, _p, _p, _i, _p, _sz, _p],
+    "llama3_decode_step": [_cfgp, _wp, _i, _p, _i, _p, _p, _p, _i, _i, _i, _p, _p, _sz, _p],
     "llama3_layer_forward_docs": [_cfgp, _wp, _p, _i, _p, _p, _p, _i, _i, _i, _i, _p, _p, _sz, _p],
     "llama3_attention_docs": [_cfgp, _p, _p, _p, _i, _i, _i, _i, _p, _p, _p, _sz, _p],
     "llama3_lm_head_argmax": [_cfgp, _p, _p, _p, _i, _ll, _p, _p, _p, _sz, _p],
@@ -199,6 +200,21 @@ def llama3_layer_decode_chained(cfg, w, rope, rope_len, x, k_cache, v_cache, cac
         ctypes.byref(cfg), ctypes.byref(w), _ptr(rope), rope_len, _ptr(x), _ptr(k_cache), _ptr(v_cache),
         cache_cap, batch, start_pos, _ptr(positions), _ptr(next_attention_norm), 1 if input_normalised else 0,
         _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def llama3_decode_step(cfg, weights, rope, rope_len, x, k_caches, v_caches, cache_cap, batch, start_pos, positions,
+                       ws, ws_bytes, stream=None):
+    """One decode step through every block of the stack, in order: ``weights``
+    is a sequence of llama3_layer_weights structs, ``k_caches``/``v_caches``
+    the blocks' cache tensors."""
+    n = len(weights)
+    arr = (llama3_layer_weights * n)(*weights)
+    kp = (ctypes.c_void_p * n)(*[t.data_ptr() for t in k_caches])
+    vp = (ctypes.c_void_p * n)(*[t.data_ptr() for t in v_caches])
+    _check("llama3_decode_step", lib().llama3_decode_step(
+        ctypes.byref(cfg), arr, n, _ptr(rope), rope_len, _ptr(x), ctypes.cast(kp, ctypes.c_void_p),
+        ctypes.cast(vp, ctypes.c_void_p), cache_cap, batch, start_pos, _ptr(positions), _ptr(ws), ws_bytes,
+        _stream(stream)))
 
 
 def llama3_lm_head_argmax(cfg, norm_w, w_out, h, rows, row_stride, ids_out, logits_out, ws, ws_bytes,

@@ -428,18 +428,13 @@ EpiParams empty_epi() {
 // sum_k W[n, k] X[t, k], with W1|W3 stacked through `w_second`.
 // Skinny GEMM with the weights as the MMA's M side and split-K: fp32 partials
 // P[split][token][feature], reduced by a separate kernel.
-int swapped_partial_gemm(const void* w, int rows_w, const void* w_second, int rows_w2, int out_offset2,
-                         const void* x, int rows_x, int k, float* P, int ldo, int* splits_out,
-                         cudaStream_t st) {
-  CUtensorMap ma, ma2, mb;
-  const int bn = rows_x <= 16 ? 16 : rows_x <= 32 ? 32 : rows_x <= 64 ? 64 : rows_x <= 128 ? 128 : 256;
-  L3_TRY(make_map(&ma, w, rows_w, k, 128));
-  if (w_second) L3_TRY(make_map(&ma2, w_second, rows_w2, k, 128)); else ma2 = ma;
-  L3_TRY(make_map(&mb, x, rows_x, k, bn));
+// Schedule of a weight-streaming GEMM: rows_w (+ rows_w2 stacked) weight rows
+// as the MMA M side, rows_x tokens as N (tile width bn), k deep.
+GemmShape plan_swapped(int rows_w, int rows_w2, int rows_x, int k, int bn) {
   const int tiles = ((rows_w + 127) / 128 + (rows_w2 + 127) / 128) * ((rows_x + bn - 1) / bn);
   const int kblocks = (k + 63) / 64;
   const int splits = choose_splits(tiles, kblocks, num_sms());
-  GemmShape sh = make_shape(rows_w, w_second ? rows_w2 : 0, rows_x, k, bn, splits);
+  GemmShape sh = make_shape(rows_w, rows_w2, rows_x, k, bn, splits);
   // Stream-K over (m-tile, k-block) when it beats the best even split: every
   // CTA streams an equal share of the weights, and a tile shared by several
   // CTAs gets one partial slab per CTA (the tile's last CTA zeroes the slabs
@@ -454,6 +449,18 @@ int swapped_partial_gemm(const void* w, int rows_w, const void* w_second, int ro
       sh.splits = sk.slabs;
     }
   }
+  return sh;
+}
+
+int swapped_partial_gemm(const void* w, int rows_w, const void* w_second, int rows_w2, int out_offset2,
+                         const void* x, int rows_x, int k, float* P, int ldo, int* splits_out,
+                         cudaStream_t st) {
+  CUtensorMap ma, ma2, mb;
+  const int bn = rows_x <= 16 ? 16 : rows_x <= 32 ? 32 : rows_x <= 64 ? 64 : rows_x <= 128 ? 128 : 256;
+  L3_TRY(make_map(&ma, w, rows_w, k, 128));
+  if (w_second) L3_TRY(make_map(&ma2, w_second, rows_w2, k, 128)); else ma2 = ma;
+  L3_TRY(make_map(&mb, x, rows_x, k, bn));
+  GemmShape sh = plan_swapped(rows_w, w_second ? rows_w2 : 0, rows_x, k, bn);
   EpiParams ep = empty_epi();
   ep.out = P;
   ep.ldo = ldo;
@@ -1174,6 +1181,26 @@ int llama3_layer_decode_chained(const llama3_config* cfg, const llama3_layer_wei
                                       start_pos, ws, ws_bytes, stream);
   return llama3_layer_decode(cfg, w, rope, rope_len, x, k_cache, v_cache, cache_cap, batch, start_pos, ws, ws_bytes,
                              stream);
+}
+
+int llama3_decode_step(const llama3_config* cfg, const llama3_layer_weights* layers, int n_layers,
+                       const float* rope, int rope_len, void* x, void* const* k_caches, void* const* v_caches,
+                       int cache_cap, int batch, int start_pos, const int32_t* positions, void* ws,
+                       size_t ws_bytes, llama3_stream_t stream) {
+  if (!layers || n_layers < 1 || !k_caches || !v_caches) return LLAMA3_ERR_ARG;
+  if (positions && (reinterpret_cast<uintptr_t>(positions) & 3)) return LLAMA3_ERR_ALIGN;
+  Workspace L;
+  for (int i = 0; i < n_layers; ++i)
+    L3_TRY(check_layer_args(cfg, &layers[i], rope, rope_len, x, k_caches[i], v_caches[i], cache_cap, batch, 1,
+                            start_pos, ws, ws_bytes, &L));
+  (void)L;
+  // the block loop, each block handing the next one its normalised input
+  for (int i = 0; i < n_layers; ++i) {
+    const void* next_norm = i + 1 < n_layers ? layers[i + 1].attention_norm : nullptr;
+    L3_TRY(llama3_layer_decode_chained(cfg, &layers[i], rope, rope_len, x, k_caches[i], v_caches[i], cache_cap,
+                                       batch, start_pos, positions, next_norm, i > 0, ws, ws_bytes, stream));
+  }
+  return LLAMA3_OK;
 }
 
 int llama3_layer_forward_docs(const llama3_config* cfg, const llama3_layer_weights* w, const float* rope,

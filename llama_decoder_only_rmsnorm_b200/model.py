@@ -59,10 +59,17 @@ class Llama3Stack:
                                    self.cache_cap, self.batch, seq, start_pos, self.ws, self.ws_bytes, stream)
 
     def _decode_chain(self, x, start_pos, positions, stream, layers):
-        # Each block leaves the next block's normalised input in the workspace
-        # (llama3_layer_decode_chained); a block is told so only when the call
-        # before it, on the same workspace, was the block right before it.
-        idx = list(range(len(self.layers)) if layers is None else layers)
+        # Every block in order: one call for the whole step (llama3_decode_step).
+        if layers is None or list(layers) == list(range(len(self.layers))):
+            B.llama3_decode_step(self.cfg, self.wstructs, self.rope, self.rope_len, x,
+                                 [kc for kc, _ in self.caches], [vc for _, vc in self.caches], self.cache_cap,
+                                 self.batch, start_pos, positions, self.ws, self.ws_bytes, stream)
+            return
+        # Any other order: one call per block.  Each block leaves the next
+        # block's normalised input in the workspace (llama3_layer_decode_chained);
+        # a block is told so only when the call before it, on the same
+        # workspace, was the block right before it.
+        idx = list(layers)
         for n, i in enumerate(idx):
             kc, vc = self.caches[i]
             nxt = idx[n + 1] if n + 1 < len(idx) else None

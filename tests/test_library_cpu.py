@@ -107,6 +107,27 @@ def test_lm_head_and_helpers_reject_bad_arguments():
     assert lib.llama3_attention(ctypes.byref(c), FAKE, FAKE, FAKE, 8, 1, 9, 0, FAKE, FAKE, 1 << 30, None) == 1
 
 
+def test_decode_step_rejects_bad_arguments_before_launch():
+    lib = B.lib()
+    c = cfg8b()
+    ws = (B.llama3_layer_weights * 2)(_weights(), _weights())
+    caches = (ctypes.c_void_p * 2)(FAKE, FAKE)
+    cp = ctypes.cast(caches, ctypes.c_void_p)
+    step = lambda **k: lib.llama3_decode_step(ctypes.byref(c), k.get("w", ws), k.get("n", 2), FAKE, 9000, FAKE,
+                                              k.get("kc", cp), cp, k.get("cap", 8193), k.get("batch", 32),
+                                              k.get("pos", 8192), k.get("positions", None), FAKE,
+                                              k.get("ws_bytes", 1 << 40), None)
+    assert step(n=0) == 1
+    assert step(w=None) == 1
+    assert step(kc=None) == 1
+    assert step(pos=8193) == 1                        # start_pos + 1 > cache capacity
+    assert step(batch=0) == 1
+    assert step(positions=ctypes.c_void_p(FAKE + 2)) == 2
+    assert step(ws_bytes=16) == 3
+    bad = (ctypes.c_void_p * 2)(FAKE, FAKE + 8)       # second block's cache not 16-byte aligned
+    assert step(kc=ctypes.cast(bad, ctypes.c_void_p)) == 2
+
+
 def test_kernel_path_and_wait_limit_switches():
     assert B.llama3_set_kernel_path(1) == 0
     assert B.llama3_set_kernel_path(0) == 1
