@@ -27,7 +27,9 @@
 //  * P (bf16, two per 32-bit column) is written back into TMEM over the
 //    scores just read (keys 0-127 -> columns 0-63) and P.V takes its A operand
 //    from TMEM, so P never goes through shared memory; K and V are both
-//    double-buffered in shared memory.
+//    double-buffered in shared memory.  P is handed over in two halves (keys
+//    0-63, then 64-127), so the first half's P.V runs on the tensor core
+//    while the softmax is still on the second half's exponentials.
 //  * A whole warp runs the MMA loop (warp-uniform addresses and descriptors)
 //    and one elected lane issues; a head's next S goes right behind the P.V
 //    that reads its columns, since the MMAs of one thread run in issue order.
@@ -118,7 +120,7 @@ struct FlashCfg {
   static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
   static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
   static constexpr int OFF_BAR = OFF_V + VST * KV_BYTES;
-  static constexpr int N_BARS = 2 + 2 + 2 * KST + 2 * VST + 2 + 2 + 2;
+  static constexpr int N_BARS = 2 + 2 + 2 * KST + 2 * VST + 2 + 2 + 2 + 2;
   static constexpr int SMEM_BYTES = 1024 + OFF_BAR + N_BARS * 8 + 16;
   static_assert(SMEM_BYTES <= 232448, "shared memory");
   static_assert(HD % 32 == 0 && HD <= 128, "head_dim");
@@ -161,22 +163,18 @@ __device__ __forceinline__ void flash_pack_store(uint32_t (&r)[32], uint32_t tad
   for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
   tmem_st16(taddr, pk);
 }
-// The whole row: all 128 exponentials before any pack or store, so that the
-// four chunks overlap; then the bf16 pairs go to the 64 TMEM columns at taddr
-// (keys 0-127 -> columns 0-63).  Returns the row's sum over the tile.
+// Half a row (64 scores): both chunks' exponentials before any pack or store,
+// so that they overlap; then the bf16 pairs go to the 32 TMEM columns at
+// taddr.  Returns the half row's sum.
 template <bool MASKED>
-__device__ __forceinline__ float flash_exp_row(uint32_t (&ra)[32], uint32_t (&rb)[32], uint32_t (&rc)[32],
-                                                uint32_t (&rd)[32], float scl, float neg_m, uint32_t taddr) {
-  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f, s4 = 0.f, s5 = 0.f, s6 = 0.f, s7 = 0.f;
+__device__ __forceinline__ float flash_exp_half(uint32_t (&ra)[32], uint32_t (&rb)[32], float scl, float neg_m,
+                                                 uint32_t taddr) {
+  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
   flash_exp_inplace<MASKED>(ra, scl, neg_m, s0, s1);
   flash_exp_inplace<MASKED>(rb, scl, neg_m, s2, s3);
-  flash_exp_inplace<MASKED>(rc, scl, neg_m, s4, s5);
-  flash_exp_inplace<MASKED>(rd, scl, neg_m, s6, s7);
   flash_pack_store(ra, taddr);
   flash_pack_store(rb, taddr + 16);
-  flash_pack_store(rc, taddr + 32);
-  flash_pack_store(rd, taddr + 48);
-  return ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
+  return (s0 + s1) + (s2 + s3);
 }
 
 template <bool MASKED>
@@ -194,7 +192,7 @@ __device__ __forceinline__ float flash_row_max(uint32_t (&r)[32], int key0, int 
 
 // The barriers the three roles share (all in shared memory).
 struct FlashBars {
-  uint64_t *q_full, *q_empty, *k_full, *k_empty, *v_full, *v_empty, *s_full, *p_full, *o_done;
+  uint64_t *q_full, *q_empty, *k_full, *k_empty, *v_full, *v_empty, *s_full, *p_full, *o_done, *p_half;
 };
 
 // Producer (one thread): per work unit the Q tiles of its one or two heads,
@@ -288,16 +286,17 @@ __device__ __forceinline__ void flash_issue_mma(uint8_t* smem, const FlashBars& 
     }
     __syncwarp();
   };
-  auto issue_pv = [&](int s, int vst, bool accumulate) {
+  // keys 16k.. for k in [k0, k1): P in columns 8k.., V rows 16k..
+  auto issue_pv = [&](int s, int vst, bool accumulate, int k0, int k1) {
     const uint32_t d = tmem_base + s * 256 + 128;
-    const uint32_t pa = tmem_base + s * 256;   // P: keys 16k.. in columns 8k..
+    const uint32_t pa = tmem_base + s * 256;
     const uint32_t va = smem_u32(smem + C::OFF_V + vst * C::KV_BYTES);
     if (leader) {
 #pragma unroll
-      for (int k = 0; k < 8; ++k)
+      for (int k = k0; k < k1; ++k)
         tc_mma_f16_ts(d, pa + k * 8, sw128_desc(va + k * 2048, 1024, C::TILE_BYTES), IDESC_O,
                       (accumulate || k > 0) ? 1u : 0u);
-      tc_commit(&o_done[s]);
+      if (k1 == 8) tc_commit(&o_done[s]);
     }
     __syncwarp();
   };
@@ -323,10 +322,15 @@ __device__ __forceinline__ void flash_issue_mma(uint8_t* smem, const FlashBars& 
       const bool more = j + 1 < nt;
       bool k_ready = false;
       for (int s = 0; s < nslots; ++s) {
+        // keys 0-63 of P.V as soon as the softmax has written their P,
+        // while it works on keys 64-127; then the rest and the next S
+        if (!mbar_wait_warp(&B.p_half[s], (pph >> s) & 1u, wait_ns)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv(s, vs, j > jt0, 0, 4);
         if (!mbar_wait_warp(&p_full[s], (pph >> s) & 1u, wait_ns)) { ok = false; break; }
         pph ^= 1u << s;
         tc_fence_after();
-        issue_pv(s, vs, j > jt0);
+        issue_pv(s, vs, true, 4, 8);
         if (more) {
           if (!k_ready && !mbar_wait_warp(&k_full[ks], kph, wait_ns)) { ok = false; break; }
           k_ready = true;
@@ -365,8 +369,9 @@ __global__ void __launch_bounds__(kFlashThreads, 1)
   uint64_t* s_full = v_empty + C::VST;
   uint64_t* p_full = s_full + 2;
   uint64_t* o_done = p_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_done + 2);
-  const FlashBars fbars{q_full, q_empty, k_full, k_empty, v_full, v_empty, s_full, p_full, o_done};
+  uint64_t* p_half = o_done + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(p_half + 2);
+  const FlashBars fbars{q_full, q_empty, k_full, k_empty, v_full, v_empty, s_full, p_full, o_done, p_half};
 
   // warp index through a shuffle: the compiler then treats it as uniform
   // across the warp, so the whole-warp MMA issuer below keeps its addresses
@@ -376,6 +381,7 @@ __global__ void __launch_bounds__(kFlashThreads, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&q_full[s], 1); mbar_init(&q_empty[s], 1);
       mbar_init(&s_full[s], 1); mbar_init(&p_full[s], 128); mbar_init(&o_done[s], 1);
+      mbar_init(&p_half[s], 128);
     }
     for (int s = 0; s < C::KST; ++s) { mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1); }
     for (int s = 0; s < C::VST; ++s) { mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1); }
@@ -472,10 +478,22 @@ __global__ void __launch_bounds__(kFlashThreads, 1)
         }
         const float scl = fs.scale_log2;
         const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;   // a row with no visible key yet: p = 0
+        // P in two hand-offs: keys 0-63 (columns 0-31), then keys 64-127
+        // (columns 32-63), so that the first half's P.V overlaps the second
+        // half's exponentials
+        float la, lb;
         if (need_mask)
-          l += flash_exp_row<true>(ra, rb, rc, rd, scl, neg_m, s_tmem);
+          la = flash_exp_half<true>(ra, rb, scl, neg_m, s_tmem);
         else
-          l += flash_exp_row<false>(ra, rb, rc, rd, scl, neg_m, s_tmem);
+          la = flash_exp_half<false>(ra, rb, scl, neg_m, s_tmem);
+        tc_wait_st();
+        tc_fence_before();
+        mbar_arrive(&p_half[slot]);
+        if (need_mask)
+          lb = flash_exp_half<true>(rc, rd, scl, neg_m, s_tmem + 32);
+        else
+          lb = flash_exp_half<false>(rc, rd, scl, neg_m, s_tmem + 32);
+        l += la + lb;
         tc_wait_st();
         tc_fence_before();
         if (!(fs.withhold == 2 && k_ == 0 && j == jt0 && row == 0 && slot == 0)) mbar_arrive(&p_full[slot]);
