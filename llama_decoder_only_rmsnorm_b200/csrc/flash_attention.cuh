@@ -40,6 +40,9 @@
 //    unwritten cache entry is ever touched.
 //  * Causal tile skipping: a query tile visits only key tiles up to its last
 //    position; work units are issued longest first, in snake order.
+//  * The epilogue goes through 2 KB of shared memory per softmax warp, 32
+//    columns at a time, so the global stores write 64 contiguous bytes per
+//    row instead of one 16-byte piece in each of 32 rows.
 // The split of registers is only valid for a launch of 384 threads at 168
 // registers each (128*104 + 256*200 = 384*168); the host checks the compiled
 // register count before every launch.
@@ -121,7 +124,9 @@ struct FlashCfg {
   static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
   static constexpr int OFF_BAR = OFF_V + VST * KV_BYTES;
   static constexpr int N_BARS = 2 + 2 + 2 * KST + 2 * VST + 2 + 2 + 2 + 2;
-  static constexpr int SMEM_BYTES = 1024 + OFF_BAR + N_BARS * 8 + 16;
+  // output staging: 2 KB (32 rows x 32 bf16) per softmax warp
+  static constexpr int OFF_STAGE = (OFF_BAR + N_BARS * 8 + 16 + 127) / 128 * 128;
+  static constexpr int SMEM_BYTES = 1024 + OFF_STAGE + 8 * 2048;
   static_assert(SMEM_BYTES <= 232448, "shared memory");
   static_assert(HD % 32 == 0 && HD <= 128, "head_dim");
 };
@@ -503,26 +508,38 @@ __global__ void __launch_bounds__(kFlashThreads, 1)
       if (!mbar_wait_warp(&o_done[slot], oph, wait_ns)) break;
       oph ^= 1u;
       tc_fence_after();
-      const int t = qt * 128 + row;
       const int h = g * fs.n_rep + pair * 2 + slot;
       const float inv = 1.f / l;
-      bf16* orow = out + ((size_t)b * fs.S + t) * fs.ldo + (size_t)h * HD;
+      // 32 columns at a time through this warp's 2 KB of shared memory
+      // (row r at 64 r bytes, its 16-byte piece k in slot k ^ ((r >> 1) & 3),
+      // so neither the row-wise writes nor the piece-wise reads conflict),
+      // then stored with four lanes per row: 64 contiguous bytes per row
+      uint8_t* stage = smem + C::OFF_STAGE + (warp - 4) * 2048;
+      const int t0 = qt * 128 + quarter * 32;
+      bf16* obase = out + ((size_t)b * fs.S + t0) * fs.ldo + (size_t)h * HD;
 #pragma unroll 1
       for (int c = 0; c < HD / 32; ++c) {
         uint32_t r[32];
         tmem_ld32(o_tmem + c * 32, r);
         tc_wait_ld();
-        if (t < fs.S) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint4 o;
-            o.x = pack_bf16x2(__uint_as_float(r[8 * q + 0]) * inv, __uint_as_float(r[8 * q + 1]) * inv);
-            o.y = pack_bf16x2(__uint_as_float(r[8 * q + 2]) * inv, __uint_as_float(r[8 * q + 3]) * inv);
-            o.z = pack_bf16x2(__uint_as_float(r[8 * q + 4]) * inv, __uint_as_float(r[8 * q + 5]) * inv);
-            o.w = pack_bf16x2(__uint_as_float(r[8 * q + 6]) * inv, __uint_as_float(r[8 * q + 7]) * inv);
-            *reinterpret_cast<uint4*>(orow + c * 32 + q * 8) = o;
-          }
+        for (int k = 0; k < 4; ++k) {
+          uint4 o;
+          o.x = pack_bf16x2(__uint_as_float(r[8 * k + 0]) * inv, __uint_as_float(r[8 * k + 1]) * inv);
+          o.y = pack_bf16x2(__uint_as_float(r[8 * k + 2]) * inv, __uint_as_float(r[8 * k + 3]) * inv);
+          o.z = pack_bf16x2(__uint_as_float(r[8 * k + 4]) * inv, __uint_as_float(r[8 * k + 5]) * inv);
+          o.w = pack_bf16x2(__uint_as_float(r[8 * k + 6]) * inv, __uint_as_float(r[8 * k + 7]) * inv);
+          *reinterpret_cast<uint4*>(stage + lane * 64 + ((k ^ ((lane >> 1) & 3)) << 4)) = o;
         }
+        __syncwarp();
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const int rr = m * 8 + (lane >> 2), k = lane & 3;
+          const uint4 o = *reinterpret_cast<const uint4*>(stage + rr * 64 + ((k ^ ((rr >> 1) & 3)) << 4));
+          if (t0 + rr < fs.S)
+            *reinterpret_cast<uint4*>(obase + (size_t)rr * fs.ldo + c * 32 + k * 8) = o;
+        }
+        __syncwarp();
       }
       tc_fence_before();
     }
