@@ -19,6 +19,7 @@
 #include "sampling.cuh"
 #include "simt.cuh"
 #include "tc_gemm.cuh"
+#include "tc_gemm_pair.cuh"
 
 using namespace l3;
 
@@ -26,6 +27,10 @@ namespace {
 
 thread_local int t_last_cuda = 0;
 int g_kernel_path = 0;       // 0 = tcgen05 for bf16, 1 = SIMT everywhere
+// Prefill GEMMs run on CTA pairs (tc_gemm_pair.cuh) once there are at least
+// 256 token rows: on the 8B prefill step that measured 107.1 against 109.2 ms
+// with single-CTA tiles (interleaved runs on one box), bit-identical results.
+bool use_pair_gemm(int m) { return m >= 256; }
 int g_wait_ms = 2000;        // bounded device waits
 int g_withhold = 0;          // failure-detection test hook (llama3_set_test_withheld_arrival)
 constexpr int kMaxDevices = 64;
@@ -428,6 +433,63 @@ int launch_gemm(int kind, const CUtensorMap& a, const CUtensorMap& a2, const CUt
   return launch_check();
 }
 
+// Prefill GEMM shape for CTA pairs: 256-row tiles of A, raster groups of 16
+// of them (the same 4096 rows as the single-CTA raster's 32 tiles of 128).
+GemmShape make_shape_pair(int rows_a, int rows_b, int k, int bn) {
+  GemmShape s = make_shape(rows_a, 0, rows_b, k, bn, 1);
+  s.tiles_m1 = s.tiles_m = (rows_a + 255) / 256;
+  s.units = s.tiles_m * s.tiles_n;
+  s.group_m = std::max(1, std::min(L3_GROUP_M / 2, s.tiles_m));
+  return s;
+}
+
+template <int BN, int STAGES, int EPI, bool DUAL>
+int launch_gemm_pair(int kind, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2,
+                     const GemmShape& sh, const EpiParams& ep, cudaStream_t st) {
+  using Cfg = TcGemmPairCfg<BN, STAGES, DUAL>;
+  auto kern = tc_gemm_pair_kernel<BN, STAGES, EPI, DUAL>;
+  int dev = 0;
+  L3_TRY(current_device(&dev));
+  static bool attr_done[kMaxDevices];
+  if (!attr_done[dev]) {
+    L3_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES));
+    attr_done[dev] = true;
+  }
+  if (sh.units <= 0) return LLAMA3_OK;
+  GemmShape s = sh;
+  s.withhold = g_withhold == 1 ? 1 : 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // One persistent pair per cluster slot the device can hold at once (two SMs
+  // of one GPC each); pairs never wait on one another, so a smaller count
+  // would only be slower, never stuck.
+  static int max_pairs[kMaxDevices];
+  if (!max_pairs[dev]) {
+    cfg.gridDim = dim3(2 * std::max(1, num_sms() / 2));
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) n = std::max(1, num_sms() / 2);
+    max_pairs[dev] = std::min(n, std::max(1, num_sms() / 2));
+  }
+  const int pairs = std::min(s.units, max_pairs[dev]);
+  cfg.gridDim = dim3(2 * pairs);
+  const bool after_norm = kind == LLAMA3_KERNEL_GEMM_QKV || kind == LLAMA3_KERNEL_GEMM_W13;
+  cfg.numAttrs = (g_pdl && !after_norm) ? 2 : 1;
+  const unsigned long long wns = wait_ns();
+  L3_LAUNCH(kind, st, cudaLaunchKernelEx(&cfg, kern, a, b, b2, s, ep, wns));
+  return launch_check();
+}
+
 EpiParams empty_epi() {
   EpiParams e;
   memset(&e, 0, sizeof(e));
@@ -707,14 +769,18 @@ int layer_tc_prefill(const llama3_config* c, const llama3_layer_weights* w, cons
   bf16* g = ws_at<bf16>(ws, L.g);
   float* Ap = ws_at<float>(ws, L.attn_part);
   CUtensorMap mxn, mo, mg, mwqkv, mwo, mw1, mw3, mw2;
+  // CTA-pair GEMMs take each weight tile in halves, one per CTA (box rows BN / 2)
+  const bool pair = use_pair_gemm(M);
+  const int bb = pair ? kPrefillBN / 2 : kPrefillBN;
+  const int bd = pair ? 64 : 128;
   L3_TRY(make_map(&mxn, xn, M, D, 128));
   L3_TRY(make_map(&mo, o, M, H * hd, 128));
   L3_TRY(make_map(&mg, g, M, F, 128));
-  L3_TRY(make_map(&mwqkv, w->wqkv, nqkv, D, kPrefillBN));
-  L3_TRY(make_map(&mwo, w->wo, D, H * hd, kPrefillBN));
-  L3_TRY(make_map(&mw1, w->w1, F, D, 128));
-  L3_TRY(make_map(&mw3, w->w3, F, D, 128));
-  L3_TRY(make_map(&mw2, w->w2, D, F, kPrefillBN));
+  L3_TRY(make_map(&mwqkv, w->wqkv, nqkv, D, bb));
+  L3_TRY(make_map(&mwo, w->wo, D, H * hd, bb));
+  L3_TRY(make_map(&mw1, w->w1, F, D, bd));
+  L3_TRY(make_map(&mw3, w->w3, F, D, bd));
+  L3_TRY(make_map(&mw2, w->w2, D, F, bb));
 
   // attention half
   L3_TRY(rmsnorm_any(c, x, D, w->attention_norm, xn, M, st));
@@ -722,29 +788,45 @@ int layer_tc_prefill(const llama3_config* c, const llama3_layer_weights* w, cons
     EpiParams ep = empty_epi();
     ep.seq = S; ep.start_pos = P; ep.n_heads = H; ep.n_kv = KV; ep.head_dim = hd; ep.cache_cap = cap;
     ep.rope = rope; ep.q_out = q; ep.k_cache = kc; ep.v_cache = vc;
-    L3_TRY((launch_gemm<kPrefillBN, 4, EPI_QKV_ROPE, false>(LLAMA3_KERNEL_GEMM_QKV, mxn, mxn, mwqkv, mwqkv,
-                                                             make_shape(M, 0, nqkv, D, kPrefillBN, 1), ep, st)));
+    if (pair)
+      L3_TRY((launch_gemm_pair<kPrefillBN, 6, EPI_QKV_ROPE, false>(
+          LLAMA3_KERNEL_GEMM_QKV, mxn, mwqkv, mwqkv, make_shape_pair(M, nqkv, D, kPrefillBN), ep, st)));
+    else
+      L3_TRY((launch_gemm<kPrefillBN, 4, EPI_QKV_ROPE, false>(LLAMA3_KERNEL_GEMM_QKV, mxn, mxn, mwqkv, mwqkv,
+                                                               make_shape(M, 0, nqkv, D, kPrefillBN, 1), ep, st)));
   }
   L3_TRY(attention_dispatch(c, q, kc, vc, cap, B, S, P, o, Ap, st, doc_start));
   {
     EpiParams ep = empty_epi();
     ep.out = x; ep.res = x; ep.ldo = D;
-    L3_TRY((launch_gemm<kPrefillBN, 4, EPI_RESIDUAL, false>(LLAMA3_KERNEL_GEMM_WO, mo, mo, mwo, mwo,
-                                                             make_shape(M, 0, D, H * hd, kPrefillBN, 1), ep, st)));
+    if (pair)
+      L3_TRY((launch_gemm_pair<kPrefillBN, 6, EPI_RESIDUAL, false>(
+          LLAMA3_KERNEL_GEMM_WO, mo, mwo, mwo, make_shape_pair(M, D, H * hd, kPrefillBN), ep, st)));
+    else
+      L3_TRY((launch_gemm<kPrefillBN, 4, EPI_RESIDUAL, false>(LLAMA3_KERNEL_GEMM_WO, mo, mo, mwo, mwo,
+                                                               make_shape(M, 0, D, H * hd, kPrefillBN, 1), ep, st)));
   }
   // FFN half
   L3_TRY(rmsnorm_any(c, x, D, w->ffn_norm, xn, M, st));
   {
     EpiParams ep = empty_epi();
     ep.out = g; ep.ldo = F;
-    L3_TRY((launch_gemm<128, 4, EPI_SWIGLU, true>(LLAMA3_KERNEL_GEMM_W13, mxn, mxn, mw1, mw3,
-                                                   make_shape(M, 0, F, D, 128, 1), ep, st)));
+    if (pair)
+      L3_TRY((launch_gemm_pair<128, 6, EPI_SWIGLU, true>(LLAMA3_KERNEL_GEMM_W13, mxn, mw1, mw3,
+                                                          make_shape_pair(M, F, D, 128), ep, st)));
+    else
+      L3_TRY((launch_gemm<128, 4, EPI_SWIGLU, true>(LLAMA3_KERNEL_GEMM_W13, mxn, mxn, mw1, mw3,
+                                                     make_shape(M, 0, F, D, 128, 1), ep, st)));
   }
   {
     EpiParams ep = empty_epi();
     ep.out = x; ep.res = x; ep.ldo = D;
-    L3_TRY((launch_gemm<kPrefillBN, 4, EPI_RESIDUAL, false>(LLAMA3_KERNEL_GEMM_W2, mg, mg, mw2, mw2,
-                                                             make_shape(M, 0, D, F, kPrefillBN, 1), ep, st)));
+    if (pair)
+      L3_TRY((launch_gemm_pair<kPrefillBN, 6, EPI_RESIDUAL, false>(
+          LLAMA3_KERNEL_GEMM_W2, mg, mw2, mw2, make_shape_pair(M, D, F, kPrefillBN), ep, st)));
+    else
+      L3_TRY((launch_gemm<kPrefillBN, 4, EPI_RESIDUAL, false>(LLAMA3_KERNEL_GEMM_W2, mg, mg, mw2, mw2,
+                                                               make_shape(M, 0, D, F, kPrefillBN, 1), ep, st)));
   }
   return LLAMA3_OK;
 }
@@ -1087,6 +1169,12 @@ int llama3_linear(const llama3_config* cfg, const void* x, const void* w, const 
     EpiParams ep = empty_epi();
     ep.out = y; ep.res = residual; ep.ldo = n;
     L3_TRY(make_map(&ma, x, m, k, 128));
+    if (use_pair_gemm(m)) {
+      L3_TRY(make_map(&mb, w, n, k, kPrefillBN / 2));
+      const GemmShape sh = make_shape_pair(m, n, k, kPrefillBN);
+      if (residual) return launch_gemm_pair<kPrefillBN, 6, EPI_RESIDUAL, false>(LLAMA3_KERNEL_GEMM_WO, ma, mb, mb, sh, ep, st);
+      return launch_gemm_pair<kPrefillBN, 6, EPI_STORE, false>(LLAMA3_KERNEL_GEMM_WO, ma, mb, mb, sh, ep, st);
+    }
     L3_TRY(make_map(&mb, w, n, k, kPrefillBN));
     GemmShape sh = make_shape(m, 0, n, k, kPrefillBN, 1);
     if (residual) return launch_gemm<kPrefillBN, 4, EPI_RESIDUAL, false>(LLAMA3_KERNEL_GEMM_WO, ma, ma, mb, mb, sh, ep, st);

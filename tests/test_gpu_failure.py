@@ -37,8 +37,8 @@ def _hook_off():
 
 
 def test_gemm_accumulator_wait_gives_up_then_next_call_is_exact():
-    # 20 x 23 tiles of 128 x 256 on at most 148 CTAs: at least three tiles per
-    # CTA, so the withheld release of the first accumulator is waited for
+    # 10 x 23 tiles of 256 x 256 on at most 74 CTA pairs: at least three tiles
+    # per pair, so the withheld release of the first accumulator is waited for
     m, n, k = 2560, 5888, 64
     g = torch.Generator(device="cpu").manual_seed(41)
     x = torch.randn((m, k), generator=g).to(torch.bfloat16).to(DEV)
