@@ -395,10 +395,11 @@ def run_ours(args):
     F = PREFILL.ffn_hidden
     w13_flop = 2.0 * S * (2 * F) * D
     achieved = w13_flop / (k_ms / 1e3) / 1e12 if k_ms else None
-    roofline = {"bound": "tensor", "kernel": "tc_gemm w1|w3 + SwiGLU (M=8192, N=2x14336, K=4096)",
+    roofline = {"bound": "tensor", "kernel": "tc_gemm_pair w1|w3 + SwiGLU (M=8192, N=2x14336, K=4096; CTA pairs)",
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": (achieved / peak) if achieved else None, "peak_source": peak_src,
                 "traffic": recorded_traffic("gemm_w13", ["llama_decoder_only_rmsnorm_b200/csrc/tc_gemm.cuh",
+                                                         "llama_decoder_only_rmsnorm_b200/csrc/tc_gemm_pair.cuh",
                                                          "llama_decoder_only_rmsnorm_b200/csrc/llama3.cu"]),
                 "kernel_ms": k_ms, "timed_launches": len(w13)}
     total_flop = n_layers * (2.0 * S * 6.979e9 / 32) + 2.0 * D * PREFILL.vocab  # linear layers + LM head row
