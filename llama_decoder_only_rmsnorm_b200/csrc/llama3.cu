@@ -478,7 +478,10 @@ int launch_gemm_pair(int kind, const CUtensorMap& a, const CUtensorMap& b, const
   if (!max_pairs[dev]) {
     cfg.gridDim = dim3(2 * std::max(1, num_sms() / 2));
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) n = std::max(1, num_sms() / 2);
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) {
+      (void)cudaGetLastError();   // a failed query must not be reported as the launch's error
+      n = std::max(1, num_sms() / 2);
+    }
     max_pairs[dev] = std::min(n, std::max(1, num_sms() / 2));
   }
   const int pairs = std::min(s.units, max_pairs[dev]);
