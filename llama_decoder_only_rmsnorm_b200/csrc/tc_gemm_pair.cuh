@@ -43,7 +43,9 @@ struct TcGemmPairCfg {
   static constexpr int ACC_BUFS = 2;
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = STAGES * A_BYTES;
-  static constexpr int SLACK = 16384;                // keeps any operand read inside the allocation
+  // 16 KB of spare shared memory after the B ring: a margin kept from the
+  // first version of this kernel; the MMAs read only the ring itself.
+  static constexpr int SLACK = 16384;
   static constexpr int OFF_BAR = OFF_B + STAGES * NB * B_BYTES + SLACK;
   static constexpr int BAR_BYTES = (2 * STAGES + 2 * ACC_BUFS) * 8 + 16;
   static constexpr int SMEM_BYTES = 1024 + OFF_BAR + BAR_BYTES;
