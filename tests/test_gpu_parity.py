@@ -97,6 +97,27 @@ def test_linear_in_place_residual():
     assert_close(y, want, "bf16", "in-place residual")
 
 
+@pytest.mark.parametrize("n,k,residual", [(768, 512, False), (4096, 4096, True), (264, 200, True)])
+def test_linear_cta_pairs_match_single_cta_bit_for_bit(n, k, residual):
+    """From 256 rows on, the prefill GEMMs run on CTA pairs (256-row tiles,
+    half of each weight tile per CTA); below, on single CTAs.  Both reduce
+    every output element over k in the same order, so the first 255 rows of
+    a 512-row product equal, bit for bit, the same rows computed alone."""
+    g = torch.Generator(device="cpu").manual_seed(n + k)
+    x = torch.randn((512, k), generator=g).to(torch.bfloat16).to(DEV)
+    w = (torch.randn((n, k), generator=g) * 0.05).to(torch.bfloat16).to(DEV)
+    r = torch.randn((512, n), generator=g).to(torch.bfloat16).to(DEV) if residual else None
+    cfg = B.make_config(512, 8, 8, 1024)
+    y_pair = G.empty((512, n), dtype=torch.bfloat16, device=DEV)
+    B.llama3_linear(cfg, x, w, r, y_pair, 512, n, k)
+    y_single = G.empty((255, n), dtype=torch.bfloat16, device=DEV)
+    B.llama3_linear(cfg, x[:255].contiguous(), w, r[:255].contiguous() if residual else None, y_single, 255, n, k)
+    torch.cuda.synchronize()
+    assert torch.equal(y_pair[:255], y_single)
+    want = f64(x) @ f64(w).T + (f64(r) if residual else 0.0)
+    assert_close(y_pair, want, "bf16", f"CTA-pair linear {n}x{k}")
+
+
 # --------------------------------------------------------------- attention
 def _attn_case(Bn, S, P, H, KV, hd, seed):
     g = torch.Generator(device="cpu").manual_seed(seed)
